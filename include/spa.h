@@ -1,0 +1,228 @@
+/*
+ * spa.h -- C ABI of libspa: paged / selected-token sparse attention over a
+ * block-table KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the staged pipeline described on the onnxruntime pages
+ * "[WebGPU] Add PagedAttention metadata and GPT-OSS support" (PR #32277),
+ * "[WebGPU] Add SparsePagedAttention" (PR #32533), "[WebGPU] Add
+ * DynamicSparseAttention" (PR #32529) and PR #33472 (INT8 KV cache):
+ *   1. metadata prepare    -> spa_prepare_metadata
+ *   2. KV append scatter   -> spa_append_kv
+ *   3.-5. gather, scaled QK + joint softmax with a learned sink,
+ *         split-KV partials + log-sum-exp combine -> spa_attention
+ *
+ * Conventions for every entry point:
+ *   - Every pointer is a DEVICE pointer unless marked [host].  All buffers are
+ *     owned by the caller; the library allocates no device memory, never
+ *     synchronises the stream and never reads device memory from the host, so
+ *     every call may be captured into a CUDA graph.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - The return value reports HOST-side problems only (SPA_OK or a negative
+ *     SPA_ERR_* code; spa_error_string() gives a message).  When an error is
+ *     returned nothing was enqueued.
+ *   - Problems visible only on the device (malformed lengths, bad block ids,
+ *     bad selected indices, host bounds exceeded) are OR-ed into the int32
+ *     word `*status` (SPA_ST_* bits).  The caller clears it; kernels never
+ *     clear it.  Whatever the inputs, every memory access stays inside the
+ *     buffers whose sizes the arguments describe.  When a bit other than
+ *     SPA_ST_BAD_IDX is set, the outputs of the affected requests are
+ *     unspecified.
+ *   - Integer layouts are int32, row-major, densely packed.
+ */
+#ifndef SPA_H_
+#define SPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so that the header needs no CUDA headers. */
+typedef struct CUstream_st* spa_stream_t;
+
+/* Element encodings. */
+typedef enum {
+  SPA_F32 = 0,  /* IEEE binary32                                   */
+  SPA_F16 = 1,  /* IEEE binary16                                   */
+  SPA_BF16 = 2, /* bfloat16                                        */
+  SPA_I8 = 3    /* signed int8 with per-channel fp32 scales (cache) */
+} spa_dtype_t;
+
+/* Host-side return codes. */
+#define SPA_OK 0
+#define SPA_ERR_INVALID_ARG (-1) /* null required pointer, bad size, H_q % H_kv != 0, bad dtype combination */
+#define SPA_ERR_UNSUPPORTED (-2) /* non-causal, main selection combined with window/aux, unsupported D */
+#define SPA_ERR_WORKSPACE (-3)   /* workspace missing, too small or misaligned */
+#define SPA_ERR_CUDA (-4)        /* a kernel launch failed; see spa_error_string(SPA_ERR_CUDA) */
+
+/* Device status bits (OR-ed into *status). */
+#define SPA_ST_BAD_CU 0x1     /* cu_seqlens_q not non-decreasing from 0 to T, or a negative past length */
+#define SPA_ST_CAPACITY 0x2   /* a position lies beyond the block table (pos >= MB * block_size) */
+#define SPA_ST_BAD_BLOCK 0x4  /* a block-table entry needed by a position is outside [0, num_blocks) */
+#define SPA_ST_BOUNDS 0x8     /* a device length exceeds the host bound max_seqlen_q / max_seqlen_k */
+#define SPA_ST_BAD_IDX 0x10   /* a selected index is < -1 or beyond its range; it was skipped */
+
+/*
+ * spa_prepare_metadata -- step 1, exact per-request and per-token metadata on
+ * the device, replacing a device-to-host readback per layer.
+ * Source: "[WebGPU] Add PagedAttention metadata and GPT-OSS support",
+ * Description / Changes (host replay-wide bounds; exact seqlen_k and
+ * seqlens_q derived on device) and review item T1 (seqlen_k = -1 for an
+ * empty request); "[WebGPU] Add SparsePagedAttention", File summaries
+ * (token_meta: sanitised per-token metadata).
+ *
+ * Inputs:
+ *   cu_seqlens_q [B+1]  cumulative query lengths; request b owns packed tokens
+ *                       [cu[b], cu[b+1]).  Malformed values are clamped to a
+ *                       non-decreasing sequence in [0, T] starting at 0 and
+ *                       flagged SPA_ST_BAD_CU.
+ *   past_seqlens [B]    tokens already resident in the cache (negative -> 0, flagged).
+ *   block_table [B, MB] physical block id of each logical block (-1 = unmapped).
+ *   B, T                [host] number of requests / packed query tokens.
+ *   max_seqlen_q, max_seqlen_k [host] replay-wide bounds; a request with
+ *                       q_len > max_seqlen_q or past + q_len > max_seqlen_k
+ *                       sets SPA_ST_BOUNDS.
+ *   MB, block_size, num_blocks [host] block-table width, tokens per block,
+ *                       number of physical blocks in the cache.
+ * Outputs:
+ *   seqlens_q [B]       q_len[b] = cu'[b+1] - cu'[b]
+ *   seqlen_k  [B]       past[b] + q_len[b] - 1 (so -1 for a request with no tokens)
+ *   token_batch [T]     request owning token t (-1 if none)
+ *   token_pos   [T]     absolute position past[b] + t - cu'[b] (-1 if no owner)
+ *   slot_mapping [T]    block_table[b, pos / bs] * bs + pos % bs, or -1 when the
+ *                       position is beyond the table (SPA_ST_CAPACITY) or its
+ *                       block id is invalid (SPA_ST_BAD_BLOCK)
+ *   status              OR-ed status bits.
+ * B = 0 or T = 0 is valid (outputs of length 0 are not touched).
+ */
+int spa_prepare_metadata(const int32_t* cu_seqlens_q, const int32_t* past_seqlens,
+                         const int32_t* block_table, int32_t B, int32_t T, int32_t max_seqlen_q,
+                         int32_t max_seqlen_k, int32_t MB, int32_t block_size, int32_t num_blocks,
+                         int32_t* seqlens_q, int32_t* seqlen_k, int32_t* token_batch,
+                         int32_t* token_pos, int32_t* slot_mapping, int32_t* status,
+                         spa_stream_t stream);
+
+/*
+ * spa_append_kv -- step 2, scatter the current tokens' K/V rows into the paged
+ * cache through slot_mapping.
+ * Source: "[WebGPU] Add SparsePagedAttention", File summaries (scatter current
+ * K/V into the cache using slot_mapping); PR #33472, Key Changes (INT8 KV
+ * cache append with key_scale / value_scale).
+ *
+ *   k_new, v_new [T, H_kv, D]  activation dtype `act` (SPA_F32/F16/BF16).
+ *   k_cache, v_cache [num_blocks, block_size, H_kv, D]  dtype `cache`, which is
+ *                     either `act` (exact copy) or SPA_I8.
+ *   k_scale, v_scale [H_kv, D] fp32, required iff cache == SPA_I8:
+ *                     q8 = clamp(rint(float(x) / scale[h, d]), -128, 127),
+ *                     IEEE fp32 division, round half to even.
+ *   slot_mapping [T]  destination slot of token t; -1 skips the token; a slot
+ *                     outside [0, num_blocks * block_size) is skipped and sets
+ *                     SPA_ST_BAD_BLOCK.
+ * T = 0 is valid.  D must be a multiple of 8 (and of 16 for SPA_I8).
+ */
+int spa_append_kv(const void* k_new, const void* v_new, int32_t act, void* k_cache, void* v_cache,
+                  int32_t cache, const float* k_scale, const float* v_scale,
+                  const int32_t* slot_mapping, int32_t T, int32_t H_kv, int32_t D,
+                  int32_t block_size, int32_t num_blocks, int32_t* status, spa_stream_t stream);
+
+/*
+ * Arguments of spa_attention (steps 3-5).  `struct_size` must be set to
+ * sizeof(spa_attention_args_t) so that the struct can grow compatibly.
+ * Sources: "[WebGPU] Add DynamicSparseAttention", Description / Attention
+ * (selected main-cache and local-plus-auxiliary modes, joint FP32 stable
+ * softmax with optional sink, guarded int32 indices) and QKV and cache (GQA
+ * head mapping); "[WebGPU] Add PagedAttention metadata and GPT-OSS support",
+ * Description (local window, learned head sink) and review item Q3 (window
+ * start); "[WebGPU] Add SparsePagedAttention", File summaries (main and
+ * auxiliary partial FP32 softmax state, finalize merge with the sink).
+ */
+typedef struct spa_attention_args {
+  size_t struct_size;
+  /* queries and output, [T, H_q, D] in `act` (SPA_F32 / SPA_F16 / SPA_BF16) */
+  const void* q;
+  void* out;
+  int32_t act;
+  int32_t T, B, H_q, H_kv, D; /* [host]; H_q must be a positive multiple of H_kv; D in {64, 128} */
+  /* paged cache [num_blocks, block_size, H_kv, D] in `cache` (== act, or SPA_I8 with scales) */
+  const void* k_cache;
+  const void* v_cache;
+  int32_t cache;
+  const float* k_scale; /* [H_kv, D], SPA_I8 only */
+  const float* v_scale; /* [H_kv, D], SPA_I8 only */
+  const int32_t* block_table; /* [B, MB] */
+  int32_t MB, block_size, num_blocks; /* [host] */
+  /* metadata from spa_prepare_metadata */
+  const int32_t* cu_seqlens_q; /* [B+1] */
+  const int32_t* seqlens_q;    /* [B]   */
+  const int32_t* seqlen_k;     /* [B]   total - 1 */
+  const int32_t* token_batch;  /* [T]   */
+  const int32_t* token_pos;    /* [T]   */
+  int32_t max_seqlen_q, max_seqlen_k; /* [host] replay-wide bounds used for launch sizing */
+  int32_t is_causal; /* must be 1 */
+  int32_t window;    /* > 0: key j visible to position p iff p - window < j <= p; <= 0: off */
+  /* selected indices, -1 padded: [T, H_kv, sel_width] (sel_per_request = 0) or
+     [B, H_kv, sel_width] (sel_per_request = 1); NULL = no selection */
+  const int32_t* selected_idx;
+  int32_t sel_width;
+  int32_t sel_per_request;
+  int32_t sel_target; /* 0: indices address the main cache (no window allowed);
+                         1: indices address the auxiliary store; the main cache
+                            then contributes its causal window (or all causal
+                            keys when window <= 0) */
+  /* auxiliary store [B, aux_cap, H_kv, D], same dtype and scales as the main cache */
+  const void* aux_k;
+  const void* aux_v;
+  int32_t aux_cap;
+  const int32_t* aux_seqlens; /* [B] valid entries per request */
+  const float* sinks; /* [H_q] learned sink logits, not multiplied by scale; NULL = no sink */
+  float scale;        /* 0 selects 1/sqrt(D) */
+  float* lse;         /* [T, H_q] optional: log of the softmax denominator incl. the sink */
+  int32_t num_splits; /* 0 = automatic; otherwise the number of key splits per unit */
+  int32_t* status;    /* OR-ed status bits */
+} spa_attention_args_t;
+
+/* Bytes of workspace spa_attention needs for these arguments (0 if none).
+   Returns 0 as well for invalid arguments; spa_attention then reports the error. */
+size_t spa_attention_workspace_size(const spa_attention_args_t* a);
+
+/*
+ * spa_attention -- steps 3-5.  For token t (request b, position p) and q
+ * head h (kv head h / (H_q / H_kv)):
+ *   s_j = scale * <q[t,h], k_j> over the attended set S(t, h_kv),
+ *   m = max(max_j s_j, sink_h), l = sum_j exp(s_j - m) + exp(sink_h - m),
+ *   out[t,h] = sum_j exp(s_j - m) v_j / l  (0 when S is empty and there is no sink),
+ *   lse[t,h] = m + log(l).
+ * The attended set is, for the main cache, the causal window (or all causal
+ * keys) or the valid selected indices <= p; plus, with sel_target = 1, the
+ * valid auxiliary entries of the request.  Keys are processed in splits whose
+ * FP32 partial states are merged by log-sum-exp; the result does not depend
+ * on num_splits beyond rounding.
+ * workspace: device buffer of at least spa_attention_workspace_size() bytes,
+ * 256-byte aligned, contents irrelevant on entry; it may be NULL when the
+ * size is 0.  Calls that share a workspace must be ordered on one stream.
+ */
+int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
+                  spa_stream_t stream);
+
+/*
+ * spa_attention_plan -- host-only introspection of what spa_attention would
+ * launch for these arguments: the number of key splits per unit, the number
+ * of kernel launches, and the kernel family (0 = CUDA-core decode,
+ * 1 = tensor-core decode, 2 = tcgen05 prefill).  Any output pointer may be
+ * NULL.  Returns the same code spa_attention would return for the arguments
+ * before launching anything.
+ */
+int spa_attention_plan(const spa_attention_args_t* a, int32_t* num_splits, int32_t* num_launches,
+                       int32_t* kernel_kind);
+
+/* Static message for a return code; for SPA_ERR_CUDA the message of the
+   last failed launch in this thread. */
+const char* spa_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPA_H_ */

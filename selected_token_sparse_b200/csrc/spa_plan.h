@@ -1,0 +1,27 @@
+// Host-side launch plan of spa_attention.
+#pragma once
+
+#include <stddef.h>
+
+#include "spa.h"
+
+namespace spa {
+
+enum PlanKind { kPlanScalar = 0, kPlanMma = 1, kPlanPrefill = 2 };
+
+struct Plan {
+  int kind;
+  int group_by_request;
+  int max_q;
+  int max_rows;
+  int num_splits;
+  int split_len;
+  int units;
+  size_t ws_acc_bytes;
+  size_t ws_ml_bytes;
+};
+
+int validate_attention(const spa_attention_args_t* a);
+int make_plan(const spa_attention_args_t* a, Plan* pl);
+
+}  // namespace spa

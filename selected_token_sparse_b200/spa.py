@@ -1,0 +1,238 @@
+"""Thin Python binding of libspa (ctypes).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors must be CUDA tensors; outputs are allocated with torch on
+the input's device (the library itself never allocates).  Work is enqueued on
+torch's current stream.  If libspa.so is missing the import fails loudly --
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspa.so")
+
+SPA_F32, SPA_F16, SPA_BF16, SPA_I8 = 0, 1, 2, 3
+SPA_OK, SPA_ERR_INVALID_ARG, SPA_ERR_UNSUPPORTED, SPA_ERR_WORKSPACE, SPA_ERR_CUDA = 0, -1, -2, -3, -4
+ST_BAD_CU, ST_CAPACITY, ST_BAD_BLOCK, ST_BOUNDS, ST_BAD_IDX = 0x1, 0x2, 0x4, 0x8, 0x10
+
+EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_attention",
+            "spa_attention_workspace_size", "spa_attention_plan", "spa_error_string")
+
+_DT = {torch.float32: SPA_F32, torch.float16: SPA_F16, torch.bfloat16: SPA_BF16, torch.int8: SPA_I8}
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+
+
+class AttentionArgs(ctypes.Structure):
+    """Mirror of spa_attention_args_t (include/spa.h)."""
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("q", _vp), ("out", _vp), ("act", _i32),
+        ("T", _i32), ("B", _i32), ("H_q", _i32), ("H_kv", _i32), ("D", _i32),
+        ("k_cache", _vp), ("v_cache", _vp), ("cache", _i32),
+        ("k_scale", _vp), ("v_scale", _vp),
+        ("block_table", _vp),
+        ("MB", _i32), ("block_size", _i32), ("num_blocks", _i32),
+        ("cu_seqlens_q", _vp), ("seqlens_q", _vp), ("seqlen_k", _vp),
+        ("token_batch", _vp), ("token_pos", _vp),
+        ("max_seqlen_q", _i32), ("max_seqlen_k", _i32),
+        ("is_causal", _i32), ("window", _i32),
+        ("selected_idx", _vp), ("sel_width", _i32), ("sel_per_request", _i32), ("sel_target", _i32),
+        ("aux_k", _vp), ("aux_v", _vp), ("aux_cap", _i32), ("aux_seqlens", _vp),
+        ("sinks", _vp), ("scale", ctypes.c_float), ("lse", _vp),
+        ("num_splits", _i32), ("status", _vp),
+    ]
+
+
+class SpaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {error_string(code)} (code {code})")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"libspa.so not found at {path}; build it with "
+                           "`python -m selected_token_sparse_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.spa_prepare_metadata.restype = ctypes.c_int
+    lib.spa_prepare_metadata.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                         _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.spa_append_kv.restype = ctypes.c_int
+    lib.spa_append_kv.argtypes = [_vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32,
+                                  _i32, _i32, _vp, _vp]
+    lib.spa_attention_workspace_size.restype = ctypes.c_size_t
+    lib.spa_attention_workspace_size.argtypes = [ctypes.POINTER(AttentionArgs)]
+    lib.spa_attention.restype = ctypes.c_int
+    lib.spa_attention.argtypes = [ctypes.POINTER(AttentionArgs), _vp, ctypes.c_size_t, _vp]
+    lib.spa_attention_plan.restype = ctypes.c_int
+    lib.spa_attention_plan.argtypes = [ctypes.POINTER(AttentionArgs), _vp, _vp, _vp]
+    lib.spa_error_string.restype = ctypes.c_char_p
+    lib.spa_error_string.argtypes = [ctypes.c_int]
+    return lib
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        _LIB = load_library()
+    return _LIB
+
+
+def error_string(code: int) -> str:
+    return lib().spa_error_string(code).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libspa takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libspa takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(code: int, what: str):
+    if code != SPA_OK:
+        raise SpaError(code, what)
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def prepare_metadata(cu_seqlens_q: torch.Tensor, past_seqlens: torch.Tensor,
+                     block_table: torch.Tensor, T: int, max_seqlen_q: int, max_seqlen_k: int,
+                     block_size: int, num_blocks: int, status: Optional[torch.Tensor] = None,
+                     out: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+    """Step 1: per-request seqlens_q / seqlen_k and per-token batch / pos / slot."""
+    dev = cu_seqlens_q.device
+    B = cu_seqlens_q.numel() - 1
+    MB = block_table.shape[1] if block_table.dim() == 2 else 0
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = {"seqlens_q": torch.empty(B, **i32), "seqlen_k": torch.empty(B, **i32),
+               "token_batch": torch.empty(T, **i32), "token_pos": torch.empty(T, **i32),
+               "slot_mapping": torch.empty(T, **i32)}
+    if status is None:
+        status = new_status(dev)
+    out["status"] = status
+    rc = lib().spa_prepare_metadata(
+        _ptr(cu_seqlens_q), _ptr(past_seqlens), _ptr(block_table), B, T, max_seqlen_q,
+        max_seqlen_k, MB, block_size, num_blocks, _ptr(out["seqlens_q"]), _ptr(out["seqlen_k"]),
+        _ptr(out["token_batch"]), _ptr(out["token_pos"]), _ptr(out["slot_mapping"]),
+        _ptr(status), _stream(dev))
+    _check(rc, "spa_prepare_metadata")
+    out["cu_seqlens_q"] = cu_seqlens_q
+    return out
+
+
+def append_kv(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+              v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+              k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
+              status: Optional[torch.Tensor] = None) -> None:
+    """Step 2: scatter k_new/v_new [T, H_kv, D] into the paged cache [NB, bs, H_kv, D]."""
+    T, H_kv, D = k_new.shape
+    NB, bs = k_cache.shape[0], k_cache.shape[1]
+    if status is None:
+        status = new_status(k_new.device)
+    rc = lib().spa_append_kv(_ptr(k_new), _ptr(v_new), _DT[k_new.dtype], _ptr(k_cache),
+                             _ptr(v_cache), _DT[k_cache.dtype], _ptr(k_scale), _ptr(v_scale),
+                             _ptr(slot_mapping), T, H_kv, D, bs, NB, _ptr(status),
+                             _stream(k_new.device))
+    _check(rc, "spa_append_kv")
+
+
+def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_table: torch.Tensor, meta: Dict[str, torch.Tensor], *,
+                   max_seqlen_q: int, max_seqlen_k: int, out: torch.Tensor,
+                   lse: Optional[torch.Tensor] = None, window: int = 0,
+                   selected_idx: Optional[torch.Tensor] = None, sel_per_request: int = 1,
+                   sel_target: int = 0, aux_k: Optional[torch.Tensor] = None,
+                   aux_v: Optional[torch.Tensor] = None, aux_seqlens: Optional[torch.Tensor] = None,
+                   sinks: Optional[torch.Tensor] = None, scale: float = 0.0,
+                   k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
+                   num_splits: int = 0, status: Optional[torch.Tensor] = None,
+                   is_causal: int = 1) -> AttentionArgs:
+    T, H_q, D = q.shape
+    a = AttentionArgs()
+    a.struct_size = ctypes.sizeof(AttentionArgs)
+    a.q, a.out, a.act = _ptr(q), _ptr(out), _DT[q.dtype]
+    a.T, a.B, a.H_q, a.H_kv, a.D = T, meta["seqlens_q"].numel(), H_q, k_cache.shape[2], D
+    a.k_cache, a.v_cache, a.cache = _ptr(k_cache), _ptr(v_cache), _DT[k_cache.dtype]
+    a.k_scale, a.v_scale = _ptr(k_scale), _ptr(v_scale)
+    a.block_table = _ptr(block_table)
+    a.MB, a.block_size, a.num_blocks = block_table.shape[1], k_cache.shape[1], k_cache.shape[0]
+    a.cu_seqlens_q = _ptr(meta["cu_seqlens_q"])
+    a.seqlens_q, a.seqlen_k = _ptr(meta["seqlens_q"]), _ptr(meta["seqlen_k"])
+    a.token_batch, a.token_pos = _ptr(meta["token_batch"]), _ptr(meta["token_pos"])
+    a.max_seqlen_q, a.max_seqlen_k = max_seqlen_q, max_seqlen_k
+    a.is_causal, a.window = is_causal, window
+    a.selected_idx = _ptr(selected_idx)
+    a.sel_width = selected_idx.shape[-1] if selected_idx is not None else 0
+    a.sel_per_request, a.sel_target = sel_per_request, sel_target
+    a.aux_k, a.aux_v = _ptr(aux_k), _ptr(aux_v)
+    a.aux_cap = aux_k.shape[1] if aux_k is not None else 0
+    a.aux_seqlens = _ptr(aux_seqlens)
+    a.sinks, a.scale, a.lse = _ptr(sinks), float(scale), _ptr(lse)
+    a.num_splits = num_splits
+    a.status = _ptr(status if status is not None else meta.get("status"))
+    return a
+
+
+def workspace_size(args: AttentionArgs) -> int:
+    return int(lib().spa_attention_workspace_size(ctypes.byref(args)))
+
+
+def attention_plan(args: AttentionArgs) -> Dict[str, int]:
+    """What spa_attention would launch: splits, launches, kernel kind."""
+    ns, nl, kk = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    rc = lib().spa_attention_plan(ctypes.byref(args), ctypes.addressof(ns), ctypes.addressof(nl),
+                                  ctypes.addressof(kk))
+    _check(rc, "spa_attention_plan")
+    return {"num_splits": ns.value, "launches": nl.value, "kind": kk.value}
+
+
+def run_attention(args: AttentionArgs, workspace: Optional[torch.Tensor]) -> None:
+    """Enqueue spa_attention for prepared arguments on the current stream."""
+    need = workspace_size(args)
+    if need and (workspace is None or workspace.numel() < need):
+        raise SpaError(SPA_ERR_WORKSPACE, "spa_attention")
+    ws = _ptr(workspace) if need else None
+    dev = workspace.device if workspace is not None else torch.device("cuda")
+    rc = lib().spa_attention(ctypes.byref(args), ws, need, _stream(dev))
+    _check(rc, "spa_attention")
+
+
+def attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_table: torch.Tensor, meta: Dict[str, torch.Tensor], *, max_seqlen_q: int,
+              max_seqlen_k: int, out: Optional[torch.Tensor] = None, want_lse: bool = False,
+              workspace: Optional[torch.Tensor] = None, **kw):
+    """Steps 3-5: sparse / paged attention; returns (out, lse or None)."""
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if want_lse else None
+    a = attention_args(q, k_cache, v_cache, block_table, meta, max_seqlen_q=max_seqlen_q,
+                       max_seqlen_k=max_seqlen_k, out=out, lse=lse, **kw)
+    need = workspace_size(a)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib().spa_attention(ctypes.byref(a), _ptr(workspace) if need else None, need,
+                             _stream(q.device))
+    _check(rc, "spa_attention")
+    return out, lse

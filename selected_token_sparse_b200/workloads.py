@@ -32,21 +32,45 @@ import numpy as np
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to bfloat16 (round-to-nearest-even) and return the bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    bias = 0x7FFF + ((u >> 16) & 1)
-    return ((u + bias) >> 16).astype(np.uint16)
+    """Round finite float32 values to bfloat16 (round-to-nearest-even); return the bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).reshape(-1).view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+    step = 1 << 24
+    for i in range(0, u.size, step):
+        c = u[i:i + step]
+        # finite values stay below 2**32 after adding the bias
+        out[i:i + step] = ((c + (np.uint32(0x7FFF) + ((c >> np.uint32(16)) & np.uint32(1))))
+                           >> np.uint32(16)).astype(np.uint16)
+    return out.reshape(np.shape(x))
+
+
+_NORMAL_TABLE = {}
+
+
+def _normal_table(act: str) -> np.ndarray:
+    """N(0, 1) quantiles at the midpoints of 65536 equal-probability cells,
+    encoded in the activation dtype."""
+    if act not in _NORMAL_TABLE:
+        from scipy.special import ndtri
+        z = ndtri((np.arange(65536, dtype=np.float64) + 0.5) / 65536.0).astype(np.float32)
+        if act == "f32":
+            tab = z
+        elif act == "f16":
+            tab = z.astype(np.float16)
+        else:
+            tab = f32_to_bf16_bits(z)
+        _NORMAL_TABLE[act] = tab
+    return _NORMAL_TABLE[act]
 
 
 def _act_array(rng: np.random.Generator, shape, act: str) -> np.ndarray:
-    x = rng.standard_normal(size=shape, dtype=np.float32)
-    if act == "f32":
-        return x
-    if act == "f16":
-        return x.astype(np.float16)
-    if act == "bf16":
-        return f32_to_bf16_bits(x)
-    raise ValueError(act)
+    """Seeded N(0, 1) draws in the activation dtype: 16 uniform random bits per
+    element select one of 65536 equal-probability normal quantiles."""
+    if act not in ("f32", "f16", "bf16"):
+        raise ValueError(act)
+    n = int(np.prod(shape))
+    bits = rng.integers(0, 65536, size=n, dtype=np.uint16)
+    return _normal_table(act)[bits].reshape(shape)
 
 
 @dataclasses.dataclass

@@ -1,0 +1,172 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Metadata, slots, cache contents, index handling and
+status bits are compared bit for bit; outputs within max-abs 1e-5 (fp32) or
+3e-3 (fp16 / bf16; INT8 caches are compared with the oracle run on the
+dequantised values)."""
+import numpy as np
+import pytest
+import torch
+
+from selected_token_sparse_b200 import pipeline, workloads as W
+from tests.gpu_util import compare, oracle_step
+
+pytestmark = pytest.mark.gpu
+
+
+def run(wl, **kw):
+    return pipeline.run_step(wl, **kw)
+
+
+@pytest.mark.parametrize("name", W.WORKLOADS)
+def test_workload_small(name):
+    wl = W.by_name(name, small=True)
+    compare(wl, run(wl), oracle_step(wl))
+
+
+@pytest.mark.parametrize("name", W.WORKLOADS)
+def test_workload_full_size(name):
+    """The five workloads at full size; prefill outputs are sampled rows."""
+    wl = W.by_name(name, small=False)
+    tokens = None
+    if name == "ragged_prefill_f16":
+        rng = np.random.default_rng(0)
+        cu = wl["cu_seqlens_q"]
+        picks = set()
+        for b in range(wl.B):
+            picks |= {int(cu[b]), int(cu[b]) + 1, int(cu[b + 1]) - 1, int(cu[b + 1]) - 2}
+            picks |= set(int(x) for x in rng.integers(cu[b], cu[b + 1], size=6))
+        tokens = sorted(picks)
+    got = run(wl)
+    ref = oracle_step(wl, tokens=tokens)
+    compare(wl, got, ref, tokens=tokens)
+
+
+@pytest.mark.parametrize("name", ["tiny_decode_f32", "gptoss_paged_decode_f16",
+                                  "selected_decode_bf16", "local_plus_selected_int8"])
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 32])
+def test_forced_splits(name, splits):
+    wl = W.by_name(name, small=True)
+    compare(wl, run(wl, num_splits=splits), oracle_step(wl))
+
+
+@pytest.mark.parametrize("name", W.WORKLOADS)
+def test_deterministic(name):
+    wl = W.by_name(name, small=True)
+    a, b = run(wl), run(wl)
+    assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["lse"], b["lse"], equal_nan=True)
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+
+EDGE = {
+    "empty_requests_decode": dict(act="f16", B=4, H_q=8, H_kv=2, D=64, block_size=16,
+                                  q_lens=[1, 0, 1, 0], past=[40, 17, 0, 0], window=16),
+    "no_tokens": dict(act="f16", B=2, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[0, 0],
+                      past=[5, 0]),
+    "window_larger_than_history": dict(act="bf16", B=3, H_q=8, H_kv=1, D=128, block_size=64,
+                                       q_lens=[1, 1, 1], past=[3, 64, 200], window=1000),
+    "window_one": dict(act="f16", B=2, H_q=4, H_kv=4, D=64, block_size=16, q_lens=[1, 1],
+                       past=[10, 0], window=1),
+    "no_sink_mha": dict(act="f32", B=2, H_q=2, H_kv=2, D=64, block_size=16, q_lens=[1, 1],
+                        past=[30, 5], window=8, has_sinks=False),
+    "gqa16": dict(act="bf16", B=2, H_q=32, H_kv=2, D=64, block_size=16, q_lens=[1, 1],
+                  past=[100, 33], window=64),
+    "all_padding_selection": dict(act="f16", B=2, H_q=4, H_kv=2, D=64, block_size=16,
+                                  q_lens=[1, 1], past=[20, 9], sel_mode="main", sel_width=8,
+                                  sel_valid=0),
+    "all_padding_selection_no_sink": dict(act="f16", B=2, H_q=4, H_kv=2, D=64, block_size=16,
+                                          q_lens=[1, 1], past=[20, 9], sel_mode="main",
+                                          sel_width=8, sel_valid=0, has_sinks=False),
+    "per_token_selection_multi_query": dict(act="bf16", B=2, H_q=8, H_kv=2, D=128, block_size=64,
+                                            q_lens=[4, 3], past=[150, 70], sel_mode="main",
+                                            sel_per_request=0, sel_width=40, sel_valid=33),
+    "per_request_selection_multi_query": dict(act="f16", B=2, H_q=8, H_kv=2, D=64, block_size=16,
+                                              q_lens=[5, 2], past=[60, 7], sel_mode="main",
+                                              sel_per_request=1, sel_width=30, sel_valid=25),
+    "aux_short_lengths": dict(act="f16", cache="i8", B=3, H_q=12, H_kv=2, D=128, block_size=64,
+                              q_lens=[2, 1, 3], past=[100, 5, 64], window=32, sel_mode="aux",
+                              sel_width=20, aux_cap=50, aux_lens=[50, 10, 0]),
+    "aux_without_window": dict(act="bf16", B=2, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[1, 2],
+                               past=[20, 30], window=0, sel_mode="aux", sel_width=12, aux_cap=30),
+    "int8_bf16_act": dict(act="bf16", cache="i8", B=2, H_q=8, H_kv=2, D=128, block_size=64,
+                          q_lens=[1, 1], past=[300, 77], window=128),
+    "int8_f32_act": dict(act="f32", cache="i8", B=2, H_q=4, H_kv=2, D=64, block_size=16,
+                         q_lens=[1, 1], past=[50, 7], window=20),
+    "explicit_scale": dict(act="f16", B=2, H_q=4, H_kv=2, D=128, block_size=16, q_lens=[1, 1],
+                           past=[50, 7], window=20, scale=0.3),
+    "chunked_prefill_dense": dict(act="f16", B=3, H_q=8, H_kv=2, D=64, block_size=16,
+                                  q_lens=[7, 1, 12], past=[20, 3, 0]),
+    "chunked_prefill_window": dict(act="bf16", B=2, H_q=4, H_kv=1, D=128, block_size=64,
+                                   q_lens=[40, 9], past=[100, 0], window=24),
+    "long_prefill_per_token_fallback": dict(act="f32", B=2, H_q=4, H_kv=2, D=64, block_size=16,
+                                            q_lens=[70, 33], past=[0, 5]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(EDGE))
+def test_edge_case(case):
+    wl = W.make_workload(name=case, seed=11, **EDGE[case])
+    compare(wl, run(wl), oracle_step(wl))
+
+
+def test_bad_selected_indices_flagged_and_skipped():
+    wl = W.make_workload(act="f16", B=2, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[1, 1],
+                         past=[30, 12], sel_mode="main", sel_width=10, sel_valid=7, seed=5)
+    sel = wl.arrays["selected_idx"]
+    sel[0, 0, 7] = 31 + 5        # beyond the request's length
+    sel[1, 1, 8] = -9            # below the padding value
+    ref = oracle_step(wl)
+    assert ref["status"] == 0x10
+    compare(wl, run(wl), ref)
+
+
+def test_bad_aux_indices_flagged_and_skipped():
+    wl = W.make_workload(act="f16", cache="i8", B=2, H_q=8, H_kv=2, D=128, block_size=64,
+                         q_lens=[2, 1], past=[70, 3], window=16, sel_mode="aux", sel_width=12,
+                         aux_cap=40, aux_lens=[40, 9], seed=6)
+    sel = wl.arrays["selected_idx"]
+    sel[1, 0, 11] = 20           # within capacity, beyond request 1's aux length
+    sel[0, 1, 10] = 40           # beyond capacity
+    ref = oracle_step(wl)
+    assert ref["status"] == 0x10
+    compare(wl, run(wl), ref)
+
+
+@pytest.mark.parametrize("which", ["decreasing_cu", "short_cu", "bad_block", "capacity",
+                                   "negative_past"])
+def test_malformed_metadata_status(which):
+    """Malformed inputs: status bits and metadata match the oracle, caches stay
+    bit-exact (no write outside a valid slot); outputs are unspecified."""
+    wl = W.make_workload(act="f16", B=3, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[2, 1, 3],
+                         past=[20, 5, 40], window=8, spare_blocks=2, seed=9)
+    a = wl.arrays
+    if which == "decreasing_cu":
+        a["cu_seqlens_q"][2] = 1
+    elif which == "short_cu":
+        a["cu_seqlens_q"][3] = 4
+    elif which == "bad_block":
+        a["block_table"][2, 2] = wl.NB + 3
+        a["block_table"][0, 0] = -1
+    elif which == "capacity":
+        a["past_seqlens"][0] = wl.MB * wl.block_size - 1
+    elif which == "negative_past":
+        a["past_seqlens"][1] = -4
+    ref = oracle_step(wl)
+    assert ref["status"] != 0
+    got = run(wl)
+    compare(wl, got, ref, check_out=False)
+
+
+def test_status_accumulates_and_is_not_cleared():
+    wl = W.make_workload(act="f16", B=1, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[1],
+                         past=[5], sel_mode="main", sel_width=4, sel_valid=2, seed=3)
+    wl.arrays["selected_idx"][0, 0, 3] = 100
+    d = pipeline.to_device(wl)
+    st = pipeline.Step(wl, d)
+    st.status.fill_(0x40)
+    st()
+    torch.cuda.synchronize()
+    assert int(st.status.item()) == 0x50
