@@ -1,8 +1,491 @@
-// Tensor-core decode kernel (placeholder until written).
+// Steps 3-5 on tensor cores for 16-bit activations (fp16 / bf16 caches, and
+// INT8 caches dequantised to fp16 in shared memory).
+//
+// Decode attention is a skinny contraction: one CTA owns a unit (all G q
+// heads of one kv head, for one token or all tokens of one request: R = G*S_q
+// rows) and one split of its candidate keys, so every gathered K/V row is read
+// from HBM once and used by all R rows.  At G*2 flops per byte the math must
+// not run on the FP32 pipe, but R is far below a 128-row tcgen05 tile, so the
+// contraction uses warp-level m16n8k16 MMAs (rows padded to 16) while the
+// kernel's real work is the gather:
+//
+//   * candidates (window positions, or selected / auxiliary slots) are resolved
+//     through the block table with every guard of the scalar path, by the
+//     threads that copy the rows, and
+//   * K/V rows are copied as 16-byte cp.async chunks into a 3-stage ring of
+//     64-key tiles in XOR-swizzled shared memory (conflict-free ldmatrix),
+//     keeping two tiles in flight while one is consumed.
+//
+// Warps split a key tile (KW slices) and/or the row tiles (RT); each keeps
+// its own online-softmax state (log2 units) and merges through shared memory
+// at the end.  With one split the learned sink is folded in and the output
+// written; otherwise FP32 partial states go to the workspace for the
+// log-sum-exp combine ("[WebGPU] Add SparsePagedAttention", File summaries;
+// "[WebGPU] Add DynamicSparseAttention", Attention: joint FP32 stable softmax
+// with optional sink; onnxruntime PR #33472: INT8 per-channel K/V scales).
+#include <type_traits>
+
 #include "spa_attn.cuh"
 
 namespace spa {
-int mma_supported(int, int, int, int) { return 0; }
-int mma_key_tile() { return 64; }
-int launch_attention_mma(const AttnParams&, int, int, int, cudaStream_t) { return SPA_ERR_UNSUPPORTED; }
+
+constexpr int kMmaKT = 64;      // keys per tile
+constexpr int kMmaStages = 3;   // cp.async ring depth
+
+int mma_key_tile() { return kMmaKT; }
+
+template <typename T> struct MmaName;
+template <> struct MmaName<__half> { static constexpr bool bf16 = false; };
+template <> struct MmaName<__nv_bfloat16> { static constexpr bool bf16 = true; };
+
+template <typename MT>
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, const uint32_t* b) {
+  if constexpr (MmaName<MT>::bf16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  }
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* p) {
+  uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const void* p) {
+  uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+template <typename MT>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (MmaName<MT>::bf16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` in a swizzled tile with `cpr` chunks per row.
+__device__ __forceinline__ int swz(int r, int c, int cpr) { return (r * cpr + (c ^ (r & 7))) * 16; }
+
+template <typename ActT, typename CacheT, int D, int RT, int KW>
+struct MmaCfg {
+  using MT = typename std::conditional<sizeof(CacheT) == 1, __half, ActT>::type;
+  static constexpr bool kInt8 = sizeof(CacheT) == 1;
+  static constexpr int NW = RT * KW;
+  static constexpr int NT = NW * 32;
+  static constexpr int KS = kMmaKT / KW;        // keys per warp slice
+  static constexpr int CPR = D * 2 / 16;        // 16-byte chunks per 16-bit row
+  static constexpr int RAW_CPR = D * (int)sizeof(CacheT) / 16;
+  static constexpr int TILE16 = kMmaKT * D * 2;               // one converted K or V tile
+  static constexpr int RAW_TILE = kMmaKT * D * (int)sizeof(CacheT);
+  static constexpr int ROWS = RT * 16;
+  // shared memory layout (bytes)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RAW = OFF_Q + ROWS * D * 2;                 // stages x (K, V) raw
+  static constexpr int OFF_CONV = OFF_RAW + kMmaStages * 2 * RAW_TILE;  // int8 only: (K, V) fp16
+  static constexpr int OFF_KPOS = OFF_CONV + (kInt8 ? 2 * TILE16 : 0);
+  static constexpr int OFF_SCALE = OFF_KPOS + kMmaStages * kMmaKT * 4;
+  static constexpr int OFF_PROW = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
+  static constexpr int END = OFF_PROW + 128 * 4;
+  // the cross-warp merge reuses the K/V ring once every tile is consumed
+  static constexpr int OFF_RED = OFF_RAW;
+  static constexpr int RED_BYTES = (KW > 1) ? NW * 32 * (D / 2 + 4) * 4 : 0;
+  static constexpr int SMEM = (OFF_RED + RED_BYTES > END) ? OFF_RED + RED_BYTES : END;
+};
+
+template <typename ActT, typename CacheT, int D, int RT, int KW>
+__global__ void __launch_bounds__(RT * KW * 32)
+decode_mma_kernel(const AttnParams p) {
+  using C = MmaCfg<ActT, CacheT, D, RT, KW>;
+  using MT = typename C::MT;
+  constexpr int KT = kMmaKT, NT = C::NT, KS = C::KS, CPR = C::CPR, RAW_CPR = C::RAW_CPR;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wr = warp % RT;   // row tile of this warp
+  const int wk = warp / RT;   // key slice of this warp
+
+  Unit U;
+  const bool has_rows = decode_unit(p, blockIdx.x, U);
+  if (p.group_by_request && !has_rows) return;
+  const int split = blockIdx.y;
+  const int G = p.G;
+  const int nq = p.group_by_request ? U.nq : 1;
+  const int R = nq * G;
+  const int t0 = has_rows ? U.t0 : blockIdx.x / p.H_kv;
+  const int h_kv = blockIdx.x % p.H_kv;
+
+  unsigned char* q_s = smem + C::OFF_Q;
+  int* kpos_s = reinterpret_cast<int*>(smem + C::OFF_KPOS);
+  float* ksc_s = reinterpret_cast<float*>(smem + C::OFF_SCALE);
+  float* vsc_s = ksc_s + D;
+  int* prow_s = reinterpret_cast<int*>(smem + C::OFF_PROW);
+
+  // ---- Q rows -> swizzled smem (16-bit, converted for the INT8 path)
+  const ActT* q = static_cast<const ActT*>(p.q);
+  for (int e = tid; e < C::ROWS * CPR; e += NT) {
+    const int r = e / CPR, c = e % CPR;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const int t = t0 + r / G, h = h_kv * G + r % G;
+      const ActT* src = q + ((long long)t * p.H_q + h) * D + c * 8;
+      if constexpr (std::is_same<MT, ActT>::value) {
+        v = *reinterpret_cast<const uint4*>(src);
+      } else {
+        alignas(16) __half tmp[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tmp[i] = __float2half_rn(to_f32(src[i]));
+        v = *reinterpret_cast<const uint4*>(tmp);
+      }
+    }
+    *reinterpret_cast<uint4*>(q_s + swz(r, c, CPR)) = v;
+  }
+  for (int i = tid; i < 128; i += NT) prow_s[i] = (i < nq && has_rows) ? p.token_pos[t0 + i] : -1;
+  if constexpr (C::kInt8) {
+    for (int d = tid; d < D; d += NT) {
+      ksc_s[d] = p.k_scale[h_kv * D + d];
+      vsc_s[d] = p.v_scale[h_kv * D + d];
+    }
+  }
+
+  // ---- candidate range of this split
+  const int n_total = has_rows ? U.n_main + U.n_aux : 0;
+  const int c_begin = split * p.split_len;
+  const int c_end = min(c_begin + p.split_len, n_total);
+  const int ntiles = c_end > c_begin ? (c_end - c_begin + KT - 1) / KT : 0;
+  const CacheT* kc = static_cast<const CacheT*>(p.k_cache);
+  const CacheT* vc = static_cast<const CacheT*>(p.v_cache);
+  const CacheT* ak = static_cast<const CacheT*>(p.aux_k);
+  const CacheT* av = static_cast<const CacheT*>(p.aux_v);
+  int bits = 0;
+
+  // Issue the copies of tile `it` into its ring stage.  Thread `tid` copies
+  // chunk (tid % RAW_CPR) of rows tid / RAW_CPR, + NT / RAW_CPR, ...; it resolves
+  // those rows' candidates itself.
+  auto issue = [&](int it) {
+    const int stage = it % kMmaStages;
+    unsigned char* kraw = smem + C::OFF_RAW + stage * 2 * C::RAW_TILE;
+    unsigned char* vraw = kraw + C::RAW_TILE;
+    const int c = tid % RAW_CPR;
+    for (int row = tid / RAW_CPR; row < KT; row += NT / RAW_CPR) {
+      const int cand = c_begin + it * KT + row;
+      int kp = kPosInvalid;
+      bool from_aux = false;
+      long long off = -1;
+      if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      const bool ok = off >= 0;
+      const CacheT* kb = from_aux ? ak : kc;
+      const CacheT* vb = from_aux ? av : vc;
+      const CacheT* ksrc = ok ? kb + off + c * (16 / sizeof(CacheT)) : kc;
+      const CacheT* vsrc = ok ? vb + off + c * (16 / sizeof(CacheT)) : vc;
+      const int dst = C::kInt8 ? (row * RAW_CPR + c) * 16 : swz(row, c, CPR);
+      cp_async_16(kraw + dst, ksrc, ok);
+      cp_async_16(vraw + dst, vsrc, ok);
+      if (c == 0) kpos_s[stage * KT + row] = kp;
+    }
+  };
+
+  // per-warp state: rows (lane/4) and (lane/4 + 8) of row tile wr
+  float m_r[2] = {-INFINITY, -INFINITY};
+  float l_r[2] = {0.f, 0.f};
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  uint32_t qf[D / 16][4];
+
+#pragma unroll
+  for (int s = 0; s < kMmaStages - 1; ++s) {
+    if (s < ntiles) issue(s);
+    cp_async_commit();
+  }
+  __syncthreads();
+  // Q fragments for this warp's row tile stay in registers
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const int r = wr * 16 + (lane & 15);
+    const int ch = kk * 2 + (lane >> 4);
+    ldsm_x4(qf[kk], q_s + swz(r, ch, CPR));
+  }
+  const int r0 = wr * 16 + (lane >> 2);
+  const int r1 = r0 + 8;
+  const int prow0 = r0 < R ? prow_s[r0 / G] : -1;
+  const int prow1 = r1 < R ? prow_s[r1 / G] : -1;
+  const float sl2 = p.scale_log2;
+
+  for (int it = 0; it < ntiles; ++it) {
+    if (it + kMmaStages - 1 < ntiles) issue(it + kMmaStages - 1);
+    cp_async_commit();
+    cp_async_wait<kMmaStages - 1>();
+    __syncthreads();
+    const int stage = it % kMmaStages;
+    const unsigned char* ks;
+    const unsigned char* vs;
+    if constexpr (C::kInt8) {
+      // dequantise the raw int8 stage into fp16 tiles (per-channel scales)
+      const int8_t* kraw = reinterpret_cast<const int8_t*>(smem + C::OFF_RAW + stage * 2 * C::RAW_TILE);
+      const int8_t* vraw = kraw + C::RAW_TILE;
+      unsigned char* kconv = smem + C::OFF_CONV;
+      unsigned char* vconv = kconv + C::TILE16;
+      for (int e = tid; e < KT * RAW_CPR * 2; e += NT) {
+        const bool isv = e >= KT * RAW_CPR;
+        const int ee = isv ? e - KT * RAW_CPR : e;
+        const int row = ee / RAW_CPR, c = ee % RAW_CPR;
+        const int8_t* src = (isv ? vraw : kraw) + (row * RAW_CPR + c) * 16;
+        const float* sc = (isv ? vsc_s : ksc_s) + c * 16;
+        const int4 raw = *reinterpret_cast<const int4*>(src);
+        const int8_t* b8 = reinterpret_cast<const int8_t*>(&raw);
+        alignas(16) __half h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = __float2half_rn(static_cast<float>(b8[i]) * sc[i]);
+        unsigned char* dst = isv ? vconv : kconv;
+        *reinterpret_cast<uint4*>(dst + swz(row, 2 * c, CPR)) = *reinterpret_cast<const uint4*>(h);
+        *reinterpret_cast<uint4*>(dst + swz(row, 2 * c + 1, CPR)) =
+            *reinterpret_cast<const uint4*>(h + 8);
+      }
+      __syncthreads();
+      ks = kconv;
+      vs = vconv;
+    } else {
+      ks = smem + C::OFF_RAW + stage * 2 * C::RAW_TILE;
+      vs = ks + C::RAW_TILE;
+    }
+    const int* kpos = kpos_s + stage * KT;
+
+    // S = Q K^T for this warp's 16 rows x KS keys
+    float s[KS / 8][4];
+#pragma unroll
+    for (int j = 0; j < KS / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+      for (int j = 0; j < KS / 8; j += 2) {
+        uint32_t b[4];
+        const int mi = lane >> 3;
+        const int krow = wk * KS + j * 8 + (mi >> 1) * 8 + (lane & 7);
+        ldsm_x4(b, ks + swz(krow, kk * 2 + (mi & 1), CPR));
+        mma16816<MT>(s[j], qf[kk], b);
+        mma16816<MT>(s[j + 1], qf[kk], b + 2);
+      }
+    }
+    // mask, scale, online softmax (rows r0, r1)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < KS / 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = wk * KS + j * 8 + (lane & 3) * 2 + e;
+        const int kp = kpos[key];
+        s[j][e] = key_visible(kp, prow0, p.window) ? s[j][e] * sl2 : -INFINITY;
+        s[j][2 + e] = key_visible(kp, prow1, p.window) ? s[j][2 + e] * sl2 : -INFINITY;
+        mx0 = fmaxf(mx0, s[j][e]);
+        mx1 = fmaxf(mx1, s[j][2 + e]);
+      }
+    }
+#pragma unroll
+    for (int o2 = 1; o2 <= 2; o2 <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+    }
+    const float mn0 = fmaxf(m_r[0], mx0), mn1 = fmaxf(m_r[1], mx1);
+    const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_r[0] - mn0);
+    const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_r[1] - mn1);
+    m_r[0] = mn0;
+    m_r[1] = mn1;
+    float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < KS / 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        s[j][e] = (s[j][e] == -INFINITY) ? 0.f : exp2f(s[j][e] - mn0);
+        s[j][2 + e] = (s[j][2 + e] == -INFINITY) ? 0.f : exp2f(s[j][2 + e] - mn1);
+        ls0 += s[j][e];
+        ls1 += s[j][2 + e];
+      }
+    }
+    l_r[0] = l_r[0] * al0 + ls0;
+    l_r[1] = l_r[1] * al1 + ls1;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o[n][0] *= al0;
+      o[n][1] *= al0;
+      o[n][2] *= al1;
+      o[n][3] *= al1;
+    }
+    // O += P V
+#pragma unroll
+    for (int kk = 0; kk < KS / 16; ++kk) {
+      uint32_t a[4];
+      a[0] = pack2<MT>(s[2 * kk][0], s[2 * kk][1]);
+      a[1] = pack2<MT>(s[2 * kk][2], s[2 * kk][3]);
+      a[2] = pack2<MT>(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      a[3] = pack2<MT>(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int n = 0; n < D / 8; n += 2) {
+        uint32_t b[4];
+        const int mi = lane >> 3;
+        const int vrow = wk * KS + kk * 16 + (mi & 1) * 8 + (lane & 7);
+        ldsm_x4_t(b, vs + swz(vrow, n + (mi >> 1), CPR));
+        mma16816<MT>(o[n], a, b);
+        mma16816<MT>(o[n + 1], a, b + 2);
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  flag(p.status, bits);
+
+  // row sums across the quad
+#pragma unroll
+  for (int o2 = 1; o2 <= 2; o2 <<= 1) {
+    l_r[0] += __shfl_xor_sync(0xffffffffu, l_r[0], o2);
+    l_r[1] += __shfl_xor_sync(0xffffffffu, l_r[1], o2);
+  }
+
+  // merge the KW key slices of each row tile (into the wk == 0 warp)
+  if constexpr (KW > 1) {
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+    constexpr int PER = D / 2 + 4;
+    float* mine = red + (warp * 32 + lane) * PER;
+    if (wk > 0) {
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        mine[n * 4 + 0] = o[n][0];
+        mine[n * 4 + 1] = o[n][1];
+        mine[n * 4 + 2] = o[n][2];
+        mine[n * 4 + 3] = o[n][3];
+      }
+      mine[D / 2 + 0] = m_r[0];
+      mine[D / 2 + 1] = m_r[1];
+      mine[D / 2 + 2] = l_r[0];
+      mine[D / 2 + 3] = l_r[1];
+    }
+    __syncthreads();
+    if (wk == 0) {
+#pragma unroll
+      for (int k2 = 1; k2 < KW; ++k2) {
+        const float* other = red + ((k2 * RT + wr) * 32 + lane) * PER;
+        const float om0 = other[D / 2 + 0], om1 = other[D / 2 + 1];
+        const float mn0 = fmaxf(m_r[0], om0), mn1 = fmaxf(m_r[1], om1);
+        const float a0 = (mn0 == -INFINITY) ? 0.f : exp2f(m_r[0] - mn0);
+        const float b0 = (mn0 == -INFINITY) ? 0.f : exp2f(om0 - mn0);
+        const float a1 = (mn1 == -INFINITY) ? 0.f : exp2f(m_r[1] - mn1);
+        const float b1 = (mn1 == -INFINITY) ? 0.f : exp2f(om1 - mn1);
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] = o[n][0] * a0 + other[n * 4 + 0] * b0;
+          o[n][1] = o[n][1] * a0 + other[n * 4 + 1] * b0;
+          o[n][2] = o[n][2] * a1 + other[n * 4 + 2] * b1;
+          o[n][3] = o[n][3] * a1 + other[n * 4 + 3] * b1;
+        }
+        l_r[0] = l_r[0] * a0 + other[D / 2 + 2] * b0;
+        l_r[1] = l_r[1] * a1 + other[D / 2 + 3] * b1;
+        m_r[0] = mn0;
+        m_r[1] = mn1;
+      }
+    }
+  }
+  if (wk != 0) return;
+
+  // write rows r0, r1 of this row tile
+#pragma unroll
+  for (int hrow = 0; hrow < 2; ++hrow) {
+    const int r = hrow ? r1 : r0;
+    if (r >= R) continue;
+    const int t = t0 + r / G, h = h_kv * G + r % G;
+    const long long row = (long long)t * p.H_q + h;
+    if (p.num_splits == 1) {
+      const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+      float a, inv_l, lse;
+      finalize_row(m_r[hrow], l_r[hrow], sink2, a, inv_l, lse);
+      const float f = a * inv_l;
+      ActT* out = static_cast<ActT*>(p.out) + row * D;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        const int d = n * 8 + (lane & 3) * 2;
+        out[d] = from_f32<ActT>(o[n][hrow * 2 + 0] * f);
+        out[d + 1] = from_f32<ActT>(o[n][hrow * 2 + 1] * f);
+      }
+      if ((lane & 3) == 0 && p.lse) p.lse[row] = lse;
+    } else {
+      const long long wrow = (long long)split * p.T * p.H_q + row;
+      float* acc = p.ws_acc + wrow * D;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        const int d = n * 8 + (lane & 3) * 2;
+        *reinterpret_cast<float2*>(acc + d) = make_float2(o[n][hrow * 2], o[n][hrow * 2 + 1]);
+      }
+      if ((lane & 3) == 0) {
+        p.ws_ml[wrow * 2 + 0] = m_r[hrow];
+        p.ws_ml[wrow * 2 + 1] = l_r[hrow];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dispatch
+// ---------------------------------------------------------------------------
+
+int mma_supported(int act, int cache, int D, int max_rows) {
+  if (act != SPA_F16 && act != SPA_BF16) return 0;
+  if (!(cache == act || cache == SPA_I8)) return 0;
+  if (D != 64 && D != 128) return 0;
+  return max_rows >= 1 && max_rows <= 128;
+}
+
+template <typename ActT, typename CacheT, int D, int RT, int KW>
+static int launch_rt(const AttnParams& p, cudaStream_t stream) {
+  using C = MmaCfg<ActT, CacheT, D, RT, KW>;
+  auto kern = decode_mma_kernel<ActT, CacheT, D, RT, KW>;
+  if (C::SMEM > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
+  dim3 grid(units, p.num_splits);
+  kern<<<grid, C::NT, C::SMEM, stream>>>(p);
+  return 0;
+}
+
+template <typename ActT, typename CacheT, int D>
+static int launch_d(const AttnParams& p, int max_rows, cudaStream_t stream) {
+  const int rt = (max_rows + 15) / 16;
+  switch (rt) {
+    case 1: return launch_rt<ActT, CacheT, D, 1, 4>(p, stream);
+    case 2: return launch_rt<ActT, CacheT, D, 2, 2>(p, stream);
+    case 3: return launch_rt<ActT, CacheT, D, 3, 1>(p, stream);
+    case 4: return launch_rt<ActT, CacheT, D, 4, 1>(p, stream);
+    case 5:
+    case 6: return launch_rt<ActT, CacheT, D, 6, 1>(p, stream);
+    default: return launch_rt<ActT, CacheT, D, 8, 1>(p, stream);
+  }
+}
+
+template <typename ActT, typename CacheT>
+static int launch_dd(const AttnParams& p, int max_rows, cudaStream_t stream) {
+  if (p.D == 64) return launch_d<ActT, CacheT, 64>(p, max_rows, stream);
+  return launch_d<ActT, CacheT, 128>(p, max_rows, stream);
+}
+
+int launch_attention_mma(const AttnParams& p, int act, int cache, int max_rows, cudaStream_t stream) {
+  if (act == SPA_F16) {
+    if (cache == SPA_I8) return launch_dd<__half, int8_t>(p, max_rows, stream);
+    return launch_dd<__half, __half>(p, max_rows, stream);
+  }
+  if (cache == SPA_I8) return launch_dd<__nv_bfloat16, int8_t>(p, max_rows, stream);
+  return launch_dd<__nv_bfloat16, __nv_bfloat16>(p, max_rows, stream);
+}
+
 }  // namespace spa

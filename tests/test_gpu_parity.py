@@ -20,7 +20,7 @@ def run(wl, **kw):
 @pytest.mark.parametrize("name", W.WORKLOADS)
 def test_workload_small(name):
     wl = W.by_name(name, small=True)
-    compare(wl, run(wl), oracle_step(wl))
+    compare(wl, run(wl), oracle_step(wl), strict=True)
 
 
 @pytest.mark.parametrize("name", W.WORKLOADS)
@@ -38,7 +38,7 @@ def test_workload_full_size(name):
         tokens = sorted(picks)
     got = run(wl)
     ref = oracle_step(wl, tokens=tokens)
-    compare(wl, got, ref, tokens=tokens)
+    compare(wl, got, ref, tokens=tokens, strict=True)
 
 
 @pytest.mark.parametrize("name", ["tiny_decode_f32", "gptoss_paged_decode_f16",
