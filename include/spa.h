@@ -63,6 +63,7 @@ typedef enum {
 #define SPA_ST_BAD_BLOCK 0x4  /* a block-table entry needed by a position is outside [0, num_blocks) */
 #define SPA_ST_BOUNDS 0x8     /* a device length exceeds the host bound max_seqlen_q / max_seqlen_k */
 #define SPA_ST_BAD_IDX 0x10   /* a selected index is < -1 or beyond its range; it was skipped */
+#define SPA_ST_TIMEOUT 0x20   /* a bounded on-chip wait expired; the affected outputs are unspecified */
 
 /*
  * spa_prepare_metadata -- step 1, exact per-request and per-token metadata on

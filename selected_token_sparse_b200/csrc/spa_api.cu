@@ -172,7 +172,8 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   const float scale = a->scale == 0.f ? (float)(1.0 / std::sqrt((double)a->D)) : a->scale;
   p->scale_log2 = scale * kLog2e;
   p->group_by_request = pl.group_by_request;
-  p->max_q = pl.max_q;
+  p->max_q = pl.kind == kPlanPrefill ? a->max_seqlen_q : pl.max_q;
+  p->max_k = a->max_seqlen_k;
   p->num_splits = pl.num_splits;
   p->split_len = pl.split_len;
   p->status = a->status;

@@ -37,6 +37,7 @@ struct AttnParams {
   float scale_log2;      // softmax scale * log2(e)
   int group_by_request;  // 1: unit = (request, kv head), rows = q_len * G; 0: unit = (token, kv head)
   int max_q;             // tokens per unit bound (host max_seqlen_q, or 1)
+  int max_k;             // host bound max_seqlen_k
   int num_splits;
   int split_len;         // candidates per split (multiple of the kernel's key tile)
   float* ws_acc;         // [num_splits, T, H_q, D]

@@ -95,8 +95,9 @@ struct MmaCfg {
   static constexpr int RAW_TILE = kMmaKT * D * (int)sizeof(CacheT);
   static constexpr int ROWS = RT * 16;
   // shared memory layout (bytes)
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_RAW = OFF_Q + ROWS * D * 2;                 // stages x (K, V) raw
+  static constexpr int OFF_Q = 0;                                      // Q (int8 path: q*ks, high part)
+  static constexpr int OFF_QLO = OFF_Q + ROWS * D * 2;                 // int8 path: low part
+  static constexpr int OFF_RAW = OFF_QLO + (kInt8 ? ROWS * D * 2 : 0); // stages x (K, V) raw
   static constexpr int OFF_CONV = OFF_RAW + kMmaStages * 2 * RAW_TILE;  // int8 only: (K, V) fp16
   static constexpr int OFF_KPOS = OFF_CONV + (kInt8 ? 2 * TILE16 : 0);
   static constexpr int OFF_SCALE = OFF_KPOS + kMmaStages * kMmaKT * 4;
@@ -106,6 +107,7 @@ struct MmaCfg {
   static constexpr int OFF_RED = OFF_RAW;
   static constexpr int RED_BYTES = (KW > 1) ? NW * 32 * (D / 2 + 4) * 4 : 0;
   static constexpr int SMEM = (OFF_RED + RED_BYTES > END) ? OFF_RED + RED_BYTES : END;
+  static_assert(OFF_RED + RED_BYTES <= OFF_KPOS, "merge buffer must not reach the scales / positions");
 };
 
 template <typename ActT, typename CacheT, int D, int RT, int KW>
@@ -135,32 +137,43 @@ decode_mma_kernel(const AttnParams p) {
   float* vsc_s = ksc_s + D;
   int* prow_s = reinterpret_cast<int*>(smem + C::OFF_PROW);
 
-  // ---- Q rows -> swizzled smem (16-bit, converted for the INT8 path)
+  // ---- Q rows -> swizzled smem.  INT8 caches keep K exact (|k8| <= 128 is
+  // exact in fp16): the key scale is folded into q in fp32 and q*ks is split
+  // into fp16 high and low parts, so S = k8.hi + k8.lo carries ~22 bits.
   const ActT* q = static_cast<const ActT*>(p.q);
-  for (int e = tid; e < C::ROWS * CPR; e += NT) {
-    const int r = e / CPR, c = e % CPR;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < R) {
-      const int t = t0 + r / G, h = h_kv * G + r % G;
-      const ActT* src = q + ((long long)t * p.H_q + h) * D + c * 8;
-      if constexpr (std::is_same<MT, ActT>::value) {
-        v = *reinterpret_cast<const uint4*>(src);
-      } else {
-        alignas(16) __half tmp[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) tmp[i] = __float2half_rn(to_f32(src[i]));
-        v = *reinterpret_cast<const uint4*>(tmp);
-      }
-    }
-    *reinterpret_cast<uint4*>(q_s + swz(r, c, CPR)) = v;
-  }
-  for (int i = tid; i < 128; i += NT) prow_s[i] = (i < nq && has_rows) ? p.token_pos[t0 + i] : -1;
   if constexpr (C::kInt8) {
     for (int d = tid; d < D; d += NT) {
       ksc_s[d] = p.k_scale[h_kv * D + d];
       vsc_s[d] = p.v_scale[h_kv * D + d];
     }
+    __syncthreads();
   }
+  for (int e = tid; e < C::ROWS * CPR; e += NT) {
+    const int r = e / CPR, c = e % CPR;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    uint4 vlo = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const int t = t0 + r / G, h = h_kv * G + r % G;
+      const ActT* src = q + ((long long)t * p.H_q + h) * D + c * 8;
+      if constexpr (!C::kInt8) {
+        v = *reinterpret_cast<const uint4*>(src);
+      } else {
+        alignas(16) __half hi[8];
+        alignas(16) __half lo[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float x = to_f32(src[i]) * ksc_s[c * 8 + i];
+          hi[i] = __float2half_rn(x);
+          lo[i] = __float2half_rn(x - __half2float(hi[i]));
+        }
+        v = *reinterpret_cast<const uint4*>(hi);
+        vlo = *reinterpret_cast<const uint4*>(lo);
+      }
+    }
+    *reinterpret_cast<uint4*>(q_s + swz(r, c, CPR)) = v;
+    if constexpr (C::kInt8) *reinterpret_cast<uint4*>(smem + C::OFF_QLO + swz(r, c, CPR)) = vlo;
+  }
+  for (int i = tid; i < 128; i += NT) prow_s[i] = (i < nq && has_rows) ? p.token_pos[t0 + i] : -1;
 
   // ---- candidate range of this split
   const int n_total = has_rows ? U.n_main + U.n_aux : 0;
@@ -205,7 +218,7 @@ decode_mma_kernel(const AttnParams p) {
   float o[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  uint32_t qf[D / 16][4];
+  uint32_t qf[C::kInt8 ? 1 : D / 16][4];
 
 #pragma unroll
   for (int s = 0; s < kMmaStages - 1; ++s) {
@@ -213,12 +226,14 @@ decode_mma_kernel(const AttnParams p) {
     cp_async_commit();
   }
   __syncthreads();
-  // Q fragments for this warp's row tile stay in registers
+  // Q fragments for this warp's row tile stay in registers (16-bit caches)
+  if constexpr (!C::kInt8) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const int r = wr * 16 + (lane & 15);
-    const int ch = kk * 2 + (lane >> 4);
-    ldsm_x4(qf[kk], q_s + swz(r, ch, CPR));
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = wr * 16 + (lane & 15);
+      const int ch = kk * 2 + (lane >> 4);
+      ldsm_x4(qf[kk], q_s + swz(r, ch, CPR));
+    }
   }
   const int r0 = wr * 16 + (lane >> 2);
   const int r1 = r0 + 8;
@@ -245,12 +260,11 @@ decode_mma_kernel(const AttnParams p) {
         const int ee = isv ? e - KT * RAW_CPR : e;
         const int row = ee / RAW_CPR, c = ee % RAW_CPR;
         const int8_t* src = (isv ? vraw : kraw) + (row * RAW_CPR + c) * 16;
-        const float* sc = (isv ? vsc_s : ksc_s) + c * 16;
         const int4 raw = *reinterpret_cast<const int4*>(src);
         const int8_t* b8 = reinterpret_cast<const int8_t*>(&raw);
         alignas(16) __half h[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) h[i] = __float2half_rn(static_cast<float>(b8[i]) * sc[i]);
+        for (int i = 0; i < 16; ++i) h[i] = __int2half_rn(static_cast<int>(b8[i]));   // exact
         unsigned char* dst = isv ? vconv : kconv;
         *reinterpret_cast<uint4*>(dst + swz(row, 2 * c, CPR)) = *reinterpret_cast<const uint4*>(h);
         *reinterpret_cast<uint4*>(dst + swz(row, 2 * c + 1, CPR)) =
@@ -271,14 +285,28 @@ decode_mma_kernel(const AttnParams p) {
     for (int j = 0; j < KS / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t qh[4], ql[4];
+      if constexpr (C::kInt8) {
+        const int r = wr * 16 + (lane & 15);
+        const int ch = kk * 2 + (lane >> 4);
+        ldsm_x4(qh, q_s + swz(r, ch, CPR));
+        ldsm_x4(ql, smem + C::OFF_QLO + swz(r, ch, CPR));
+      }
 #pragma unroll
       for (int j = 0; j < KS / 8; j += 2) {
         uint32_t b[4];
         const int mi = lane >> 3;
         const int krow = wk * KS + j * 8 + (mi >> 1) * 8 + (lane & 7);
         ldsm_x4(b, ks + swz(krow, kk * 2 + (mi & 1), CPR));
-        mma16816<MT>(s[j], qf[kk], b);
-        mma16816<MT>(s[j + 1], qf[kk], b + 2);
+        if constexpr (C::kInt8) {
+          mma16816<MT>(s[j], qh, b);
+          mma16816<MT>(s[j + 1], qh, b + 2);
+          mma16816<MT>(s[j], ql, b);
+          mma16816<MT>(s[j + 1], ql, b + 2);
+        } else {
+          mma16816<MT>(s[j], qf[kk], b);
+          mma16816<MT>(s[j + 1], qf[kk], b + 2);
+        }
       }
     }
     // mask, scale, online softmax (rows r0, r1)
@@ -400,6 +428,16 @@ decode_mma_kernel(const AttnParams p) {
     }
   }
   if (wk != 0) return;
+  if constexpr (C::kInt8) {   // O = vs * sum_j p_j v8_j (V stayed exact)
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      const int d = n * 8 + (lane & 3) * 2;
+      o[n][0] *= vsc_s[d];
+      o[n][1] *= vsc_s[d + 1];
+      o[n][2] *= vsc_s[d];
+      o[n][3] *= vsc_s[d + 1];
+    }
+  }
 
   // write rows r0, r1 of this row tile
 #pragma unroll
