@@ -279,16 +279,16 @@ def run_ours(args):
         d = {k: (v.clone() if k in ("k_cache", "v_cache", "q", "k_new", "v_new", "block_table",
                                    "cu_seqlens_q", "past_seqlens", "selected_idx") else v)
              for k, v in base.items()}
-        insts.append(pipeline.Step(wl, d))
+        insts.append(pipeline.Step(wl, d, num_splits=args.splits))
     del base
     step0 = insts[0]
     a0 = spa.attention_args(step0.d["q"], step0.d["k_cache"], step0.d["v_cache"],
                             step0.d["block_table"], dict(step0.meta,
                                                          cu_seqlens_q=step0.d["cu_seqlens_q"]),
                             max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
-                            out=step0.out, **step0.kw)
+                            out=step0.out, num_splits=args.splits, **step0.kw)
     plan = spa.attention_plan(a0)
-    launches_per_step = 2 + plan["launches"]
+    launches_per_step = (1 if step0.fused else 2) + plan["launches"]
     kind_name = {0: "decode_scalar", 1: "decode_mma", 2: "prefill_tcgen05"}[plan["kind"]]
 
     stream = torch.cuda.Stream(dev)
@@ -313,7 +313,8 @@ def run_ours(args):
             a = spa.attention_args(st.d["q"], st.d["k_cache"], st.d["v_cache"],
                                    st.d["block_table"], dict(st.meta, cu_seqlens_q=st.d["cu_seqlens_q"]),
                                    max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
-                                   out=st.out, lse=None, num_splits=0, status=st.status, **st.kw)
+                                   out=st.out, lse=None, num_splits=args.splits, status=st.status,
+                                   **st.kw)
             spa.run_attention(a, st.workspace)
         return f
 
@@ -436,7 +437,8 @@ def run_ours(args):
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": f"rotating {R} device instances, attended+q/k/v bytes per cycle "
                          f"{R * per_inst / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB",
-                   "timing": "CUDA graphs of whole steps, CUDA events on the launching stream"},
+                   "timing": "CUDA graphs of whole steps, CUDA events on the launching stream",
+                   "num_splits": plan["num_splits"]},
         "tokens_per_s": world * wl.T / (ms_per_step * 1e-3),
         "attended_kv_bytes_per_step": alg_bytes,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
@@ -507,6 +509,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--instances", type=int, default=0)
+    ap.add_argument("--splits", type=int, default=0, help="key splits per unit (0 = automatic)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -129,6 +129,25 @@ int spa_append_kv(const void* k_new, const void* v_new, int32_t act, void* k_cac
                   int32_t block_size, int32_t num_blocks, int32_t* status, spa_stream_t stream);
 
 /*
+ * spa_prepare_append_kv -- steps 1 and 2 in one launch: the metadata of
+ * spa_prepare_metadata and the scatter of spa_append_kv, with outputs (the
+ * five metadata arrays, both caches and the status bits) identical bit for
+ * bit to calling those two entry points in sequence with the same arguments.
+ * Source: "[WebGPU] Add SparsePagedAttention", File summaries (token_meta and
+ * scatter_kv stages) -- fused here so that one warp derives a token's slot and
+ * writes its K/V rows.  Argument meaning, layouts and error behaviour are those
+ * of the two entry points; H_kv and D describe k_new / v_new and the caches.
+ */
+int spa_prepare_append_kv(const int32_t* cu_seqlens_q, const int32_t* past_seqlens,
+                          const int32_t* block_table, int32_t B, int32_t T, int32_t max_seqlen_q,
+                          int32_t max_seqlen_k, int32_t MB, int32_t block_size, int32_t num_blocks,
+                          int32_t* seqlens_q, int32_t* seqlen_k, int32_t* token_batch,
+                          int32_t* token_pos, int32_t* slot_mapping, const void* k_new,
+                          const void* v_new, int32_t act, void* k_cache, void* v_cache, int32_t cache,
+                          const float* k_scale, const float* v_scale, int32_t H_kv, int32_t D,
+                          int32_t* status, spa_stream_t stream);
+
+/*
  * Arguments of spa_attention (steps 3-5).  `struct_size` must be set to
  * sizeof(spa_attention_args_t) so that the struct can grow compatibly.
  * Sources: "[WebGPU] Add DynamicSparseAttention", Description / Attention
@@ -201,8 +220,12 @@ size_t spa_attention_workspace_size(const spa_attention_args_t* a);
  * FP32 partial states are merged by log-sum-exp; the result does not depend
  * on num_splits beyond rounding.
  * workspace: device buffer of at least spa_attention_workspace_size() bytes,
- * 256-byte aligned, contents irrelevant on entry; it may be NULL when the
- * size is 0.  Calls that share a workspace must be ordered on one stream.
+ * 256-byte aligned; it may be NULL when the size is 0.  It must be zero-filled
+ * before its first use: it holds per-unit split tickets that every call
+ * leaves at zero again (the partial states around them need no
+ * initialisation).  Calls that share a workspace must be ordered on one
+ * stream.  The whole operation is one kernel launch: the last CTA to finish
+ * a unit's splits merges them.
  */
 int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
                   spa_stream_t stream);

@@ -18,8 +18,10 @@ int launch_prepare_metadata(const int32_t*, const int32_t*, const int32_t*, int,
                             cudaStream_t);
 int launch_append_kv(const void*, const void*, int, void*, void*, int, const float*, const float*,
                      const int32_t*, int, int, int, int, int, int32_t*, cudaStream_t);
+int launch_prepare_append(const int32_t*, const int32_t*, const int32_t*, int, int, int, int, int, int, int,
+                          int32_t*, int32_t*, int32_t*, int32_t*, int32_t*, const void*, const void*, int,
+                          void*, void*, int, const float*, const float*, int, int, int32_t*, cudaStream_t);
 int launch_attention_scalar_impl(const AttnParams&, int, int, int, cudaStream_t);
-int launch_combine_impl(const AttnParams&, int, cudaStream_t);
 size_t scalar_smem_bytes(int D, int max_rows, int nq);
 int launch_attention_mma(const AttnParams& p, int act, int cache, int max_rows, cudaStream_t stream);
 int mma_supported(int act, int cache, int D, int max_rows);
@@ -94,7 +96,7 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   // group all tokens of a request when their rows fit one CTA and the
   // candidate list is per request
   const bool per_request_list = !a->selected_idx || a->sel_per_request;
-  pl->group_by_request = per_request_list && (long long)maxq * G <= 128 && maxq > 1;
+  pl->group_by_request = per_request_list && (long long)maxq * G <= 128;
   pl->max_q = pl->group_by_request ? maxq : 1;
   pl->max_rows = pl->max_q * G;
   pl->kind = mma_supported(a->act, a->cache, a->D, pl->max_rows) ? kPlanMma : kPlanScalar;
@@ -128,6 +130,7 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
     const size_t rows = (size_t)a->T * a->H_q;
     pl->ws_acc_bytes = align256(rows * a->D * sizeof(float) * pl->num_splits);
     pl->ws_ml_bytes = align256(rows * 2 * sizeof(float) * pl->num_splits);
+    pl->ws_count_bytes = align256((size_t)units * sizeof(int));
   }
   if (pl->kind == kPlanScalar &&
       scalar_smem_bytes(a->D, pl->max_rows, pl->max_q) > 200 * 1024)
@@ -180,6 +183,7 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   if (pl.num_splits > 1) {
     p->ws_acc = static_cast<float*>(ws);
     p->ws_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.ws_acc_bytes);
+    p->ws_count = reinterpret_cast<int*>(static_cast<char*>(ws) + pl.ws_acc_bytes + pl.ws_ml_bytes);
   }
 }
 
@@ -195,18 +199,10 @@ int run_attention(const spa_attention_args_t* a, const Plan& pl, void* ws, cudaS
   if (pl.kind == kPlanMma) rc = launch_attention_mma(p, a->act, a->cache, pl.max_rows, stream);
   else rc = launch_attention_scalar_impl(p, a->act, a->cache, pl.max_rows, stream);
   if (rc != SPA_OK) return rc;
-  if ((rc = check_launch()) != SPA_OK) return rc;
-  if (pl.num_splits > 1) {
-    launch_combine_impl(p, a->act, stream);
-    if ((rc = check_launch()) != SPA_OK) return rc;
-  }
-  return SPA_OK;
+  return check_launch();
 }
 
-int launches_of(const Plan& pl) {
-  if (pl.kind == kPlanPrefill) return 1;
-  return pl.num_splits > 1 ? 2 : 1;
-}
+int launches_of(const Plan&) { return 1; }
 
 const char* cuda_message() { return g_cuda_msg; }
 int check_launch_public() { return check_launch(); }
@@ -255,12 +251,44 @@ int spa_append_kv(const void* k_new, const void* v_new, int32_t act, void* k_cac
   return check_launch();
 }
 
+int spa_prepare_append_kv(const int32_t* cu_seqlens_q, const int32_t* past_seqlens,
+                          const int32_t* block_table, int32_t B, int32_t T, int32_t max_seqlen_q,
+                          int32_t max_seqlen_k, int32_t MB, int32_t block_size, int32_t num_blocks,
+                          int32_t* seqlens_q, int32_t* seqlen_k, int32_t* token_batch,
+                          int32_t* token_pos, int32_t* slot_mapping, const void* k_new,
+                          const void* v_new, int32_t act, void* k_cache, void* v_cache, int32_t cache,
+                          const float* k_scale, const float* v_scale, int32_t H_kv, int32_t D,
+                          int32_t* status, spa_stream_t stream) {
+  // the union of both entry points' checks
+  if (B < 0 || T < 0 || MB < 0 || block_size <= 0 || num_blocks < 0) return SPA_ERR_INVALID_ARG;
+  if (B > 16384) return SPA_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * block_size >= (1LL << 31)) return SPA_ERR_INVALID_ARG;
+  if (!cu_seqlens_q) return SPA_ERR_INVALID_ARG;
+  if (B > 0 && (!past_seqlens || !seqlens_q || !seqlen_k || (MB > 0 && !block_table)))
+    return SPA_ERR_INVALID_ARG;
+  if (T > 0 && (!token_batch || !token_pos || !slot_mapping)) return SPA_ERR_INVALID_ARG;
+  if (!act_ok(act) || !(cache == act || cache == SPA_I8)) return SPA_ERR_INVALID_ARG;
+  if (H_kv <= 0 || D <= 0 || (D * elt_bytes(act)) % 16 != 0) return SPA_ERR_INVALID_ARG;
+  if (cache == SPA_I8 && (D % 16 != 0 || !k_scale || !v_scale)) return SPA_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!k_new || !v_new || !k_cache || !v_cache) return SPA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new) |
+         reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15)
+      return SPA_ERR_INVALID_ARG;
+  }
+  launch_prepare_append(cu_seqlens_q, past_seqlens, block_table, B, T, max_seqlen_q, max_seqlen_k, MB,
+                        block_size, num_blocks, seqlens_q, seqlen_k, token_batch, token_pos, slot_mapping,
+                        k_new, v_new, act, k_cache, v_cache, cache, k_scale, v_scale, H_kv, D, status,
+                        (cudaStream_t)stream);
+  return check_launch();
+}
+
 size_t spa_attention_workspace_size(const spa_attention_args_t* a) {
   if (validate_attention(a) != SPA_OK) return 0;
   if (a->T == 0 || a->B == 0) return 0;
   Plan pl;
   if (make_plan(a, &pl) != SPA_OK) return 0;
-  return pl.ws_acc_bytes + pl.ws_ml_bytes;
+  return pl.ws_acc_bytes + pl.ws_ml_bytes + pl.ws_count_bytes;
 }
 
 int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
@@ -270,7 +298,7 @@ int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspa
   if (a->T == 0 || a->B == 0) return SPA_OK;
   Plan pl;
   if ((rc = make_plan(a, &pl)) != SPA_OK) return rc;
-  const size_t need = pl.ws_acc_bytes + pl.ws_ml_bytes;
+  const size_t need = pl.ws_acc_bytes + pl.ws_ml_bytes + pl.ws_count_bytes;
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return SPA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPA_ERR_WORKSPACE;

@@ -9,7 +9,7 @@
 //
 // Pure bandwidth: one thread moves one 16-byte chunk of the destination row,
 // so loads and stores are 16-byte vectors and a warp covers whole rows.
-#include "spa_common.cuh"
+#include "spa_attn.cuh"
 
 namespace spa {
 
@@ -21,6 +21,8 @@ append_copy_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_
                    uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                    const int32_t* __restrict__ slot_mapping, int T, int H_kv, int chunks_per_row,
                    long long num_slots, int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   const long long per_tensor = (long long)T * H_kv * chunks_per_row;
   int bits = 0;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < 2 * per_tensor;
@@ -55,6 +57,8 @@ append_int8_kernel(const ActT* __restrict__ k_new, const ActT* __restrict__ v_ne
                    const float* __restrict__ k_scale, const float* __restrict__ v_scale,
                    const int32_t* __restrict__ slot_mapping, int T, int H_kv, int D,
                    long long num_slots, int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   const int chunks_per_row = D / 16;
   const long long per_tensor = (long long)T * H_kv * chunks_per_row;
   int bits = 0;
@@ -103,26 +107,25 @@ int launch_append_kv(const void* k_new, const void* v_new, int act, void* k_cach
     const int elt = act == SPA_F32 ? 4 : 2;
     const int chunks = D * elt / 16;
     const long long work = 2LL * T * H_kv * chunks;
-    append_copy_kernel<<<grid_for(work), kAppendThreads, 0, stream>>>(
-        (const uint4*)k_new, (const uint4*)v_new, (uint4*)k_cache, (uint4*)v_cache, slot_mapping,
-        T, H_kv, chunks, num_slots, status);
-    return 0;
+    return launch_pdl(append_copy_kernel, dim3(grid_for(work)), dim3(kAppendThreads), 0, stream,
+                      (const uint4*)k_new, (const uint4*)v_new, (uint4*)k_cache, (uint4*)v_cache,
+                      slot_mapping, T, H_kv, chunks, num_slots, status);
   }
   const long long work = 2LL * T * H_kv * (D / 16);
   const int g = grid_for(work);
   switch (act) {
     case SPA_F32:
-      append_int8_kernel<float><<<g, kAppendThreads, 0, stream>>>(
+      launch_pdl(append_int8_kernel<float>, dim3(g), dim3(kAppendThreads), 0, stream,
           (const float*)k_new, (const float*)v_new, (int8_t*)k_cache, (int8_t*)v_cache, k_scale,
           v_scale, slot_mapping, T, H_kv, D, num_slots, status);
       break;
     case SPA_F16:
-      append_int8_kernel<__half><<<g, kAppendThreads, 0, stream>>>(
+      launch_pdl(append_int8_kernel<__half>, dim3(g), dim3(kAppendThreads), 0, stream,
           (const __half*)k_new, (const __half*)v_new, (int8_t*)k_cache, (int8_t*)v_cache, k_scale,
           v_scale, slot_mapping, T, H_kv, D, num_slots, status);
       break;
     default:
-      append_int8_kernel<__nv_bfloat16><<<g, kAppendThreads, 0, stream>>>(
+      launch_pdl(append_int8_kernel<__nv_bfloat16>, dim3(g), dim3(kAppendThreads), 0, stream,
           (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, (int8_t*)k_cache,
           (int8_t*)v_cache, k_scale, v_scale, slot_mapping, T, H_kv, D, num_slots, status);
       break;

@@ -120,6 +120,9 @@ decode_mma_kernel(const AttnParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wr = warp % RT;   // row tile of this warp
   const int wk = warp / RT;   // key slice of this warp
+  __shared__ int last_flag;
+  pdl_wait();
+  pdl_trigger();
 
   Unit U;
   const bool has_rows = decode_unit(p, blockIdx.x, U);
@@ -173,7 +176,7 @@ decode_mma_kernel(const AttnParams p) {
     *reinterpret_cast<uint4*>(q_s + swz(r, c, CPR)) = v;
     if constexpr (C::kInt8) *reinterpret_cast<uint4*>(smem + C::OFF_QLO + swz(r, c, CPR)) = vlo;
   }
-  for (int i = tid; i < 128; i += NT) prow_s[i] = (i < nq && has_rows) ? p.token_pos[t0 + i] : -1;
+  for (int i = tid; i < 128; i += NT) prow_s[i] = (i < nq && has_rows) ? U.p_first + i : -1;
 
   // ---- candidate range of this split
   const int n_total = has_rows ? U.n_main + U.n_aux : 0;
@@ -427,7 +430,7 @@ decode_mma_kernel(const AttnParams p) {
       }
     }
   }
-  if (wk != 0) return;
+  if (wk == 0) {
   if constexpr (C::kInt8) {   // O = vs * sum_j p_j v8_j (V stayed exact)
 #pragma unroll
     for (int n = 0; n < D / 8; ++n) {
@@ -473,6 +476,8 @@ decode_mma_kernel(const AttnParams p) {
       }
     }
   }
+  }  // wk == 0
+  if (p.num_splits > 1) finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
 }
 
 // ---------------------------------------------------------------------------
@@ -493,8 +498,7 @@ static int launch_rt(const AttnParams& p, cudaStream_t stream) {
   if (C::SMEM > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
   dim3 grid(units, p.num_splits);
-  kern<<<grid, C::NT, C::SMEM, stream>>>(p);
-  return 0;
+  return launch_pdl(kern, grid, dim3(C::NT), C::SMEM, stream, p);
 }
 
 template <typename ActT, typename CacheT, int D>

@@ -46,6 +46,9 @@ decode_scalar_kernel(const AttnParams p) {
   constexpr int MAXO = kScalarMaxRows * D / NT;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int last_flag;
+  pdl_wait();
+  pdl_trigger();
 
   Unit U;
   const bool has_rows = decode_unit(p, blockIdx.x, U);
@@ -84,7 +87,7 @@ decode_scalar_kernel(const AttnParams p) {
     m_s[r] = -INFINITY;
     l_s[r] = 0.f;
   }
-  for (int i = tid; i < nq; i += NT) prow_s[i] = has_rows ? p.token_pos[t0 + i] : -1;
+  for (int i = tid; i < nq; i += NT) prow_s[i] = has_rows ? U.p_first + i : -1;
 
   float acc[MAXO];
 #pragma unroll
@@ -211,6 +214,7 @@ decode_scalar_kernel(const AttnParams p) {
         }
       }
     }
+    finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
   }
 }
 
@@ -222,8 +226,7 @@ static int launch_scalar_t(const AttnParams& p, int max_rows, cudaStream_t strea
   if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
   dim3 grid(units, p.num_splits);
-  kern<<<grid, kScalarThreads, smem, stream>>>(p);
-  return 0;
+  return launch_pdl(kern, grid, dim3(kScalarThreads), smem, stream, p);
 }
 
 template <typename ActT, typename CacheT>
@@ -231,9 +234,6 @@ static int launch_scalar_d(const AttnParams& p, int max_rows, cudaStream_t strea
   if (p.D == 64) return launch_scalar_t<ActT, CacheT, 64>(p, max_rows, stream);
   return launch_scalar_t<ActT, CacheT, 128>(p, max_rows, stream);
 }
-
-int launch_attention_scalar_dispatch(const AttnParams& p, int act, int cache, int max_rows,
-                                     cudaStream_t stream);
 
 int launch_attention_scalar_impl(const AttnParams& p, int act, int cache, int max_rows,
                                  cudaStream_t stream) {
@@ -248,73 +248,6 @@ int launch_attention_scalar_impl(const AttnParams& p, int act, int cache, int ma
       if (cache == SPA_I8) return launch_scalar_d<__nv_bfloat16, int8_t>(p, max_rows, stream);
       return launch_scalar_d<__nv_bfloat16, __nv_bfloat16>(p, max_rows, stream);
   }
-}
-
-// ---------------------------------------------------------------------------
-// Log-sum-exp combine of split partials with the sink; one warp per (t, h).
-// ---------------------------------------------------------------------------
-template <typename ActT, int D>
-__global__ void __launch_bounds__(128) combine_kernel(const AttnParams p) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * 4 + warp;
-  if (row >= (long long)p.T * p.H_q) return;
-  const int t = (int)(row / p.H_q), h = (int)(row % p.H_q);
-  ActT* out = static_cast<ActT*>(p.out) + row * D;
-  constexpr int PER = D / 32;
-  if (p.token_batch[t] < 0) {
-#pragma unroll
-    for (int i = 0; i < PER; ++i) out[lane + 32 * i] = from_f32<ActT>(0.f);
-    if (lane == 0 && p.lse) p.lse[row] = -INFINITY;
-    return;
-  }
-  const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
-  const long long stride = (long long)p.T * p.H_q;
-  float M = sink2;
-  for (int s = 0; s < p.num_splits; ++s) M = fmaxf(M, p.ws_ml[(s * stride + row) * 2]);
-  float o[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) o[i] = 0.f;
-  float lse = -INFINITY;
-  if (M != -INFINITY) {
-    float Lsum = (sink2 == -INFINITY) ? 0.f : exp2f(sink2 - M);
-    for (int s = 0; s < p.num_splits; ++s) {
-      const float ms = p.ws_ml[(s * stride + row) * 2];
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      Lsum += w * p.ws_ml[(s * stride + row) * 2 + 1];
-      const float* a = p.ws_acc + (s * stride + row) * D;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) o[i] = fmaf(w, a[lane + 32 * i], o[i]);
-    }
-    const float inv = 1.0f / Lsum;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) o[i] *= inv;
-    lse = (M + log2f(Lsum)) * kLn2;
-  }
-#pragma unroll
-  for (int i = 0; i < PER; ++i) out[lane + 32 * i] = from_f32<ActT>(o[i]);
-  if (lane == 0 && p.lse) p.lse[row] = lse;
-}
-
-int launch_combine_impl(const AttnParams& p, int act, cudaStream_t stream) {
-  const long long rows = (long long)p.T * p.H_q;
-  if (rows == 0) return 0;
-  const int grid = (int)((rows + 3) / 4);
-  switch (act) {
-    case SPA_F32:
-      if (p.D == 64) combine_kernel<float, 64><<<grid, 128, 0, stream>>>(p);
-      else combine_kernel<float, 128><<<grid, 128, 0, stream>>>(p);
-      break;
-    case SPA_F16:
-      if (p.D == 64) combine_kernel<__half, 64><<<grid, 128, 0, stream>>>(p);
-      else combine_kernel<__half, 128><<<grid, 128, 0, stream>>>(p);
-      break;
-    default:
-      if (p.D == 64) combine_kernel<__nv_bfloat16, 64><<<grid, 128, 0, stream>>>(p);
-      else combine_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(p);
-      break;
-  }
-  return 0;
 }
 
 size_t scalar_smem_bytes(int D, int max_rows, int nq) {

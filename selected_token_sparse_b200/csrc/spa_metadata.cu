@@ -1,4 +1,4 @@
-// Step 1 -- metadata prepare.
+// Step 1 -- metadata prepare (and its fusion with step 2, the KV append).
 //
 // Derives the exact per-request lengths and the per-token (request, position,
 // slot) metadata on the device, so that no device-to-host copy is needed per
@@ -8,25 +8,23 @@
 // not a linear scan ("[WebGPU] Add SparsePagedAttention", review note on the
 // O(batch_size) scan per token and on malformed cumulative lengths).
 //
-// One launch.  Every block rebuilds the sanitised cumulative lengths
+// Every block rebuilds the sanitised cumulative lengths
 //   cs[0] = 0,  cs[b] = min(max(cu[1..b], 0), T)
 // (a clamped prefix maximum) in shared memory with a block-wide scan; block 0
-// also writes the per-request outputs and status bits; every thread then
-// handles tokens in a grid-stride loop.
-#include "spa_common.cuh"
+// also writes the per-request outputs and status bits.
+//
+// prepare_append_kernel fuses the scatter of the current tokens' K/V rows
+// into the same launch (one warp per token: the lanes find the token's slot,
+// then copy its rows as 16-byte vectors, quantising for an INT8 cache); its
+// outputs are bit-identical to spa_prepare_metadata followed by spa_append_kv.
+#include "spa_attn.cuh"
 
 namespace spa {
 
 constexpr int kMetaThreads = 256;
 
-__global__ void __launch_bounds__(kMetaThreads)
-prepare_metadata_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
-                        const int32_t* __restrict__ block_table, int B, int T, int max_q,
-                        int max_k, int MB, int bs, int num_blocks, int32_t* __restrict__ seqlens_q,
-                        int32_t* __restrict__ seqlen_k, int32_t* __restrict__ token_batch,
-                        int32_t* __restrict__ token_pos, int32_t* __restrict__ slot_mapping,
-                        int32_t* __restrict__ status) {
-  extern __shared__ int32_t cs[];  // [B + 1]
+// Sanitised cumulative lengths into cs[0..B] (all threads of the block).
+__device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, int T, int32_t* cs) {
   __shared__ int32_t warp_max[kMetaThreads / 32];
   __shared__ int32_t chunk_carry[kMetaThreads];
   const int tid = threadIdx.x;
@@ -41,8 +39,7 @@ prepare_metadata_kernel(const int32_t* __restrict__ cu, const int32_t* __restric
     run = max(run, v);
     cs[i] = run;
   }
-  // inclusive scan (max) of chunk maxima across the block
-  int lane = tid & 31, warp = tid >> 5;
+  const int lane = tid & 31, warp = tid >> 5;
   int x = (c0 < c1) ? run : 0;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -53,66 +50,174 @@ prepare_metadata_kernel(const int32_t* __restrict__ cu, const int32_t* __restric
   __syncthreads();
   int prev_warps = 0;
   for (int w = 0; w < warp; ++w) prev_warps = max(prev_warps, warp_max[w]);
-  int incl = max(x, prev_warps);
-  chunk_carry[tid] = incl;
+  chunk_carry[tid] = max(x, prev_warps);
   __syncthreads();
-  int carry = (tid == 0) ? 0 : chunk_carry[tid - 1];
+  const int carry = (tid == 0) ? 0 : chunk_carry[tid - 1];
   for (int i = c0; i < c1; ++i) cs[i] = min(max(cs[i], carry), T);
   __syncthreads();
+}
 
-  if (blockIdx.x == 0) {
-    int bits = 0;
-    for (int b = tid; b <= B; b += kMetaThreads) {
-      int raw = (b == 0) ? cu[0] : cu[b];
-      if (raw != cs[b]) bits |= kStBadCu;
-      if (b == B && cs[B] != T) bits |= kStBadCu;
-    }
-    for (int b = tid; b < B; b += kMetaThreads) {
-      int p = past[b];
-      if (p < 0) {
-        bits |= kStBadCu;
-        p = 0;
-      }
-      int q_len = cs[b + 1] - cs[b];
-      long long total = (long long)p + q_len;
-      seqlens_q[b] = q_len;
-      seqlen_k[b] = (int32_t)(total - 1);
-      if (q_len > max_q || total > (long long)max_k) bits |= kStBounds;
-    }
-    flag(status, bits);
-  }
-
+// Per-request outputs and the request-level status bits (block 0 only).
+__device__ __forceinline__ int per_request(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
+                                           const int32_t* cs, int B, int T, int max_q, int max_k,
+                                           int32_t* __restrict__ seqlens_q, int32_t* __restrict__ seqlen_k) {
   int bits = 0;
-  for (int t = blockIdx.x * kMetaThreads + tid; t < T; t += gridDim.x * kMetaThreads) {
-    // owner = upper_bound(cs[0..B], t) - 1, valid iff t < cs[B]
-    int lo = 0, hi = n;  // search in [lo, hi)
-    while (lo < hi) {
-      int mid = (lo + hi) >> 1;
-      if (cs[mid] <= t) lo = mid + 1; else hi = mid;
+  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
+    if (cu[b] != cs[b]) bits |= kStBadCu;
+    if (b == B && cs[B] != T) bits |= kStBadCu;
+  }
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    int pb = past[b];
+    if (pb < 0) {
+      bits |= kStBadCu;
+      pb = 0;
     }
-    int b = lo - 1;
-    if (t >= cs[B] || b < 0 || b >= B) {
-      token_batch[t] = -1;
-      token_pos[t] = -1;
-      slot_mapping[t] = -1;
-      continue;
-    }
-    int p0 = max(past[b], 0);
-    int pos = p0 + (t - cs[b]);
-    token_batch[t] = b;
-    token_pos[t] = pos;
-    int lb = pos / bs;
-    int slot = -1;
-    if (lb >= MB) {
-      bits |= kStCapacity;
-    } else {
-      int blk = block_table[(long long)b * MB + lb];
-      if (blk < 0 || blk >= num_blocks) bits |= kStBadBlock;
-      else slot = blk * bs + pos % bs;
-    }
-    slot_mapping[t] = slot;
+    const int q_len = cs[b + 1] - cs[b];
+    const long long total = (long long)pb + q_len;
+    seqlens_q[b] = q_len;
+    seqlen_k[b] = (int32_t)(total - 1);
+    if (q_len > max_q || total > (long long)max_k) bits |= kStBounds;
+  }
+  return bits;
+}
+
+struct TokenMeta {
+  int b, pos, slot;
+};
+
+// Owner request, absolute position and cache slot of token t.
+__device__ __forceinline__ TokenMeta token_meta(int t, const int32_t* cs, int B,
+                                                const int32_t* __restrict__ past,
+                                                const int32_t* __restrict__ block_table, int MB, int bs,
+                                                int num_blocks, int& bits) {
+  TokenMeta m = {-1, -1, -1};
+  int lo = 0, hi = B + 1;  // owner = upper_bound(cs[0..B], t) - 1
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (cs[mid] <= t) lo = mid + 1; else hi = mid;
+  }
+  const int b = lo - 1;
+  if (t >= cs[B] || b < 0 || b >= B) return m;
+  m.b = b;
+  m.pos = max(past[b], 0) + (t - cs[b]);
+  const int lb = m.pos / bs;
+  if (lb >= MB) {
+    bits |= kStCapacity;
+  } else {
+    const int blk = block_table[(long long)b * MB + lb];
+    if (blk < 0 || blk >= num_blocks) bits |= kStBadBlock;
+    else m.slot = blk * bs + m.pos % bs;
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(kMetaThreads)
+prepare_metadata_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
+                        const int32_t* __restrict__ block_table, int B, int T, int max_q,
+                        int max_k, int MB, int bs, int num_blocks, int32_t* __restrict__ seqlens_q,
+                        int32_t* __restrict__ seqlen_k, int32_t* __restrict__ token_batch,
+                        int32_t* __restrict__ token_pos, int32_t* __restrict__ slot_mapping,
+                        int32_t* __restrict__ status) {
+  extern __shared__ int32_t cs[];  // [B + 1]
+  pdl_wait();
+  pdl_trigger();
+  build_cs(cu, B, T, cs);
+  if (blockIdx.x == 0) flag(status, per_request(cu, past, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
+  int bits = 0;
+  for (int t = blockIdx.x * kMetaThreads + threadIdx.x; t < T; t += gridDim.x * kMetaThreads) {
+    const TokenMeta m = token_meta(t, cs, B, past, block_table, MB, bs, num_blocks, bits);
+    token_batch[t] = m.b;
+    token_pos[t] = m.pos;
+    slot_mapping[t] = m.slot;
   }
   flag(status, bits);
+}
+
+// Copy (or quantise) token t's K and V rows for all kv heads into `slot`, by one warp.
+template <typename ActT, typename CacheT>
+__device__ __forceinline__ void append_token_rows(const ActT* __restrict__ k_new,
+                                                  const ActT* __restrict__ v_new,
+                                                  CacheT* __restrict__ k_cache, CacheT* __restrict__ v_cache,
+                                                  const float* __restrict__ k_scale,
+                                                  const float* __restrict__ v_scale, int t, int slot,
+                                                  int H_kv, int D, int lane) {
+  const long long src_row = (long long)t * H_kv * D;
+  const long long dst_row = (long long)slot * H_kv * D;
+  if constexpr (sizeof(CacheT) != 1) {
+    // exact copy, 16-byte vectors
+    constexpr int EPV = 16 / sizeof(ActT);
+    const int nvec = H_kv * D / EPV;
+    const uint4* ks = reinterpret_cast<const uint4*>(k_new + src_row);
+    const uint4* vs = reinterpret_cast<const uint4*>(v_new + src_row);
+    uint4* kd = reinterpret_cast<uint4*>(k_cache + dst_row);
+    uint4* vd = reinterpret_cast<uint4*>(v_cache + dst_row);
+    for (int i = lane; i < nvec; i += 32) {
+      kd[i] = ks[i];
+      vd[i] = vs[i];
+    }
+  } else {
+    // q8 = clamp(rint(x / scale), -128, 127) per channel, 16 channels per lane step
+    const int ngrp = H_kv * D / 16;
+    for (int i = lane; i < 2 * ngrp; i += 32) {
+      const bool isv = i >= ngrp;
+      const int gi = isv ? i - ngrp : i;
+      const int e0 = gi * 16;                  // element offset within the token's H_kv*D row
+      const int h = e0 / D, d0 = e0 % D;
+      const ActT* src = (isv ? v_new : k_new) + src_row + e0;
+      const float* sc = (isv ? v_scale : k_scale) + (long long)h * D + d0;
+      alignas(16) int8_t qv[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float r = rintf(__fdiv_rn(to_f32(src[e]), sc[e]));
+        r = fminf(fmaxf(r, -128.0f), 127.0f);
+        qv[e] = static_cast<int8_t>(static_cast<int>(r));
+      }
+      int8_t* dst = reinterpret_cast<int8_t*>(isv ? v_cache : k_cache) + dst_row + e0;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(qv);
+    }
+  }
+}
+
+template <typename ActT, typename CacheT>
+__global__ void __launch_bounds__(kMetaThreads)
+prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
+                      const int32_t* __restrict__ block_table, int B, int T, int max_q, int max_k, int MB,
+                      int bs, int num_blocks, int32_t* __restrict__ seqlens_q,
+                      int32_t* __restrict__ seqlen_k, int32_t* __restrict__ token_batch,
+                      int32_t* __restrict__ token_pos, int32_t* __restrict__ slot_mapping,
+                      const ActT* __restrict__ k_new, const ActT* __restrict__ v_new,
+                      CacheT* __restrict__ k_cache, CacheT* __restrict__ v_cache,
+                      const float* __restrict__ k_scale, const float* __restrict__ v_scale, int H_kv,
+                      int D, int32_t* __restrict__ status) {
+  extern __shared__ int32_t cs[];  // [B + 1]
+  pdl_wait();
+  pdl_trigger();
+  build_cs(cu, B, T, cs);
+  if (blockIdx.x == 0) flag(status, per_request(cu, past, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
+  const int lane = threadIdx.x & 31;
+  const int wpb = kMetaThreads / 32;
+  int bits = 0;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    int tb = 0;  // every lane computes the same metadata; lane 0 reports and writes it
+    const TokenMeta m = token_meta(t, cs, B, past, block_table, MB, bs, num_blocks, tb);
+    if (lane == 0) {
+      bits |= tb;
+      token_batch[t] = m.b;
+      token_pos[t] = m.pos;
+      slot_mapping[t] = m.slot;
+    }
+    if (m.slot >= 0)
+      append_token_rows<ActT, CacheT>(k_new, v_new, k_cache, v_cache, k_scale, v_scale, t, m.slot, H_kv, D,
+                                      lane);
+  }
+  flag(status, bits);
+}
+
+static size_t cs_smem(int B) { return sizeof(int32_t) * (size_t)(B + 1); }
+
+template <typename K>
+static void allow_smem(K kern, size_t smem) {
+  if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
 int launch_prepare_metadata(const int32_t* cu, const int32_t* past, const int32_t* block_table,
@@ -123,15 +228,53 @@ int launch_prepare_metadata(const int32_t* cu, const int32_t* past, const int32_
   int grid = (T + kMetaThreads - 1) / kMetaThreads;
   if (grid < 1) grid = 1;
   if (grid > 148 * 8) grid = 148 * 8;
-  size_t smem = sizeof(int32_t) * (size_t)(B + 1);
-  if (smem > 48 * 1024) {
-    cudaFuncSetAttribute(prepare_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
+  const size_t smem = cs_smem(B);
+  allow_smem(prepare_metadata_kernel, smem);
+  return launch_pdl(prepare_metadata_kernel, dim3(grid), dim3(kMetaThreads), smem, stream, cu, past,
+                    block_table, B, T, max_q, max_k, MB, bs, num_blocks, seqlens_q, seqlen_k, token_batch,
+                    token_pos, slot_mapping, status);
+}
+
+template <typename ActT, typename CacheT>
+static int launch_pa(const int32_t* cu, const int32_t* past, const int32_t* block_table, int B, int T,
+                     int max_q, int max_k, int MB, int bs, int num_blocks, int32_t* seqlens_q,
+                     int32_t* seqlen_k, int32_t* token_batch, int32_t* token_pos, int32_t* slot_mapping,
+                     const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                     const float* k_scale, const float* v_scale, int H_kv, int D, int32_t* status,
+                     cudaStream_t stream) {
+  const int wpb = kMetaThreads / 32;
+  int grid = (T + wpb - 1) / wpb;
+  if (grid < 1) grid = 1;
+  if (grid > 148 * 8) grid = 148 * 8;
+  const size_t smem = cs_smem(B);
+  auto kern = prepare_append_kernel<ActT, CacheT>;
+  allow_smem(kern, smem);
+  return launch_pdl(kern, dim3(grid), dim3(kMetaThreads), smem, stream, cu, past, block_table, B, T, max_q,
+                    max_k, MB, bs, num_blocks, seqlens_q, seqlen_k, token_batch, token_pos, slot_mapping,
+                    static_cast<const ActT*>(k_new), static_cast<const ActT*>(v_new),
+                    static_cast<CacheT*>(k_cache), static_cast<CacheT*>(v_cache), k_scale, v_scale, H_kv, D,
+                    status);
+}
+
+int launch_prepare_append(const int32_t* cu, const int32_t* past, const int32_t* block_table, int B, int T,
+                          int max_q, int max_k, int MB, int bs, int num_blocks, int32_t* seqlens_q,
+                          int32_t* seqlen_k, int32_t* token_batch, int32_t* token_pos,
+                          int32_t* slot_mapping, const void* k_new, const void* v_new, int act,
+                          void* k_cache, void* v_cache, int cache, const float* k_scale,
+                          const float* v_scale, int H_kv, int D, int32_t* status, cudaStream_t stream) {
+#define SPA_PA(A, C)                                                                                     \
+  return launch_pa<A, C>(cu, past, block_table, B, T, max_q, max_k, MB, bs, num_blocks, seqlens_q,       \
+                         seqlen_k, token_batch, token_pos, slot_mapping, k_new, v_new, k_cache, v_cache, \
+                         k_scale, v_scale, H_kv, D, status, stream)
+  if (cache == SPA_I8) {
+    if (act == SPA_F32) SPA_PA(float, int8_t);
+    if (act == SPA_F16) SPA_PA(__half, int8_t);
+    SPA_PA(__nv_bfloat16, int8_t);
   }
-  prepare_metadata_kernel<<<grid, kMetaThreads, smem, stream>>>(
-      cu, past, block_table, B, T, max_q, max_k, MB, bs, num_blocks, seqlens_q, seqlen_k,
-      token_batch, token_pos, slot_mapping, status);
-  return 0;
+  if (act == SPA_F32) SPA_PA(float, float);
+  if (act == SPA_F16) SPA_PA(__half, __half);
+  SPA_PA(__nv_bfloat16, __nv_bfloat16);
+#undef SPA_PA
 }
 
 }  // namespace spa

@@ -19,6 +19,7 @@ struct Plan {
   int units;
   size_t ws_acc_bytes;
   size_t ws_ml_bytes;
+  size_t ws_count_bytes;
 };
 
 int validate_attention(const spa_attention_args_t* a);

@@ -133,6 +133,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
 
   // ---- geometry (uniform across the CTA)
   PfGeom g;
@@ -467,8 +469,7 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   auto kern = prefill_tcgen05_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   dim3 grid(p.H_q, n_qt, p.B);
-  kern<<<grid, 128, C::SMEM, stream>>>(p, tq, tk, tv, n_qt, box_rows, max_tiles);
-  return SPA_OK;
+  return launch_pdl(kern, grid, dim3(128), C::SMEM, stream, p, tq, tk, tv, n_qt, box_rows, max_tiles);
 }
 
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream) {

@@ -43,7 +43,7 @@ class Step:
     """Pre-allocated buffers for repeated steps of one workload on one device."""
 
     def __init__(self, wl, d: Dict[str, torch.Tensor], num_splits: int = 0,
-                 want_lse: bool = False):
+                 want_lse: bool = False, fused: bool = True):
         self.wl, self.d = wl, d
         dev = d["q"].device
         i32 = dict(dtype=torch.int32, device=dev)
@@ -60,16 +60,24 @@ class Step:
         args = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], d["block_table"], meta,
                                   max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
                                   out=self.out, lse=self.lse, num_splits=num_splits, **self.kw)
-        n = spa.workspace_size(args)
-        self.workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+        self.workspace = spa.new_workspace(spa.workspace_size(args), dev)
+        self.fused = fused
 
     def __call__(self):
         wl, d = self.wl, self.d
-        meta = spa.prepare_metadata(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"], wl.T,
-                                    wl.max_seqlen_q, wl.max_seqlen_k, wl.block_size, wl.NB,
-                                    status=self.status, out=self.meta)
-        spa.append_kv(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"], meta["slot_mapping"],
-                      k_scale=d.get("k_scale"), v_scale=d.get("v_scale"), status=self.status)
+        if self.fused:
+            meta = spa.prepare_append_kv(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],
+                                         wl.T, wl.max_seqlen_q, wl.max_seqlen_k, d["k_new"],
+                                         d["v_new"], d["k_cache"], d["v_cache"],
+                                         k_scale=d.get("k_scale"), v_scale=d.get("v_scale"),
+                                         status=self.status, out=self.meta)
+        else:
+            meta = spa.prepare_metadata(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],
+                                        wl.T, wl.max_seqlen_q, wl.max_seqlen_k, wl.block_size,
+                                        wl.NB, status=self.status, out=self.meta)
+            spa.append_kv(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"],
+                          meta["slot_mapping"], k_scale=d.get("k_scale"),
+                          v_scale=d.get("v_scale"), status=self.status)
         a = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], d["block_table"], meta,
                                max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
                                out=self.out, lse=self.lse, num_splits=self.num_splits,
@@ -78,10 +86,10 @@ class Step:
         return self.out
 
 
-def run_step(wl, device="cuda", num_splits: int = 0, want_lse: bool = True):
+def run_step(wl, device="cuda", num_splits: int = 0, want_lse: bool = True, fused: bool = True):
     """Run one step on fresh device copies; returns host numpy results."""
     d = to_device(wl, device)
-    st = Step(wl, d, num_splits=num_splits, want_lse=want_lse)
+    st = Step(wl, d, num_splits=num_splits, want_lse=want_lse, fused=fused)
     st()
     torch.cuda.synchronize(device)
     res = {k: v.cpu().numpy() for k, v in st.meta.items()}

@@ -21,7 +21,7 @@ SPA_F32, SPA_F16, SPA_BF16, SPA_I8 = 0, 1, 2, 3
 SPA_OK, SPA_ERR_INVALID_ARG, SPA_ERR_UNSUPPORTED, SPA_ERR_WORKSPACE, SPA_ERR_CUDA = 0, -1, -2, -3, -4
 ST_BAD_CU, ST_CAPACITY, ST_BAD_BLOCK, ST_BOUNDS, ST_BAD_IDX = 0x1, 0x2, 0x4, 0x8, 0x10
 
-EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_attention",
+EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_prepare_append_kv", "spa_attention",
             "spa_attention_workspace_size", "spa_attention_plan", "spa_error_string")
 
 _DT = {torch.float32: SPA_F32, torch.float16: SPA_F16, torch.bfloat16: SPA_BF16, torch.int8: SPA_I8}
@@ -68,6 +68,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spa_append_kv.restype = ctypes.c_int
     lib.spa_append_kv.argtypes = [_vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32,
                                   _i32, _i32, _vp, _vp]
+    lib.spa_prepare_append_kv.restype = ctypes.c_int
+    lib.spa_prepare_append_kv.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32,
+                                          _vp, _vp, _i32, _i32, _vp, _vp]
     lib.spa_attention_workspace_size.restype = ctypes.c_size_t
     lib.spa_attention_workspace_size.argtypes = [ctypes.POINTER(AttentionArgs)]
     lib.spa_attention.restype = ctypes.c_int
@@ -158,6 +162,36 @@ def append_kv(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
     _check(rc, "spa_append_kv")
 
 
+def prepare_append_kv(cu_seqlens_q: torch.Tensor, past_seqlens: torch.Tensor,
+                      block_table: torch.Tensor, T: int, max_seqlen_q: int, max_seqlen_k: int,
+                      k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, k_scale: Optional[torch.Tensor] = None,
+                      v_scale: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                      out: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+    """Steps 1 + 2 in one launch (same results as prepare_metadata then append_kv)."""
+    dev = cu_seqlens_q.device
+    B = cu_seqlens_q.numel() - 1
+    MB = block_table.shape[1] if block_table.dim() == 2 else 0
+    NB, bs, H_kv, D = k_cache.shape
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = {"seqlens_q": torch.empty(B, **i32), "seqlen_k": torch.empty(B, **i32),
+               "token_batch": torch.empty(T, **i32), "token_pos": torch.empty(T, **i32),
+               "slot_mapping": torch.empty(T, **i32)}
+    if status is None:
+        status = new_status(dev)
+    out["status"] = status
+    rc = lib().spa_prepare_append_kv(
+        _ptr(cu_seqlens_q), _ptr(past_seqlens), _ptr(block_table), B, T, max_seqlen_q,
+        max_seqlen_k, MB, bs, NB, _ptr(out["seqlens_q"]), _ptr(out["seqlen_k"]),
+        _ptr(out["token_batch"]), _ptr(out["token_pos"]), _ptr(out["slot_mapping"]),
+        _ptr(k_new), _ptr(v_new), _DT[k_new.dtype], _ptr(k_cache), _ptr(v_cache),
+        _DT[k_cache.dtype], _ptr(k_scale), _ptr(v_scale), H_kv, D, _ptr(status), _stream(dev))
+    _check(rc, "spa_prepare_append_kv")
+    out["cu_seqlens_q"] = cu_seqlens_q
+    return out
+
+
 def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                    block_table: torch.Tensor, meta: Dict[str, torch.Tensor], *,
                    max_seqlen_q: int, max_seqlen_k: int, out: torch.Tensor,
@@ -193,6 +227,11 @@ def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     a.num_splits = num_splits
     a.status = _ptr(status if status is not None else meta.get("status"))
     return a
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled workspace (its split tickets must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def workspace_size(args: AttentionArgs) -> int:
@@ -231,7 +270,7 @@ def attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                        max_seqlen_k=max_seqlen_k, out=out, lse=lse, **kw)
     need = workspace_size(a)
     if need and (workspace is None or workspace.numel() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = new_workspace(need, q.device)
     rc = lib().spa_attention(ctypes.byref(a), _ptr(workspace) if need else None, need,
                              _stream(q.device))
     _check(rc, "spa_attention")

@@ -13,7 +13,7 @@ from tests.gpu_util import compare, oracle_step
 pytestmark = pytest.mark.gpu
 
 
-def run(wl, **kw):
+def run(wl, **kw):  # noqa: D103
     return pipeline.run_step(wl, **kw)
 
 
@@ -170,3 +170,62 @@ def test_status_accumulates_and_is_not_cleared():
     st()
     torch.cuda.synchronize()
     assert int(st.status.item()) == 0x50
+
+
+# ---------------------------------------------------------------------------
+# fused prepare + append against the staged entry points; workspace reuse
+# ---------------------------------------------------------------------------
+
+def _all_equal(a, b):
+    for k in ("seqlens_q", "seqlen_k", "token_batch", "token_pos", "slot_mapping"):
+        assert np.array_equal(a[k], b[k]), k
+    assert a["status"] == b["status"]
+    for k in ("k_cache", "v_cache"):
+        assert torch.equal(a[k].view(torch.uint8) if a[k].element_size() == 1 else
+                           a[k].view(torch.int16) if a[k].element_size() == 2 else
+                           a[k].view(torch.int32),
+                           b[k].view(torch.uint8) if b[k].element_size() == 1 else
+                           b[k].view(torch.int16) if b[k].element_size() == 2 else
+                           b[k].view(torch.int32)), k
+
+
+@pytest.mark.parametrize("name", W.WORKLOADS)
+def test_fused_prepare_append_matches_staged(name):
+    wl = W.by_name(name, small=True)
+    a = run(wl, fused=True)
+    b = run(wl, fused=False)
+    _all_equal(a, b)
+    assert np.array_equal(a["out"], b["out"])
+
+
+@pytest.mark.parametrize("which", ["decreasing_cu", "bad_block", "capacity"])
+def test_fused_prepare_append_malformed(which):
+    wl = W.make_workload(act="f16", cache="i8", B=3, H_q=8, H_kv=2, D=64, block_size=16,
+                         q_lens=[2, 1, 3], past=[20, 5, 40], window=8, spare_blocks=2, seed=19)
+    a_ = wl.arrays
+    if which == "decreasing_cu":
+        a_["cu_seqlens_q"][2] = 1
+    elif which == "bad_block":
+        a_["block_table"][2, 2] = wl.NB + 3
+    else:
+        a_["past_seqlens"][0] = wl.MB * wl.block_size - 1
+    _all_equal(run(wl, fused=True), run(wl, fused=False))
+
+
+@pytest.mark.parametrize("name", ["selected_decode_bf16", "local_plus_selected_int8"])
+def test_workspace_reuse_across_calls(name):
+    """Split tickets are left at zero, so the same workspace serves call after call."""
+    wl = W.by_name(name, small=True)
+    d = pipeline.to_device(wl)
+    st = pipeline.Step(wl, d, num_splits=3, want_lse=True)
+    outs = []
+    for _ in range(3):
+        st()
+        torch.cuda.synchronize()
+        outs.append(st.out.clone())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    ref = oracle_step(wl)
+    got = {k: v.cpu().numpy() for k, v in st.meta.items()}
+    got.update(status=int(st.status.item()), out=outs[-1].float().cpu().numpy().astype(np.float64),
+               k_cache=d["k_cache"].cpu(), v_cache=d["v_cache"].cpu())
+    compare(wl, got, ref)
