@@ -56,6 +56,7 @@ typedef enum {
 #define SPA_ERR_UNSUPPORTED (-2) /* non-causal, main selection combined with window/aux, unsupported D */
 #define SPA_ERR_WORKSPACE (-3)   /* workspace missing, too small or misaligned */
 #define SPA_ERR_CUDA (-4)        /* a kernel launch failed; see spa_error_string(SPA_ERR_CUDA) */
+#define SPA_ERR_SCRATCH_LIMIT (-5) /* spa_attention_noalloc: the call needs more than SPA_NOALLOC_SCRATCH_BYTES */
 
 /* Device status bits (OR-ed into *status). */
 #define SPA_ST_BAD_CU 0x1     /* cu_seqlens_q not non-decreasing from 0 to T, or a negative past length */
@@ -229,6 +230,32 @@ size_t spa_attention_workspace_size(const spa_attention_args_t* a);
  */
 int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
                   spa_stream_t stream);
+
+/*
+ * spa_attention_noalloc -- spa_attention for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this entry point exists for
+ * callers of this library that cannot provide a workspace -- code running
+ * inside a CUDA graph capture (where cudaMalloc is not allowed), plugins whose
+ * host runtime owns all device memory, tools that must keep the process's
+ * device footprint fixed.  It computes exactly what spa_attention computes
+ * (same kernels, same arguments) but takes its scratch from an array built
+ * into the library: SPA_NOALLOC_SCRATCH_BYTES on every GPU that loads the
+ * library, held until the process exits.  It calls no cudaMalloc / cudaFree
+ * and no allocating routine.
+ *   - A call whose plan needs more scratch than SPA_NOALLOC_SCRATCH_BYTES
+ *     (spa_attention_workspace_size() of the same arguments) returns
+ *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.
+ *   - The first call on each device resolves the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *     If the address cannot be resolved the call returns SPA_ERR_CUDA.
+ *   - Every call on a device shares the array and sees what the previous call
+ *     left in it; the values that must start at zero are cleared on `stream`
+ *     before the kernel runs (one memset).  Calls that may overlap on the GPU
+ *     (different streams, different host threads) race on the array and must
+ *     be ordered by the caller.
+ */
+#define SPA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int spa_attention_noalloc(const spa_attention_args_t* a, spa_stream_t stream);
 
 /*
  * spa_attention_plan -- host-only introspection of what spa_attention would

@@ -327,6 +327,9 @@ const char* spa_error_string(int code) {
     case SPA_ERR_UNSUPPORTED: return "unsupported combination of arguments";
     case SPA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
     case SPA_ERR_CUDA: return g_cuda_msg;
+    case SPA_ERR_SCRATCH_LIMIT:
+      return "the call needs more scratch than the library's static array (SPA_NOALLOC_SCRATCH_BYTES); "
+             "use spa_attention with a caller workspace";
     default: return "unknown error code";
   }
 }
