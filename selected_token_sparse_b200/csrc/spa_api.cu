@@ -114,8 +114,9 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   if (a->num_splits > 0) {
     splits = a->num_splits;
   } else {
-    const long long target = 2LL * 148;
-    splits = (target + units - 1) / units;
+    // units that already fill the GPU run unsplit (no partials, no merge);
+    // otherwise split as far as one wave of two CTAs per SM allows
+    splits = units >= 148 ? 1 : (2LL * 148) / units;
     if (splits > tiles) splits = tiles;
     if (splits > 64) splits = 64;
     if (splits < 1) splits = 1;

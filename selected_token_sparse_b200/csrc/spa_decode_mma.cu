@@ -31,6 +31,8 @@ namespace spa {
 
 constexpr int kMmaKT = 64;      // keys per tile
 constexpr int kMmaStages = 3;   // cp.async ring depth
+constexpr int kMmaCandTiles = 8;                     // tiles whose candidates are resolved at once
+constexpr int kMmaCandChunk = kMmaCandTiles * 64;    // = kMmaCandTiles * kMmaKT
 
 int mma_key_tile() { return kMmaKT; }
 
@@ -102,7 +104,8 @@ struct MmaCfg {
   static constexpr int OFF_KPOS = OFF_CONV + (kInt8 ? 2 * TILE16 : 0);
   static constexpr int OFF_SCALE = OFF_KPOS + kMmaStages * kMmaKT * 4;
   static constexpr int OFF_PROW = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
-  static constexpr int END = OFF_PROW + 128 * 4;
+  static constexpr int OFF_CAND = OFF_PROW + 128 * 4;                  // resolved candidates
+  static constexpr int END = OFF_CAND + kMmaCandChunk * (8 + 4);
   // the cross-warp merge reuses the K/V ring once every tile is consumed
   static constexpr int OFF_RED = OFF_RAW;
   static constexpr int RED_BYTES = (KW > 1) ? NW * 32 * (D / 2 + 4) * 4 : 0;
@@ -190,19 +193,34 @@ decode_mma_kernel(const AttnParams p) {
   int bits = 0;
 
   // Issue the copies of tile `it` into its ring stage.  Thread `tid` copies
-  // chunk (tid % RAW_CPR) of rows tid / RAW_CPR, + NT / RAW_CPR, ...; it resolves
-  // those rows' candidates itself.
+  // chunk (tid % RAW_CPR) of rows tid / RAW_CPR, + NT / RAW_CPR, ...
+  // Candidates are resolved (selection slot / window position -> block table
+  // -> row offset, with every guard) a chunk of tiles at a time by all threads
+  // at once, so the index loads of many rows are in flight together and the
+  // copy loop below reads ready offsets.
+  long long* cand_off = reinterpret_cast<long long*>(smem + C::OFF_CAND);
+  int* cand_kpos = reinterpret_cast<int*>(smem + C::OFF_CAND + kMmaCandChunk * 8);
+  auto resolve_chunk = [&](int first_tile) {
+    for (int i = tid; i < kMmaCandChunk; i += NT) {
+      const int cand = c_begin + first_tile * KT + i;
+      int kp = kPosInvalid;
+      bool from_aux = false;
+      long long off = -1;
+      if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      cand_off[i] = off;
+      cand_kpos[i] = kp;
+    }
+  };
   auto issue = [&](int it) {
     const int stage = it % kMmaStages;
     unsigned char* kraw = smem + C::OFF_RAW + stage * 2 * C::RAW_TILE;
     unsigned char* vraw = kraw + C::RAW_TILE;
     const int c = tid % RAW_CPR;
     for (int row = tid / RAW_CPR; row < KT; row += NT / RAW_CPR) {
-      const int cand = c_begin + it * KT + row;
-      int kp = kPosInvalid;
-      bool from_aux = false;
-      long long off = -1;
-      if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      const int ci = (it % kMmaCandTiles) * KT + row;
+      const int kp = cand_kpos[ci];
+      const long long off = cand_off[ci];
+      const bool from_aux = kp == kPosAux;
       const bool ok = off >= 0;
       const CacheT* kb = from_aux ? ak : kc;
       const CacheT* vb = from_aux ? av : vc;
@@ -223,6 +241,8 @@ decode_mma_kernel(const AttnParams p) {
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   uint32_t qf[C::kInt8 ? 1 : D / 16][4];
 
+  if (ntiles > 0) resolve_chunk(0);
+  __syncthreads();
 #pragma unroll
   for (int s = 0; s < kMmaStages - 1; ++s) {
     if (s < ntiles) issue(s);
@@ -245,7 +265,13 @@ decode_mma_kernel(const AttnParams p) {
   const float sl2 = p.scale_log2;
 
   for (int it = 0; it < ntiles; ++it) {
-    if (it + kMmaStages - 1 < ntiles) issue(it + kMmaStages - 1);
+    const int nxt = it + kMmaStages - 1;
+    if (nxt < ntiles && nxt % kMmaCandTiles == 0) {
+      // every thread is past the copies that read the previous chunk
+      resolve_chunk(nxt);
+      __syncthreads();
+    }
+    if (nxt < ntiles) issue(nxt);
     cp_async_commit();
     cp_async_wait<kMmaStages - 1>();
     __syncthreads();
