@@ -2,24 +2,30 @@
 // fifth-generation tensor cores (tcgen05, TMEM accumulators, TMA).
 //
 // The dense QK^T and PV tiles of a causal (optionally windowed) prefill are
-// real contractions, so they run as 128x128xD tcgen05.mma tiles:
+// real contractions, so they run as 128x128xD tcgen05.mma tiles, and the
+// kernel is organised so that the tensor core and the softmax overlap:
 //
-//   CTA  = one q head x one 128-row q tile of one request; launched longest
-//          tiles first (q tiles in reverse order) so the ragged tail balances.
-//   TMA  = Q tile (3-D map over [T, H_q, D]) once; per 128-key step a K and a V
-//          tile gathered from the paged cache with a 4-D map over
-//          [num_blocks, block_size, H_kv, D] whose block coordinate comes from
-//          the block table (one box per cache block; an unmapped block is
-//          loaded from an out-of-range coordinate, i.e. zeros, and masked).
-//          128-byte swizzle, no multicast.
-//   MMA  = one elected thread: S = Q K^T (SS form, fp32 in TMEM columns
-//          [0,128)), then O += P V (TS form: P read from TMEM, V MN-major).
-//   softmax = 128 threads, thread i owns row i (TMEM lane i): masks the
-//          causal / window / unmapped keys, keeps a running max in log2
-//          units that is only raised (and O, l rescaled) when a tile's max
-//          exceeds it by more than 8, so P <= 2^8 fits fp16 / bf16 and most
-//          tiles skip the O rescale; P overwrites S in TMEM as packed pairs.
-//   sink = folded into the final normalisation (denominator only).
+//   CTA    = one q head x one request x a PAIR of 128-row q tiles (A, B);
+//            launched longest pairs first (q tiles in reverse order).
+//   TMEM   = S_A | S_B | O_A | O_B (4 x 128 columns); P of a tile overwrites
+//            its S as packed 16-bit pairs and feeds the PV MMA from TMEM.
+//   warp 8 = TMA producer and MMA issuer (one elected thread): Q_A, Q_B once;
+//            K and V tiles through a 2-stage ring from the paged cache (4-D
+//            tensor map over [num_blocks, block_size, H_kv, D]; the block id is
+//            a coordinate taken from the block table; an unmapped block is read
+//            from an out-of-range coordinate, i.e. zeros, and masked; 128-byte
+//            swizzle; no multicast).  Per 128-key step j it issues
+//              S_A = Q_A K_j^T, S_B = Q_B K_j^T, then O_A += P_A V_j and
+//              O_B += P_B V_j as each softmax group hands over its P,
+//            so S_B and PV_A run on the tensor core while the other group's
+//            softmax runs on the CUDA cores.
+//   warps 0-3 / 4-7 = softmax of tile A / B: thread i owns row i (TMEM lane i);
+//            masks only the tiles that cross the causal diagonal, the window
+//            edge, the end of the keys or an unmapped block; keeps a running
+//            max in log2 units that is raised (O rescaled in TMEM) only when a
+//            tile's max exceeds it by more than 8, so P <= 2^8; the scale is
+//            folded into one FFMA ahead of ex2.approx.
+//   sink   = folded into the final normalisation (denominator only).
 //
 // The key loop starts at the earliest window tile, rounded down to the tile
 // size, and keeps per-row visibility checks ("[WebGPU] Add PagedAttention
@@ -28,7 +34,8 @@
 // (joint FP32 stable softmax with optional sink).
 //
 // Every mbarrier wait is bounded; on expiry the kernel sets SPA_ST_TIMEOUT,
-// drains what it issued (again bounded), frees its TMEM and returns.
+// the other roles give up at their next wait, the issuing thread drains its
+// copies and MMAs (bounded), the CTA frees its TMEM and returns.
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -40,31 +47,39 @@ namespace spa {
 
 using namespace sm100;
 
-constexpr int kPfBM = 128;   // q rows per CTA (TMEM lanes)
+constexpr int kPfBM = 128;   // q rows per tile (TMEM lanes)
 constexpr int kPfBN = 128;   // keys per step
-constexpr uint32_t kPfTmemCols = 256;
+constexpr uint32_t kPfTmemCols = 512;
 constexpr uint32_t kPfWaitLimit = 1u << 20;   // polls before a wait is declared lost
+constexpr int kPfThreads = 9 * 32;            // 2 softmax groups + the TMA / MMA warp
 
 template <int D>
 struct PfCfg {
   static constexpr int NCH = D / 64;                  // 128-byte chunks along D
   static constexpr int CHUNK = 128 * 128;             // one chunk of a 128-row tile (bytes)
-  static constexpr int TILE = NCH * CHUNK;            // Q, K or V tile
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE;
-  static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_BAR = OFF_V + TILE;        // 5 mbarriers
-  static constexpr int OFF_TMEM = OFF_BAR + 64;       // TMEM base address holder
-  static constexpr int OFF_MASK = OFF_TMEM + 16;      // box validity per tile (2 slots)
-  static constexpr int OFF_FLAG = OFF_MASK + 16;      // abort flag
-  static constexpr int BYTES = OFF_FLAG + 16;
-  // + alignment slack; at least 80 KB so that no more than two CTAs (2 x 256
-  // TMEM columns) are ever resident on one SM
-  static constexpr int SMEM = (BYTES + 1024 > 80 * 1024) ? BYTES + 1024 : 80 * 1024;
+  static constexpr int TILE = NCH * CHUNK;            // one Q, K or V tile
+  static constexpr int OFF_QA = 0;
+  static constexpr int OFF_QB = OFF_QA + TILE;
+  static constexpr int OFF_K = OFF_QB + TILE;         // 2 stages
+  static constexpr int OFF_V = OFF_K + 2 * TILE;      // 2 stages
+  static constexpr int OFF_BAR = OFF_V + 2 * TILE;    // mbarriers
+  static constexpr int NBAR = 11;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_FLAG = OFF_TMEM + 8;
+  static constexpr int BYTES = OFF_FLAG + 8;
+  // + alignment slack; above half of the SM's shared memory so that exactly
+  // one CTA (holding all 512 TMEM columns) is resident per SM
+  static constexpr int SMEM = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
   static constexpr uint32_t TX_TILE = (uint32_t)TILE;
 };
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <typename T>
 __device__ __forceinline__ uint32_t pack_pair(float lo, float hi);
@@ -80,7 +95,8 @@ __device__ __forceinline__ uint32_t pack_pair<__nv_bfloat16>(float lo, float hi)
 }
 
 struct PfGeom {
-  int b, h, h_kv, t_begin, q0, rows, past, L, k_lo, k_hi, ntiles;
+  int b, h, h_kv, t_begin, q_len, past, L, k_lo, k_hi, ntiles;
+  int q0[2], rows[2];   // per q tile: first row within the request, rows present (0 = absent)
 };
 
 // Block id of the cache block holding key `key` (or -1), with status bits for
@@ -99,32 +115,27 @@ __device__ __forceinline__ int pf_block(const AttnParams& p, int b, int key, boo
   return blk;
 }
 
-// Issue the TMA loads of one K or V tile (keys [kb, kb + 128)); returns the
-// validity mask of its boxes (bit i: box i maps to a cache block).
-__device__ __forceinline__ uint32_t pf_issue_kv(const AttnParams& p, const PfGeom& g,
-                                                const CUtensorMap* map, unsigned char* dst,
-                                                uint64_t* bar, int kb, int box_rows, int nch,
-                                                int& bits, uint32_t tx) {
+// TMA loads of one K or V tile (keys [kb, kb + 128)) into `dst`.
+__device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g, const CUtensorMap* map,
+                                            unsigned char* dst, uint64_t* bar, int kb, int box_rows,
+                                            int nch, int& bits, uint32_t tx) {
   mbar_arrive_expect_tx(bar, tx);
-  uint32_t mask = 0;
   const int nbox = kPfBN / box_rows;
   for (int i = 0; i < nbox; ++i) {
     const int key0 = kb + i * box_rows;
     const int blk = pf_block(p, g.b, key0, key0 < g.k_hi, bits);
-    if (blk >= 0) mask |= 1u << i;
     const int cblk = blk >= 0 ? blk : p.NB;  // out of range: the box reads zeros
     const int row = key0 % p.bs;
     for (int c = 0; c < nch; ++c)
       tma_load_4d(dst + c * (128 * 128) + i * box_rows * 128, map, bar, c * 64, g.h_kv, row, cblk);
   }
-  return mask;
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                       int n_qt, int box_rows, int max_tiles) {
+                       int n_pairs, int box_rows, int box_shift, int max_tiles) {
   using C = PfCfg<D>;
   constexpr uint32_t FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = idesc_f16(FMT, kPfBM, kPfBN, 0);
@@ -132,52 +143,61 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
   pdl_trigger();
 
   // ---- geometry (uniform across the CTA)
   PfGeom g;
   g.h = blockIdx.x;
-  g.b = blockIdx.z;
-  const int qt = n_qt - 1 - (int)blockIdx.y;
+  g.b = blockIdx.y;
+  const int pair = n_pairs - 1 - (int)blockIdx.z;
   g.t_begin = clampi(p.cu[g.b], 0, p.T);
-  const int q_len = clampi(p.seqlens_q[g.b], 0, p.T - g.t_begin);
-  g.q0 = qt * kPfBM;
-  if (g.q0 >= q_len) return;
-  g.rows = min(kPfBM, q_len - g.q0);
+  g.q_len = clampi(p.seqlens_q[g.b], 0, p.T - g.t_begin);
+  g.q0[0] = pair * 2 * kPfBM;
+  g.q0[1] = g.q0[0] + kPfBM;
+  if (g.q0[0] >= g.q_len) return;
+  g.rows[0] = min(kPfBM, g.q_len - g.q0[0]);
+  g.rows[1] = max(0, min(kPfBM, g.q_len - g.q0[1]));
   g.L = max(p.seqlen_k[g.b] + 1, 0);
-  g.past = max(g.L - q_len, 0);
+  g.past = max(g.L - g.q_len, 0);
   g.h_kv = g.h / p.G;
-  const int p_first = g.past + g.q0;
-  const int p_last = p_first + g.rows - 1;
+  const int last_row = g.rows[1] > 0 ? g.q0[1] + g.rows[1] - 1 : g.q0[0] + g.rows[0] - 1;
+  const int p_first = g.past + g.q0[0];
+  const int p_last = g.past + last_row;
   g.k_lo = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
   g.k_lo = (g.k_lo / kPfBN) * kPfBN;
   g.k_hi = min(p_last + 1, g.L);
   g.ntiles = g.k_hi > g.k_lo ? (g.k_hi - g.k_lo + kPfBN - 1) / kPfBN : 0;
   g.ntiles = min(g.ntiles, max_tiles);
+  const bool two = g.rows[1] > 0;   // the second q tile exists
+  const int ntq = two ? 2 : 1;
 
-  unsigned char* sQ = smem + C::OFF_Q;
+  unsigned char* const sQA = smem + C::OFF_QA;
+  unsigned char* const sQB = smem + C::OFF_QB;
   unsigned char* sK = smem + C::OFF_K;
   unsigned char* sV = smem + C::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_q = bars + 0;
-  uint64_t* bar_k = bars + 1;
-  uint64_t* bar_v = bars + 2;
-  uint64_t* bar_s = bars + 3;
-  uint64_t* bar_o = bars + 4;
+  uint64_t* bar_kf = bars + 1;    // [2] K stage full
+  uint64_t* bar_vf = bars + 3;    // [2] V stage full
+  uint64_t* bar_s = bars + 5;     // [2] S of tile A / B written
+  uint64_t* bar_o = bars + 7;     // [2] PV of tile A / B done
+  uint64_t* bar_p = bars + 9;     // [2] P of tile A / B in TMEM (4 warps arrive)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
-  volatile uint32_t* kmask = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MASK);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
 
-  int bits = 0;
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_kf + i, 1);
+      mbar_init(bar_vf + i, 1);
+      mbar_init(bar_s + i, 1);
+      mbar_init(bar_o + i, 1);
+      mbar_init(bar_p + i, 4);
+    }
     fence_mbar_init();
     *abort_flag = 0;
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
   }
   if (warp == 0) {
     tmem_alloc(tmem_holder, kPfTmemCols);
@@ -187,211 +207,252 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_S = tmem;         // S (fp32, 128 cols); P (packed, 64 cols) overlays it
-  const uint32_t tmem_O = tmem + 128;   // O (fp32, D cols)
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  int bits = 0;
 
-  // outstanding async work issued by thread 0 (for the drain on abort)
-  int pend_q = 0, pend_k = 0, pend_v = 0, pend_s = 0, pend_o = 0;
-  uint32_t ph_k = 0, ph_v = 0, ph_o = 0;
-
-  if (tid == 0 && g.ntiles > 0) {
-    mbar_arrive_expect_tx(bar_q, C::TX_TILE);
-    for (int c = 0; c < C::NCH; ++c)
-      tma_load_3d(sQ + c * C::CHUNK, &tm_q, bar_q, c * 64, g.h, g.t_begin + g.q0);
-    pend_q = 1;
-    kmask[0] = pf_issue_kv(p, g, &tm_k, sK, bar_k, g.k_lo, box_rows, C::NCH, bits, C::TX_TILE);
-    pend_k = 1;
-    pf_issue_kv(p, g, &tm_v, sV, bar_v, g.k_lo, box_rows, C::NCH, bits, C::TX_TILE);
-    pend_v = 1;
-  }
-  __syncthreads();
-
-  // softmax state of row `tid`
-  const int prow = g.past + g.q0 + tid;
-  float m_used = -INFINITY;   // log2 units
-  float l_sum = 0.f;
-  const float sl2 = p.scale_log2;
-
-  for (int j = 0; j < g.ntiles; ++j) {
-    const int kb = g.k_lo + j * kPfBN;
-    // ---- producer / MMA thread: V_j, then S_j = Q K_j^T
-    if (tid == 0) {
-      bool ok = true;
-      if (j > 0) {
-        ok = mbar_wait(bar_o, ph_o, kPfWaitLimit);   // PV_{j-1} done: V buffer and P free
-        if (ok) {
-          ph_o ^= 1;
-          pend_o = 0;
-          pf_issue_kv(p, g, &tm_v, sV, bar_v, kb, box_rows, C::NCH, bits, C::TX_TILE);
-          pend_v = 1;
-        }
+  if (warp == 8) {
+    // =================== TMA producer and MMA issuer (one thread) ===================
+    if (lane == 0 && g.ntiles > 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(bar_q, ntq * C::TX_TILE);
+      for (int c = 0; c < C::NCH; ++c) {
+        tma_load_3d(sQA + c * C::CHUNK, &tm_q, bar_q, c * 64, g.h, g.t_begin + g.q0[0]);
+        if (two) tma_load_3d(sQB + c * C::CHUNK, &tm_q, bar_q, c * 64, g.h, g.t_begin + g.q0[1]);
       }
-      if (ok && j == 0) {
-        ok = mbar_wait(bar_q, 0, kPfWaitLimit);
-        if (ok) pend_q = 0;
+      int n_kv = 0;   // K/V tiles whose loads were issued
+      for (int j = 0; j < 2 && j < g.ntiles; ++j, ++n_kv) {
+        pf_issue_kv(p, g, &tm_k, sK + j * C::TILE, bar_kf + j, g.k_lo + j * kPfBN, box_rows, C::NCH, bits,
+                    C::TX_TILE);
+        pf_issue_kv(p, g, &tm_v, sV + j * C::TILE, bar_vf + j, g.k_lo + j * kPfBN, box_rows, C::NCH, bits,
+                    C::TX_TILE);
       }
-      if (ok) ok = mbar_wait(bar_k, ph_k, kPfWaitLimit);
-      if (ok) {
-        ph_k ^= 1;
-        pend_k = 0;
-        tc_fence_after();
+      int n_s0 = 0, n_s1 = 0, n_o0 = 0, n_o1 = 0;   // commits issued per barrier
+      int kv_seen = 0;                        // K/V tiles whose arrival was observed
+      bool ok = mbar_wait(bar_q, 0, kPfWaitLimit, abort_flag);
+      const bool q_seen = ok;
+      for (int j = 0; j < g.ntiles && ok; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        ok = mbar_wait(bar_kf + st, ph, kPfWaitLimit, abort_flag);
+        for (int t = 0; t < ntq && ok; ++t) {
+          // S_t of step j overwrites P_t of step j-1: PV_t(j-1) must be done
+          if (j > 0) ok = mbar_wait(bar_o + t, (j - 1) & 1, kPfWaitLimit, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t tS = tmem + t * 128;
+          unsigned char* const sq = t ? sQB : sQA;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int c = kk / 4, koff = (kk % 4) * 32;
-          const uint64_t ad = smem_desc_sw128(smem_u32(sQ + c * C::CHUNK + koff), 16, 1024);
-          const uint64_t bd = smem_desc_sw128(smem_u32(sK + c * C::CHUNK + koff), 16, 1024);
-          mma_ss(tmem_S, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int c = kk / 4, koff = (kk % 4) * 32;
+            const uint64_t ad = smem_desc_sw128(smem_u32(sq + c * C::CHUNK + koff), 16, 1024);
+            const uint64_t bd = smem_desc_sw128(smem_u32(sK + st * C::TILE + c * C::CHUNK + koff), 16, 1024);
+            mma_ss(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar_s + t);
+          if (t) ++n_s1; else ++n_s0;
         }
-        tc_commit(bar_s);
-        pend_s = 1;
-      } else {
+        if (!ok) break;
+        // every MMA of step j-1 is complete here (PV of each tile of step j-1
+        // was waited on above), so step j+1's K and V may take that stage
+        if (j >= 1 && j + 1 < g.ntiles) {
+          const int s2 = (j + 1) & 1;
+          pf_issue_kv(p, g, &tm_k, sK + s2 * C::TILE, bar_kf + s2, g.k_lo + (j + 1) * kPfBN, box_rows, C::NCH,
+                      bits, C::TX_TILE);
+          pf_issue_kv(p, g, &tm_v, sV + s2 * C::TILE, bar_vf + s2, g.k_lo + (j + 1) * kPfBN, box_rows, C::NCH,
+                      bits, C::TX_TILE);
+          ++n_kv;
+        }
+        ok = mbar_wait(bar_vf + st, ph, kPfWaitLimit, abort_flag);
+        if (ok) kv_seen = j + 1;
+        for (int t = 0; t < ntq && ok; ++t) {
+          ok = mbar_wait(bar_p + t, j & 1, kPfWaitLimit, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t tP = tmem + t * 128;
+          const uint32_t tO = tmem + 256 + t * 128;
+#pragma unroll
+          for (int kk = 0; kk < kPfBN / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(smem_u32(sV + st * C::TILE + kk * 2048), C::CHUNK, 1024);
+            mma_ts(tO, tP + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar_o + t);
+          if (t) ++n_o1; else ++n_o0;
+        }
+      }
+      if (!ok) {
         *abort_flag = 1;
+        bits |= SPA_ST_TIMEOUT;
+        // drain, bounded: the latest commit of each barrier covers every MMA
+        // issued before it; then the copies whose arrival was not observed
+        if (n_s0 > 0) mbar_wait(bar_s + 0, (n_s0 - 1) & 1, kPfWaitLimit);
+        if (n_s1 > 0) mbar_wait(bar_s + 1, (n_s1 - 1) & 1, kPfWaitLimit);
+        if (n_o0 > 0) mbar_wait(bar_o + 0, (n_o0 - 1) & 1, kPfWaitLimit);
+        if (n_o1 > 0) mbar_wait(bar_o + 1, (n_o1 - 1) & 1, kPfWaitLimit);
+        if (!q_seen) mbar_wait(bar_q, 0, kPfWaitLimit);
+        for (int j = kv_seen; j < n_kv; ++j) {
+          mbar_wait(bar_kf + (j & 1), (j >> 1) & 1, kPfWaitLimit);
+          mbar_wait(bar_vf + (j & 1), (j >> 1) & 1, kPfWaitLimit);
+        }
       }
     }
-    // ---- everyone: wait for S_j (the decision to go on is CTA-uniform)
-    const bool got_s = mbar_wait(bar_s, j & 1, kPfWaitLimit, abort_flag);
-    if (__syncthreads_or(!got_s || *abort_flag)) {
-      if (tid == 0) *abort_flag = 1;
-      break;
-    }
-    if (tid == 0) {
-      pend_s = 0;
-      // K buffer is free: prefetch K_{j+1}
-      if (j + 1 < g.ntiles) {
-        kmask[(j + 1) & 1] = pf_issue_kv(p, g, &tm_k, sK, bar_k, kb + kPfBN, box_rows, C::NCH, bits,
-                                         C::TX_TILE);
-        pend_k = 1;
+  } else {
+    // =================== softmax group t (warps 4t .. 4t+3) ===================
+    const int t = warp >> 2;
+    const int r = tid & 127;                      // row within the q tile (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tS = tmem + t * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + t * 128 + lane_off;
+    const int q0_t = t ? g.q0[1] : g.q0[0];
+    const int rows_t = t ? g.rows[1] : g.rows[0];
+    const bool active = rows_t > 0;
+    const int prow = g.past + q0_t + r;
+    const int p_lo = g.past + q0_t;                         // first row of this tile
+    const int p_hi = g.past + q0_t + max(rows_t, 1) - 1;
+    float m_used = -INFINITY;   // log2 units
+    float l_sum = 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < g.ntiles && active; ++j) {
+      ok = mbar_wait(bar_s + t, j & 1, kPfWaitLimit, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
       }
-    }
-    tc_fence_after();
-    {
-      const uint32_t vmask = kmask[j & 1];
-      uint32_t s[kPfBN];
-#pragma unroll
-      for (int c = 0; c < kPfBN / 32; ++c) tmem_ld32(tmem_S + lane_off + c * 32, s + c * 32);
-      tmem_wait_ld();
+      tc_fence_after();
+      const int kb = g.k_lo + j * kPfBN;
+      // which cache blocks of this tile are mapped (bit i: box i), and does any
+      // key of the tile need a mask for any row of this q tile?
+      const int nbox = kPfBN >> box_shift;   // <= 8 (block_size >= 16)
+      uint32_t boxmask = 0;
+      for (int i = 0; i < nbox; ++i) {
+        const int key0 = kb + (i << box_shift);
+        const int lb = key0 / p.bs;
+        const int blk = lb < p.MB ? p.block_table[(long long)g.b * p.MB + lb] : -1;
+        if (blk >= 0 && blk < p.NB) boxmask |= 1u << i;
+      }
+      const bool all_mapped = boxmask == (1u << nbox) - 1u;
+      const bool full = all_mapped && kb + kPfBN - 1 <= p_lo && kb + kPfBN <= g.k_hi &&
+                        (p.window <= 0 || kb > p_hi - p.window);
+      // visibility of key column c (only consulted on tiles that need a mask):
+      // the row's causal / window / end-of-keys limits as a column interval
+      // [c_lo, c_hi), and the mapped-block bitmask
+      const int c_hi = min(min(prow + 1, g.k_hi) - kb, kPfBN);
+      const int c_lo = p.window > 0 ? max(prow - p.window + 1 - kb, 0) : 0;
+      auto visible = [&](int c) {
+        return c >= c_lo && c < c_hi && ((boxmask >> (c >> box_shift)) & 1u);
+      };
+      // pass 1: row max over 32-column chunks of S (keeps few registers live);
+      // on tiles that need a mask, hidden keys are written back as -inf so
+      // that pass 2 is the same for every tile
       float mx = -INFINITY;
+#pragma unroll 1
+      for (int c4 = 0; c4 < kPfBN / 32; ++c4) {
+        uint32_t v[32];
+        tmem_ld32(tS + c4 * 32, v);
+        tmem_wait_ld();
+        if (!full) {
 #pragma unroll
-      for (int c = 0; c < kPfBN; ++c) {
-        const int key = kb + c;
-        const bool vis = key < g.k_hi && key <= prow && (p.window <= 0 || key > prow - p.window) &&
-                         ((vmask >> (c / box_rows)) & 1u);
-        const float v = vis ? u2f(s[c]) * sl2 : -INFINITY;
-        s[c] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+          for (int e = 0; e < 32; ++e)
+            if (!visible(c4 * 32 + e)) v[e] = __float_as_uint(-INFINITY);
+          tmem_st32(tS + c4 * 32, v);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, u2f(v[e]));
       }
+      if (!full) tmem_wait_st();
+      mx *= sl2;   // scores in log2 units (scale > 0)
       // lazy rescale: raise the reference max only when it grows by > 8 (x256).
       // The TMEM loads / stores of O are warp-collective, so the whole warp
       // takes the branch when any of its rows needs it (alpha = 1 otherwise).
       const bool need = mx > m_used + 8.0f;
       const float m_new = need ? mx : m_used;
-      const float alpha = need ? ((m_used == -INFINITY) ? 0.f : exp2f(m_used - m_new)) : 1.f;
+      const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2(m_used - m_new)) : 1.f;
       if (j > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
         uint32_t o[32];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          tmem_ld32(tmem_O + lane_off + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(u2f(o[e]) * alpha);
-          tmem_st32(tmem_O + lane_off + c * 32, o);
+          tmem_st32(tO + c * 32, o);
         }
       }
       l_sum *= alpha;
       m_used = m_new;
-      uint32_t pk[kPfBN / 2];
+      const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+      // pass 2: P = 2^(s*scale - m) for 64 keys at a time, packed in pairs into
+      // the TMEM columns that held those keys' scores (already read)
       float ls = 0.f;
 #pragma unroll
-      for (int c = 0; c < kPfBN; c += 2) {
-        const float a = u2f(s[c]), bb = u2f(s[c + 1]);
-        const float pa = (a == -INFINITY) ? 0.f : exp2f(a - m_used);
-        const float pb = (bb == -INFINITY) ? 0.f : exp2f(bb - m_used);
-        ls += pa + pb;
-        pk[c / 2] = pack_pair<T>(pa, pb);
+      for (int hh = 0; hh < kPfBN / 64; ++hh) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          const int c0 = hh * 64 + half * 32;
+          tmem_ld32(tS + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float pa = ex2(fmaf(u2f(v[e]), sl2, nm));   // -inf -> 0
+            const float pb = ex2(fmaf(u2f(v[e + 1]), sl2, nm));
+            ls += pa + pb;
+            pk[half * 16 + e / 2] = pack_pair<T>(pa, pb);
+          }
+        }
+        tmem_st32(tS + hh * 32, pk);
       }
       l_sum += ls;
-#pragma unroll
-      for (int c = 0; c < kPfBN / 64; ++c) tmem_st32(tmem_S + lane_off + c * 32, pk + c * 32);
       tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p + t);
     }
-    tc_fence_before();
-    __syncthreads();
-    // ---- MMA thread: O += P V_j
-    if (tid == 0) {
+    // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
+    bool have_o = active && ok && g.ntiles > 0;
+    if (have_o) have_o = mbar_wait(bar_o + t, (g.ntiles - 1) & 1, kPfWaitLimit, abort_flag);
+    have_o = __all_sync(0xffffffffu, have_o);
+    if (active && !(*abort_flag) && (have_o || g.ntiles == 0)) {
       tc_fence_after();
-      if (mbar_wait(bar_v, ph_v, kPfWaitLimit)) {
-        ph_v ^= 1;
-        pend_v = 0;
+      const bool mine = r < rows_t;
+      const int tok = g.t_begin + q0_t + r;
+      const long long orow = (long long)tok * p.H_q + g.h;
+      const float sink2 = p.sinks ? p.sinks[g.h] * kLog2e : -INFINITY;
+      float a, inv_l, lse;
+      finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
+      const float f = a * inv_l;
+      T* out = static_cast<T*>(p.out) + orow * D;
 #pragma unroll
-        for (int kk = 0; kk < kPfBN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(smem_u32(sV + kk * 2048), C::CHUNK, 1024);
-          mma_ts(tmem_O, tmem_S + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (have_o) {   // warp-uniform: every lane takes part in the warp-wide load
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        tc_commit(bar_o);
-        pend_o = 1;
-      } else {
-        *abort_flag = 1;
-      }
-    }
-    __syncthreads();
-    if (*abort_flag) break;
-  }
-
-  // ---- epilogue: wait for the last PV, normalise with the sink, store
-  __syncthreads();
-  bool have_o = g.ntiles > 0 && !*abort_flag;
-  if (have_o) {
-    const bool got = mbar_wait(bar_o, (g.ntiles - 1) & 1, kPfWaitLimit, abort_flag);
-    if (__syncthreads_or(!got)) {
-      if (tid == 0) *abort_flag = 1;
-    } else if (tid == 0) {
-      pend_o = 0;
-    }
-  }
-  __syncthreads();
-  have_o = have_o && !*abort_flag;
-  if (*abort_flag) {
-    bits |= SPA_ST_TIMEOUT;
-    if (tid == 0) {   // drain whatever is still in flight, bounded
-      if (pend_q) mbar_wait(bar_q, 0, kPfWaitLimit);
-      if (pend_k) mbar_wait(bar_k, ph_k, kPfWaitLimit);
-      if (pend_v) mbar_wait(bar_v, ph_v, kPfWaitLimit);
-      if (pend_s || pend_o) mbar_wait(bar_o, ph_o, kPfWaitLimit);
-    }
-  } else {
-    const bool mine = tid < g.rows;
-    const int t = g.t_begin + g.q0 + tid;
-    const long long orow = (long long)t * p.H_q + g.h;
-    const float sink2 = p.sinks ? p.sinks[g.h] * kLog2e : -INFINITY;
-    float a, inv_l, lse;
-    finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
-    const float f = a * inv_l;
-    T* out = static_cast<T*>(p.out) + orow * D;
+        if (mine) {
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      if (have_o) {   // CTA-uniform: every thread takes part in the warp-wide load
-        tmem_ld32(tmem_O + lane_off + c * 32, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
-      }
-      if (mine) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 v;
-          v.x = pack_pair<T>(u2f(o[e + 0]) * f, u2f(o[e + 1]) * f);
-          v.y = pack_pair<T>(u2f(o[e + 2]) * f, u2f(o[e + 3]) * f);
-          v.z = pack_pair<T>(u2f(o[e + 4]) * f, u2f(o[e + 5]) * f);
-          v.w = pack_pair<T>(u2f(o[e + 6]) * f, u2f(o[e + 7]) * f);
-          *reinterpret_cast<uint4*>(out + c * 32 + e) = v;
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack_pair<T>(u2f(o[e + 0]) * f, u2f(o[e + 1]) * f);
+            v.y = pack_pair<T>(u2f(o[e + 2]) * f, u2f(o[e + 3]) * f);
+            v.z = pack_pair<T>(u2f(o[e + 4]) * f, u2f(o[e + 5]) * f);
+            v.w = pack_pair<T>(u2f(o[e + 6]) * f, u2f(o[e + 7]) * f);
+            *reinterpret_cast<uint4*>(out + c * 32 + e) = v;
+          }
         }
       }
+      if (mine && p.lse) p.lse[orow] = lse;
+    } else if (active) {
+      *abort_flag = 1;
     }
-    if (mine && p.lse) p.lse[orow] = lse;
   }
+  __syncthreads();
+  if (*abort_flag) bits |= SPA_ST_TIMEOUT;
   flag(p.status, bits);
   tc_fence_before();
   __syncthreads();
@@ -452,6 +513,8 @@ template <typename T, int D>
 static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t stream) {
   using C = PfCfg<D>;
   const int box_rows = p.bs < kPfBN ? p.bs : kPfBN;
+  int box_shift = 0;
+  while ((1 << box_shift) < box_rows) ++box_shift;
   CUtensorMap tq, tk, tv;
   const cuuint64_t qd[3] = {(cuuint64_t)D, (cuuint64_t)p.H_q, (cuuint64_t)p.T};
   const cuuint64_t qs[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.H_q * D * 2};
@@ -464,12 +527,15 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   if ((rc = encode(&tq, dt, 3, p.q, qd, qs, qb)) != SPA_OK) return rc;
   if ((rc = encode(&tk, dt, 4, p.k_cache, kd, ks, kbx)) != SPA_OK) return rc;
   if ((rc = encode(&tv, dt, 4, p.v_cache, kd, ks, kbx)) != SPA_OK) return rc;
-  const int n_qt = (p.max_q + kPfBM - 1) / kPfBM;
+  const int n_pairs = (p.max_q + 2 * kPfBM - 1) / (2 * kPfBM);
+  if (n_pairs > 65535) return SPA_ERR_UNSUPPORTED;
   const int max_tiles = (p.max_k + kPfBN - 1) / kPfBN + 1;
   auto kern = prefill_tcgen05_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  dim3 grid(p.H_q, n_qt, p.B);
-  return launch_pdl(kern, grid, dim3(128), C::SMEM, stream, p, tq, tk, tv, n_qt, box_rows, max_tiles);
+  // grid: heads fastest, then requests, then q-tile pairs from the last (longest) down
+  dim3 grid(p.H_q, p.B, n_pairs);
+  return launch_pdl(kern, grid, dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_pairs, box_rows,
+                    box_shift, max_tiles);
 }
 
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream) {
