@@ -289,7 +289,7 @@ def run_ours(args):
                             out=step0.out, num_splits=args.splits, **step0.kw)
     plan = spa.attention_plan(a0)
     launches_per_step = (1 if step0.fused else 2) + plan["launches"]
-    kind_name = {0: "decode_scalar", 1: "decode_mma", 2: "prefill_tcgen05"}[plan["kind"]]
+    kind_name = {0: "decode_scalar", 1: "decode_mma", 2: "prefill_tcgen05", 3: "decode_tc"}[plan["kind"]]
 
     stream = torch.cuda.Stream(dev)
     torch.cuda.synchronize(dev)

@@ -261,7 +261,7 @@ int spa_attention_noalloc(const spa_attention_args_t* a, spa_stream_t stream);
  * spa_attention_plan -- host-only introspection of what spa_attention would
  * launch for these arguments: the number of key splits per unit, the number
  * of kernel launches, and the kernel family (0 = CUDA-core decode,
- * 1 = tensor-core decode, 2 = tcgen05 prefill).  Any output pointer may be
+ * 1 = warp-MMA decode, 2 = tcgen05 prefill, 3 = tcgen05 multi-row decode).  Any output pointer may be
  * NULL.  Returns the same code spa_attention would return for the arguments
  * before launching anything.
  */

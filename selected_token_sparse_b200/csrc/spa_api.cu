@@ -26,6 +26,9 @@ size_t scalar_smem_bytes(int D, int max_rows, int nq);
 int launch_attention_mma(const AttnParams& p, int act, int cache, int max_rows, cudaStream_t stream);
 int mma_supported(int act, int cache, int D, int max_rows);
 int mma_key_tile();
+int tc_supported(int act, int cache, int D, int max_rows);
+int tc_key_tile();
+int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream);
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream);
 int prefill_supported(const spa_attention_args_t* a);
 
@@ -99,8 +102,11 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   pl->group_by_request = per_request_list && (long long)maxq * G <= 128;
   pl->max_q = pl->group_by_request ? maxq : 1;
   pl->max_rows = pl->max_q * G;
-  pl->kind = mma_supported(a->act, a->cache, a->D, pl->max_rows) ? kPlanMma : kPlanScalar;
-  const int KT = pl->kind == kPlanMma ? mma_key_tile() : scalar_key_tile();
+  if (tc_supported(a->act, a->cache, a->D, pl->max_rows)) pl->kind = kPlanTc;
+  else if (mma_supported(a->act, a->cache, a->D, pl->max_rows)) pl->kind = kPlanMma;
+  else pl->kind = kPlanScalar;
+  const int KT = pl->kind == kPlanTc ? tc_key_tile()
+                                     : (pl->kind == kPlanMma ? mma_key_tile() : scalar_key_tile());
   long long n_main;
   if (sel_main) n_main = a->sel_width;
   else if (a->window > 0) n_main = std::min<long long>((long long)a->window + pl->max_q - 1, a->max_seqlen_k);
@@ -115,8 +121,10 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
     splits = a->num_splits;
   } else {
     // units that already fill the GPU run unsplit (no partials, no merge);
-    // otherwise split as far as one wave of two CTAs per SM allows
-    splits = units >= 148 ? 1 : (2LL * 148) / units;
+    // otherwise split as far as one wave allows (two CTAs per SM, one for
+    // the tcgen05 kernel, which holds most of the shared memory)
+    const long long slots = pl->kind == kPlanTc ? 148 : 2LL * 148;
+    splits = units >= 148 ? 1 : slots / units;
     if (splits > tiles) splits = tiles;
     if (splits > 64) splits = 64;
     if (splits < 1) splits = 1;
@@ -197,7 +205,8 @@ int run_attention(const spa_attention_args_t* a, const Plan& pl, void* ws, cudaS
     if (rc != SPA_OK) return rc;
     return check_launch();
   }
-  if (pl.kind == kPlanMma) rc = launch_attention_mma(p, a->act, a->cache, pl.max_rows, stream);
+  if (pl.kind == kPlanTc) rc = launch_attention_tc(p, a->act, a->cache, stream);
+  else if (pl.kind == kPlanMma) rc = launch_attention_mma(p, a->act, a->cache, pl.max_rows, stream);
   else rc = launch_attention_scalar_impl(p, a->act, a->cache, pl.max_rows, stream);
   if (rc != SPA_OK) return rc;
   return check_launch();

@@ -1,0 +1,462 @@
+// Steps 3-5 for units with many query rows (multi-token decode: G q heads x
+// S_q tokens sharing one kv head's candidate list, up to 128 rows) on the
+// fifth-generation tensor cores.
+//
+// With tens of rows per kv head every gathered K/V row feeds a 96- or
+// 128-row contraction, so the unit is one M = 128 tcgen05 tile:
+//
+//   * the unit's rows (token i, head g) -> row i*G + g of a Q tile in shared
+//     memory, 128-byte-swizzled K-major; INT8 caches keep K exact (|k8| <= 128
+//     is exact in fp16) and fold the key scale into q, split into fp16 high
+//     and low tiles, so S = Q_hi K^T + Q_lo K^T carries ~22 bits;
+//   * candidates (window positions, selected or auxiliary slots) are resolved
+//     up front through the block table with every guard; rows are gathered
+//     with cp.async into a double-buffered staging area (the next 128-key
+//     tile streams in while this one is computed); INT8 rows are converted to
+//     fp16 integers into the swizzled K and V tiles (V is the MN-major B
+//     operand of PV, the same bytes), 16-bit rows are copied there as is;
+//   * S = Q K^T (tcgen05.mma into TMEM), 128 softmax threads (thread i owns
+//     row i) mask by key position (causal / window for the main cache,
+//     always visible for auxiliary entries), keep a lazily raised max in log2
+//     units, write P over S in TMEM, then O += P V (A from TMEM);
+//   * O is scaled by the value scale (INT8), then either normalised with the
+//     sink and written (one split) or written as a partial state merged by the
+//     CTA that takes the unit's last ticket.
+//
+// Sources: "[WebGPU] Add DynamicSparseAttention" (Attention: selected and
+// local-plus-auxiliary modes, joint FP32 stable softmax with optional sink),
+// "[WebGPU] Add SparsePagedAttention" (partial FP32 state, finalize merge),
+// onnxruntime PR #33472 (INT8 per-channel K/V scales; 12 q heads per kv head
+// with S <= 8 decode).
+#include <type_traits>
+
+#include "spa_attn.cuh"
+#include "spa_sm100.cuh"
+
+namespace spa {
+
+using namespace sm100;
+
+constexpr int kTcKT = 128;                      // keys per tile (MMA N)
+constexpr int kTcCandTiles = 4;                 // tiles whose candidates are resolved at once
+constexpr int kTcCand = kTcCandTiles * kTcKT;
+constexpr uint32_t kTcTmemCols = 256;           // S [0,128) | O [128, 128 + D)
+constexpr uint32_t kTcWaitLimit = 1u << 20;
+
+int tc_key_tile() { return kTcKT; }
+
+template <typename ActT, typename CacheT, int D>
+struct TcCfg {
+  static constexpr bool kInt8 = sizeof(CacheT) == 1;
+  using MT = typename std::conditional<kInt8, __half, ActT>::type;
+  static constexpr int NCH = D / 64;
+  static constexpr int TILE = NCH * 128 * 128;        // one 128-row 16-bit tile, swizzled
+  static constexpr int ROW_BYTES = D * (int)sizeof(CacheT);
+  static constexpr int RAW = kTcKT * ROW_BYTES;       // one staged K or V tile (INT8 only)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_QLO = OFF_Q + TILE;
+  static constexpr int OFF_KV = OFF_QLO + (kInt8 ? TILE : 0);
+  // 16-bit caches: 2 stages x (K, V) swizzled tiles; INT8: one (K, V) pair of
+  // converted tiles plus 2 stages x (K, V) raw staging
+  static constexpr int KV_BYTES = kInt8 ? 2 * TILE + 2 * 2 * RAW : 2 * 2 * TILE;
+  static constexpr int OFF_KPOS = OFF_KV + KV_BYTES;              // [2][128] key positions
+  static constexpr int OFF_CAND = OFF_KPOS + 2 * kTcKT * 4;      // candidate offsets + positions
+  static constexpr int OFF_SCALE = OFF_CAND + kTcCand * 12;      // INT8: ks, vs
+  static constexpr int OFF_BAR = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
+  static constexpr int OFF_MISC = OFF_BAR + 16;                  // tmem holder, flags
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM = BYTES + 1024;
+};
+
+// byte offset of 16-byte unit u (0 .. D/8-1) of row r in a 128-row swizzled tile
+__device__ __forceinline__ int sw_off(int r, int u) {
+  const int c = u >> 3, uu = u & 7;
+  return c * 16384 + (r >> 3) * 1024 + (r & 7) * 128 + ((uu ^ (r & 7)) << 4);
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pk_pair(float lo, float hi) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <typename ActT, typename CacheT, int D>
+__global__ void __launch_bounds__(128, 1)
+decode_tc_kernel(const AttnParams p) {
+  using C = TcCfg<ActT, CacheT, D>;
+  using MT = typename C::MT;
+  constexpr uint32_t FMT = std::is_same<MT, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t IDESC_S = idesc_f16(FMT, 128, kTcKT, 0);
+  constexpr uint32_t IDESC_O = idesc_f16(FMT, 128, D, 1);
+  constexpr int KT = kTcKT, NT = 128;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5;
+  __shared__ int last_flag;
+  pdl_wait();
+  pdl_trigger();
+
+  Unit U;
+  const bool has_rows = decode_unit(p, blockIdx.x, U);
+  if (p.group_by_request && !has_rows) return;
+  const int split = blockIdx.y;
+  const int G = p.G;
+  const int nq = p.group_by_request ? U.nq : 1;
+  const int R = nq * G;
+  const int t0 = has_rows ? U.t0 : blockIdx.x / p.H_kv;
+  const int h_kv = blockIdx.x % p.H_kv;
+  const int n_total = has_rows ? U.n_main + U.n_aux : 0;
+  const int c_begin = split * p.split_len;
+  const int c_end = min(c_begin + p.split_len, n_total);
+  const int ntiles = c_end > c_begin ? (c_end - c_begin + KT - 1) / KT : 0;
+
+  unsigned char* sQ = smem + C::OFF_Q;
+  unsigned char* sQlo = smem + C::OFF_QLO;
+  int* kpos_s = reinterpret_cast<int*>(smem + C::OFF_KPOS);
+  long long* cand_off = reinterpret_cast<long long*>(smem + C::OFF_CAND);
+  int* cand_kpos = reinterpret_cast<int*>(smem + C::OFF_CAND + kTcCand * 8);
+  float* ksc = reinterpret_cast<float*>(smem + C::OFF_SCALE);
+  float* vsc = ksc + D;
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_o = bar_s + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, kTcTmemCols);
+    tmem_relinquish();
+  }
+  if constexpr (C::kInt8) {
+    for (int d = tid; d < D; d += NT) {
+      ksc[d] = p.k_scale[h_kv * D + d];
+      vsc[d] = p.v_scale[h_kv * D + d];
+    }
+  }
+  int bits = 0;
+  auto resolve_chunk = [&](int first_tile) {
+    for (int i = tid; i < kTcCand; i += NT) {
+      const int cand = c_begin + first_tile * KT + i;
+      int kp = kPosInvalid;
+      bool from_aux = false;
+      long long off = -1;
+      if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      cand_off[i] = off;
+      cand_kpos[i] = kp;
+    }
+  };
+  if (ntiles > 0) resolve_chunk(0);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t tS = tmem + lane_off;
+  const uint32_t tO = tmem + 128 + lane_off;
+
+  // ---- Q tile: thread r owns row r (token r / G, head r % G)
+  {
+    const int r = tid;
+    const ActT* q = static_cast<const ActT*>(p.q);
+    const bool ok = r < R;
+    const ActT* qrow = q + ((long long)(t0 + (ok ? r / G : 0)) * p.H_q + h_kv * G + (ok ? r % G : 0)) * D;
+#pragma unroll 4
+    for (int u = 0; u < D / 8; ++u) {
+      uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
+      if (ok) {
+        if constexpr (!C::kInt8) {
+          hi = *reinterpret_cast<const uint4*>(qrow + u * 8);
+        } else {
+          alignas(16) __half h8[8], l8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = to_f32(qrow[u * 8 + e]) * ksc[u * 8 + e];
+            h8[e] = __float2half_rn(x);
+            l8[e] = __float2half_rn(x - __half2float(h8[e]));
+          }
+          hi = *reinterpret_cast<const uint4*>(h8);
+          lo = *reinterpret_cast<const uint4*>(l8);
+        }
+      }
+      *reinterpret_cast<uint4*>(sQ + sw_off(r, u)) = hi;
+      if constexpr (C::kInt8) *reinterpret_cast<uint4*>(sQlo + sw_off(r, u)) = lo;
+    }
+  }
+
+  // ---- gather of tile `it` into stage it % 2 (cp.async, 16-byte chunks)
+  const CacheT* kc = static_cast<const CacheT*>(p.k_cache);
+  const CacheT* vc = static_cast<const CacheT*>(p.v_cache);
+  const CacheT* ak = static_cast<const CacheT*>(p.aux_k);
+  const CacheT* av = static_cast<const CacheT*>(p.aux_v);
+  constexpr int CPR = C::ROW_BYTES / 16;   // 16-byte chunks per gathered row
+  auto issue = [&](int it) {
+    const int st = it & 1;
+    for (int e = tid; e < KT * CPR * 2; e += NT) {
+      const bool isv = e >= KT * CPR;
+      const int ee = isv ? e - KT * CPR : e;
+      const int row = ee / CPR, ch = ee % CPR;
+      const int ci = (it % kTcCandTiles) * KT + row;
+      const long long off = cand_off[ci];
+      const int kp = cand_kpos[ci];
+      const bool okr = off >= 0;
+      const CacheT* base = isv ? (kp == kPosAux ? av : vc) : (kp == kPosAux ? ak : kc);
+      const CacheT* src = okr ? base + off + ch * (16 / sizeof(CacheT)) : kc;
+      unsigned char* dst;
+      if constexpr (C::kInt8) {
+        dst = smem + C::OFF_KV + 2 * C::TILE + (st * 2 + (isv ? 1 : 0)) * C::RAW + row * C::ROW_BYTES + ch * 16;
+      } else {
+        dst = smem + C::OFF_KV + (st * 2 + (isv ? 1 : 0)) * C::TILE + sw_off(row, ch);
+      }
+      cp_async_16(dst, src, okr);
+      if (!isv && ch == 0) kpos_s[st * KT + row] = kp;
+    }
+  };
+
+  float m_used = -INFINITY, l_sum = 0.f;
+  const float sl2 = p.scale_log2;
+  const int prow = (tid < R && has_rows) ? U.p_first + tid / G : -1;
+  bool lost = false;
+  if (ntiles > 0) issue(0);
+  cp_async_commit();
+  for (int it = 0; it < ntiles; ++it) {
+    const int st = it & 1;
+    const int nxt = it + 1;
+    if (nxt < ntiles && nxt % kTcCandTiles == 0) {
+      __syncthreads();   // copies of the previous chunk are issued
+      resolve_chunk(nxt);
+      __syncthreads();
+    }
+    if (nxt < ntiles) issue(nxt);   // stage nxt & 1 was released by PV(it - 1)
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const unsigned char* kt;
+    const unsigned char* vt;
+    if constexpr (C::kInt8) {
+      // PV(it - 1) finished reading the converted tiles (waited below)
+      unsigned char* kcv = smem + C::OFF_KV;
+      unsigned char* vcv = kcv + C::TILE;
+      const unsigned char* raw = smem + C::OFF_KV + 2 * C::TILE + st * 2 * C::RAW;
+      for (int e = tid; e < KT * CPR * 2; e += NT) {
+        const bool isv = e >= KT * CPR;
+        const int ee = isv ? e - KT * CPR : e;
+        const int row = ee / CPR, ch = ee % CPR;
+        const int4 rv = *reinterpret_cast<const int4*>(raw + (isv ? C::RAW : 0) + row * C::ROW_BYTES + ch * 16);
+        const int8_t* b8 = reinterpret_cast<const int8_t*>(&rv);
+        alignas(16) __half h16[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) h16[k] = __int2half_rn(static_cast<int>(b8[k]));
+        unsigned char* dst = isv ? vcv : kcv;
+        *reinterpret_cast<uint4*>(dst + sw_off(row, 2 * ch)) = *reinterpret_cast<const uint4*>(h16);
+        *reinterpret_cast<uint4*>(dst + sw_off(row, 2 * ch + 1)) = *reinterpret_cast<const uint4*>(h16 + 8);
+      }
+      kt = kcv;
+      vt = vcv;
+    } else {
+      kt = smem + C::OFF_KV + st * 2 * C::TILE;
+      vt = kt + C::TILE;
+    }
+    // generic-proxy smem writes (Q, converted tiles, cp.async data) must be
+    // visible to the tensor core's async proxy
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int c = kk / 4, koff = (kk % 4) * 32;
+        const uint64_t bd = smem_desc_sw128(smem_u32(kt + c * 16384 + koff), 16, 1024);
+        mma_ss(tmem, smem_desc_sw128(smem_u32(sQ + c * 16384 + koff), 16, 1024), bd, IDESC_S,
+               kk > 0 ? 1u : 0u);
+        if constexpr (C::kInt8)
+          mma_ss(tmem, smem_desc_sw128(smem_u32(sQlo + c * 16384 + koff), 16, 1024), bd, IDESC_S, 1u);
+      }
+      tc_commit(bar_s);
+    }
+    const bool got = mbar_wait(bar_s, it & 1, kTcWaitLimit);
+    if (__syncthreads_or(!got)) {
+      lost = true;
+      break;
+    }
+    tc_fence_after();
+    // ---- softmax of row tid over this tile's keys
+    const int* kp = kpos_s + st * KT;
+    float mx = -INFINITY;
+#pragma unroll 1
+    for (int c4 = 0; c4 < KT / 32; ++c4) {
+      uint32_t v[32];
+      tmem_ld32(tS + c4 * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const bool vis = key_visible(kp[c4 * 32 + e], prow, p.window);
+        const float x = vis ? __uint_as_float(v[e]) : -INFINITY;
+        v[e] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      tmem_st32(tS + c4 * 32, v);
+    }
+    tmem_wait_st();
+    mx *= sl2;
+    const bool need = mx > m_used + 8.0f;
+    const float m_new = need ? mx : m_used;
+    const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2a(m_used - m_new)) : 1.f;
+    if (it > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
+      uint32_t o[32];
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st32(tO + c * 32, o);
+      }
+    }
+    l_sum *= alpha;
+    m_used = m_new;
+    const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+    float ls = 0.f;
+#pragma unroll 1
+    for (int hh = 0; hh < KT / 64; ++hh) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(tS + hh * 64 + half * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float pa = ex2a(fmaf(__uint_as_float(v[e]), sl2, nm));
+          const float pb = ex2a(fmaf(__uint_as_float(v[e + 1]), sl2, nm));
+          ls += pa + pb;
+          pk[half * 16 + e / 2] = pk_pair<MT>(pa, pb);
+        }
+      }
+      tmem_st32(tS + hh * 32, pk);
+    }
+    l_sum += ls;
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < KT / 16; ++kk) {
+        const uint64_t bd = smem_desc_sw128(smem_u32(vt + kk * 2048), 16384, 1024);
+        mma_ts(tmem + 128, tmem + kk * 8, bd, IDESC_O, (it > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(bar_o);
+    }
+    // the next tile's staging / conversion and S reuse what PV reads
+    const bool gone = mbar_wait(bar_o, it & 1, kTcWaitLimit);
+    if (__syncthreads_or(!gone)) {
+      lost = true;
+      break;
+    }
+    tc_fence_after();
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  if (lost) bits |= SPA_ST_TIMEOUT;
+
+  // ---- epilogue: row tid; O (x value scale) -> output or partial state
+  const bool have_o = ntiles > 0 && !lost;
+  const int r = tid;
+  const int tt = t0 + r / max(G, 1), h = h_kv * G + r % G;
+  const long long row = (long long)tt * p.H_q + h;
+  const bool mine = r < R;
+  float f = 1.f, lse = -INFINITY;
+  if (p.num_splits == 1) {
+    const float sink2 = (p.sinks && mine) ? p.sinks[h] * kLog2e : -INFINITY;
+    float a, inv_l;
+    finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
+    f = a * inv_l;
+  }
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    if (have_o) {
+      tmem_ld32(tO + c * 32, o);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0u;
+    }
+    if (!mine) continue;
+    float ov[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ov[e] = __uint_as_float(o[e]) * (C::kInt8 ? vsc[c * 32 + e] : 1.f);
+    if (p.num_splits == 1) {
+      ActT* out = static_cast<ActT*>(p.out) + row * D + c * 32;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) out[e] = from_f32<ActT>(ov[e] * f);
+    } else {
+      float* acc = p.ws_acc + ((long long)split * p.T * p.H_q + row) * D + c * 32;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(acc + e) = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
+    }
+  }
+  if (mine) {
+    if (p.num_splits == 1) {
+      if (p.lse) p.lse[row] = lse;
+    } else {
+      const long long wrow = (long long)split * p.T * p.H_q + row;
+      p.ws_ml[wrow * 2 + 0] = m_used;
+      p.ws_ml[wrow * 2 + 1] = l_sum;
+    }
+  }
+  flag(p.status, bits);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTcTmemCols);
+  }
+  if (p.num_splits > 1) finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
+}
+
+int tc_supported(int act, int cache, int D, int max_rows) {
+  if (act != SPA_F16 && act != SPA_BF16) return 0;
+  if (!(cache == act || cache == SPA_I8)) return 0;
+  if (D != 64 && D != 128) return 0;
+  return max_rows > 32 && max_rows <= 128;
+}
+
+template <typename ActT, typename CacheT, int D>
+static int launch_tc_t(const AttnParams& p, cudaStream_t stream) {
+  using C = TcCfg<ActT, CacheT, D>;
+  static_assert(C::SMEM <= 227 * 1024, "shared memory");
+  auto kern = decode_tc_kernel<ActT, CacheT, D>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
+  return launch_pdl(kern, dim3(units, p.num_splits), dim3(128), C::SMEM, stream, p);
+}
+
+int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream) {
+  if (act == SPA_F16) {
+    if (cache == SPA_I8) return p.D == 64 ? launch_tc_t<__half, int8_t, 64>(p, stream)
+                                          : launch_tc_t<__half, int8_t, 128>(p, stream);
+    return p.D == 64 ? launch_tc_t<__half, __half, 64>(p, stream) : launch_tc_t<__half, __half, 128>(p, stream);
+  }
+  if (cache == SPA_I8) return p.D == 64 ? launch_tc_t<__nv_bfloat16, int8_t, 64>(p, stream)
+                                        : launch_tc_t<__nv_bfloat16, int8_t, 128>(p, stream);
+  return p.D == 64 ? launch_tc_t<__nv_bfloat16, __nv_bfloat16, 64>(p, stream)
+                   : launch_tc_t<__nv_bfloat16, __nv_bfloat16, 128>(p, stream);
+}
+
+}  // namespace spa

@@ -7,7 +7,7 @@
 
 namespace spa {
 
-enum PlanKind { kPlanScalar = 0, kPlanMma = 1, kPlanPrefill = 2 };
+enum PlanKind { kPlanScalar = 0, kPlanMma = 1, kPlanPrefill = 2, kPlanTc = 3 };
 
 struct Plan {
   int kind;

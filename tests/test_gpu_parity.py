@@ -103,6 +103,18 @@ EDGE = {
                                    q_lens=[40, 9], past=[100, 0], window=24),
     "long_prefill_per_token_fallback": dict(act="f32", B=2, H_q=4, H_kv=2, D=64, block_size=16,
                                             q_lens=[70, 33], past=[0, 5]),
+    # units of more than 32 rows (G x S_q) take the tcgen05 decode kernel
+    "tc_bf16_window_64_rows": dict(act="bf16", B=3, H_q=32, H_kv=2, D=128, block_size=64,
+                                   q_lens=[4, 2, 3], past=[200, 30, 0], window=100),
+    "tc_int8_d64_aux_40_rows": dict(act="f16", cache="i8", B=2, H_q=20, H_kv=2, D=64, block_size=16,
+                                    q_lens=[4, 4], past=[130, 70], window=40, sel_mode="aux",
+                                    sel_width=50, aux_cap=90, aux_lens=[90, 33]),
+    "tc_sel_main_48_rows": dict(act="f16", B=2, H_q=16, H_kv=2, D=128, block_size=64, q_lens=[6, 5],
+                                past=[400, 250], sel_mode="main", sel_per_request=1, sel_width=300,
+                                sel_valid=280),
+    "tc_empty_selection": dict(act="bf16", cache="i8", B=2, H_q=48, H_kv=4, D=128, block_size=64,
+                               q_lens=[8, 3], past=[60, 10], sel_mode="main", sel_per_request=1,
+                               sel_width=16, sel_valid=0),
 }
 
 
