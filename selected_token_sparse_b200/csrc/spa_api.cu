@@ -25,7 +25,7 @@ int launch_attention_scalar_impl(const AttnParams&, int, int, int, cudaStream_t)
 size_t scalar_smem_bytes(int D, int max_rows, int nq);
 int launch_attention_mma(const AttnParams& p, int act, int cache, int max_rows, cudaStream_t stream);
 int mma_supported(int act, int cache, int D, int max_rows);
-int mma_key_tile();
+int mma_key_tile(int D, int max_rows);
 int tc_supported(int act, int cache, int D, int max_rows);
 int tc_key_tile();
 int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream);
@@ -106,7 +106,7 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   else if (mma_supported(a->act, a->cache, a->D, pl->max_rows)) pl->kind = kPlanMma;
   else pl->kind = kPlanScalar;
   const int KT = pl->kind == kPlanTc ? tc_key_tile()
-                                     : (pl->kind == kPlanMma ? mma_key_tile() : scalar_key_tile());
+                                     : (pl->kind == kPlanMma ? mma_key_tile(a->D, pl->max_rows) : scalar_key_tile());
   long long n_main;
   if (sel_main) n_main = a->sel_width;
   else if (a->window > 0) n_main = std::min<long long>((long long)a->window + pl->max_q - 1, a->max_seqlen_k);

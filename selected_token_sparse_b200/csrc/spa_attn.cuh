@@ -2,6 +2,7 @@
 #pragma once
 
 #include <climits>
+#include <type_traits>
 
 #include "spa_common.cuh"
 
@@ -166,39 +167,104 @@ __device__ __forceinline__ void finalize_row(float m, float l, float sink2, floa
   lse = (mf + log2f(lf)) * kLn2;
 }
 
-// Log-sum-exp merge of the split partial states of one output row with the
-// sink, by one warp (lanes over D); writes out[row] and lse[row].
-template <typename ActT, int D>
-__device__ __forceinline__ void merge_row(const AttnParams& p, long long row, int h, int lane) {
-  constexpr int PER = D / 32;
-  const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
-  const long long stride = (long long)p.T * p.H_q;
-  float M = sink2;
-  for (int s = 0; s < p.num_splits; ++s) M = fmaxf(M, __ldcg(p.ws_ml + (s * stride + row) * 2));
-  float o[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) o[i] = 0.f;
-  float lse = -INFINITY;
-  if (M != -INFINITY) {
-    float Lsum = (sink2 == -INFINITY) ? 0.f : exp2f(sink2 - M);
-    for (int s = 0; s < p.num_splits; ++s) {
-      const float ms = __ldcg(p.ws_ml + (s * stride + row) * 2);
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      Lsum += w * __ldcg(p.ws_ml + (s * stride + row) * 2 + 1);
-      const float* a = p.ws_acc + (s * stride + row) * D;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) o[i] = fmaf(w, __ldcg(a + lane + 32 * i), o[i]);
-    }
-    const float inv = 1.0f / Lsum;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) o[i] *= inv;
-    lse = (M + log2f(Lsum)) * kLn2;
+// Log-sum-exp merge of the split partial states of a unit's rows with the
+// sink ("[WebGPU] Add SparsePagedAttention", finalize: every split's running
+// max m_s and sum l_s are rescaled to the global max M; the sink joins the
+// denominator).  The whole CTA works on it with independent loads so the L2
+// latency of the workspace reads overlaps:
+//   pass 1, one thread per row: M = max(sink, m_s), L = sum_s 2^(m_s - M) l_s
+//           (+ 2^(sink - M)), lse = (M + log2 L) ln 2, kept in shared memory;
+//   pass 2, one thread per 4 output columns: o = sum_s 2^(m_s - M) acc_s / L.
+// Rows go in chunks of kMergeRows (the shared arrays' size).
+constexpr int kMergeRows = 128;
+
+template <typename ActT>
+__device__ __forceinline__ void store4(ActT* dst, float a, float b, float c, float d) {
+  if constexpr (std::is_same<ActT, float>::value) {
+    *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
+  } else {
+    ActT v[4] = {from_f32<ActT>(a), from_f32<ActT>(b), from_f32<ActT>(c), from_f32<ActT>(d)};
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(v);
   }
-  ActT* out = static_cast<ActT*>(p.out) + row * D;
+}
+
+template <typename ActT, int D>
+__device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, int h_kv) {
+  __shared__ float sM[kMergeRows], sInv[kMergeRows];
+  constexpr int C4 = D / 4;
+  const long long stride = (long long)p.T * p.H_q;
+  const int R = nq * p.G, S = p.num_splits;
+  for (int r0 = 0; r0 < R; r0 += kMergeRows) {
+    const int nr = min(kMergeRows, R - r0);
+    for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+      const int r = r0 + i;
+      const int h = h_kv * p.G + r % p.G;
+      const long long row = (long long)(t0 + r / p.G) * p.H_q + h;
+      const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+      float M = sink2;
+#pragma unroll 4
+      for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(p.ws_ml + (s * stride + row) * 2));
+      float inv = 0.f, lse = -INFINITY;
+      if (M != -INFINITY) {
+        float Lsum = (sink2 == -INFINITY) ? 0.f : exp2f(sink2 - M);
+#pragma unroll 4
+        for (int s = 0; s < S; ++s) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml + (s * stride + row) * 2));
+          if (ml.x != -INFINITY) Lsum += exp2f(ml.x - M) * ml.y;
+        }
+        inv = 1.0f / Lsum;
+        lse = (M + log2f(Lsum)) * kLn2;
+      }
+      sM[i] = M;
+      sInv[i] = inv;
+      if (p.lse) p.lse[row] = lse;
+    }
+    __syncthreads();
+    // four output items per thread in flight; out-of-range items re-read the
+    // chunk's last item and store nothing
+    const int n_items = nr * C4;
+    for (int base = threadIdx.x; base < n_items; base += 4 * blockDim.x) {
+      int ii[4];
+      long long rw[4];
+      float Mi[4];
+      float4 o[4];
 #pragma unroll
-  for (int i = 0; i < PER; ++i) out[lane + 32 * i] = from_f32<ActT>(o[i]);
-  if (lane == 0 && p.lse) p.lse[row] = lse;
+      for (int j = 0; j < 4; ++j) {
+        ii[j] = min(base + j * (int)blockDim.x, n_items - 1);
+        const int r = r0 + ii[j] / C4;
+        rw[j] = (long long)(t0 + r / p.G) * p.H_q + h_kv * p.G + r % p.G;
+        Mi[j] = sM[ii[j] / C4];
+        o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll 2
+      for (int s = 0; s < S; ++s) {
+        float ms[4];
+        float4 a[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          ms[j] = __ldcg(p.ws_ml + (s * stride + rw[j]) * 2);
+          a[j] = __ldcg(reinterpret_cast<const float4*>(p.ws_acc + (s * stride + rw[j]) * D + (ii[j] % C4) * 4));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (ms[j] == -INFINITY || Mi[j] == -INFINITY) continue;
+          const float w = exp2f(ms[j] - Mi[j]);
+          o[j].x = fmaf(w, a[j].x, o[j].x);
+          o[j].y = fmaf(w, a[j].y, o[j].y);
+          o[j].z = fmaf(w, a[j].z, o[j].z);
+          o[j].w = fmaf(w, a[j].w, o[j].w);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (base + j * (int)blockDim.x >= n_items) continue;
+        const float inv = sInv[ii[j] / C4];
+        store4<ActT>(static_cast<ActT*>(p.out) + rw[j] * D + (ii[j] % C4) * 4, o[j].x * inv, o[j].y * inv,
+                     o[j].z * inv, o[j].w * inv);
+      }
+    }
+    __syncthreads();
+  }
 }
 
 // Called by every thread of a split CTA once its partial states are written.
@@ -218,12 +284,7 @@ __device__ __forceinline__ void finish_split(const AttnParams& p, int unit, int 
   __syncthreads();
   if (!*smem_flag) return;
   __threadfence();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int R = nq * p.G;
-  for (int r = warp; r < R; r += nw) {
-    const int t = t0 + r / p.G, h = h_kv * p.G + r % p.G;
-    merge_row<ActT, D>(p, (long long)t * p.H_q + h, h, lane);
-  }
+  merge_rows<ActT, D>(p, t0, nq, h_kv);
 }
 
 int scalar_key_tile();

@@ -29,12 +29,18 @@
 
 namespace spa {
 
-constexpr int kMmaKT = 64;      // keys per tile
-constexpr int kMmaStages = 3;   // cp.async ring depth
-constexpr int kMmaCandTiles = 8;                     // tiles whose candidates are resolved at once
-constexpr int kMmaCandChunk = kMmaCandTiles * 64;    // = kMmaCandTiles * kMmaKT
+constexpr int kMmaCandChunk = 512;   // candidates resolved at once
 
-int mma_key_tile() { return kMmaKT; }
+// Keys per tile: one 128-key tile (one softmax pass, four 32-key warp slices)
+// for single-row-tile units with D = 64, otherwise 64-key tiles in a 3-deep ring.
+constexpr int mma_kt(int D, int rt) { return (D == 64 && rt == 1) ? 128 : 64; }
+int mma_key_tile(int D, int max_rows) { return mma_kt(D, (max_rows + 15) / 16); }
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <typename T> struct MmaName;
 template <> struct MmaName<__half> { static constexpr bool bf16 = false; };
@@ -88,21 +94,24 @@ template <typename ActT, typename CacheT, int D, int RT, int KW>
 struct MmaCfg {
   using MT = typename std::conditional<sizeof(CacheT) == 1, __half, ActT>::type;
   static constexpr bool kInt8 = sizeof(CacheT) == 1;
+  static constexpr int KT = mma_kt(D, RT);
+  static constexpr int STAGES = KT == 128 ? 2 : 3;  // cp.async ring depth
+  static constexpr int CAND_TILES = kMmaCandChunk / KT;
   static constexpr int NW = RT * KW;
   static constexpr int NT = NW * 32;
-  static constexpr int KS = kMmaKT / KW;        // keys per warp slice
+  static constexpr int KS = KT / KW;            // keys per warp slice
   static constexpr int CPR = D * 2 / 16;        // 16-byte chunks per 16-bit row
   static constexpr int RAW_CPR = D * (int)sizeof(CacheT) / 16;
-  static constexpr int TILE16 = kMmaKT * D * 2;               // one converted K or V tile
-  static constexpr int RAW_TILE = kMmaKT * D * (int)sizeof(CacheT);
+  static constexpr int TILE16 = KT * D * 2;                   // one converted K or V tile
+  static constexpr int RAW_TILE = KT * D * (int)sizeof(CacheT);
   static constexpr int ROWS = RT * 16;
   // shared memory layout (bytes)
   static constexpr int OFF_Q = 0;                                      // Q (int8 path: q*ks, high part)
   static constexpr int OFF_QLO = OFF_Q + ROWS * D * 2;                 // int8 path: low part
   static constexpr int OFF_RAW = OFF_QLO + (kInt8 ? ROWS * D * 2 : 0); // stages x (K, V) raw
-  static constexpr int OFF_CONV = OFF_RAW + kMmaStages * 2 * RAW_TILE;  // int8 only: (K, V) fp16
+  static constexpr int OFF_CONV = OFF_RAW + STAGES * 2 * RAW_TILE;  // int8 only: (K, V) fp16
   static constexpr int OFF_KPOS = OFF_CONV + (kInt8 ? 2 * TILE16 : 0);
-  static constexpr int OFF_SCALE = OFF_KPOS + kMmaStages * kMmaKT * 4;
+  static constexpr int OFF_SCALE = OFF_KPOS + STAGES * KT * 4;
   static constexpr int OFF_PROW = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
   static constexpr int OFF_CAND = OFF_PROW + 128 * 4;                  // resolved candidates
   static constexpr int END = OFF_CAND + kMmaCandChunk * (8 + 4);
@@ -118,7 +127,8 @@ __global__ void __launch_bounds__(RT * KW * 32)
 decode_mma_kernel(const AttnParams p) {
   using C = MmaCfg<ActT, CacheT, D, RT, KW>;
   using MT = typename C::MT;
-  constexpr int KT = kMmaKT, NT = C::NT, KS = C::KS, CPR = C::CPR, RAW_CPR = C::RAW_CPR;
+  constexpr int KT = C::KT, NT = C::NT, KS = C::KS, CPR = C::CPR, RAW_CPR = C::RAW_CPR;
+  constexpr int kMmaStages = C::STAGES, kMmaCandTiles = C::CAND_TILES;
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wr = warp % RT;   // row tile of this warp
@@ -126,6 +136,24 @@ decode_mma_kernel(const AttnParams p) {
   __shared__ int last_flag;
   pdl_wait();
   pdl_trigger();
+
+  // Q rows of the unit in 16-byte chunks (row r = token r / G, head r % G).
+  // A per-token unit knows its token from the block index, so its loads are
+  // in flight while the unit's metadata loads resolve.
+  constexpr int QPER = (C::ROWS * CPR + NT - 1) / NT;
+  const ActT* q = static_cast<const ActT*>(p.q);
+  uint4 qv[QPER];
+  auto load_q = [&](int tq, int rows) {
+#pragma unroll
+    for (int k = 0; k < QPER; ++k) {
+      const int e = tid + k * NT, r = e / CPR, c = e % CPR;
+      qv[k] = make_uint4(0, 0, 0, 0);
+      if (e < C::ROWS * CPR && r < rows)
+        qv[k] = *reinterpret_cast<const uint4*>(q + ((long long)(tq + r / p.G) * p.H_q +
+                                                     (blockIdx.x % p.H_kv) * p.G + r % p.G) * D + c * 8);
+    }
+  };
+  if (!p.group_by_request) load_q(blockIdx.x / p.H_kv, p.G);
 
   Unit U;
   const bool has_rows = decode_unit(p, blockIdx.x, U);
@@ -143,10 +171,11 @@ decode_mma_kernel(const AttnParams p) {
   float* vsc_s = ksc_s + D;
   int* prow_s = reinterpret_cast<int*>(smem + C::OFF_PROW);
 
+  if (p.group_by_request) load_q(t0, R);
+
   // ---- Q rows -> swizzled smem.  INT8 caches keep K exact (|k8| <= 128 is
   // exact in fp16): the key scale is folded into q in fp32 and q*ks is split
   // into fp16 high and low parts, so S = k8.hi + k8.lo carries ~22 bits.
-  const ActT* q = static_cast<const ActT*>(p.q);
   if constexpr (C::kInt8) {
     for (int d = tid; d < D; d += NT) {
       ksc_s[d] = p.k_scale[h_kv * D + d];
@@ -154,30 +183,25 @@ decode_mma_kernel(const AttnParams p) {
     }
     __syncthreads();
   }
-  for (int e = tid; e < C::ROWS * CPR; e += NT) {
-    const int r = e / CPR, c = e % CPR;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    uint4 vlo = make_uint4(0, 0, 0, 0);
-    if (r < R) {
-      const int t = t0 + r / G, h = h_kv * G + r % G;
-      const ActT* src = q + ((long long)t * p.H_q + h) * D + c * 8;
-      if constexpr (!C::kInt8) {
-        v = *reinterpret_cast<const uint4*>(src);
-      } else {
-        alignas(16) __half hi[8];
-        alignas(16) __half lo[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float x = to_f32(src[i]) * ksc_s[c * 8 + i];
-          hi[i] = __float2half_rn(x);
-          lo[i] = __float2half_rn(x - __half2float(hi[i]));
-        }
-        v = *reinterpret_cast<const uint4*>(hi);
-        vlo = *reinterpret_cast<const uint4*>(lo);
+  for (int k = 0; k < QPER; ++k) {
+    const int e = tid + k * NT, r = e / CPR, c = e % CPR;
+    if (e >= C::ROWS * CPR) continue;
+    uint4 v = qv[k];
+    if constexpr (C::kInt8) {
+      const ActT* x8 = reinterpret_cast<const ActT*>(&qv[k]);
+      alignas(16) __half hi[8];
+      alignas(16) __half lo[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float x = to_f32(x8[i]) * ksc_s[c * 8 + i];
+        hi[i] = __float2half_rn(x);
+        lo[i] = __float2half_rn(x - __half2float(hi[i]));
       }
+      v = *reinterpret_cast<const uint4*>(hi);
+      *reinterpret_cast<uint4*>(smem + C::OFF_QLO + swz(r, c, CPR)) = *reinterpret_cast<const uint4*>(lo);
     }
     *reinterpret_cast<uint4*>(q_s + swz(r, c, CPR)) = v;
-    if constexpr (C::kInt8) *reinterpret_cast<uint4*>(smem + C::OFF_QLO + swz(r, c, CPR)) = vlo;
   }
   for (int i = tid; i < 128; i += NT) prow_s[i] = (i < nq && has_rows) ? U.p_first + i : -1;
 
@@ -358,8 +382,10 @@ decode_mma_kernel(const AttnParams p) {
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
     }
     const float mn0 = fmaxf(m_r[0], mx0), mn1 = fmaxf(m_r[1], mx1);
-    const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_r[0] - mn0);
-    const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_r[1] - mn1);
+    const float al0 = (mn0 == -INFINITY) ? 1.f : ex2f(m_r[0] - mn0);
+    const float al1 = (mn1 == -INFINITY) ? 1.f : ex2f(m_r[1] - mn1);
+    // masked scores are -inf and give 0 once the row max is finite
+    const float ms0 = (mn0 == -INFINITY) ? 0.f : mn0, ms1 = (mn1 == -INFINITY) ? 0.f : mn1;
     m_r[0] = mn0;
     m_r[1] = mn1;
     float ls0 = 0.f, ls1 = 0.f;
@@ -367,8 +393,8 @@ decode_mma_kernel(const AttnParams p) {
     for (int j = 0; j < KS / 8; ++j) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        s[j][e] = (s[j][e] == -INFINITY) ? 0.f : exp2f(s[j][e] - mn0);
-        s[j][2 + e] = (s[j][2 + e] == -INFINITY) ? 0.f : exp2f(s[j][2 + e] - mn1);
+        s[j][e] = ex2f(s[j][e] - ms0);
+        s[j][2 + e] = ex2f(s[j][2 + e] - ms1);
         ls0 += s[j][e];
         ls1 += s[j][2 + e];
       }
@@ -438,10 +464,10 @@ decode_mma_kernel(const AttnParams p) {
         const float* other = red + ((k2 * RT + wr) * 32 + lane) * PER;
         const float om0 = other[D / 2 + 0], om1 = other[D / 2 + 1];
         const float mn0 = fmaxf(m_r[0], om0), mn1 = fmaxf(m_r[1], om1);
-        const float a0 = (mn0 == -INFINITY) ? 0.f : exp2f(m_r[0] - mn0);
-        const float b0 = (mn0 == -INFINITY) ? 0.f : exp2f(om0 - mn0);
-        const float a1 = (mn1 == -INFINITY) ? 0.f : exp2f(m_r[1] - mn1);
-        const float b1 = (mn1 == -INFINITY) ? 0.f : exp2f(om1 - mn1);
+        const float a0 = (mn0 == -INFINITY) ? 0.f : ex2f(m_r[0] - mn0);
+        const float b0 = (mn0 == -INFINITY) ? 0.f : ex2f(om0 - mn0);
+        const float a1 = (mn1 == -INFINITY) ? 0.f : ex2f(m_r[1] - mn1);
+        const float b1 = (mn1 == -INFINITY) ? 0.f : ex2f(om1 - mn1);
 #pragma unroll
         for (int n = 0; n < D / 8; ++n) {
           o[n][0] = o[n][0] * a0 + other[n * 4 + 0] * b0;
@@ -484,8 +510,7 @@ decode_mma_kernel(const AttnParams p) {
 #pragma unroll
       for (int n = 0; n < D / 8; ++n) {
         const int d = n * 8 + (lane & 3) * 2;
-        out[d] = from_f32<ActT>(o[n][hrow * 2 + 0] * f);
-        out[d + 1] = from_f32<ActT>(o[n][hrow * 2 + 1] * f);
+        *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(o[n][hrow * 2 + 0] * f, o[n][hrow * 2 + 1] * f);
       }
       if ((lane & 3) == 0 && p.lse) p.lse[row] = lse;
     } else {

@@ -38,6 +38,7 @@ namespace spa {
 using namespace sm100;
 
 constexpr int kTcKT = 128;                      // keys per tile (MMA N)
+constexpr int kTcThreads = 256;                 // two warps per TMEM lane quadrant
 constexpr int kTcCandTiles = 4;                 // tiles whose candidates are resolved at once
 constexpr int kTcCand = kTcCandTiles * kTcKT;
 constexpr uint32_t kTcTmemCols = 256;           // S [0,128) | O [128, 128 + D)
@@ -59,11 +60,12 @@ struct TcCfg {
   // 16-bit caches: 2 stages x (K, V) swizzled tiles; INT8: one (K, V) pair of
   // converted tiles plus 2 stages x (K, V) raw staging
   static constexpr int KV_BYTES = kInt8 ? 2 * TILE + 2 * 2 * RAW : 2 * 2 * TILE;
-  static constexpr int OFF_KPOS = OFF_KV + KV_BYTES;              // [2][128] key positions
-  static constexpr int OFF_CAND = OFF_KPOS + 2 * kTcKT * 4;      // candidate offsets + positions
-  static constexpr int OFF_SCALE = OFF_CAND + kTcCand * 12;      // INT8: ks, vs
+  static constexpr int OFF_KVIS = OFF_KV + KV_BYTES;              // [2][128] visible row-position intervals
+  static constexpr int OFF_CAND = OFF_KVIS + 2 * kTcKT * 8;      // candidate offsets + positions
+  static constexpr int OFF_RED = OFF_CAND + kTcCand * 12;        // [2][128] row max, [2][128] row sum
+  static constexpr int OFF_SCALE = OFF_RED + 4 * 128 * 4;        // INT8: ks, vs
   static constexpr int OFF_BAR = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
-  static constexpr int OFF_MISC = OFF_BAR + 16;                  // tmem holder, flags
+  static constexpr int OFF_MISC = OFF_BAR + 16;                  // tmem holder
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;
 };
@@ -91,19 +93,47 @@ __device__ __forceinline__ float ex2a(float x) {
   return y;
 }
 
+// Four signed bytes -> two fp16 pairs holding the same integers, exactly:
+// with the sign bit flipped a byte is u = x + 128 in [0, 255]; placed under
+// the fp16 exponent of 1024 (high byte 0x64) it reads 1024 + u, and
+// subtracting 1152 leaves x.
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t x = w ^ 0x80808080u;
+  uint32_t a = __byte_perm(x, 0x64646464u, 0x4140);
+  uint32_t b = __byte_perm(x, 0x64646464u, 0x4342);
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152
+  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
+  __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
+  lo = *reinterpret_cast<uint32_t*>(&ha);
+  hi = *reinterpret_cast<uint32_t*>(&hb);
+}
+
+template <typename ActT>
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  uint4 r;
+  r.x = pk_pair<ActT>(x[0], x[1]);
+  r.y = pk_pair<ActT>(x[2], x[3]);
+  r.z = pk_pair<ActT>(x[4], x[5]);
+  r.w = pk_pair<ActT>(x[6], x[7]);
+  return r;
+}
+
 template <typename ActT, typename CacheT, int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const AttnParams p) {
   using C = TcCfg<ActT, CacheT, D>;
   using MT = typename C::MT;
   constexpr uint32_t FMT = std::is_same<MT, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = idesc_f16(FMT, 128, kTcKT, 0);
   constexpr uint32_t IDESC_O = idesc_f16(FMT, 128, D, 1);
-  constexpr int KT = kTcKT, NT = 128;
+  constexpr int KT = kTcKT, NT = kTcThreads;
+  constexpr int HK = KT / 2, HD = D / 2;   // key columns / O columns per warp half
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + lane;   // the S / O row (TMEM lane) this thread works on
   __shared__ int last_flag;
   pdl_wait();
   pdl_trigger();
@@ -121,12 +151,16 @@ decode_tc_kernel(const AttnParams p) {
   const int c_begin = split * p.split_len;
   const int c_end = min(c_begin + p.split_len, n_total);
   const int ntiles = c_end > c_begin ? (c_end - c_begin + KT - 1) / KT : 0;
+  // query positions of the unit's rows: [p_lo, p_hi]
+  const int p_lo = has_rows ? U.p_first : 0, p_hi = has_rows ? U.p_last : -1;
 
   unsigned char* sQ = smem + C::OFF_Q;
   unsigned char* sQlo = smem + C::OFF_QLO;
-  int* kpos_s = reinterpret_cast<int*>(smem + C::OFF_KPOS);
+  int2* kvis_s = reinterpret_cast<int2*>(smem + C::OFF_KVIS);
   long long* cand_off = reinterpret_cast<long long*>(smem + C::OFF_CAND);
   int* cand_kpos = reinterpret_cast<int*>(smem + C::OFF_CAND + kTcCand * 8);
+  float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);
+  float* red_l = red_max + 2 * 128;
   float* ksc = reinterpret_cast<float*>(smem + C::OFF_SCALE);
   float* vsc = ksc + D;
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -160,57 +194,48 @@ decode_tc_kernel(const AttnParams p) {
       cand_kpos[i] = kp;
     }
   };
+  // Q rows (row r = token r / G, head r % G) in coalesced 16-byte units; the
+  // loads are in flight while the candidates resolve
+  constexpr int QU = D / 8;
+  constexpr int QPER = 128 * QU / NT;
+  uint4 qv[QPER];
+  {
+    const ActT* q = static_cast<const ActT*>(p.q);
+#pragma unroll
+    for (int k = 0; k < QPER; ++k) {
+      const int i = tid + k * NT, r = i / QU, u = i % QU;
+      qv[k] = make_uint4(0, 0, 0, 0);
+      if (r < R)
+        qv[k] = *reinterpret_cast<const uint4*>(q + ((long long)(t0 + r / G) * p.H_q + h_kv * G + r % G) * D + u * 8);
+    }
+  }
   if (ntiles > 0) resolve_chunk(0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
   const uint32_t tS = tmem + lane_off;
-  const uint32_t tO = tmem + 128 + lane_off;
+  const uint32_t tO = tmem + 128 + lane_off + half * HD;
 
-  // ---- Q tile: thread r owns row r (token r / G, head r % G)
-  {
-    const int r = tid;
-    const ActT* q = static_cast<const ActT*>(p.q);
-    const bool ok = r < R;
-    const ActT* qrow = q + ((long long)(t0 + (ok ? r / G : 0)) * p.H_q + h_kv * G + (ok ? r % G : 0)) * D;
-#pragma unroll 4
-    for (int u = 0; u < D / 8; ++u) {
-      uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
-      if (ok) {
-        if constexpr (!C::kInt8) {
-          hi = *reinterpret_cast<const uint4*>(qrow + u * 8);
-        } else {
-          alignas(16) __half h8[8], l8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float x = to_f32(qrow[u * 8 + e]) * ksc[u * 8 + e];
-            h8[e] = __float2half_rn(x);
-            l8[e] = __float2half_rn(x - __half2float(h8[e]));
-          }
-          hi = *reinterpret_cast<const uint4*>(h8);
-          lo = *reinterpret_cast<const uint4*>(l8);
-        }
-      }
-      *reinterpret_cast<uint4*>(sQ + sw_off(r, u)) = hi;
-      if constexpr (C::kInt8) *reinterpret_cast<uint4*>(sQlo + sw_off(r, u)) = lo;
-    }
-  }
-
-  // ---- gather of tile `it` into stage it % 2 (cp.async, 16-byte chunks)
+  // ---- gather of tile `it` into stage it % 2 (cp.async, 16-byte chunks).
+  // Each key also gets the interval [a, b] of query positions that see it
+  // (auxiliary entries: all; empty slots: none; main-cache key j: j .. j +
+  // window - 1, or j .. with no window).  Returns whether every key this
+  // thread placed is visible to every row of the unit.
   const CacheT* kc = static_cast<const CacheT*>(p.k_cache);
   const CacheT* vc = static_cast<const CacheT*>(p.v_cache);
   const CacheT* ak = static_cast<const CacheT*>(p.aux_k);
   const CacheT* av = static_cast<const CacheT*>(p.aux_v);
   constexpr int CPR = C::ROW_BYTES / 16;   // 16-byte chunks per gathered row
-  auto issue = [&](int it) {
+  auto issue = [&](int it) -> bool {
     const int st = it & 1;
+    bool all_vis = true;
     for (int e = tid; e < KT * CPR * 2; e += NT) {
       const bool isv = e >= KT * CPR;
       const int ee = isv ? e - KT * CPR : e;
-      const int row = ee / CPR, ch = ee % CPR;
-      const int ci = (it % kTcCandTiles) * KT + row;
+      const int r = ee / CPR, ch = ee % CPR;
+      const int ci = (it % kTcCandTiles) * KT + r;
       const long long off = cand_off[ci];
       const int kp = cand_kpos[ci];
       const bool okr = off >= 0;
@@ -218,21 +243,58 @@ decode_tc_kernel(const AttnParams p) {
       const CacheT* src = okr ? base + off + ch * (16 / sizeof(CacheT)) : kc;
       unsigned char* dst;
       if constexpr (C::kInt8) {
-        dst = smem + C::OFF_KV + 2 * C::TILE + (st * 2 + (isv ? 1 : 0)) * C::RAW + row * C::ROW_BYTES + ch * 16;
+        dst = smem + C::OFF_KV + 2 * C::TILE + (st * 2 + (isv ? 1 : 0)) * C::RAW + r * C::ROW_BYTES + ch * 16;
       } else {
-        dst = smem + C::OFF_KV + (st * 2 + (isv ? 1 : 0)) * C::TILE + sw_off(row, ch);
+        dst = smem + C::OFF_KV + (st * 2 + (isv ? 1 : 0)) * C::TILE + sw_off(r, ch);
       }
       cp_async_16(dst, src, okr);
-      if (!isv && ch == 0) kpos_s[st * KT + row] = kp;
+      if (!isv && ch == 0) {
+        int a = kp, b = INT_MAX;
+        if (kp == kPosAux) {
+          a = INT_MIN;
+        } else if (kp == kPosInvalid) {
+          a = INT_MAX;
+          b = INT_MIN;
+        } else if (p.window > 0 && kp <= INT_MAX - p.window) {
+          b = kp + p.window - 1;
+        }
+        kvis_s[st * KT + r] = make_int2(a, b);
+        all_vis = all_vis && a <= p_lo && b >= p_hi;
+      }
     }
+    return all_vis;
   };
+  bool vis_cur = true;
+  if (ntiles > 0) vis_cur = issue(0);
+  cp_async_commit();
+
+  // ---- Q tile in swizzled shared memory (overlaps the first gather); INT8
+  // caches fold the key scale into q and split it into fp16 high and low tiles
+  {
+#pragma unroll
+    for (int k = 0; k < QPER; ++k) {
+      const int i = tid + k * NT, r = i / QU, u = i % QU;
+      if constexpr (!C::kInt8) {
+        *reinterpret_cast<uint4*>(sQ + sw_off(r, u)) = qv[k];
+      } else {
+        const ActT* x8 = reinterpret_cast<const ActT*>(&qv[k]);
+        alignas(16) __half h8[8], l8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = to_f32(x8[e]) * ksc[u * 8 + e];
+          h8[e] = __float2half_rn(x);
+          l8[e] = __float2half_rn(x - __half2float(h8[e]));
+        }
+        *reinterpret_cast<uint4*>(sQ + sw_off(r, u)) = *reinterpret_cast<const uint4*>(h8);
+        *reinterpret_cast<uint4*>(sQlo + sw_off(r, u)) = *reinterpret_cast<const uint4*>(l8);
+      }
+    }
+  }
 
   float m_used = -INFINITY, l_sum = 0.f;
   const float sl2 = p.scale_log2;
-  const int prow = (tid < R && has_rows) ? U.p_first + tid / G : -1;
+  const int prow = (row < R && has_rows) ? U.p_first + row / G : -1;
   bool lost = false;
-  if (ntiles > 0) issue(0);
-  cp_async_commit();
   for (int it = 0; it < ntiles; ++it) {
     const int st = it & 1;
     const int nxt = it + 1;
@@ -241,10 +303,12 @@ decode_tc_kernel(const AttnParams p) {
       resolve_chunk(nxt);
       __syncthreads();
     }
-    if (nxt < ntiles) issue(nxt);   // stage nxt & 1 was released by PV(it - 1)
+    bool vis_nxt = true;
+    if (nxt < ntiles) vis_nxt = issue(nxt);   // stage nxt & 1 was released by PV(it - 1)
     cp_async_commit();
     cp_async_wait<1>();
-    __syncthreads();
+    const bool tile_vis = __syncthreads_and(vis_cur);
+    vis_cur = vis_nxt;
     const unsigned char* kt;
     const unsigned char* vt;
     if constexpr (C::kInt8) {
@@ -252,18 +316,20 @@ decode_tc_kernel(const AttnParams p) {
       unsigned char* kcv = smem + C::OFF_KV;
       unsigned char* vcv = kcv + C::TILE;
       const unsigned char* raw = smem + C::OFF_KV + 2 * C::TILE + st * 2 * C::RAW;
+#pragma unroll 2
       for (int e = tid; e < KT * CPR * 2; e += NT) {
         const bool isv = e >= KT * CPR;
         const int ee = isv ? e - KT * CPR : e;
-        const int row = ee / CPR, ch = ee % CPR;
-        const int4 rv = *reinterpret_cast<const int4*>(raw + (isv ? C::RAW : 0) + row * C::ROW_BYTES + ch * 16);
-        const int8_t* b8 = reinterpret_cast<const int8_t*>(&rv);
-        alignas(16) __half h16[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) h16[k] = __int2half_rn(static_cast<int>(b8[k]));
+        const int r = ee / CPR, ch = ee % CPR;
+        const uint4 rv = *reinterpret_cast<const uint4*>(raw + (isv ? C::RAW : 0) + r * C::ROW_BYTES + ch * 16);
+        uint4 h0, h1;
+        i8x4_to_h2x2(rv.x, h0.x, h0.y);
+        i8x4_to_h2x2(rv.y, h0.z, h0.w);
+        i8x4_to_h2x2(rv.z, h1.x, h1.y);
+        i8x4_to_h2x2(rv.w, h1.z, h1.w);
         unsigned char* dst = isv ? vcv : kcv;
-        *reinterpret_cast<uint4*>(dst + sw_off(row, 2 * ch)) = *reinterpret_cast<const uint4*>(h16);
-        *reinterpret_cast<uint4*>(dst + sw_off(row, 2 * ch + 1)) = *reinterpret_cast<const uint4*>(h16 + 8);
+        *reinterpret_cast<uint4*>(dst + sw_off(r, 2 * ch)) = h0;
+        *reinterpret_cast<uint4*>(dst + sw_off(r, 2 * ch + 1)) = h1;
       }
       kt = kcv;
       vt = vcv;
@@ -294,32 +360,42 @@ decode_tc_kernel(const AttnParams p) {
       break;
     }
     tc_fence_after();
-    // ---- softmax of row tid over this tile's keys
-    const int* kp = kpos_s + st * KT;
-    float mx = -INFINITY;
-#pragma unroll 1
-    for (int c4 = 0; c4 < KT / 32; ++c4) {
-      uint32_t v[32];
-      tmem_ld32(tS + c4 * 32, v);
-      tmem_wait_ld();
+    // ---- softmax of row `row` over this half's 64 keys of the tile; the two
+    // halves exchange their maxima through shared memory
+    uint32_t v[HK];
+    tmem_ld32(tS + half * HK, v);
+    tmem_ld32(tS + half * HK + 32, v + 32);
+    tmem_wait_ld();
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+    if (tile_vis) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const bool vis = key_visible(kp[c4 * 32 + e], prow, p.window);
-        const float x = vis ? __uint_as_float(v[e]) : -INFINITY;
-        v[e] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      for (int e = 0; e < HK; e += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+        mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
       }
-      tmem_st32(tS + c4 * 32, v);
+    } else {
+      const int4* kv4 = reinterpret_cast<const int4*>(kvis_s + st * KT + half * HK);
+#pragma unroll
+      for (int e = 0; e < HK; e += 2) {
+        const int4 w = kv4[e / 2];
+        const float x0 = (prow >= w.x && prow <= w.y) ? __uint_as_float(v[e]) : -INFINITY;
+        const float x1 = (prow >= w.z && prow <= w.w) ? __uint_as_float(v[e + 1]) : -INFINITY;
+        v[e] = __float_as_uint(x0);
+        v[e + 1] = __float_as_uint(x1);
+        mx0 = fmaxf(mx0, x0);
+        mx1 = fmaxf(mx1, x1);
+      }
     }
-    tmem_wait_st();
-    mx *= sl2;
+    red_max[half * 128 + row] = fmaxf(mx0, mx1);
+    __syncthreads();
+    const float mx = fmaxf(red_max[row], red_max[128 + row]) * sl2;
     const bool need = mx > m_used + 8.0f;
     const float m_new = need ? mx : m_used;
     const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2a(m_used - m_new)) : 1.f;
     if (it > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
       uint32_t o[32];
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
 #pragma unroll
@@ -327,29 +403,22 @@ decode_tc_kernel(const AttnParams p) {
         tmem_st32(tO + c * 32, o);
       }
     }
-    l_sum *= alpha;
     m_used = m_new;
     const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
-    float ls = 0.f;
-#pragma unroll 1
-    for (int hh = 0; hh < KT / 64; ++hh) {
-      uint32_t pk[32];
+    float ls0 = 0.f, ls1 = 0.f;
+    uint32_t pk[HK / 2];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t v[32];
-        tmem_ld32(tS + hh * 64 + half * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float pa = ex2a(fmaf(__uint_as_float(v[e]), sl2, nm));
-          const float pb = ex2a(fmaf(__uint_as_float(v[e + 1]), sl2, nm));
-          ls += pa + pb;
-          pk[half * 16 + e / 2] = pk_pair<MT>(pa, pb);
-        }
-      }
-      tmem_st32(tS + hh * 32, pk);
+    for (int e = 0; e < HK; e += 2) {
+      const float pa = ex2a(fmaf(__uint_as_float(v[e]), sl2, nm));
+      const float pb = ex2a(fmaf(__uint_as_float(v[e + 1]), sl2, nm));
+      ls0 += pa;
+      ls1 += pb;
+      pk[e / 2] = pk_pair<MT>(pa, pb);
     }
-    l_sum += ls;
+    // packed P of keys [half*64, half*64 + 64) -> columns [half*32, half*32 + 32);
+    // every S column was read into registers before the barrier above
+    tmem_st32(tS + half * (HK / 2), pk);
+    l_sum = l_sum * alpha + (ls0 + ls1);
     tmem_wait_st();
     tc_fence_before();
     __syncthreads();
@@ -371,15 +440,17 @@ decode_tc_kernel(const AttnParams p) {
     tc_fence_after();
   }
   cp_async_wait<0>();
+  red_l[half * 128 + row] = l_sum;
   __syncthreads();
+  l_sum = red_l[row] + red_l[128 + row];
   if (lost) bits |= SPA_ST_TIMEOUT;
 
-  // ---- epilogue: row tid; O (x value scale) -> output or partial state
+  // ---- epilogue: row `row`, this half's D/2 columns; O (x value scale) ->
+  // output or partial state
   const bool have_o = ntiles > 0 && !lost;
-  const int r = tid;
-  const int tt = t0 + r / max(G, 1), h = h_kv * G + r % G;
-  const long long row = (long long)tt * p.H_q + h;
-  const bool mine = r < R;
+  const int tt = t0 + row / max(G, 1), h = h_kv * G + row % G;
+  const long long orow = (long long)tt * p.H_q + h;
+  const bool mine = row < R;
   float f = 1.f, lse = -INFINITY;
   if (p.num_splits == 1) {
     const float sink2 = (p.sinks && mine) ? p.sinks[h] * kLog2e : -INFINITY;
@@ -388,7 +459,7 @@ decode_tc_kernel(const AttnParams p) {
     f = a * inv_l;
   }
 #pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = 0; c < HD / 32; ++c) {
     uint32_t o[32];
     if (have_o) {
       tmem_ld32(tO + c * 32, o);
@@ -398,24 +469,27 @@ decode_tc_kernel(const AttnParams p) {
       for (int e = 0; e < 32; ++e) o[e] = 0u;
     }
     if (!mine) continue;
+    const int col = half * HD + c * 32;
     float ov[32];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) ov[e] = __uint_as_float(o[e]) * (C::kInt8 ? vsc[c * 32 + e] : 1.f);
+    for (int e = 0; e < 32; ++e) ov[e] = __uint_as_float(o[e]) * (C::kInt8 ? vsc[col + e] : 1.f);
     if (p.num_splits == 1) {
-      ActT* out = static_cast<ActT*>(p.out) + row * D + c * 32;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) out[e] = from_f32<ActT>(ov[e] * f);
+      for (int e = 0; e < 32; ++e) ov[e] *= f;
+      uint4* out = reinterpret_cast<uint4*>(static_cast<ActT*>(p.out) + orow * D + col);
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) out[e / 8] = pack8<ActT>(ov + e);
     } else {
-      float* acc = p.ws_acc + ((long long)split * p.T * p.H_q + row) * D + c * 32;
+      float* acc = p.ws_acc + ((long long)split * p.T * p.H_q + orow) * D + col;
 #pragma unroll
       for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(acc + e) = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
     }
   }
-  if (mine) {
+  if (mine && half == 0) {
     if (p.num_splits == 1) {
-      if (p.lse) p.lse[row] = lse;
+      if (p.lse) p.lse[orow] = lse;
     } else {
-      const long long wrow = (long long)split * p.T * p.H_q + row;
+      const long long wrow = (long long)split * p.T * p.H_q + orow;
       p.ws_ml[wrow * 2 + 0] = m_used;
       p.ws_ml[wrow * 2 + 1] = l_sum;
     }
@@ -444,7 +518,7 @@ static int launch_tc_t(const AttnParams& p, cudaStream_t stream) {
   auto kern = decode_tc_kernel<ActT, CacheT, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
-  return launch_pdl(kern, dim3(units, p.num_splits), dim3(128), C::SMEM, stream, p);
+  return launch_pdl(kern, dim3(units, p.num_splits), dim3(kTcThreads), C::SMEM, stream, p);
 }
 
 int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream) {

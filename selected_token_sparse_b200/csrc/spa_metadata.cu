@@ -178,6 +178,10 @@ __device__ __forceinline__ void append_token_rows(const ActT* __restrict__ k_new
   }
 }
 
+// 16-byte vectors of a token's K (and V) rows each lane loads before the
+// metadata is known (16-bit caches), so the copy does not wait for them
+constexpr int kAppendPre = 2;
+
 template <typename ActT, typename CacheT>
 __global__ void __launch_bounds__(kMetaThreads)
 prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
@@ -189,31 +193,73 @@ prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict_
                       CacheT* __restrict__ k_cache, CacheT* __restrict__ v_cache,
                       const float* __restrict__ k_scale, const float* __restrict__ v_scale, int H_kv,
                       int D, int32_t* __restrict__ status) {
-  extern __shared__ int32_t cs[];  // [B + 1]
+  extern __shared__ int32_t cs[];  // [B + 1] cumulative lengths, then [B] past lengths
+  int32_t* past_s = cs + B + 1;
   pdl_wait();
   pdl_trigger();
-  build_cs(cu, B, T, cs);
-  if (blockIdx.x == 0) flag(status, per_request(cu, past, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
   const int lane = threadIdx.x & 31;
   const int wpb = kMetaThreads / 32;
+  const int t_first = blockIdx.x * wpb + (threadIdx.x >> 5);
+  constexpr bool kCopy = sizeof(CacheT) != 1;
+  constexpr int EPV = 16 / sizeof(ActT);
+  const int nvec = H_kv * D / EPV;
+  uint4 kpre[kAppendPre], vpre[kAppendPre];
+  if constexpr (kCopy) {
+    if (t_first < T) {
+      const uint4* ks = reinterpret_cast<const uint4*>(k_new + (long long)t_first * H_kv * D);
+      const uint4* vs = reinterpret_cast<const uint4*>(v_new + (long long)t_first * H_kv * D);
+#pragma unroll
+      for (int i = 0; i < kAppendPre; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nvec) {
+          kpre[i] = ks[v];
+          vpre[i] = vs[v];
+        }
+      }
+    }
+  }
+  for (int b = threadIdx.x; b < B; b += blockDim.x) past_s[b] = past[b];
+  build_cs(cu, B, T, cs);   // ends with a block barrier: past_s is visible too
+  if (blockIdx.x == 0) flag(status, per_request(cu, past_s, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
   int bits = 0;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+  for (int t = t_first; t < T; t += gridDim.x * wpb) {
     int tb = 0;  // every lane computes the same metadata; lane 0 reports and writes it
-    const TokenMeta m = token_meta(t, cs, B, past, block_table, MB, bs, num_blocks, tb);
+    const TokenMeta m = token_meta(t, cs, B, past_s, block_table, MB, bs, num_blocks, tb);
     if (lane == 0) {
       bits |= tb;
       token_batch[t] = m.b;
       token_pos[t] = m.pos;
       slot_mapping[t] = m.slot;
     }
-    if (m.slot >= 0)
-      append_token_rows<ActT, CacheT>(k_new, v_new, k_cache, v_cache, k_scale, v_scale, t, m.slot, H_kv, D,
-                                      lane);
+    if (m.slot < 0) continue;
+    if constexpr (kCopy) {
+      if (t == t_first) {
+        uint4* kd = reinterpret_cast<uint4*>(k_cache + (long long)m.slot * H_kv * D);
+        uint4* vd = reinterpret_cast<uint4*>(v_cache + (long long)m.slot * H_kv * D);
+#pragma unroll
+        for (int i = 0; i < kAppendPre; ++i) {
+          const int v = lane + 32 * i;
+          if (v < nvec) {
+            kd[v] = kpre[i];
+            vd[v] = vpre[i];
+          }
+        }
+        const uint4* ks = reinterpret_cast<const uint4*>(k_new + (long long)t * H_kv * D);
+        const uint4* vs = reinterpret_cast<const uint4*>(v_new + (long long)t * H_kv * D);
+        for (int v = lane + 32 * kAppendPre; v < nvec; v += 32) {
+          kd[v] = ks[v];
+          vd[v] = vs[v];
+        }
+        continue;
+      }
+    }
+    append_token_rows<ActT, CacheT>(k_new, v_new, k_cache, v_cache, k_scale, v_scale, t, m.slot, H_kv, D, lane);
   }
   flag(status, bits);
 }
 
 static size_t cs_smem(int B) { return sizeof(int32_t) * (size_t)(B + 1); }
+static size_t cs_past_smem(int B) { return sizeof(int32_t) * (size_t)(2 * B + 1); }
 
 template <typename K>
 static void allow_smem(K kern, size_t smem) {
@@ -246,7 +292,7 @@ static int launch_pa(const int32_t* cu, const int32_t* past, const int32_t* bloc
   int grid = (T + wpb - 1) / wpb;
   if (grid < 1) grid = 1;
   if (grid > 148 * 8) grid = 148 * 8;
-  const size_t smem = cs_smem(B);
+  const size_t smem = cs_past_smem(B);
   auto kern = prepare_append_kernel<ActT, CacheT>;
   allow_smem(kern, smem);
   return launch_pdl(kern, dim3(grid), dim3(kMetaThreads), smem, stream, cu, past, block_table, B, T, max_q,
