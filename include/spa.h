@@ -232,6 +232,41 @@ int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspa
                   spa_stream_t stream);
 
 /*
+ * spa_prepare_append_attention -- steps 1 to 5 as one call: the outputs of
+ * spa_prepare_append_kv followed by spa_attention with the same arguments,
+ * bit for bit (the metadata arrays, both caches, out, lse and status).
+ * Source: "[WebGPU] Add SparsePagedAttention", File summaries (prepare the
+ * token metadata, scatter the current K/V into the cache, then attend) --
+ * here one kernel launch when the plan picks the warp-MMA decode kernel on a
+ * 16-bit cache of the activation dtype (each CTA derives its unit's metadata
+ * from cu_seqlens_q and past_seqlens in shared memory, writes its share of
+ * the metadata and of the appended rows, and reads this step's own new rows
+ * from k_new / v_new); otherwise the two launches of the staged sequence.
+ *   a               the attention arguments; a->seqlens_q, a->seqlen_k,
+ *                   a->token_batch and a->token_pos are OUTPUTS here (the
+ *                   step-1 arrays, written with spa_prepare_metadata's
+ *                   meaning); a->cu_seqlens_q, block_table, MB, block_size,
+ *                   num_blocks, max_seqlen_q, max_seqlen_k, k_cache, v_cache,
+ *                   cache, k_scale, v_scale, H_kv, D and status play their
+ *                   spa_prepare_append_kv roles as well.
+ *   past_seqlens [B], k_new, v_new [T, H_kv, D] (dtype a->act, 16-byte
+ *                   aligned), slot_mapping [T] (output): as in
+ *                   spa_prepare_append_kv.
+ *   workspace       as in spa_attention (spa_attention_workspace_size(a)).
+ * Errors: those of both entry points; nothing is launched on an error.
+ * Memory the caches alias between this step's new slots and older positions
+ * (a malformed block table) is read as the staged sequence would only when
+ * the two launches are used.
+ */
+int spa_prepare_append_attention(const spa_attention_args_t* a, const int32_t* past_seqlens,
+                                 const void* k_new, const void* v_new, int32_t* slot_mapping, void* workspace,
+                                 size_t workspace_bytes, spa_stream_t stream);
+
+/* Kernel launches spa_prepare_append_attention makes for these arguments (1 or
+   2), or a negative error code.  Host only. */
+int spa_prepare_append_attention_launches(const spa_attention_args_t* a);
+
+/*
  * spa_attention_noalloc -- spa_attention for callers that cannot allocate
  * device memory.  The pages have no counterpart: this entry point exists for
  * callers of this library that cannot provide a workspace -- code running

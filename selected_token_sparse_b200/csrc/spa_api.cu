@@ -29,6 +29,8 @@ int mma_key_tile(int D, int max_rows);
 int tc_supported(int act, int cache, int D, int max_rows);
 int tc_key_tile();
 int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream);
+int launch_step_mma(const AttnParams& p, int act, int max_rows, cudaStream_t stream);
+int mma_step_fits(int D, int max_rows, int B);
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream);
 int prefill_supported(const spa_attention_args_t* a);
 
@@ -214,6 +216,12 @@ int run_attention(const spa_attention_args_t* a, const Plan& pl, void* ws, cudaS
 
 int launches_of(const Plan&) { return 1; }
 
+// The fused step runs as one launch when the plan picks the warp-MMA kernel
+// on a cache of the activation dtype and the metadata fits shared memory.
+static bool step_fusable(const spa_attention_args_t* a, const Plan& pl) {
+  return pl.kind == kPlanMma && a->cache == a->act && a->B <= 4096 && mma_step_fits(a->D, pl.max_rows, a->B);
+}
+
 const char* cuda_message() { return g_cuda_msg; }
 int check_launch_public() { return check_launch(); }
 
@@ -314,6 +322,76 @@ int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspa
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPA_ERR_WORKSPACE;
   }
   return run_attention(a, pl, workspace, (cudaStream_t)stream);
+}
+
+// Validation of the step-1/2 arguments the fused step adds to `a`.
+static int validate_step(const spa_attention_args_t* a, const int32_t* past_seqlens, const void* k_new,
+                         const void* v_new, const int32_t* slot_mapping) {
+  if (a->B > 16384) return SPA_ERR_UNSUPPORTED;
+  if ((long long)a->num_blocks * a->block_size >= (1LL << 31)) return SPA_ERR_INVALID_ARG;
+  if (a->B > 0 && (!past_seqlens || !a->seqlens_q || !a->seqlen_k)) return SPA_ERR_INVALID_ARG;
+  if (a->T > 0 && (!a->token_batch || !a->token_pos || !slot_mapping || !k_new || !v_new))
+    return SPA_ERR_INVALID_ARG;
+  if ((a->D * elt_bytes(a->act)) % 16 != 0) return SPA_ERR_INVALID_ARG;
+  if (a->cache == SPA_I8 && a->D % 16 != 0) return SPA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15) return SPA_ERR_INVALID_ARG;
+  return SPA_OK;
+}
+
+int spa_prepare_append_attention(const spa_attention_args_t* a, const int32_t* past_seqlens,
+                                 const void* k_new, const void* v_new, int32_t* slot_mapping, void* workspace,
+                                 size_t workspace_bytes, spa_stream_t stream) {
+  int rc = validate_attention(a);
+  if (rc != SPA_OK) return rc;
+  if ((rc = validate_step(a, past_seqlens, k_new, v_new, slot_mapping)) != SPA_OK) return rc;
+  int32_t* seqlens_q = const_cast<int32_t*>(a->seqlens_q);
+  int32_t* seqlen_k = const_cast<int32_t*>(a->seqlen_k);
+  int32_t* token_batch = const_cast<int32_t*>(a->token_batch);
+  int32_t* token_pos = const_cast<int32_t*>(a->token_pos);
+  const cudaStream_t st = (cudaStream_t)stream;
+  auto staged_prepare = [&]() {
+    launch_prepare_append(a->cu_seqlens_q, past_seqlens, a->block_table, a->B, a->T, a->max_seqlen_q,
+                          a->max_seqlen_k, a->MB, a->block_size, a->num_blocks, seqlens_q, seqlen_k, token_batch,
+                          token_pos, slot_mapping, k_new, v_new, a->act, const_cast<void*>(a->k_cache),
+                          const_cast<void*>(a->v_cache), a->cache, a->k_scale, a->v_scale, a->H_kv, a->D,
+                          a->status, st);
+    return check_launch();
+  };
+  if (a->T == 0 || a->B == 0) return staged_prepare();
+  Plan pl;
+  if ((rc = make_plan(a, &pl)) != SPA_OK) return rc;
+  const size_t need = pl.ws_acc_bytes + pl.ws_ml_bytes + pl.ws_count_bytes;
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return SPA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return SPA_ERR_WORKSPACE;
+  }
+  if (!step_fusable(a, pl)) {
+    if ((rc = staged_prepare()) != SPA_OK) return rc;
+    return run_attention(a, pl, workspace, st);
+  }
+  AttnParams p;
+  fill_params(a, pl, workspace, &p);
+  p.past = past_seqlens;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.seqlens_q_out = seqlens_q;
+  p.seqlen_k_out = seqlen_k;
+  p.token_batch_out = token_batch;
+  p.token_pos_out = token_pos;
+  p.slot_out = slot_mapping;
+  p.max_seqlen_q = a->max_seqlen_q;
+  p.max_seqlen_k = a->max_seqlen_k;
+  if ((rc = launch_step_mma(p, a->act, pl.max_rows, st)) != SPA_OK) return rc;
+  return check_launch();
+}
+
+int spa_prepare_append_attention_launches(const spa_attention_args_t* a) {
+  int rc = validate_attention(a);
+  if (rc != SPA_OK) return rc;
+  if (a->T == 0 || a->B == 0) return 1;
+  Plan pl;
+  if ((rc = make_plan(a, &pl)) != SPA_OK) return rc;
+  return step_fusable(a, pl) ? 1 : 1 + launches_of(pl);
 }
 
 int spa_attention_plan(const spa_attention_args_t* a, int32_t* num_splits, int32_t* num_launches,

@@ -45,6 +45,18 @@ struct AttnParams {
   float* ws_ml;          // [num_splits, T, H_q, 2]
   int* ws_count;         // [units] split tickets; zero between calls
   int32_t* status;
+  // fused step (metadata + append + attention in one launch): inputs of step
+  // 1-2, and the metadata arrays as outputs
+  const int32_t* past;
+  const void* k_new;
+  const void* v_new;
+  int32_t* seqlens_q_out;
+  int32_t* seqlen_k_out;
+  int32_t* token_batch_out;
+  int32_t* token_pos_out;
+  int32_t* slot_out;
+  int max_seqlen_q;      // host bounds for the step-1 status bits
+  int max_seqlen_k;
 };
 
 // Programmatic dependent launch: let the next kernel in the stream be
@@ -61,28 +73,47 @@ struct Unit {
   int aux_n;              // valid auxiliary entries of the request
   const int32_t* selrow;  // selection row or nullptr
   bool sel_main, sel_aux;
+  // fused step only: positions [new_lo, new_hi) are this step's tokens of the
+  // request, whose K/V rows are read from k_new / v_new (token new_t0 + j - new_lo)
+  int new_lo, new_hi, new_t0;
 };
 
-__device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& U) {
+// Step-1 metadata as the attention kernels read it: the arrays written by the
+// metadata entry points.
+struct StagedMeta {
+  const AttnParams& p;
+  __device__ __forceinline__ int cu(int g) const { return p.cu[g]; }
+  __device__ __forceinline__ int seqlens_q(int b) const { return p.seqlens_q[b]; }
+  __device__ __forceinline__ int seqlen_k(int b) const { return p.seqlen_k[b]; }
+  __device__ __forceinline__ void token(int t, int& b, int& pos) const {
+    b = p.token_batch[t];
+    pos = p.token_pos[t];
+  }
+};
+
+template <typename Meta>
+__device__ __forceinline__ bool decode_unit_with(const AttnParams& p, const Meta& m, int u, Unit& U) {
   U.h_kv = u % p.H_kv;
   const int g = u / p.H_kv;
+  int tpos = -1;
+  U.new_lo = U.new_hi = U.new_t0 = 0;
   if (p.group_by_request) {
     U.b = g;
-    U.t0 = clampi(p.cu[g], 0, p.T);
-    U.nq = clampi(p.seqlens_q[g], 0, p.T - U.t0);
+    U.t0 = clampi(m.cu(g), 0, p.T);
+    U.nq = clampi(m.seqlens_q(g), 0, p.T - U.t0);
     U.nq = min(U.nq, p.max_q);
   } else {
     U.t0 = g;
-    U.b = p.token_batch[g];
+    m.token(g, U.b, tpos);
     U.nq = 1;
   }
   if (U.b < 0 || U.b >= p.B || U.nq <= 0) return false;
-  U.L = max(p.seqlen_k[U.b] + 1, 0);
+  U.L = max(m.seqlen_k(U.b) + 1, 0);
   if (p.group_by_request) {
     // the request's tokens sit at past, past + 1, ... with past = L - q_len
-    U.p_first = max(U.L - p.seqlens_q[U.b], 0);
+    U.p_first = max(U.L - m.seqlens_q(U.b), 0);
   } else {
-    U.p_first = p.token_pos[U.t0];
+    U.p_first = tpos;
   }
   U.p_last = U.p_first + U.nq - 1;
   U.sel_main = p.sel != nullptr && p.sel_target == 0;
@@ -100,6 +131,10 @@ __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& U)
   U.n_aux = U.sel_aux ? p.sel_width : 0;
   U.aux_n = U.sel_aux ? min(p.aux_len[U.b], p.aux_cap) : 0;
   return true;
+}
+
+__device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& U) {
+  return decode_unit_with(p, StagedMeta{p}, u, U);
 }
 
 // Resolve candidate c of a unit to a cache element offset (or -1) and a key position.

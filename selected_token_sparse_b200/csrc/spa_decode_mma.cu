@@ -26,6 +26,7 @@
 #include <type_traits>
 
 #include "spa_attn.cuh"
+#include "spa_meta.cuh"
 
 namespace spa {
 
@@ -122,7 +123,13 @@ struct MmaCfg {
   static_assert(OFF_RED + RED_BYTES <= OFF_KPOS, "merge buffer must not reach the scales / positions");
 };
 
-template <typename ActT, typename CacheT, int D, int RT, int KW>
+// FUSED: one launch of the whole step (16-bit caches).  Every CTA rebuilds
+// the sanitised cumulative lengths and reads the past lengths into shared
+// memory (after the kernel's own layout), decodes its unit from them with the
+// metadata kernels' helpers, writes its share of the step-1/2 outputs, and
+// reads candidates at this step's new positions from k_new / v_new -- the
+// bytes the append writes, so the result equals the staged sequence.
+template <typename ActT, typename CacheT, int D, int RT, int KW, bool FUSED>
 __global__ void __launch_bounds__(RT * KW * 32)
 decode_mma_kernel(const AttnParams p) {
   using C = MmaCfg<ActT, CacheT, D, RT, KW>;
@@ -154,10 +161,43 @@ decode_mma_kernel(const AttnParams p) {
     }
   };
   if (!p.group_by_request) load_q(blockIdx.x / p.H_kv, p.G);
+  // fused step, per-token unit, split 0: this thread's vector of the token's
+  // new K/V row is loaded now and stored into the cache at the end
+  constexpr int NV = D * 2 / 16;
+  const bool app_thread = FUSED && !p.group_by_request && blockIdx.y == 0 && tid < 2 * NV;
+  uint4 app_data = make_uint4(0, 0, 0, 0);
+  if constexpr (FUSED) {
+    if (app_thread) app_data = fused_load_row_vector<CacheT>(p, blockIdx.x / p.H_kv, blockIdx.x % p.H_kv, tid, NV);
+  }
 
   Unit U;
-  const bool has_rows = decode_unit(p, blockIdx.x, U);
-  if (p.group_by_request && !has_rows) return;
+  bool has_rows;
+  int bits = 0;
+  int32_t* cs_s = nullptr;
+  int32_t* past_s = nullptr;
+  if constexpr (FUSED) {
+    cs_s = reinterpret_cast<int32_t*>(smem + C::SMEM);
+    past_s = cs_s + p.B + 1;
+    for (int b = tid; b < p.B; b += NT) past_s[b] = p.past[b];
+    build_cs<NT>(p.cu, p.B, p.T, cs_s);   // ends with a block barrier
+    has_rows = decode_unit_with(p, FusedMeta{p.cu, cs_s, past_s, p.B}, blockIdx.x, U);
+    if (has_rows) {
+      U.new_lo = max(past_s[U.b], 0);
+      U.new_hi = U.new_lo + (cs_s[U.b + 1] - cs_s[U.b]);
+      U.new_t0 = cs_s[U.b];
+    }
+    if (p.group_by_request && !has_rows) {
+      if (blockIdx.y == 0) {
+        if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits);
+        fused_group_append<CacheT>(p, cs_s, past_s, blockIdx.x / p.H_kv, blockIdx.x % p.H_kv, bits);
+      }
+      flag(p.status, bits);
+      return;
+    }
+  } else {
+    has_rows = decode_unit(p, blockIdx.x, U);
+    if (p.group_by_request && !has_rows) return;
+  }
   const int split = blockIdx.y;
   const int G = p.G;
   const int nq = p.group_by_request ? U.nq : 1;
@@ -214,7 +254,8 @@ decode_mma_kernel(const AttnParams p) {
   const CacheT* vc = static_cast<const CacheT*>(p.v_cache);
   const CacheT* ak = static_cast<const CacheT*>(p.aux_k);
   const CacheT* av = static_cast<const CacheT*>(p.aux_v);
-  int bits = 0;
+  const CacheT* kn = static_cast<const CacheT*>(p.k_new);
+  const CacheT* vn = static_cast<const CacheT*>(p.v_new);
 
   // Issue the copies of tile `it` into its ring stage.  Thread `tid` copies
   // chunk (tid % RAW_CPR) of rows tid / RAW_CPR, + NT / RAW_CPR, ...
@@ -231,6 +272,11 @@ decode_mma_kernel(const AttnParams p) {
       bool from_aux = false;
       long long off = -1;
       if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      if constexpr (FUSED) {
+        // this step's tokens: read the row the append writes from its source
+        if (off >= 0 && kp >= U.new_lo && kp < U.new_hi)
+          off = (((long long)(U.new_t0 + kp - U.new_lo) * p.H_kv + U.h_kv) * D) | kNewRow;
+      }
       cand_off[i] = off;
       cand_kpos[i] = kp;
     }
@@ -243,11 +289,18 @@ decode_mma_kernel(const AttnParams p) {
     for (int row = tid / RAW_CPR; row < KT; row += NT / RAW_CPR) {
       const int ci = (it % kMmaCandTiles) * KT + row;
       const int kp = cand_kpos[ci];
-      const long long off = cand_off[ci];
+      long long off = cand_off[ci];
       const bool from_aux = kp == kPosAux;
       const bool ok = off >= 0;
       const CacheT* kb = from_aux ? ak : kc;
       const CacheT* vb = from_aux ? av : vc;
+      if constexpr (FUSED) {
+        if (ok && (off & kNewRow)) {
+          off &= ~kNewRow;
+          kb = kn;
+          vb = vn;
+        }
+      }
       const CacheT* ksrc = ok ? kb + off + c * (16 / sizeof(CacheT)) : kc;
       const CacheT* vsrc = ok ? vb + off + c * (16 / sizeof(CacheT)) : vc;
       const int dst = C::kInt8 ? (row * RAW_CPR + c) * 16 : swz(row, c, CPR);
@@ -272,6 +325,11 @@ decode_mma_kernel(const AttnParams p) {
     if (s < ntiles) issue(s);
     cp_async_commit();
   }
+  TokenLoad app_tl;
+  if constexpr (FUSED) {
+    if (!p.group_by_request && split == 0)
+      app_tl = token_meta_load(blockIdx.x / p.H_kv, cs_s, p.B, past_s, p.block_table, p.MB, p.bs);
+  }
   __syncthreads();
   // Q fragments for this warp's row tile stay in registers (16-bit caches)
   if constexpr (!C::kInt8) {
@@ -284,6 +342,12 @@ decode_mma_kernel(const AttnParams p) {
   }
   const int r0 = wr * 16 + (lane >> 2);
   const int r1 = r0 + 8;
+  // the epilogue's sink logits, in flight from here
+  float sink_raw[2] = {-INFINITY, -INFINITY};
+  if (p.sinks && p.num_splits == 1) {
+    if (r0 < R) sink_raw[0] = ld_early(p.sinks + h_kv * G + r0 % G);
+    if (r1 < R) sink_raw[1] = ld_early(p.sinks + h_kv * G + r1 % G);
+  }
   const int prow0 = r0 < R ? prow_s[r0 / G] : -1;
   const int prow1 = r1 < R ? prow_s[r1 / G] : -1;
   const float sl2 = p.scale_log2;
@@ -430,7 +494,6 @@ decode_mma_kernel(const AttnParams p) {
   }
   cp_async_wait<0>();
   __syncthreads();
-  flag(p.status, bits);
 
   // row sums across the quad
 #pragma unroll
@@ -439,62 +502,81 @@ decode_mma_kernel(const AttnParams p) {
     l_r[1] += __shfl_xor_sync(0xffffffffu, l_r[1], o2);
   }
 
-  // merge the KW key slices of each row tile (into the wk == 0 warp)
+  // Merge of the KW key slices of each row tile: every warp publishes its
+  // state, then warp (wr, wk) combines and writes the wk-th share of the
+  // output columns (8-column blocks [wk * NPW, (wk + 1) * NPW)).
+  constexpr int NB8 = D / 8;
+  constexpr int NPW = NB8 / KW;
+  const int n_lo = wk * NPW;
+  float fo[NPW][4];
+  float mf[2], lf[2];
   if constexpr (KW > 1) {
     float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
     constexpr int PER = D / 2 + 4;
     float* mine = red + (warp * 32 + lane) * PER;
-    if (wk > 0) {
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        mine[n * 4 + 0] = o[n][0];
-        mine[n * 4 + 1] = o[n][1];
-        mine[n * 4 + 2] = o[n][2];
-        mine[n * 4 + 3] = o[n][3];
-      }
-      mine[D / 2 + 0] = m_r[0];
-      mine[D / 2 + 1] = m_r[1];
-      mine[D / 2 + 2] = l_r[0];
-      mine[D / 2 + 3] = l_r[1];
-    }
+    for (int n = 0; n < NB8; ++n)
+      *reinterpret_cast<float4*>(mine + n * 4) = make_float4(o[n][0], o[n][1], o[n][2], o[n][3]);
+    *reinterpret_cast<float4*>(mine + D / 2) = make_float4(m_r[0], m_r[1], l_r[0], l_r[1]);
     __syncthreads();
-    if (wk == 0) {
+    float4 ml[KW];
 #pragma unroll
-      for (int k2 = 1; k2 < KW; ++k2) {
-        const float* other = red + ((k2 * RT + wr) * 32 + lane) * PER;
-        const float om0 = other[D / 2 + 0], om1 = other[D / 2 + 1];
-        const float mn0 = fmaxf(m_r[0], om0), mn1 = fmaxf(m_r[1], om1);
-        const float a0 = (mn0 == -INFINITY) ? 0.f : ex2f(m_r[0] - mn0);
-        const float b0 = (mn0 == -INFINITY) ? 0.f : ex2f(om0 - mn0);
-        const float a1 = (mn1 == -INFINITY) ? 0.f : ex2f(m_r[1] - mn1);
-        const float b1 = (mn1 == -INFINITY) ? 0.f : ex2f(om1 - mn1);
+    for (int k2 = 0; k2 < KW; ++k2)
+      ml[k2] = *reinterpret_cast<const float4*>(red + ((k2 * RT + wr) * 32 + lane) * PER + D / 2);
+    mf[0] = mf[1] = -INFINITY;
 #pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-          o[n][0] = o[n][0] * a0 + other[n * 4 + 0] * b0;
-          o[n][1] = o[n][1] * a0 + other[n * 4 + 1] * b0;
-          o[n][2] = o[n][2] * a1 + other[n * 4 + 2] * b1;
-          o[n][3] = o[n][3] * a1 + other[n * 4 + 3] * b1;
-        }
-        l_r[0] = l_r[0] * a0 + other[D / 2 + 2] * b0;
-        l_r[1] = l_r[1] * a1 + other[D / 2 + 3] * b1;
-        m_r[0] = mn0;
-        m_r[1] = mn1;
+    for (int k2 = 0; k2 < KW; ++k2) {
+      mf[0] = fmaxf(mf[0], ml[k2].x);
+      mf[1] = fmaxf(mf[1], ml[k2].y);
+    }
+    float w0[KW], w1[KW];
+    lf[0] = lf[1] = 0.f;
+#pragma unroll
+    for (int k2 = 0; k2 < KW; ++k2) {
+      w0[k2] = (mf[0] == -INFINITY) ? 0.f : ex2f(ml[k2].x - mf[0]);
+      w1[k2] = (mf[1] == -INFINITY) ? 0.f : ex2f(ml[k2].y - mf[1]);
+      lf[0] = fmaf(w0[k2], ml[k2].z, lf[0]);
+      lf[1] = fmaf(w1[k2], ml[k2].w, lf[1]);
+    }
+#pragma unroll
+    for (int nn = 0; nn < NPW; ++nn) fo[nn][0] = fo[nn][1] = fo[nn][2] = fo[nn][3] = 0.f;
+#pragma unroll
+    for (int k2 = 0; k2 < KW; ++k2) {
+      const float* other = red + ((k2 * RT + wr) * 32 + lane) * PER;
+#pragma unroll
+      for (int nn = 0; nn < NPW; ++nn) {
+        const float4 x = *reinterpret_cast<const float4*>(other + (n_lo + nn) * 4);
+        fo[nn][0] = fmaf(w0[k2], x.x, fo[nn][0]);
+        fo[nn][1] = fmaf(w0[k2], x.y, fo[nn][1]);
+        fo[nn][2] = fmaf(w1[k2], x.z, fo[nn][2]);
+        fo[nn][3] = fmaf(w1[k2], x.w, fo[nn][3]);
       }
     }
+  } else {
+#pragma unroll
+    for (int nn = 0; nn < NPW; ++nn) {
+      fo[nn][0] = o[nn][0];
+      fo[nn][1] = o[nn][1];
+      fo[nn][2] = o[nn][2];
+      fo[nn][3] = o[nn][3];
+    }
+    mf[0] = m_r[0];
+    mf[1] = m_r[1];
+    lf[0] = l_r[0];
+    lf[1] = l_r[1];
   }
-  if (wk == 0) {
   if constexpr (C::kInt8) {   // O = vs * sum_j p_j v8_j (V stayed exact)
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      const int d = n * 8 + (lane & 3) * 2;
-      o[n][0] *= vsc_s[d];
-      o[n][1] *= vsc_s[d + 1];
-      o[n][2] *= vsc_s[d];
-      o[n][3] *= vsc_s[d + 1];
+    for (int nn = 0; nn < NPW; ++nn) {
+      const int d = (n_lo + nn) * 8 + (lane & 3) * 2;
+      fo[nn][0] *= vsc_s[d];
+      fo[nn][1] *= vsc_s[d + 1];
+      fo[nn][2] *= vsc_s[d];
+      fo[nn][3] *= vsc_s[d + 1];
     }
   }
 
-  // write rows r0, r1 of this row tile
+  // write this warp's columns of rows r0, r1
 #pragma unroll
   for (int hrow = 0; hrow < 2; ++hrow) {
     const int r = hrow ? r1 : r0;
@@ -502,38 +584,56 @@ decode_mma_kernel(const AttnParams p) {
     const int t = t0 + r / G, h = h_kv * G + r % G;
     const long long row = (long long)t * p.H_q + h;
     if (p.num_splits == 1) {
-      const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+      const float sink2 = p.sinks ? sink_raw[hrow] * kLog2e : -INFINITY;
       float a, inv_l, lse;
-      finalize_row(m_r[hrow], l_r[hrow], sink2, a, inv_l, lse);
+      finalize_row(mf[hrow], lf[hrow], sink2, a, inv_l, lse);
       const float f = a * inv_l;
       ActT* out = static_cast<ActT*>(p.out) + row * D;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        const int d = n * 8 + (lane & 3) * 2;
-        *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(o[n][hrow * 2 + 0] * f, o[n][hrow * 2 + 1] * f);
+      for (int nn = 0; nn < NPW; ++nn) {
+        const int d = (n_lo + nn) * 8 + (lane & 3) * 2;
+        *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(fo[nn][hrow * 2 + 0] * f, fo[nn][hrow * 2 + 1] * f);
       }
-      if ((lane & 3) == 0 && p.lse) p.lse[row] = lse;
+      if (wk == 0 && (lane & 3) == 0 && p.lse) p.lse[row] = lse;
     } else {
       const long long wrow = (long long)split * p.T * p.H_q + row;
       float* acc = p.ws_acc + wrow * D;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        const int d = n * 8 + (lane & 3) * 2;
-        *reinterpret_cast<float2*>(acc + d) = make_float2(o[n][hrow * 2], o[n][hrow * 2 + 1]);
+      for (int nn = 0; nn < NPW; ++nn) {
+        const int d = (n_lo + nn) * 8 + (lane & 3) * 2;
+        *reinterpret_cast<float2*>(acc + d) = make_float2(fo[nn][hrow * 2], fo[nn][hrow * 2 + 1]);
       }
-      if ((lane & 3) == 0) {
-        p.ws_ml[wrow * 2 + 0] = m_r[hrow];
-        p.ws_ml[wrow * 2 + 1] = l_r[hrow];
+      if (wk == 0 && (lane & 3) == 0) {
+        p.ws_ml[wrow * 2 + 0] = mf[hrow];
+        p.ws_ml[wrow * 2 + 1] = lf[hrow];
       }
     }
   }
-  }  // wk == 0
+
+  // fused step: the rest of steps 1-2 (off the attention's critical path)
+  if constexpr (FUSED) {
+    if (split == 0) {
+      if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits);
+      if (p.group_by_request) {
+        fused_group_append<CacheT>(p, cs_s, past_s, blockIdx.x / p.H_kv, h_kv, bits);
+      } else {
+        int tb = 0;
+        const int t = blockIdx.x / p.H_kv;
+        const TokenMeta m = token_meta_finish(app_tl, p.MB, p.bs, p.NB, tb);
+        fused_token_outputs(p, t, h_kv, m, tb, bits);
+        if (app_thread && m.slot >= 0) fused_store_row_vector<CacheT>(p, m.slot, h_kv, tid, NV, app_data);
+      }
+    }
+  }
+  flag(p.status, bits);
   if (p.num_splits > 1) finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
 }
 
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
+
+size_t mma_fused_extra_smem(int B);
 
 int mma_supported(int act, int cache, int D, int max_rows) {
   if (act != SPA_F16 && act != SPA_BF16) return 0;
@@ -542,43 +642,73 @@ int mma_supported(int act, int cache, int D, int max_rows) {
   return max_rows >= 1 && max_rows <= 128;
 }
 
-template <typename ActT, typename CacheT, int D, int RT, int KW>
+template <typename ActT, typename CacheT, int D, int RT, int KW, bool FUSED>
 static int launch_rt(const AttnParams& p, cudaStream_t stream) {
   using C = MmaCfg<ActT, CacheT, D, RT, KW>;
-  auto kern = decode_mma_kernel<ActT, CacheT, D, RT, KW>;
-  if (C::SMEM > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  auto kern = decode_mma_kernel<ActT, CacheT, D, RT, KW, FUSED>;
+  const size_t smem = C::SMEM + (FUSED ? mma_fused_extra_smem(p.B) : 0);
+  if (smem > 227 * 1024) return SPA_ERR_UNSUPPORTED;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
   dim3 grid(units, p.num_splits);
-  return launch_pdl(kern, grid, dim3(C::NT), C::SMEM, stream, p);
+  return launch_pdl(kern, grid, dim3(C::NT), smem, stream, p);
 }
 
-template <typename ActT, typename CacheT, int D>
+template <typename ActT, typename CacheT, int D, bool FUSED>
 static int launch_d(const AttnParams& p, int max_rows, cudaStream_t stream) {
   const int rt = (max_rows + 15) / 16;
   switch (rt) {
-    case 1: return launch_rt<ActT, CacheT, D, 1, 4>(p, stream);
-    case 2: return launch_rt<ActT, CacheT, D, 2, 2>(p, stream);
-    case 3: return launch_rt<ActT, CacheT, D, 3, 1>(p, stream);
-    case 4: return launch_rt<ActT, CacheT, D, 4, 1>(p, stream);
+    case 1: return launch_rt<ActT, CacheT, D, 1, 4, FUSED>(p, stream);
+    case 2: return launch_rt<ActT, CacheT, D, 2, 2, FUSED>(p, stream);
+    case 3: return launch_rt<ActT, CacheT, D, 3, 1, FUSED>(p, stream);
+    case 4: return launch_rt<ActT, CacheT, D, 4, 1, FUSED>(p, stream);
     case 5:
-    case 6: return launch_rt<ActT, CacheT, D, 6, 1>(p, stream);
-    default: return launch_rt<ActT, CacheT, D, 8, 1>(p, stream);
+    case 6: return launch_rt<ActT, CacheT, D, 6, 1, FUSED>(p, stream);
+    default: return launch_rt<ActT, CacheT, D, 8, 1, FUSED>(p, stream);
   }
 }
 
-template <typename ActT, typename CacheT>
+template <typename ActT, typename CacheT, bool FUSED>
 static int launch_dd(const AttnParams& p, int max_rows, cudaStream_t stream) {
-  if (p.D == 64) return launch_d<ActT, CacheT, 64>(p, max_rows, stream);
-  return launch_d<ActT, CacheT, 128>(p, max_rows, stream);
+  if (p.D == 64) return launch_d<ActT, CacheT, 64, FUSED>(p, max_rows, stream);
+  return launch_d<ActT, CacheT, 128, FUSED>(p, max_rows, stream);
 }
 
 int launch_attention_mma(const AttnParams& p, int act, int cache, int max_rows, cudaStream_t stream) {
   if (act == SPA_F16) {
-    if (cache == SPA_I8) return launch_dd<__half, int8_t>(p, max_rows, stream);
-    return launch_dd<__half, __half>(p, max_rows, stream);
+    if (cache == SPA_I8) return launch_dd<__half, int8_t, false>(p, max_rows, stream);
+    return launch_dd<__half, __half, false>(p, max_rows, stream);
   }
-  if (cache == SPA_I8) return launch_dd<__nv_bfloat16, int8_t>(p, max_rows, stream);
-  return launch_dd<__nv_bfloat16, __nv_bfloat16>(p, max_rows, stream);
+  if (cache == SPA_I8) return launch_dd<__nv_bfloat16, int8_t, false>(p, max_rows, stream);
+  return launch_dd<__nv_bfloat16, __nv_bfloat16, false>(p, max_rows, stream);
+}
+
+// Shared memory the fused step adds: cumulative lengths [B + 1] and past lengths [B].
+size_t mma_fused_extra_smem(int B) { return sizeof(int32_t) * (size_t)(2 * B + 1); }
+
+// Whether the fused step fits one CTA's shared memory (16-bit caches).
+template <int D>
+static size_t smem_rt(int rt) {
+  switch (rt) {
+    case 1: return MmaCfg<__half, __half, D, 1, 4>::SMEM;
+    case 2: return MmaCfg<__half, __half, D, 2, 2>::SMEM;
+    case 3: return MmaCfg<__half, __half, D, 3, 1>::SMEM;
+    case 4: return MmaCfg<__half, __half, D, 4, 1>::SMEM;
+    case 5:
+    case 6: return MmaCfg<__half, __half, D, 6, 1>::SMEM;
+    default: return MmaCfg<__half, __half, D, 8, 1>::SMEM;
+  }
+}
+int mma_step_fits(int D, int max_rows, int B) {
+  const int rt = (max_rows + 15) / 16;
+  const size_t base = D == 64 ? smem_rt<64>(rt) : smem_rt<128>(rt);
+  return base + mma_fused_extra_smem(B) <= 227 * 1024;
+}
+
+// The whole step in one launch (16-bit caches whose dtype is the activations').
+int launch_step_mma(const AttnParams& p, int act, int max_rows, cudaStream_t stream) {
+  if (act == SPA_F16) return launch_dd<__half, __half, true>(p, max_rows, stream);
+  return launch_dd<__nv_bfloat16, __nv_bfloat16, true>(p, max_rows, stream);
 }
 
 }  // namespace spa

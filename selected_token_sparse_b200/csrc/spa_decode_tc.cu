@@ -209,6 +209,9 @@ decode_tc_kernel(const AttnParams p) {
         qv[k] = *reinterpret_cast<const uint4*>(q + ((long long)(t0 + r / G) * p.H_q + h_kv * G + r % G) * D + u * 8);
     }
   }
+  // the epilogue's sink logit of row `row`, in flight from here
+  const float sink_raw = (p.sinks && p.num_splits == 1 && row < R) ? ld_early(p.sinks + h_kv * G + row % G)
+                                                                   : -INFINITY;
   if (ntiles > 0) resolve_chunk(0);
   tc_fence_before();
   __syncthreads();
@@ -453,7 +456,7 @@ decode_tc_kernel(const AttnParams p) {
   const bool mine = row < R;
   float f = 1.f, lse = -INFINITY;
   if (p.num_splits == 1) {
-    const float sink2 = (p.sinks && mine) ? p.sinks[h] * kLog2e : -INFINITY;
+    const float sink2 = (p.sinks && mine) ? sink_raw * kLog2e : -INFINITY;
     float a, inv_l;
     finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
     f = a * inv_l;

@@ -1,0 +1,220 @@
+// Step 1 helpers shared by the metadata kernels and the fused step kernel:
+// the sanitised cumulative lengths, the per-request outputs and the per-token
+// (request, position, slot) metadata ("[WebGPU] Add PagedAttention metadata
+// and GPT-OSS support", Description and Changes; "[WebGPU] Add
+// SparsePagedAttention", review notes on the per-token scan and on malformed
+// cumulative lengths).  Every caller runs this same code, so their outputs
+// agree bit for bit.
+#pragma once
+
+#include "spa_attn.cuh"
+
+namespace spa {
+
+// Sanitised cumulative lengths into cs[0..B] (all threads of the block).
+template <int NT>
+__device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, int T, int32_t* cs) {
+  __shared__ int32_t warp_max[NT / 32];
+  __shared__ int32_t chunk_carry[NT];
+  const int tid = threadIdx.x;
+  const int n = B + 1;
+  // contiguous chunk per thread: local prefix max, then a scan over chunk maxima
+  const int per = (n + NT - 1) / NT;
+  const int c0 = tid * per;
+  const int c1 = min(c0 + per, n);
+  int run = 0;  // cs[0] = 0 takes part in the maximum
+  for (int i = c0; i < c1; ++i) {
+    int v = (i == 0) ? 0 : cu[i];
+    run = max(run, v);
+    cs[i] = run;
+  }
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = (c0 < c1) ? run : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x = max(x, y);
+  }
+  if (lane == 31) warp_max[warp] = x;
+  __syncthreads();
+  int prev_warps = 0;
+  for (int w = 0; w < warp; ++w) prev_warps = max(prev_warps, warp_max[w]);
+  chunk_carry[tid] = max(x, prev_warps);
+  __syncthreads();
+  const int carry = (tid == 0) ? 0 : chunk_carry[tid - 1];
+  for (int i = c0; i < c1; ++i) cs[i] = min(max(cs[i], carry), T);
+  __syncthreads();
+}
+
+// seqlen_k of a request: past + q_len - 1 (past < 0 counts as 0), as int32.
+__device__ __forceinline__ int32_t request_seqlen_k(int past, int q_len) {
+  return (int32_t)((long long)max(past, 0) + q_len - 1);
+}
+
+// Per-request outputs and the request-level status bits (block 0 only).
+__device__ __forceinline__ int per_request(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
+                                           const int32_t* cs, int B, int T, int max_q, int max_k,
+                                           int32_t* __restrict__ seqlens_q, int32_t* __restrict__ seqlen_k) {
+  int bits = 0;
+  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
+    if (cu[b] != cs[b]) bits |= kStBadCu;
+    if (b == B && cs[B] != T) bits |= kStBadCu;
+  }
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    int pb = past[b];
+    if (pb < 0) {
+      bits |= kStBadCu;
+      pb = 0;
+    }
+    const int q_len = cs[b + 1] - cs[b];
+    const long long total = (long long)pb + q_len;
+    seqlens_q[b] = q_len;
+    seqlen_k[b] = request_seqlen_k(pb, q_len);
+    if (q_len > max_q || total > (long long)max_k) bits |= kStBounds;
+  }
+  return bits;
+}
+
+struct TokenMeta {
+  int b, pos, slot;
+};
+
+// Owner request (-1 if none) and absolute position (-1 if none) of token t.
+__device__ __forceinline__ void token_owner(int t, const int32_t* cs, int B, const int32_t* past, int& b,
+                                            int& pos) {
+  int lo = 0, hi = B + 1;  // owner = upper_bound(cs[0..B], t) - 1
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (cs[mid] <= t) lo = mid + 1; else hi = mid;
+  }
+  b = lo - 1;
+  pos = -1;
+  if (t >= cs[B] || b < 0 || b >= B) {
+    b = -1;
+    return;
+  }
+  pos = max(past[b], 0) + (t - cs[b]);
+}
+
+// Token metadata in two halves so that the block-table load can be in flight
+// while other work runs: the load half finds the owner and position and reads
+// the block id, the finish half validates it (status bits) and forms the slot.
+struct TokenLoad {
+  int b, pos, lb, blk;
+};
+
+__device__ __forceinline__ TokenLoad token_meta_load(int t, const int32_t* cs, int B, const int32_t* past,
+                                                     const int32_t* __restrict__ block_table, int MB, int bs) {
+  TokenLoad l;
+  token_owner(t, cs, B, past, l.b, l.pos);
+  l.lb = -1;
+  l.blk = -1;
+  if (l.b >= 0) {
+    l.lb = l.pos / bs;
+    if (l.lb < MB) l.blk = ld_early(block_table + (long long)l.b * MB + l.lb);
+  }
+  return l;
+}
+
+__device__ __forceinline__ TokenMeta token_meta_finish(const TokenLoad& l, int MB, int bs, int num_blocks,
+                                                       int& bits) {
+  TokenMeta m = {-1, -1, -1};
+  if (l.b < 0) return m;
+  m.b = l.b;
+  m.pos = l.pos;
+  if (l.lb >= MB) bits |= kStCapacity;
+  else if (l.blk < 0 || l.blk >= num_blocks) bits |= kStBadBlock;
+  else m.slot = l.blk * bs + l.pos % bs;
+  return m;
+}
+
+// Owner request, absolute position and cache slot of token t.
+__device__ __forceinline__ TokenMeta token_meta(int t, const int32_t* cs, int B,
+                                                const int32_t* __restrict__ past,
+                                                const int32_t* __restrict__ block_table, int MB, int bs,
+                                                int num_blocks, int& bits) {
+  return token_meta_finish(token_meta_load(t, cs, B, past, block_table, MB, bs), MB, bs, num_blocks, bits);
+}
+
+// Step-1 metadata computed in shared memory by the fused step kernel from
+// the raw cumulative lengths, their sanitised form cs and the past lengths,
+// with the same helpers as the metadata kernels.
+struct FusedMeta {
+  const int32_t* cu_raw;
+  const int32_t* cs;
+  const int32_t* past;
+  int B;
+  __device__ __forceinline__ int cu(int g) const { return cu_raw[g]; }
+  __device__ __forceinline__ int seqlens_q(int b) const { return cs[b + 1] - cs[b]; }
+  __device__ __forceinline__ int seqlen_k(int b) const { return request_seqlen_k(past[b], cs[b + 1] - cs[b]); }
+  __device__ __forceinline__ void token(int t, int& b, int& pos) const { token_owner(t, cs, B, past, b, pos); }
+};
+
+// Candidate offsets of a fused step that address k_new / v_new rather than
+// the cache carry this bit.
+constexpr long long kNewRow = 1LL << 62;
+
+// Steps 1 and 2 inside the attention CTAs of a fused step.
+//
+// Request-level part (CTA 0 of split 0): the per-request outputs and, with
+// request-grouped units, the metadata of tokens no request owns.
+__device__ __forceinline__ void fused_request_outputs(const AttnParams& p, const int32_t* cs, const int32_t* past,
+                                                      int& bits) {
+  bits |= per_request(p.cu, past, cs, p.B, p.T, p.max_seqlen_q, p.max_seqlen_k, p.seqlens_q_out,
+                      p.seqlen_k_out);
+  if (p.group_by_request) {
+    for (int t = cs[p.B] + threadIdx.x; t < p.T; t += blockDim.x) {
+      p.token_batch_out[t] = -1;
+      p.token_pos_out[t] = -1;
+      p.slot_out[t] = -1;
+    }
+  }
+}
+
+// Token-level part for token t and kv head h_kv (split 0): the token's
+// metadata, written by kv head 0.
+__device__ __forceinline__ void fused_token_outputs(const AttnParams& p, int t, int h_kv, const TokenMeta& m,
+                                                    int tb, int& bits) {
+  if (h_kv == 0 && threadIdx.x == 0) {
+    bits |= tb;
+    p.token_batch_out[t] = m.b;
+    p.token_pos_out[t] = m.pos;
+    p.slot_out[t] = m.slot;
+  }
+}
+
+// The token's K/V rows of one kv head go to the cache as 16-byte vectors (an
+// exact copy for 16-bit caches): vector v < nv of the K row, v - nv of the V row.
+template <typename T16>
+__device__ __forceinline__ void fused_store_row_vector(const AttnParams& p, int slot, int h_kv, int v, int nv,
+                                                       const uint4& data) {
+  const bool isv = v >= nv;
+  uint4* dp = reinterpret_cast<uint4*>(static_cast<T16*>(const_cast<void*>(isv ? p.v_cache : p.k_cache)) +
+                                       ((long long)slot * p.H_kv + h_kv) * p.D);
+  dp[isv ? v - nv : v] = data;
+}
+
+template <typename T16>
+__device__ __forceinline__ uint4 fused_load_row_vector(const AttnParams& p, int t, int h_kv, int v, int nv) {
+  const bool isv = v >= nv;
+  const uint4* sp = reinterpret_cast<const uint4*>(static_cast<const T16*>(isv ? p.v_new : p.k_new) +
+                                                   ((long long)t * p.H_kv + h_kv) * p.D);
+  return ld_early(sp + (isv ? v - nv : v));
+}
+
+// Request-grouped units: every token of the unit's request, at the end of the CTA.
+template <typename T16>
+__device__ __forceinline__ void fused_group_append(const AttnParams& p, const int32_t* cs, const int32_t* past,
+                                                   int b, int h_kv, int& bits) {
+  const int nv = p.D * (int)sizeof(T16) / 16;
+  for (int t = cs[b]; t < cs[b + 1]; ++t) {
+    int tb = 0;
+    const TokenMeta m = token_meta(t, cs, p.B, past, p.block_table, p.MB, p.bs, p.NB, tb);
+    fused_token_outputs(p, t, h_kv, m, tb, bits);
+    if (m.slot < 0) continue;
+    for (int v = threadIdx.x; v < 2 * nv; v += blockDim.x)
+      fused_store_row_vector<T16>(p, m.slot, h_kv, v, nv, fused_load_row_vector<T16>(p, t, h_kv, v, nv));
+  }
+}
+
+}  // namespace spa

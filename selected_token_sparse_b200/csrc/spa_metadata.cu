@@ -18,98 +18,11 @@
 // then copy its rows as 16-byte vectors, quantising for an INT8 cache); its
 // outputs are bit-identical to spa_prepare_metadata followed by spa_append_kv.
 #include "spa_attn.cuh"
+#include "spa_meta.cuh"
 
 namespace spa {
 
 constexpr int kMetaThreads = 256;
-
-// Sanitised cumulative lengths into cs[0..B] (all threads of the block).
-__device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, int T, int32_t* cs) {
-  __shared__ int32_t warp_max[kMetaThreads / 32];
-  __shared__ int32_t chunk_carry[kMetaThreads];
-  const int tid = threadIdx.x;
-  const int n = B + 1;
-  // contiguous chunk per thread: local prefix max, then a scan over chunk maxima
-  const int per = (n + kMetaThreads - 1) / kMetaThreads;
-  const int c0 = tid * per;
-  const int c1 = min(c0 + per, n);
-  int run = 0;  // cs[0] = 0 takes part in the maximum
-  for (int i = c0; i < c1; ++i) {
-    int v = (i == 0) ? 0 : cu[i];
-    run = max(run, v);
-    cs[i] = run;
-  }
-  const int lane = tid & 31, warp = tid >> 5;
-  int x = (c0 < c1) ? run : 0;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x = max(x, y);
-  }
-  if (lane == 31) warp_max[warp] = x;
-  __syncthreads();
-  int prev_warps = 0;
-  for (int w = 0; w < warp; ++w) prev_warps = max(prev_warps, warp_max[w]);
-  chunk_carry[tid] = max(x, prev_warps);
-  __syncthreads();
-  const int carry = (tid == 0) ? 0 : chunk_carry[tid - 1];
-  for (int i = c0; i < c1; ++i) cs[i] = min(max(cs[i], carry), T);
-  __syncthreads();
-}
-
-// Per-request outputs and the request-level status bits (block 0 only).
-__device__ __forceinline__ int per_request(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
-                                           const int32_t* cs, int B, int T, int max_q, int max_k,
-                                           int32_t* __restrict__ seqlens_q, int32_t* __restrict__ seqlen_k) {
-  int bits = 0;
-  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
-    if (cu[b] != cs[b]) bits |= kStBadCu;
-    if (b == B && cs[B] != T) bits |= kStBadCu;
-  }
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    int pb = past[b];
-    if (pb < 0) {
-      bits |= kStBadCu;
-      pb = 0;
-    }
-    const int q_len = cs[b + 1] - cs[b];
-    const long long total = (long long)pb + q_len;
-    seqlens_q[b] = q_len;
-    seqlen_k[b] = (int32_t)(total - 1);
-    if (q_len > max_q || total > (long long)max_k) bits |= kStBounds;
-  }
-  return bits;
-}
-
-struct TokenMeta {
-  int b, pos, slot;
-};
-
-// Owner request, absolute position and cache slot of token t.
-__device__ __forceinline__ TokenMeta token_meta(int t, const int32_t* cs, int B,
-                                                const int32_t* __restrict__ past,
-                                                const int32_t* __restrict__ block_table, int MB, int bs,
-                                                int num_blocks, int& bits) {
-  TokenMeta m = {-1, -1, -1};
-  int lo = 0, hi = B + 1;  // owner = upper_bound(cs[0..B], t) - 1
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (cs[mid] <= t) lo = mid + 1; else hi = mid;
-  }
-  const int b = lo - 1;
-  if (t >= cs[B] || b < 0 || b >= B) return m;
-  m.b = b;
-  m.pos = max(past[b], 0) + (t - cs[b]);
-  const int lb = m.pos / bs;
-  if (lb >= MB) {
-    bits |= kStCapacity;
-  } else {
-    const int blk = block_table[(long long)b * MB + lb];
-    if (blk < 0 || blk >= num_blocks) bits |= kStBadBlock;
-    else m.slot = blk * bs + m.pos % bs;
-  }
-  return m;
-}
 
 __global__ void __launch_bounds__(kMetaThreads)
 prepare_metadata_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
@@ -121,7 +34,7 @@ prepare_metadata_kernel(const int32_t* __restrict__ cu, const int32_t* __restric
   extern __shared__ int32_t cs[];  // [B + 1]
   pdl_wait();
   pdl_trigger();
-  build_cs(cu, B, T, cs);
+  build_cs<kMetaThreads>(cu, B, T, cs);
   if (blockIdx.x == 0) flag(status, per_request(cu, past, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
   int bits = 0;
   for (int t = blockIdx.x * kMetaThreads + threadIdx.x; t < T; t += gridDim.x * kMetaThreads) {
@@ -219,7 +132,7 @@ prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict_
     }
   }
   for (int b = threadIdx.x; b < B; b += blockDim.x) past_s[b] = past[b];
-  build_cs(cu, B, T, cs);   // ends with a block barrier: past_s is visible too
+  build_cs<kMetaThreads>(cu, B, T, cs);   // ends with a block barrier: past_s is visible too
   if (blockIdx.x == 0) flag(status, per_request(cu, past_s, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
   int bits = 0;
   for (int t = t_first; t < T; t += gridDim.x * wpb) {

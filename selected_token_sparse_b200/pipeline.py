@@ -39,12 +39,22 @@ def attention_kwargs(wl, d: Dict[str, torch.Tensor]) -> dict:
                 v_scale=d.get("v_scale"))
 
 
+MODES = ("step", "prepare_append", "staged")
+
+
 class Step:
-    """Pre-allocated buffers for repeated steps of one workload on one device."""
+    """Pre-allocated buffers for repeated steps of one workload on one device.
+
+    mode "step": spa_prepare_append_attention (one launch where the path
+    allows it); "prepare_append": spa_prepare_append_kv then spa_attention;
+    "staged": spa_prepare_metadata, spa_append_kv, spa_attention.
+    """
 
     def __init__(self, wl, d: Dict[str, torch.Tensor], num_splits: int = 0,
-                 want_lse: bool = False, fused: bool = True):
-        self.wl, self.d = wl, d
+                 want_lse: bool = False, mode: str = "step"):
+        if mode not in MODES:
+            raise ValueError(f"mode must be one of {MODES}")
+        self.wl, self.d, self.mode = wl, d, mode
         dev = d["q"].device
         i32 = dict(dtype=torch.int32, device=dev)
         B, T = wl.B, wl.T
@@ -57,39 +67,45 @@ class Step:
         self.num_splits = num_splits
         self.kw = attention_kwargs(wl, d)
         meta = dict(self.meta, cu_seqlens_q=d["cu_seqlens_q"], status=self.status)
-        args = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], d["block_table"], meta,
-                                  max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
-                                  out=self.out, lse=self.lse, num_splits=num_splits, **self.kw)
-        self.workspace = spa.new_workspace(spa.workspace_size(args), dev)
-        self.fused = fused
+        self.args = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], d["block_table"], meta,
+                                       max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
+                                       out=self.out, lse=self.lse, num_splits=num_splits,
+                                       status=self.status, **self.kw)
+        self.workspace = spa.new_workspace(spa.workspace_size(self.args), dev)
+
+    def launches(self) -> int:
+        """Kernel launches one call makes."""
+        if self.mode == "step":
+            return spa.prepare_append_attention_launches(self.args)
+        return (1 if self.mode == "prepare_append" else 2) + spa.attention_plan(self.args)["launches"]
 
     def __call__(self):
         wl, d = self.wl, self.d
-        if self.fused:
-            meta = spa.prepare_append_kv(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],
-                                         wl.T, wl.max_seqlen_q, wl.max_seqlen_k, d["k_new"],
-                                         d["v_new"], d["k_cache"], d["v_cache"],
-                                         k_scale=d.get("k_scale"), v_scale=d.get("v_scale"),
-                                         status=self.status, out=self.meta)
+        if self.mode == "step":
+            spa.run_prepare_append_attention(self.args, d["past_seqlens"], d["k_new"], d["v_new"],
+                                             self.meta["slot_mapping"], self.workspace)
+            return self.out
+        if self.mode == "prepare_append":
+            spa.prepare_append_kv(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],
+                                  wl.T, wl.max_seqlen_q, wl.max_seqlen_k, d["k_new"],
+                                  d["v_new"], d["k_cache"], d["v_cache"],
+                                  k_scale=d.get("k_scale"), v_scale=d.get("v_scale"),
+                                  status=self.status, out=self.meta)
         else:
-            meta = spa.prepare_metadata(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],
-                                        wl.T, wl.max_seqlen_q, wl.max_seqlen_k, wl.block_size,
-                                        wl.NB, status=self.status, out=self.meta)
+            spa.prepare_metadata(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],
+                                 wl.T, wl.max_seqlen_q, wl.max_seqlen_k, wl.block_size,
+                                 wl.NB, status=self.status, out=self.meta)
             spa.append_kv(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"],
-                          meta["slot_mapping"], k_scale=d.get("k_scale"),
+                          self.meta["slot_mapping"], k_scale=d.get("k_scale"),
                           v_scale=d.get("v_scale"), status=self.status)
-        a = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], d["block_table"], meta,
-                               max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
-                               out=self.out, lse=self.lse, num_splits=self.num_splits,
-                               status=self.status, **self.kw)
-        spa.run_attention(a, self.workspace)
+        spa.run_attention(self.args, self.workspace)
         return self.out
 
 
-def run_step(wl, device="cuda", num_splits: int = 0, want_lse: bool = True, fused: bool = True):
+def run_step(wl, device="cuda", num_splits: int = 0, want_lse: bool = True, mode: str = "step"):
     """Run one step on fresh device copies; returns host numpy results."""
     d = to_device(wl, device)
-    st = Step(wl, d, num_splits=num_splits, want_lse=want_lse, fused=fused)
+    st = Step(wl, d, num_splits=num_splits, want_lse=want_lse, mode=mode)
     st()
     torch.cuda.synchronize(device)
     res = {k: v.cpu().numpy() for k, v in st.meta.items()}

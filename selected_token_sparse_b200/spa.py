@@ -78,6 +78,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spa_attention.argtypes = [ctypes.POINTER(AttentionArgs), _vp, ctypes.c_size_t, _vp]
     lib.spa_attention_plan.restype = ctypes.c_int
     lib.spa_attention_plan.argtypes = [ctypes.POINTER(AttentionArgs), _vp, _vp, _vp]
+    lib.spa_prepare_append_attention.restype = ctypes.c_int
+    lib.spa_prepare_append_attention.argtypes = [ctypes.POINTER(AttentionArgs), _vp, _vp, _vp, _vp, _vp,
+                                                 ctypes.c_size_t, _vp]
+    lib.spa_prepare_append_attention_launches.restype = ctypes.c_int
+    lib.spa_prepare_append_attention_launches.argtypes = [ctypes.POINTER(AttentionArgs)]
     lib.spa_error_string.restype = ctypes.c_char_p
     lib.spa_error_string.argtypes = [ctypes.c_int]
     return lib
@@ -256,6 +261,28 @@ def run_attention(args: AttentionArgs, workspace: Optional[torch.Tensor]) -> Non
     dev = workspace.device if workspace is not None else torch.device("cuda")
     rc = lib().spa_attention(ctypes.byref(args), ws, need, _stream(dev))
     _check(rc, "spa_attention")
+
+
+def run_prepare_append_attention(args: AttentionArgs, past_seqlens: torch.Tensor, k_new: torch.Tensor,
+                                 v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                                 workspace: Optional[torch.Tensor]) -> None:
+    """Enqueue steps 1-5 (spa_prepare_append_attention) for prepared arguments on the
+    current stream; the metadata arrays `args` points at are written."""
+    need = workspace_size(args)
+    if need and (workspace is None or workspace.numel() < need):
+        raise SpaError(SPA_ERR_WORKSPACE, "spa_prepare_append_attention")
+    rc = lib().spa_prepare_append_attention(ctypes.byref(args), _ptr(past_seqlens), _ptr(k_new),
+                                            _ptr(v_new), _ptr(slot_mapping), _ptr(workspace) if need else None,
+                                            need, _stream(k_new.device))
+    _check(rc, "spa_prepare_append_attention")
+
+
+def prepare_append_attention_launches(args: AttentionArgs) -> int:
+    """Kernel launches spa_prepare_append_attention makes for these arguments (1 or 2)."""
+    rc = int(lib().spa_prepare_append_attention_launches(ctypes.byref(args)))
+    if rc < 0:
+        _check(rc, "spa_prepare_append_attention_launches")
+    return rc
 
 
 def attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

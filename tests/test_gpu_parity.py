@@ -202,12 +202,16 @@ def _all_equal(a, b):
 
 
 @pytest.mark.parametrize("name", W.WORKLOADS)
-def test_fused_prepare_append_matches_staged(name):
+@pytest.mark.parametrize("mode", ["step", "prepare_append"])
+def test_fused_entry_points_match_staged(name, mode):
+    """spa_prepare_append_attention and spa_prepare_append_kv + spa_attention give
+    the staged sequence's metadata, caches, status, out and lse bit for bit."""
     wl = W.by_name(name, small=True)
-    a = run(wl, fused=True)
-    b = run(wl, fused=False)
+    a = run(wl, mode=mode)
+    b = run(wl, mode="staged")
     _all_equal(a, b)
     assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["lse"], b["lse"], equal_nan=True)
 
 
 @pytest.mark.parametrize("which", ["decreasing_cu", "bad_block", "capacity"])
@@ -221,7 +225,61 @@ def test_fused_prepare_append_malformed(which):
         a_["block_table"][2, 2] = wl.NB + 3
     else:
         a_["past_seqlens"][0] = wl.MB * wl.block_size - 1
-    _all_equal(run(wl, fused=True), run(wl, fused=False))
+    _all_equal(run(wl, mode="prepare_append"), run(wl, mode="staged"))
+
+
+def _step_launches(wl, **kw):
+    d = pipeline.to_device(wl)
+    return pipeline.Step(wl, d, **kw).launches()
+
+
+# One-launch step (warp-MMA decode on a 16-bit cache): metadata from the raw
+# cumulative lengths in every CTA, this step's own rows read from k_new / v_new.
+STEP_CASES = {
+    # GQA decode, one token per request (per-token units)
+    "decode_f16": dict(act="f16", B=4, H_q=16, H_kv=2, D=64, block_size=16, q_lens=[1, 1, 1, 1],
+                       past=[0, 15, 40, 200], window=32),
+    # several tokens per request, grouped by request: new rows of earlier tokens
+    # of the same request are read from k_new
+    "multi_token_grouped_bf16": dict(act="bf16", B=3, H_q=8, H_kv=2, D=128, block_size=16,
+                                     q_lens=[3, 1, 4], past=[5, 0, 30]),
+    # several tokens per request with per-token selections: per-token units
+    # reading other units' new rows from k_new
+    "multi_token_per_token_sel": dict(act="f16", B=2, H_q=8, H_kv=2, D=64, block_size=16,
+                                      q_lens=[3, 2], past=[10, 4], sel_mode="main", sel_per_request=0,
+                                      sel_width=12, sel_valid=10),
+    # malformed: decreasing cumulative lengths, a bad block id, a position past the table
+    "malformed_cu": dict(act="f16", B=3, H_q=8, H_kv=2, D=64, block_size=16, q_lens=[2, 1, 3],
+                         past=[20, 5, 40], window=8, spare_blocks=2),
+    "empty_request": dict(act="f16", B=3, H_q=8, H_kv=2, D=64, block_size=16, q_lens=[1, 0, 1],
+                          past=[7, 3, 0]),
+}
+
+
+@pytest.mark.parametrize("case", list(STEP_CASES))
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_step_matches_staged(case, splits):
+    wl = W.make_workload(seed=31, has_sinks=True, **STEP_CASES[case])
+    if case == "malformed_cu":
+        wl.arrays["cu_seqlens_q"][2] = 1
+        wl.arrays["block_table"][2, 2] = wl.NB + 3
+        wl.arrays["past_seqlens"][0] = wl.MB * wl.block_size - 1
+    assert _step_launches(wl, num_splits=splits) == 1
+    a = run(wl, mode="step", num_splits=splits)
+    b = run(wl, mode="staged", num_splits=splits)
+    _all_equal(a, b)
+    assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["lse"], b["lse"], equal_nan=True)
+    if case != "malformed_cu":
+        compare(wl, a, oracle_step(wl))
+
+
+def test_step_launch_counts():
+    assert _step_launches(W.by_name("gptoss_paged_decode_f16", small=True)) == 1
+    assert _step_launches(W.by_name("selected_decode_bf16", small=True)) == 1
+    assert _step_launches(W.by_name("tiny_decode_f32", small=True)) == 2        # fp32: scalar kernel
+    assert _step_launches(W.by_name("local_plus_selected_int8", small=True)) == 2
+    assert _step_launches(W.by_name("ragged_prefill_f16", small=True)) == 2
 
 
 @pytest.mark.parametrize("name", ["selected_decode_bf16", "local_plus_selected_int8"])
