@@ -161,13 +161,15 @@ decode_mma_kernel(const AttnParams p) {
     }
   };
   if (!p.group_by_request) load_q(blockIdx.x / p.H_kv, p.G);
-  // fused step, per-token unit, split 0: this thread's vector of the token's
-  // new K/V row is loaded now and stored into the cache at the end
+  // fused step, split 0: this thread's vector of the unit's first token's
+  // new K/V row is loaded early (a per-token unit knows its token now) and
+  // stored into the cache at the end
   constexpr int NV = D * 2 / 16;
-  const bool app_thread = FUSED && !p.group_by_request && blockIdx.y == 0 && tid < 2 * NV;
+  const bool app_thread = FUSED && blockIdx.y == 0 && tid < 2 * NV;
   uint4 app_data = make_uint4(0, 0, 0, 0);
   if constexpr (FUSED) {
-    if (app_thread) app_data = fused_load_row_vector<CacheT>(p, blockIdx.x / p.H_kv, blockIdx.x % p.H_kv, tid, NV);
+    if (app_thread && !p.group_by_request)
+      app_data = fused_load_row_vector<CacheT>(p, blockIdx.x / p.H_kv, blockIdx.x % p.H_kv, tid, NV);
   }
 
   Unit U;
@@ -188,8 +190,9 @@ decode_mma_kernel(const AttnParams p) {
     }
     if (p.group_by_request && !has_rows) {
       if (blockIdx.y == 0) {
+        const int b = blockIdx.x / p.H_kv;
         if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits);
-        fused_group_append<CacheT>(p, cs_s, past_s, blockIdx.x / p.H_kv, blockIdx.x % p.H_kv, bits);
+        fused_append_tokens<CacheT>(p, cs_s, past_s, cs_s[b], cs_s[b + 1], blockIdx.x % p.H_kv, bits);
       }
       flag(p.status, bits);
       return;
@@ -325,10 +328,21 @@ decode_mma_kernel(const AttnParams p) {
     if (s < ntiles) issue(s);
     cp_async_commit();
   }
+  // fused step, split 0: the first token of the unit (-1: none) and its
+  // block-table entry, in flight until the end
+  int app_t = -1;
   TokenLoad app_tl;
   if constexpr (FUSED) {
-    if (!p.group_by_request && split == 0)
-      app_tl = token_meta_load(blockIdx.x / p.H_kv, cs_s, p.B, past_s, p.block_table, p.MB, p.bs);
+    if (split == 0) {
+      if (!p.group_by_request) {
+        app_t = blockIdx.x / p.H_kv;
+      } else {
+        const int b = blockIdx.x / p.H_kv;
+        if (cs_s[b + 1] > cs_s[b]) app_t = cs_s[b];
+        if (app_t >= 0 && app_thread) app_data = fused_load_row_vector<CacheT>(p, app_t, h_kv, tid, NV);
+      }
+      if (app_t >= 0) app_tl = token_meta_load(app_t, cs_s, p.B, past_s, p.block_table, p.MB, p.bs);
+    }
   }
   __syncthreads();
   // Q fragments for this warp's row tile stay in registers (16-bit caches)
@@ -614,14 +628,16 @@ decode_mma_kernel(const AttnParams p) {
   if constexpr (FUSED) {
     if (split == 0) {
       if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits);
-      if (p.group_by_request) {
-        fused_group_append<CacheT>(p, cs_s, past_s, blockIdx.x / p.H_kv, h_kv, bits);
-      } else {
+      if (app_t >= 0) {
         int tb = 0;
-        const int t = blockIdx.x / p.H_kv;
         const TokenMeta m = token_meta_finish(app_tl, p.MB, p.bs, p.NB, tb);
-        fused_token_outputs(p, t, h_kv, m, tb, bits);
+        fused_token_outputs(p, app_t, h_kv, m, tb, bits);
         if (app_thread && m.slot >= 0) fused_store_row_vector<CacheT>(p, m.slot, h_kv, tid, NV, app_data);
+        // a request-grouped unit's further tokens
+        if (p.group_by_request) {
+          const int b = blockIdx.x / p.H_kv;
+          fused_append_tokens<CacheT>(p, cs_s, past_s, app_t + 1, cs_s[b + 1], h_kv, bits);
+        }
       }
     }
   }

@@ -202,12 +202,12 @@ __device__ __forceinline__ uint4 fused_load_row_vector(const AttnParams& p, int 
   return ld_early(sp + (isv ? v - nv : v));
 }
 
-// Request-grouped units: every token of the unit's request, at the end of the CTA.
+// Tokens [t_lo, t_hi) of a unit, metadata and rows loaded where they are used.
 template <typename T16>
-__device__ __forceinline__ void fused_group_append(const AttnParams& p, const int32_t* cs, const int32_t* past,
-                                                   int b, int h_kv, int& bits) {
+__device__ __forceinline__ void fused_append_tokens(const AttnParams& p, const int32_t* cs, const int32_t* past,
+                                                    int t_lo, int t_hi, int h_kv, int& bits) {
   const int nv = p.D * (int)sizeof(T16) / 16;
-  for (int t = cs[b]; t < cs[b + 1]; ++t) {
+  for (int t = t_lo; t < t_hi; ++t) {
     int tb = 0;
     const TokenMeta m = token_meta(t, cs, p.B, past, p.block_table, p.MB, p.bs, p.NB, tb);
     fused_token_outputs(p, t, h_kv, m, tb, bits);
