@@ -57,6 +57,7 @@ struct AttnParams {
   int32_t* slot_out;
   int max_seqlen_q;      // host bounds for the step-1 status bits
   int max_seqlen_k;
+  int cluster_merge;     // 1: the splits of a unit are one cluster, merged in shared memory
 };
 
 // Programmatic dependent launch: let the next kernel in the stream be
@@ -297,6 +298,81 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, 
         store4<ActT>(static_cast<ActT*>(p.out) + rw[j] * D + (ii[j] % C4) * 4, o[j].x * inv, o[j].y * inv,
                      o[j].z * inv, o[j].w * inv);
       }
+    }
+    __syncthreads();
+  }
+}
+
+// Split merge through distributed shared memory.  The num_splits CTAs of a
+// unit form one cluster (rank = split); each has left its partial state at
+// the same shared-memory offsets: o [rows][D + 4] fp32 (row stride D + 4) and
+// (m, l) [rows][2], log2 units.  After a cluster barrier, CTA k merges rows
+// k, k + S, k + 2S, ... with the sink exactly as merge_rows does (pass 1: one
+// thread per row; pass 2: one thread per 4 output columns), reading the peers'
+// shared memory.  The caller ends with another cluster barrier so that no CTA
+// leaves while its state is being read.
+constexpr int kClusterMaxSplits = 8;
+
+template <typename ActT, int D>
+__device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, int nq, int h_kv,
+                                                   const float* part_o, const float* part_ml) {
+  __shared__ float sW[kMergeRows][kClusterMaxSplits];
+  __shared__ float sInv[kMergeRows];
+  constexpr int C4 = D / 4, PS = D + 4;
+  const int S = p.num_splits, k = (int)cluster_rank();
+  const int R = nq * p.G;
+  const int mine = R > k ? (R - k + S - 1) / S : 0;   // rows k, k + S, ...
+  for (int i0 = 0; i0 < mine; i0 += kMergeRows) {
+    const int n = min(kMergeRows, mine - i0);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int r = k + (i0 + i) * S;
+      const int h = h_kv * p.G + r % p.G;
+      const long long row = (long long)(t0 + r / p.G) * p.H_q + h;
+      const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+      float2 ml[kClusterMaxSplits];
+      float M = sink2;
+#pragma unroll
+      for (int s = 0; s < kClusterMaxSplits; ++s) {
+        ml[s] = make_float2(-INFINITY, 0.f);
+        if (s < S) ml[s] = ld_peer2(peer_smem(part_ml + 2 * r, s));
+        M = fmaxf(M, ml[s].x);
+      }
+      float inv = 0.f, lse = -INFINITY;
+      if (M != -INFINITY) {
+        float Lsum = (sink2 == -INFINITY) ? 0.f : exp2f(sink2 - M);
+#pragma unroll
+        for (int s = 0; s < kClusterMaxSplits; ++s) {
+          const float w = (ml[s].x == -INFINITY) ? 0.f : exp2f(ml[s].x - M);
+          sW[i][s] = w;
+          Lsum += w * ml[s].y;
+        }
+        inv = 1.0f / Lsum;
+        lse = (M + log2f(Lsum)) * kLn2;
+      } else {
+#pragma unroll
+        for (int s = 0; s < kClusterMaxSplits; ++s) sW[i][s] = 0.f;
+      }
+      sInv[i] = inv;
+      if (p.lse) p.lse[row] = lse;
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < n * C4; it += blockDim.x) {
+      const int i = it / C4, c = (it % C4) * 4;
+      const int r = k + (i0 + i) * S;
+      const long long row = (long long)(t0 + r / p.G) * p.H_q + h_kv * p.G + r % p.G;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < kClusterMaxSplits; ++s) {
+        if (s >= S) break;
+        const float w = sW[i][s];
+        const float4 a = ld_peer4(peer_smem(part_o + r * PS + c, s));
+        o.x = fmaf(w, a.x, o.x);
+        o.y = fmaf(w, a.y, o.y);
+        o.z = fmaf(w, a.z, o.z);
+        o.w = fmaf(w, a.w, o.w);
+      }
+      const float inv = sInv[i];
+      store4<ActT>(static_cast<ActT*>(p.out) + row * D + c, o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     }
     __syncthreads();
   }

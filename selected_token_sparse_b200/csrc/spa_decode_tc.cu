@@ -68,6 +68,11 @@ struct TcCfg {
   static constexpr int OFF_MISC = OFF_BAR + 16;                  // tmem holder
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;
+  // cluster split merge: partial o [128][D + 4] and (m, l) [128][2], fp32, over
+  // the K/V staging once every tile is consumed
+  static constexpr int OFF_PART = OFF_KV;
+  static constexpr int PART_ML = OFF_PART + 128 * (D + 4) * 4;
+  static_assert(PART_ML + 128 * 2 * 4 <= OFF_KV + KV_BYTES, "partial state must fit the K/V staging");
 };
 
 // byte offset of 16-byte unit u (0 .. D/8-1) of row r in a 128-row swizzled tile
@@ -482,6 +487,10 @@ decode_tc_kernel(const AttnParams p) {
       uint4* out = reinterpret_cast<uint4*>(static_cast<ActT*>(p.out) + orow * D + col);
 #pragma unroll
       for (int e = 0; e < 32; e += 8) out[e / 8] = pack8<ActT>(ov + e);
+    } else if (p.cluster_merge) {
+      float* po = reinterpret_cast<float*>(smem + C::OFF_PART) + row * (D + 4) + col;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(po + e) = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
     } else {
       float* acc = p.ws_acc + ((long long)split * p.T * p.H_q + orow) * D + col;
 #pragma unroll
@@ -491,6 +500,8 @@ decode_tc_kernel(const AttnParams p) {
   if (mine && half == 0) {
     if (p.num_splits == 1) {
       if (p.lse) p.lse[orow] = lse;
+    } else if (p.cluster_merge) {
+      *reinterpret_cast<float2*>(smem + C::PART_ML + row * 8) = make_float2(m_used, l_sum);
     } else {
       const long long wrow = (long long)split * p.T * p.H_q + orow;
       p.ws_ml[wrow * 2 + 0] = m_used;
@@ -504,7 +515,16 @@ decode_tc_kernel(const AttnParams p) {
     tc_fence_after();
     tmem_dealloc(tmem, kTcTmemCols);
   }
-  if (p.num_splits > 1) finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
+  if (p.num_splits > 1) {
+    if (p.cluster_merge) {
+      cluster_sync();
+      cluster_merge_rows<ActT, D>(p, t0, nq, h_kv, reinterpret_cast<const float*>(smem + C::OFF_PART),
+                                  reinterpret_cast<const float*>(smem + C::PART_ML));
+      cluster_sync();
+    } else {
+      finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
+    }
+  }
 }
 
 int tc_supported(int act, int cache, int D, int max_rows) {
@@ -521,6 +541,8 @@ static int launch_tc_t(const AttnParams& p, cudaStream_t stream) {
   auto kern = decode_tc_kernel<ActT, CacheT, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
+  if (p.cluster_merge)
+    return launch_pdl_cluster_y(kern, dim3(units, p.num_splits), dim3(kTcThreads), C::SMEM, stream, p.num_splits, p);
   return launch_pdl(kern, dim3(units, p.num_splits), dim3(kTcThreads), C::SMEM, stream, p);
 }
 
