@@ -138,31 +138,43 @@ __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& U)
   return decode_unit_with(p, StagedMeta{p}, u, U);
 }
 
-// Resolve candidate c of a unit to a cache element offset (or -1) and a key position.
-// `from_aux` tells which store the offset addresses.  Status bits go to `bits`.
-__device__ __forceinline__ long long resolve_candidate(const AttnParams& p, const Unit& U, int c,
-                                                       int& kpos, bool& from_aux, int& bits) {
+// Resolve candidate c of a unit to a cache element offset (or -1) and a key
+// position, in three stages so that callers resolving several candidates per
+// thread can keep every stage's loads in flight together:
+//   cand_stage1 -> the raw selection entry (selected modes) or the position;
+//   cand_stage2 -> the block id of a main-cache key (or -1);
+//   cand_finish -> guards (status bits), key position and element offset.
+// `from_aux` tells which store the offset addresses.
+__device__ __forceinline__ int cand_stage1(const AttnParams& p, const Unit& U, int c) {
+  if (c < U.n_main) return U.sel_main ? U.selrow[c] : U.lo + c;
+  return U.selrow[c - U.n_main];
+}
+
+__device__ __forceinline__ int cand_stage2(const AttnParams& p, const Unit& U, int c, int raw) {
+  if (c >= U.n_main) return -1;
+  if (U.sel_main && (raw < 0 || raw >= U.L)) return -1;
+  const int lb = raw / p.bs;
+  if (lb >= p.MB) return -1;
+  return p.block_table[(long long)U.b * p.MB + lb];
+}
+
+__device__ __forceinline__ long long cand_finish(const AttnParams& p, const Unit& U, int c, int raw, int blk,
+                                                 int& kpos, bool& from_aux, int& bits) {
   kpos = kPosInvalid;
   from_aux = false;
   if (c < U.n_main) {
-    int j;
     if (U.sel_main) {
-      const int idx = U.selrow[c];
-      if (idx == -1) return -1;
-      if (idx < -1 || idx >= U.L) {
+      if (raw == -1) return -1;
+      if (raw < -1 || raw >= U.L) {
         bits |= kStBadIdx;
         return -1;
       }
-      j = idx;
-    } else {
-      j = U.lo + c;
     }
-    const int lb = j / p.bs;
-    if (lb >= p.MB) {
+    const int j = raw;
+    if (j / p.bs >= p.MB) {
       bits |= kStCapacity;
       return -1;
     }
-    const int blk = p.block_table[(long long)U.b * p.MB + lb];
     if (blk < 0 || blk >= p.NB) {
       bits |= kStBadBlock;
       return -1;
@@ -170,15 +182,20 @@ __device__ __forceinline__ long long resolve_candidate(const AttnParams& p, cons
     kpos = j;
     return ((long long)blk * p.bs + (j % p.bs)) * p.H_kv * p.D + (long long)U.h_kv * p.D;
   }
-  const int idx = U.selrow[c - U.n_main];
-  if (idx == -1) return -1;
-  if (idx < -1 || idx >= U.aux_n) {
+  if (raw == -1) return -1;
+  if (raw < -1 || raw >= U.aux_n) {
     bits |= kStBadIdx;
     return -1;
   }
   kpos = kPosAux;
   from_aux = true;
-  return (((long long)U.b * p.aux_cap + idx) * p.H_kv + U.h_kv) * p.D;
+  return (((long long)U.b * p.aux_cap + raw) * p.H_kv + U.h_kv) * p.D;
+}
+
+__device__ __forceinline__ long long resolve_candidate(const AttnParams& p, const Unit& U, int c,
+                                                       int& kpos, bool& from_aux, int& bits) {
+  const int raw = cand_stage1(p, U, c);
+  return cand_finish(p, U, c, raw, cand_stage2(p, U, c, raw), kpos, from_aux, bits);
 }
 
 __device__ __forceinline__ bool key_visible(int kpos, int prow, int window) {

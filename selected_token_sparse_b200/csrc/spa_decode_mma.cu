@@ -269,12 +269,27 @@ decode_mma_kernel(const AttnParams p) {
   long long* cand_off = reinterpret_cast<long long*>(smem + C::OFF_CAND);
   int* cand_kpos = reinterpret_cast<int*>(smem + C::OFF_CAND + kMmaCandChunk * 8);
   auto resolve_chunk = [&](int first_tile) {
-    for (int i = tid; i < kMmaCandChunk; i += NT) {
-      const int cand = c_begin + first_tile * KT + i;
+    // every stage's loads of this thread's candidates are in flight together
+    constexpr int RPT = (kMmaCandChunk + NT - 1) / NT;
+    int raw[RPT], blk[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
+      raw[k] = (i < kMmaCandChunk && cand < c_end) ? cand_stage1(p, U, cand) : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
+      blk[k] = (i < kMmaCandChunk && cand < c_end) ? cand_stage2(p, U, cand, raw[k]) : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
+      if (i >= kMmaCandChunk) continue;
       int kp = kPosInvalid;
       bool from_aux = false;
       long long off = -1;
-      if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      if (cand < c_end) off = cand_finish(p, U, cand, raw[k], blk[k], kp, from_aux, bits);
       if constexpr (FUSED) {
         // this step's tokens: read the row the append writes from its source
         if (off >= 0 && kp >= U.new_lo && kp < U.new_hi)
@@ -459,9 +474,13 @@ decode_mma_kernel(const AttnParams p) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
     }
-    const float mn0 = fmaxf(m_r[0], mx0), mn1 = fmaxf(m_r[1], mx1);
-    const float al0 = (mn0 == -INFINITY) ? 1.f : ex2f(m_r[0] - mn0);
-    const float al1 = (mn1 == -INFINITY) ? 1.f : ex2f(m_r[1] - mn1);
+    // The reference max is raised only when a tile's max exceeds it by more
+    // than 8 (log2 units): p = 2^(s - m) then stays <= 256 (exact range in
+    // fp16 / bf16) and O is rescaled only on those tiles.
+    const bool up0 = mx0 > m_r[0] + 8.0f, up1 = mx1 > m_r[1] + 8.0f;
+    const float mn0 = up0 ? mx0 : m_r[0], mn1 = up1 ? mx1 : m_r[1];
+    const float al0 = (up0 && m_r[0] != -INFINITY) ? ex2f(m_r[0] - mn0) : 1.f;
+    const float al1 = (up1 && m_r[1] != -INFINITY) ? ex2f(m_r[1] - mn1) : 1.f;
     // masked scores are -inf and give 0 once the row max is finite
     const float ms0 = (mn0 == -INFINITY) ? 0.f : mn0, ms1 = (mn1 == -INFINITY) ? 0.f : mn1;
     m_r[0] = mn0;
@@ -479,12 +498,14 @@ decode_mma_kernel(const AttnParams p) {
     }
     l_r[0] = l_r[0] * al0 + ls0;
     l_r[1] = l_r[1] * al1 + ls1;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      o[n][0] *= al0;
-      o[n][1] *= al0;
-      o[n][2] *= al1;
-      o[n][3] *= al1;
+      for (int n = 0; n < D / 8; ++n) {
+        o[n][0] *= al0;
+        o[n][1] *= al0;
+        o[n][2] *= al1;
+        o[n][3] *= al1;
+      }
     }
     // O += P V
 #pragma unroll

@@ -189,12 +189,27 @@ decode_tc_kernel(const AttnParams p) {
   }
   int bits = 0;
   auto resolve_chunk = [&](int first_tile) {
-    for (int i = tid; i < kTcCand; i += NT) {
-      const int cand = c_begin + first_tile * KT + i;
+    // every stage's loads of this thread's candidates are in flight together
+    constexpr int RPT = kTcCand / NT;
+    static_assert(kTcCand % NT == 0, "candidates per thread");
+    int raw[RPT], blk[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int cand = c_begin + first_tile * KT + tid + k * NT;
+      raw[k] = cand < c_end ? cand_stage1(p, U, cand) : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int cand = c_begin + first_tile * KT + tid + k * NT;
+      blk[k] = cand < c_end ? cand_stage2(p, U, cand, raw[k]) : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
       int kp = kPosInvalid;
       bool from_aux = false;
       long long off = -1;
-      if (cand < c_end) off = resolve_candidate(p, U, cand, kp, from_aux, bits);
+      if (cand < c_end) off = cand_finish(p, U, cand, raw[k], blk[k], kp, from_aux, bits);
       cand_off[i] = off;
       cand_kpos[i] = kp;
     }
