@@ -36,6 +36,7 @@
 // Every mbarrier wait is bounded; on expiry the kernel sets SPA_ST_TIMEOUT,
 // the other roles give up at their next wait, the issuing thread drains its
 // copies and MMAs (bounded), the CTA frees its TMEM and returns.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -51,7 +52,7 @@ constexpr int kPfBM = 128;   // q rows per tile (TMEM lanes)
 constexpr int kPfBN = 128;   // keys per step
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint32_t kPfWaitLimit = 1u << 20;   // polls before a wait is declared lost
-constexpr int kPfThreads = 9 * 32;            // 2 softmax groups + the TMA / MMA warp
+constexpr int kPfThreads = 10 * 32;           // 2 softmax groups, the MMA warp, the K/V TMA warp
 
 template <int D>
 struct PfCfg {
@@ -63,7 +64,7 @@ struct PfCfg {
   static constexpr int OFF_K = OFF_QB + TILE;         // 2 stages
   static constexpr int OFF_V = OFF_K + 2 * TILE;      // 2 stages
   static constexpr int OFF_BAR = OFF_V + 2 * TILE;    // mbarriers
-  static constexpr int NBAR = 11;
+  static constexpr int NBAR = 15;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_FLAG = OFF_TMEM + 8;
   static constexpr int BYTES = OFF_FLAG + 8;
@@ -99,64 +100,71 @@ struct PfGeom {
   int q0[2], rows[2];   // per q tile: first row within the request, rows present (0 = absent)
 };
 
-// Block id of the cache block holding key `key` (or -1), with status bits for
-// keys that must exist (key < k_hi).
-__device__ __forceinline__ int pf_block(const AttnParams& p, int b, int key, bool needed, int& bits) {
-  const int lb = key / p.bs;
-  if (lb >= p.MB) {
-    if (needed) bits |= kStCapacity;
-    return -1;
-  }
-  const int blk = p.block_table[(long long)b * p.MB + lb];
-  if (blk < 0 || blk >= p.NB) {
-    if (needed) bits |= kStBadBlock;
-    return -1;
-  }
-  return blk;
+// Block id of box `lane` of the key tile starting at kb (-1 when the lane has
+// no box, the box lies beyond the table or the table holds -1); a volatile
+// load, so that it is issued here, a tile ahead of its use.
+__device__ __forceinline__ int pf_block_id(const AttnParams& p, int b, int kb, int lane, int nbox,
+                                           int box_shift) {
+  if (lane >= nbox) return -1;
+  const int lb = (kb + (lane << box_shift)) / p.bs;
+  return lb < p.MB ? ld_early(p.block_table + (long long)b * p.MB + lb) : -1;
 }
 
-// TMA loads of one K or V tile (keys [kb, kb + 128)) into `dst`.
-__device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g, const CUtensorMap* map,
-                                            unsigned char* dst, uint64_t* bar, int kb, int box_rows,
-                                            int nch, int& bits, uint32_t tx) {
-  mbar_arrive_expect_tx(bar, tx);
-  const int nbox = kPfBN / box_rows;
-  for (int i = 0; i < nbox; ++i) {
+// TMA loads of one key tile (keys [kb, kb + 128)) of K and of V, in boxes of
+// box_rows rows (one cache block, or 128 rows of one block).  The block ids of
+// all boxes are read first, as independent loads, and serve both tensors.
+__device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g, const CUtensorMap* map_k,
+                                            const CUtensorMap* map_v, unsigned char* dst_k,
+                                            unsigned char* dst_v, uint64_t* bar_k, uint64_t* bar_v, int kb,
+                                            int box_rows, int nch, int& bits, uint32_t tx) {
+  const int nbox = kPfBN / box_rows;   // <= 8 (block_size >= 16)
+  int raw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    raw[i] = -1;
+    if (i < nbox) {
+      const int lb = (kb + i * box_rows) / p.bs;
+      if (lb < p.MB) raw[i] = ld_early(p.block_table + (long long)g.b * p.MB + lb);
+    }
+  }
+  mbar_arrive_expect_tx(bar_k, tx);
+  mbar_arrive_expect_tx(bar_v, tx);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i >= nbox) break;
     const int key0 = kb + i * box_rows;
-    const int blk = pf_block(p, g.b, key0, key0 < g.k_hi, bits);
+    const bool needed = key0 < g.k_hi;
+    const int lb = key0 / p.bs;
+    int blk = -1;
+    if (lb >= p.MB) {
+      if (needed) bits |= kStCapacity;
+    } else if (raw[i] < 0 || raw[i] >= p.NB) {
+      if (needed) bits |= kStBadBlock;
+    } else {
+      blk = raw[i];
+    }
     const int cblk = blk >= 0 ? blk : p.NB;  // out of range: the box reads zeros
     const int row = key0 % p.bs;
-    for (int c = 0; c < nch; ++c)
-      tma_load_4d(dst + c * (128 * 128) + i * box_rows * 128, map, bar, c * 64, g.h_kv, row, cblk);
+    for (int c = 0; c < nch; ++c) {
+      tma_load_4d(dst_k + c * (128 * 128) + i * box_rows * 128, map_k, bar_k, c * 64, g.h_kv, row, cblk);
+      tma_load_4d(dst_v + c * (128 * 128) + i * box_rows * 128, map_v, bar_v, c * 64, g.h_kv, row, cblk);
+    }
   }
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kPfThreads, 1)
-prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                       int n_pairs, int box_rows, int box_shift, int max_tiles) {
-  using C = PfCfg<D>;
-  constexpr uint32_t FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
-  constexpr uint32_t IDESC_S = idesc_f16(FMT, kPfBM, kPfBN, 0);
-  constexpr uint32_t IDESC_O = idesc_f16(FMT, kPfBM, D, 1);
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  pdl_wait();
-  pdl_trigger();
-
-  // ---- geometry (uniform across the CTA)
-  PfGeom g;
-  g.h = blockIdx.x;
-  g.b = blockIdx.y;
-  const int pair = n_pairs - 1 - (int)blockIdx.z;
+// Geometry of work item `item` (q head, request, pair of 128-row q tiles;
+// items enumerate the longest pairs first).  Returns false for an empty item.
+__device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_pairs, int max_tiles, PfGeom& g) {
+  const int per_pair = p.H_q * p.B;
+  const int pz = item / per_pair, rem = item - pz * per_pair;
+  g.b = rem / p.H_q;
+  g.h = rem - g.b * p.H_q;
+  const int pair = n_pairs - 1 - pz;
   g.t_begin = clampi(p.cu[g.b], 0, p.T);
   g.q_len = clampi(p.seqlens_q[g.b], 0, p.T - g.t_begin);
   g.q0[0] = pair * 2 * kPfBM;
   g.q0[1] = g.q0[0] + kPfBM;
-  if (g.q0[0] >= g.q_len) return;
+  if (g.q0[0] >= g.q_len) return false;
   g.rows[0] = min(kPfBM, g.q_len - g.q0[0]);
   g.rows[1] = max(0, min(kPfBM, g.q_len - g.q0[1]));
   g.L = max(p.seqlen_k[g.b] + 1, 0);
@@ -170,8 +178,30 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   g.k_hi = min(p_last + 1, g.L);
   g.ntiles = g.k_hi > g.k_lo ? (g.k_hi - g.k_lo + kPfBN - 1) / kPfBN : 0;
   g.ntiles = min(g.ntiles, max_tiles);
-  const bool two = g.rows[1] > 0;   // the second q tile exists
-  const int ntq = two ? 2 : 1;
+  return true;
+}
+
+// Persistent: each CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+// The K/V ring and every barrier's phases run on across items (phases come
+// from counters, not step indices); the next item's Q is loaded as soon as
+// the current item's last P has been observed (its S MMAs are complete), and
+// a tile's first PV of an item waits until the softmax group has read the
+// previous item's O out of TMEM (bar_e).
+template <typename T, int D>
+__global__ void __launch_bounds__(kPfThreads, 1)
+prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       int n_pairs, int box_rows, int box_shift, int max_tiles, int n_items) {
+  using C = PfCfg<D>;
+  constexpr uint32_t FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t IDESC_S = idesc_f16(FMT, kPfBM, kPfBN, 0);
+  constexpr uint32_t IDESC_O = idesc_f16(FMT, kPfBM, D, 1);
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_trigger();
 
   unsigned char* const sQA = smem + C::OFF_QA;
   unsigned char* const sQB = smem + C::OFF_QB;
@@ -184,6 +214,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   uint64_t* bar_s = bars + 5;     // [2] S of tile A / B written
   uint64_t* bar_o = bars + 7;     // [2] PV of tile A / B done
   uint64_t* bar_p = bars + 9;     // [2] P of tile A / B in TMEM (4 warps arrive)
+  uint64_t* bar_e = bars + 11;    // [2] O of tile A / B read out by its epilogue (4 warps arrive)
+  uint64_t* bar_ke = bars + 13;   // [2] K/V stage empty (every MMA reading it is complete)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
 
@@ -195,6 +227,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       mbar_init(bar_s + i, 1);
       mbar_init(bar_o + i, 1);
       mbar_init(bar_p + i, 4);
+      mbar_init(bar_e + i, 4);
+      mbar_init(bar_ke + i, 1);
     }
     fence_mbar_init();
     *abort_flag = 0;
@@ -209,92 +243,174 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   const uint32_t tmem = *tmem_holder;
   int bits = 0;
 
-  if (warp == 8) {
-    // =================== TMA producer and MMA issuer (one thread) ===================
-    if (lane == 0 && g.ntiles > 0) {
-      prefetch_tmap(&tm_q);
+  // the next item, from `item` on, with key tiles (others need no tensor work)
+  auto next_work = [&](int& item, PfGeom& gg) {
+    while (item < n_items && !(pf_geom(p, item, n_pairs, max_tiles, gg) && gg.ntiles > 0)) item += gridDim.x;
+    return item < n_items;
+  };
+  if (warp == 9) {
+    // =================== K/V producer: the 2-stage ring over the CTA's key tiles ===================
+    // Tile c of the stream goes to stage c % 2 once the MMAs of tile c - 2 are
+    // complete (bar_ke), so the loads run ahead of the MMA warp.
+    if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(bar_q, ntq * C::TX_TILE);
-      for (int c = 0; c < C::NCH; ++c) {
-        tma_load_3d(sQA + c * C::CHUNK, &tm_q, bar_q, c * 64, g.h, g.t_begin + g.q0[0]);
-        if (two) tma_load_3d(sQB + c * C::CHUNK, &tm_q, bar_q, c * 64, g.h, g.t_begin + g.q0[1]);
-      }
-      int n_kv = 0;   // K/V tiles whose loads were issued
-      for (int j = 0; j < 2 && j < g.ntiles; ++j, ++n_kv) {
-        pf_issue_kv(p, g, &tm_k, sK + j * C::TILE, bar_kf + j, g.k_lo + j * kPfBN, box_rows, C::NCH, bits,
-                    C::TX_TILE);
-        pf_issue_kv(p, g, &tm_v, sV + j * C::TILE, bar_vf + j, g.k_lo + j * kPfBN, box_rows, C::NCH, bits,
-                    C::TX_TILE);
-      }
-      int n_s0 = 0, n_s1 = 0, n_o0 = 0, n_o1 = 0;   // commits issued per barrier
-      int kv_seen = 0;                        // K/V tiles whose arrival was observed
-      bool ok = mbar_wait(bar_q, 0, kPfWaitLimit, abort_flag);
-      const bool q_seen = ok;
-      for (int j = 0; j < g.ntiles && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        ok = mbar_wait(bar_kf + st, ph, kPfWaitLimit, abort_flag);
-        for (int t = 0; t < ntq && ok; ++t) {
-          // S_t of step j overwrites P_t of step j-1: PV_t(j-1) must be done
-          if (j > 0) ok = mbar_wait(bar_o + t, (j - 1) & 1, kPfWaitLimit, abort_flag);
+      int c = 0;
+      bool ok = true;
+      int item = blockIdx.x;
+      PfGeom g;
+      while (ok && next_work(item, g)) {
+        for (int j = 0; j < g.ntiles && ok; ++j) {
+          const int st = c & 1;
+          if (c >= 2) ok = mbar_wait(bar_ke + st, ((c >> 1) - 1) & 1, kPfWaitLimit, abort_flag);
           if (!ok) break;
-          tc_fence_after();
-          const uint32_t tS = tmem + t * 128;
-          unsigned char* const sq = t ? sQB : sQA;
+          pf_issue_kv(p, g, &tm_k, &tm_v, sK + st * C::TILE, sV + st * C::TILE, bar_kf + st, bar_vf + st,
+                      g.k_lo + j * kPfBN, box_rows, C::NCH, bits, C::TX_TILE);
+          ++c;
+        }
+        item += gridDim.x;
+      }
+      if (!ok) {   // the copies still in flight land before the CTA leaves (bounded)
+        *abort_flag = 1;
+        bits |= SPA_ST_TIMEOUT;
+        for (int k = c >= 2 ? c - 2 : 0; k < c; ++k) {
+          mbar_wait(bar_kf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
+          mbar_wait(bar_vf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // =================== MMA issuer and Q loads (one thread) ===================
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      auto issue_q = [&](const PfGeom& gg) {
+        const bool two = gg.rows[1] > 0;
+        mbar_arrive_expect_tx(bar_q, (two ? 2 : 1) * C::TX_TILE);
+        for (int c = 0; c < C::NCH; ++c) {
+          tma_load_3d(sQA + c * C::CHUNK, &tm_q, bar_q, c * 64, gg.h, gg.t_begin + gg.q0[0]);
+          if (two) tma_load_3d(sQB + c * C::CHUNK, &tm_q, bar_q, c * 64, gg.h, gg.t_begin + gg.q0[1]);
+        }
+      };
+      int c_use = 0;                              // key tiles consumed (stream index)
+      int q_iss = 0, q_seen = 0;
+      int s_iss[2] = {0, 0}, o_iss[2] = {0, 0}, o_seen[2] = {0, 0}, p_seen[2] = {0, 0};
+      int e_due[2] = {0, 0}, e_seen[2] = {0, 0}, ke_iss[2] = {0, 0};
+      int ci = blockIdx.x;
+      PfGeom g;
+      bool have = next_work(ci, g);
+      if (have) {
+        issue_q(g);
+        ++q_iss;
+      }
+      bool ok = true;
+      // wait for the outstanding PV of tile t (at most one)
+      auto pv_done = [&](int t) {
+        while (ok && o_seen[t] < o_iss[t]) {
+          ok = mbar_wait(bar_o + t, o_seen[t] & 1, kPfWaitLimit, abort_flag);
+          if (ok) ++o_seen[t];
+        }
+      };
+      // S_t = Q_t K^T for the key tile in `stage`
+      auto issue_s = [&](int t, int stage) {
+        tc_fence_after();
+        const uint32_t tS = tmem + t * 128;
+        unsigned char* const sq = t ? sQB : sQA;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int c = kk / 4, koff = (kk % 4) * 32;
-            const uint64_t ad = smem_desc_sw128(smem_u32(sq + c * C::CHUNK + koff), 16, 1024);
-            const uint64_t bd = smem_desc_sw128(smem_u32(sK + st * C::TILE + c * C::CHUNK + koff), 16, 1024);
-            mma_ss(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c = kk / 4, koff = (kk % 4) * 32;
+          const uint64_t ad = smem_desc_sw128(smem_u32(sq + c * C::CHUNK + koff), 16, 1024);
+          const uint64_t bd = smem_desc_sw128(smem_u32(sK + stage * C::TILE + c * C::CHUNK + koff), 16, 1024);
+          mma_ss(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_s + t);
+        ++s_iss[t];
+      };
+      // Per step j and q tile t: PV_t(j) as soon as P_t(j) is in TMEM, then
+      // S_t(j+1) once PV_t(j) is done -- each softmax group gets its next S
+      // without waiting for the other group, so one group's softmax overlaps
+      // the other's MMAs.
+      while (have && ok) {
+        const int ntq = g.rows[1] > 0 ? 2 : 1;
+        {   // step 0: S of every q tile (after the tile's previous PV)
+          const int st = c_use & 1;
+          const uint32_t ph = (c_use >> 1) & 1;
+          ok = mbar_wait(bar_kf + st, ph, kPfWaitLimit, abort_flag);
+          if (ok) {
+            ok = mbar_wait(bar_q, q_seen & 1, kPfWaitLimit, abort_flag);
+            if (ok) ++q_seen;
           }
-          tc_commit(bar_s + t);
-          if (t) ++n_s1; else ++n_s0;
+          for (int t = 0; t < ntq && ok; ++t) {
+            pv_done(t);   // S_t overwrites P_t of the tile's previous step
+            if (ok) issue_s(t, st);
+          }
+        }
+        for (int j = 0; j < g.ntiles && ok; ++j) {
+          const int st = c_use & 1;
+          const uint32_t ph = (c_use >> 1) & 1;
+          const bool more = j + 1 < g.ntiles;
+          const int st1 = (c_use + 1) & 1;
+          const uint32_t ph1 = ((c_use + 1) >> 1) & 1;
+          bool k_next = false;
+          ok = mbar_wait(bar_vf + st, ph, kPfWaitLimit, abort_flag);
+          for (int t = 0; t < ntq && ok; ++t) {
+            ok = mbar_wait(bar_p + t, p_seen[t] & 1, kPfWaitLimit, abort_flag);
+            if (ok) ++p_seen[t];
+            // the first PV of an item overwrites O_t: the previous epilogue must have read it
+            while (ok && j == 0 && e_seen[t] < e_due[t]) {
+              ok = mbar_wait(bar_e + t, e_seen[t] & 1, kPfWaitLimit, abort_flag);
+              if (ok) ++e_seen[t];
+            }
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tP = tmem + t * 128;
+            const uint32_t tO = tmem + 256 + t * 128;
+#pragma unroll
+            for (int kk = 0; kk < kPfBN / 16; ++kk) {
+              const uint64_t bd = smem_desc_sw128(smem_u32(sV + st * C::TILE + kk * 2048), C::CHUNK, 1024);
+              mma_ts(tO, tP + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(bar_o + t);
+            ++o_iss[t];
+            if (t == ntq - 1) {   // every MMA reading this stage is issued: it empties on completion
+              tc_commit(bar_ke + st);
+              ++ke_iss[st];
+            }
+            if (more) {
+              if (!k_next) {
+                ok = mbar_wait(bar_kf + st1, ph1, kPfWaitLimit, abort_flag);
+                k_next = true;
+              }
+              pv_done(t);   // P_t(j) consumed: S_t(j+1) may overwrite it
+              if (ok) issue_s(t, st1);
+            }
+          }
+          if (!ok) break;
+          ++c_use;
         }
         if (!ok) break;
-        // every MMA of step j-1 is complete here (PV of each tile of step j-1
-        // was waited on above), so step j+1's K and V may take that stage
-        if (j >= 1 && j + 1 < g.ntiles) {
-          const int s2 = (j + 1) & 1;
-          pf_issue_kv(p, g, &tm_k, sK + s2 * C::TILE, bar_kf + s2, g.k_lo + (j + 1) * kPfBN, box_rows, C::NCH,
-                      bits, C::TX_TILE);
-          pf_issue_kv(p, g, &tm_v, sV + s2 * C::TILE, bar_vf + s2, g.k_lo + (j + 1) * kPfBN, box_rows, C::NCH,
-                      bits, C::TX_TILE);
-          ++n_kv;
-        }
-        ok = mbar_wait(bar_vf + st, ph, kPfWaitLimit, abort_flag);
-        if (ok) kv_seen = j + 1;
-        for (int t = 0; t < ntq && ok; ++t) {
-          ok = mbar_wait(bar_p + t, j & 1, kPfWaitLimit, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t tP = tmem + t * 128;
-          const uint32_t tO = tmem + 256 + t * 128;
-#pragma unroll
-          for (int kk = 0; kk < kPfBN / 16; ++kk) {
-            const uint64_t bd = smem_desc_sw128(smem_u32(sV + st * C::TILE + kk * 2048), C::CHUNK, 1024);
-            mma_ts(tO, tP + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(bar_o + t);
-          if (t) ++n_o1; else ++n_o0;
+        for (int t = 0; t < ntq; ++t) ++e_due[t];
+        // every P of this item was observed, so its S MMAs are complete: Q may be replaced
+        ci += gridDim.x;
+        have = next_work(ci, g);
+        if (have) {
+          issue_q(g);
+          ++q_iss;
         }
       }
       if (!ok) {
         *abort_flag = 1;
         bits |= SPA_ST_TIMEOUT;
         // drain, bounded: the latest commit of each barrier covers every MMA
-        // issued before it; then the copies whose arrival was not observed
-        if (n_s0 > 0) mbar_wait(bar_s + 0, (n_s0 - 1) & 1, kPfWaitLimit);
-        if (n_s1 > 0) mbar_wait(bar_s + 1, (n_s1 - 1) & 1, kPfWaitLimit);
-        if (n_o0 > 0) mbar_wait(bar_o + 0, (n_o0 - 1) & 1, kPfWaitLimit);
-        if (n_o1 > 0) mbar_wait(bar_o + 1, (n_o1 - 1) & 1, kPfWaitLimit);
-        if (!q_seen) mbar_wait(bar_q, 0, kPfWaitLimit);
-        for (int j = kv_seen; j < n_kv; ++j) {
-          mbar_wait(bar_kf + (j & 1), (j >> 1) & 1, kPfWaitLimit);
-          mbar_wait(bar_vf + (j & 1), (j >> 1) & 1, kPfWaitLimit);
+        // issued before it; then the Q copies whose arrival was not observed
+        for (int t = 0; t < 2; ++t) {
+          if (s_iss[t] > 0) mbar_wait(bar_s + t, (s_iss[t] - 1) & 1, kPfWaitLimit);
+          if (o_iss[t] > o_seen[t]) mbar_wait(bar_o + t, (o_iss[t] - 1) & 1, kPfWaitLimit);
         }
+        for (int q = q_seen; q < q_iss; ++q) mbar_wait(bar_q, q & 1, kPfWaitLimit);
       }
+      // the last stage-empty arrivals land before the CTA leaves (bounded)
+      for (int st = 0; st < 2; ++st)
+        if (ke_iss[st] > 0) mbar_wait(bar_ke + st, (ke_iss[st] - 1) & 1, kPfWaitLimit);
     }
   } else {
     // =================== softmax group t (warps 4t .. 4t+3) ===================
@@ -303,153 +419,182 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem + t * 128 + lane_off;
     const uint32_t tO = tmem + 256 + t * 128 + lane_off;
-    const int q0_t = t ? g.q0[1] : g.q0[0];
-    const int rows_t = t ? g.rows[1] : g.rows[0];
-    const bool active = rows_t > 0;
-    const int prow = g.past + q0_t + r;
-    const int p_lo = g.past + q0_t;                         // first row of this tile
-    const int p_hi = g.past + q0_t + max(rows_t, 1) - 1;
-    float m_used = -INFINITY;   // log2 units
-    float l_sum = 0.f;
     const float sl2 = p.scale_log2;
+    int s_seen = 0, o_seen = 0;   // bar_s / bar_o phases this group has consumed
     bool ok = true;
-    for (int j = 0; j < g.ntiles && active; ++j) {
-      ok = mbar_wait(bar_s + t, j & 1, kPfWaitLimit, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int kb = g.k_lo + j * kPfBN;
-      // which cache blocks of this tile are mapped (bit i: box i), and does any
-      // key of the tile need a mask for any row of this q tile?
-      const int nbox = kPfBN >> box_shift;   // <= 8 (block_size >= 16)
-      uint32_t boxmask = 0;
-      for (int i = 0; i < nbox; ++i) {
-        const int key0 = kb + (i << box_shift);
-        const int lb = key0 / p.bs;
-        const int blk = lb < p.MB ? p.block_table[(long long)g.b * p.MB + lb] : -1;
-        if (blk >= 0 && blk < p.NB) boxmask |= 1u << i;
-      }
-      const bool all_mapped = boxmask == (1u << nbox) - 1u;
-      const bool full = all_mapped && kb + kPfBN - 1 <= p_lo && kb + kPfBN <= g.k_hi &&
-                        (p.window <= 0 || kb > p_hi - p.window);
-      // visibility of key column c (only consulted on tiles that need a mask):
-      // the row's causal / window / end-of-keys limits as a column interval
-      // [c_lo, c_hi), and the mapped-block bitmask
-      const int c_hi = min(min(prow + 1, g.k_hi) - kb, kPfBN);
-      const int c_lo = p.window > 0 ? max(prow - p.window + 1 - kb, 0) : 0;
-      auto visible = [&](int c) {
-        return c >= c_lo && c < c_hi && ((boxmask >> (c >> box_shift)) & 1u);
-      };
-      // pass 1: row max over 32-column chunks of S (keeps few registers live);
-      // on tiles that need a mask, hidden keys are written back as -inf so
-      // that pass 2 is the same for every tile
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c4 = 0; c4 < kPfBN / 32; ++c4) {
-        uint32_t v[32];
-        tmem_ld32(tS + c4 * 32, v);
-        tmem_wait_ld();
-        if (!full) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (!visible(c4 * 32 + e)) v[e] = __float_as_uint(-INFINITY);
-          tmem_st32(tS + c4 * 32, v);
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      PfGeom g;
+      if (!pf_geom(p, item, n_pairs, max_tiles, g)) continue;
+      const int q0_t = t ? g.q0[1] : g.q0[0];
+      const int rows_t = t ? g.rows[1] : g.rows[0];
+      if (rows_t <= 0) continue;
+      const int prow = g.past + q0_t + r;
+      const int p_lo = g.past + q0_t;                         // first row of this tile
+      const int p_hi = g.past + q0_t + rows_t - 1;
+      float m_used = -INFINITY;   // log2 units
+      float l_sum = 0.f;
+      const int nbox0 = kPfBN >> box_shift;
+      int blk_next = g.ntiles > 0 ? pf_block_id(p, g.b, g.k_lo, lane, nbox0, box_shift) : -1;
+      for (int j = 0; j < g.ntiles; ++j) {
+        ok = mbar_wait(bar_s + t, s_seen & 1, kPfWaitLimit, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
         }
+        ++s_seen;
+        tc_fence_after();
+        const int kb = g.k_lo + j * kPfBN;
+        // which cache blocks of this tile are mapped (bit i: box i; lane i read
+        // block i one tile ahead), and does any key of the tile need a mask for
+        // any row of this q tile?
+        const int nbox = kPfBN >> box_shift;   // <= 8 (block_size >= 16)
+        const uint32_t boxmask = __ballot_sync(0xffffffffu, lane < nbox && blk_next >= 0 && blk_next < p.NB);
+        if (j + 1 < g.ntiles) blk_next = pf_block_id(p, g.b, kb + kPfBN, lane, nbox, box_shift);
+        const bool all_mapped = boxmask == (1u << nbox) - 1u;
+        const bool full = all_mapped && kb + kPfBN - 1 <= p_lo && kb + kPfBN <= g.k_hi &&
+                          (p.window <= 0 || kb > p_hi - p.window);
+        // visibility of key column c (only consulted on tiles that need a mask):
+        // the row's causal / window / end-of-keys limits as a column interval
+        // [c_lo, c_hi), and the mapped-block bitmask
+        const int c_hi = min(min(prow + 1, g.k_hi) - kb, kPfBN);
+        const int c_lo = p.window > 0 ? max(prow - p.window + 1 - kb, 0) : 0;
+        // visibility of the 32 columns of chunk c4 as a bitmask: the row's
+        // causal / window / end-of-keys interval and the mapped blocks
+        auto chunk_bits = [&](int c4) -> uint32_t {
+          const int base = c4 * 32;
+          const int lo = clampi(c_lo - base, 0, 32), hi = clampi(c_hi - base, 0, 32);
+          uint32_t m = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~(lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u));
+          if (box_shift >= 5) {
+            if (!((boxmask >> (base >> box_shift)) & 1u)) m = 0u;
+          } else {   // 16-row boxes: two per chunk
+            if (!((boxmask >> (base >> 4)) & 1u)) m &= 0xffff0000u;
+            if (!((boxmask >> ((base >> 4) + 1)) & 1u)) m &= 0x0000ffffu;
+          }
+          return m;
+        };
+        // pass 1: row max over 32-column chunks of S (keeps few registers live)
+        float mx = -INFINITY;
+        if (full) {
+#pragma unroll 1
+          for (int c4 = 0; c4 < kPfBN / 32; ++c4) {
+            uint32_t v[32];
+            tmem_ld32(tS + c4 * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, u2f(v[e]));
+            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, u2f(v[e]));
+          }
+        } else {
+#pragma unroll 1
+          for (int c4 = 0; c4 < kPfBN / 32; ++c4) {
+            uint32_t v[32];
+            tmem_ld32(tS + c4 * 32, v);
+            const uint32_t m = chunk_bits(c4);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, ((m >> e) & 1u) ? u2f(v[e]) : -INFINITY);
+          }
+        }
+        mx *= sl2;   // scores in log2 units (scale > 0)
+        // lazy rescale: raise the reference max only when it grows by > 8 (x256).
+        // The TMEM loads / stores of O are warp-collective, so the whole warp
+        // takes the branch when any of its rows needs it (alpha = 1 otherwise).
+        const bool need = mx > m_used + 8.0f;
+        const float m_new = need ? mx : m_used;
+        const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2(m_used - m_new)) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
+          uint32_t o[32];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(u2f(o[e]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        l_sum *= alpha;
+        m_used = m_new;
+        const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+        // pass 2: P = 2^(s*scale - m) for 64 keys at a time, packed in pairs into
+        // the TMEM columns that held those keys' scores (already read)
+        // hidden keys (masked tiles) give p = 0
+        float ls = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < kPfBN / 64; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            const int c0 = hh * 64 + half * 32;
+            tmem_ld32(tS + c0, v);
+            const uint32_t m = full ? 0xffffffffu : chunk_bits(hh * 2 + half);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float pa = ((m >> e) & 1u) ? ex2(fmaf(u2f(v[e]), sl2, nm)) : 0.f;
+              const float pb = ((m >> (e + 1)) & 1u) ? ex2(fmaf(u2f(v[e + 1]), sl2, nm)) : 0.f;
+              ls += pa + pb;
+              pk[half * 16 + e / 2] = pack_pair<T>(pa, pb);
+            }
+          }
+          tmem_st32(tS + hh * 32, pk);
+        }
+        l_sum += ls;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p + t);
       }
-      if (!full) tmem_wait_st();
-      mx *= sl2;   // scores in log2 units (scale > 0)
-      // lazy rescale: raise the reference max only when it grows by > 8 (x256).
-      // The TMEM loads / stores of O are warp-collective, so the whole warp
-      // takes the branch when any of its rows needs it (alpha = 1 otherwise).
-      const bool need = mx > m_used + 8.0f;
-      const float m_new = need ? mx : m_used;
-      const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2(m_used - m_new)) : 1.f;
-      if (j > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
-        uint32_t o[32];
+      if (!ok) break;
+      // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
+      bool have_o = g.ntiles > 0;
+      if (have_o) {
+        have_o = mbar_wait(bar_o + t, (o_seen + g.ntiles - 1) & 1, kPfWaitLimit, abort_flag);
+        o_seen += g.ntiles;
+        if (!__all_sync(0xffffffffu, have_o)) {
+          ok = false;
+          break;
+        }
+      }
+        tc_fence_after();
+        const bool mine = r < rows_t;
+        const int tok = g.t_begin + q0_t + r;
+        const long long orow = (long long)tok * p.H_q + g.h;
+        const float sink2 = p.sinks ? p.sinks[g.h] * kLog2e : -INFINITY;
+        float a, inv_l, lse;
+        finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
+        const float f = a * inv_l;
+        T* out = static_cast<T*>(p.out) + orow * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
+          uint32_t o[32];
+          if (have_o) {   // warp-uniform: every lane takes part in the warp-wide load
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(u2f(o[e]) * alpha);
-          tmem_st32(tO + c * 32, o);
-        }
-      }
-      l_sum *= alpha;
-      m_used = m_new;
-      const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
-      // pass 2: P = 2^(s*scale - m) for 64 keys at a time, packed in pairs into
-      // the TMEM columns that held those keys' scores (already read)
-      float ls = 0.f;
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          if (mine) {
 #pragma unroll
-      for (int hh = 0; hh < kPfBN / 64; ++hh) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t v[32];
-          const int c0 = hh * 64 + half * 32;
-          tmem_ld32(tS + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float pa = ex2(fmaf(u2f(v[e]), sl2, nm));   // -inf -> 0
-            const float pb = ex2(fmaf(u2f(v[e + 1]), sl2, nm));
-            ls += pa + pb;
-            pk[half * 16 + e / 2] = pack_pair<T>(pa, pb);
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = pack_pair<T>(u2f(o[e + 0]) * f, u2f(o[e + 1]) * f);
+              v.y = pack_pair<T>(u2f(o[e + 2]) * f, u2f(o[e + 3]) * f);
+              v.z = pack_pair<T>(u2f(o[e + 4]) * f, u2f(o[e + 5]) * f);
+              v.w = pack_pair<T>(u2f(o[e + 6]) * f, u2f(o[e + 7]) * f);
+              *reinterpret_cast<uint4*>(out + c * 32 + e) = v;
+            }
           }
         }
-        tmem_st32(tS + hh * 32, pk);
+        if (mine && p.lse) p.lse[orow] = lse;
+      if (g.ntiles > 0) {   // O_t may now be overwritten by the next item
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_e + t);
       }
-      l_sum += ls;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p + t);
     }
-    // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
-    bool have_o = active && ok && g.ntiles > 0;
-    if (have_o) have_o = mbar_wait(bar_o + t, (g.ntiles - 1) & 1, kPfWaitLimit, abort_flag);
-    have_o = __all_sync(0xffffffffu, have_o);
-    if (active && !(*abort_flag) && (have_o || g.ntiles == 0)) {
-      tc_fence_after();
-      const bool mine = r < rows_t;
-      const int tok = g.t_begin + q0_t + r;
-      const long long orow = (long long)tok * p.H_q + g.h;
-      const float sink2 = p.sinks ? p.sinks[g.h] * kLog2e : -INFINITY;
-      float a, inv_l, lse;
-      finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
-      const float f = a * inv_l;
-      T* out = static_cast<T*>(p.out) + orow * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (have_o) {   // warp-uniform: every lane takes part in the warp-wide load
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if (mine) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 v;
-            v.x = pack_pair<T>(u2f(o[e + 0]) * f, u2f(o[e + 1]) * f);
-            v.y = pack_pair<T>(u2f(o[e + 2]) * f, u2f(o[e + 3]) * f);
-            v.z = pack_pair<T>(u2f(o[e + 4]) * f, u2f(o[e + 5]) * f);
-            v.w = pack_pair<T>(u2f(o[e + 6]) * f, u2f(o[e + 7]) * f);
-            *reinterpret_cast<uint4*>(out + c * 32 + e) = v;
-          }
-        }
-      }
-      if (mine && p.lse) p.lse[orow] = lse;
-    } else if (active) {
-      *abort_flag = 1;
-    }
+    if (!ok) *abort_flag = 1;
   }
   __syncthreads();
   if (*abort_flag) bits |= SPA_ST_TIMEOUT;
@@ -528,14 +673,25 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   if ((rc = encode(&tk, dt, 4, p.k_cache, kd, ks, kbx)) != SPA_OK) return rc;
   if ((rc = encode(&tv, dt, 4, p.v_cache, kd, ks, kbx)) != SPA_OK) return rc;
   const int n_pairs = (p.max_q + 2 * kPfBM - 1) / (2 * kPfBM);
-  if (n_pairs > 65535) return SPA_ERR_UNSUPPORTED;
+  const long long items = (long long)p.H_q * p.B * n_pairs;
+  if (items > 0x7fffffffLL) return SPA_ERR_UNSUPPORTED;
   const int max_tiles = (p.max_k + kPfBN - 1) / kPfBN + 1;
   auto kern = prefill_tcgen05_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  // grid: heads fastest, then requests, then q-tile pairs from the last (longest) down
-  dim3 grid(p.H_q, p.B, n_pairs);
-  return launch_pdl(kern, grid, dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_pairs, box_rows,
-                    box_shift, max_tiles);
+  // persistent: one CTA per SM (all of TMEM, over half the shared memory),
+  // items = heads fastest, then requests, then q-tile pairs from the last
+  // (longest) down
+  // Short items (a window of at most two key tiles) run persistently, one CTA
+  // per SM looping over them, so the per-CTA set-up and pipeline fill are paid
+  // once per SM; long causal items keep one CTA each, which the hardware
+  // schedules dynamically (a static assignment of the unequal causal items
+  // measured slower).
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool persistent = p.window > 0 && p.window <= 2 * kPfBN;
+  const int grid = persistent ? (int)std::min<long long>(items, std::max(sms, 1)) : (int)items;
+  return launch_pdl(kern, dim3(grid), dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_pairs, box_rows,
+                    box_shift, max_tiles, (int)items);
 }
 
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream) {

@@ -237,7 +237,7 @@ def make_workload(*, name="custom", act="f16", cache=None, B=2, H_q=8, H_kv=2, D
 # ---------------------------------------------------------------------------
 
 WORKLOADS = ("tiny_decode_f32", "gptoss_paged_decode_f16", "selected_decode_bf16",
-             "local_plus_selected_int8", "ragged_prefill_f16")
+             "local_plus_selected_int8", "ragged_prefill_f16", "windowed_chunked_prefill_f16")
 
 
 def tiny_decode_f32(seed: int = 0, small: bool = False) -> Workload:
@@ -299,6 +299,18 @@ def ragged_prefill_f16(seed: int = 4, small: bool = False) -> Workload:
     lens = [70, 130, 257, 300] if small else [512, 1024, 2048, 3072]
     return make_workload(name="ragged_prefill_f16", act="f16", B=4, H_q=32, H_kv=8, D=128,
                          block_size=64, q_lens=lens, past=[0] * 4, has_sinks=True, seed=seed)
+
+
+def windowed_chunked_prefill_f16(seed: int = 5, small: bool = False) -> Workload:
+    """Chunked prefill of GPT-OSS-like local (sliding-window) layers: B=4 chunks
+    of {2048, 1024, 512, 1536} tokens after {0, 1024, 3000, 512} resident
+    tokens, H_q=64, H_kv=8, D=64, paged block 16, window 128, sinks on, fp16."""
+    if small:
+        q_lens, past = [150, 64, 40, 97], [0, 70, 300, 33]
+    else:
+        q_lens, past = [2048, 1024, 512, 1536], [0, 1024, 3000, 512]
+    return make_workload(name="windowed_chunked_prefill_f16", act="f16", B=4, H_q=64, H_kv=8, D=64,
+                         block_size=16, q_lens=q_lens, past=past, window=128, has_sinks=True, seed=seed)
 
 
 def by_name(name: str, small: bool = False, seed: Optional[int] = None) -> Workload:
