@@ -146,6 +146,111 @@ def prepare_metadata(cu_seqlens_q: np.ndarray, past_seqlens: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# 1b. QKV prologue (optional, between metadata and append)
+# ---------------------------------------------------------------------------
+#
+# "[WebGPU] Add DynamicSparseAttention", Description: QKV and cache (packed
+# and unpacked QKV), Position processing (QK RMSNorm; partial and interleaved
+# RoPE; rotary offsets and explicit position IDs); "[WebGPU] Add
+# SparsePagedAttention", Description (the prologue -- packed-QKV split, RoPE
+# -- ahead of the block-table scatter).  Readings where the pages are silent:
+#   * packed QKV is [T, H_q + 2*H_kv, D]: q heads, then k heads, then v heads;
+#   * RMSNorm over each head's D channels, y = x / sqrt(mean(x^2) + eps) * w,
+#     one fp32 weight vector [D] for q and one for k; applied before RoPE;
+#   * RoPE rotates the first rotary_dim channels by the angle whose cos / sin
+#     are the caches' row `position` (fp32 [max_pos, rotary_dim / 2]); pairs
+#     are (i, i + rotary_dim/2) ("half-split") or (2i, 2i+1) ("interleaved"):
+#       (a, b) -> (a cos - b sin, b cos + a sin);
+#   * position = position_ids[t] when given, else token_pos[t] + offset; a
+#     position outside [0, max_pos) is left unrotated and sets BOUNDS;
+#   * q, k and v leave the prologue rounded to the activation dtype (round to
+#     nearest even), then k and v go through the append unchanged.
+
+def encode(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float64 values to `dtype`'s encoding (nearest even); bf16 as uint16 bits."""
+    x = np.asarray(x, dtype=np.float64)
+    if dtype == "f32":
+        return x.astype(np.float32)
+    if dtype == "f16":
+        return x.astype(np.float16)
+    if dtype == "bf16":
+        # the two bf16 neighbours of x, and the nearer one (ties to the even code)
+        lo = (np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64) >> 16) << 16
+        cand = [lo - (1 << 16), lo, lo + (1 << 16)]
+        vals = [c.astype(np.uint32).view(np.float32).astype(np.float64) for c in cand]
+        best = cand[1].copy()
+        bestd = np.abs(vals[1] - x)
+        for c, v in ((cand[0], vals[0]), (cand[2], vals[2])):
+            d = np.abs(v - x)
+            better = (d < bestd) | ((d == bestd) & (((c >> 16) & 1) == 0) & (((best >> 16) & 1) == 1))
+            best = np.where(better, c, best)
+            bestd = np.where(better, d, bestd)
+        return (best >> 16).astype(np.uint16)
+    raise ValueError(dtype)
+
+
+def split_packed(qkv: np.ndarray, H_q: int, H_kv: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """q [T, H_q, D], k and v [T, H_kv, D] of a packed [T, H_q + 2 H_kv, D] array."""
+    return qkv[:, :H_q], qkv[:, H_q:H_q + H_kv], qkv[:, H_q + H_kv:]
+
+
+def rms_norm(x: np.ndarray, weight: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * weight over the last axis (float64)."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + float(eps)) * np.asarray(weight, dtype=np.float64)
+
+
+def rotate(x: np.ndarray, cos: np.ndarray, sin: np.ndarray, rotary_dim: int,
+           interleaved: bool) -> np.ndarray:
+    """Rotary embedding of the first rotary_dim channels of x [D]; cos / sin [rotary_dim / 2]."""
+    y = np.array(x, dtype=np.float64)
+    half = rotary_dim // 2
+    c = np.asarray(cos, dtype=np.float64)[:half]
+    s = np.asarray(sin, dtype=np.float64)[:half]
+    if interleaved:
+        a, b = y[0:rotary_dim:2].copy(), y[1:rotary_dim:2].copy()
+        y[0:rotary_dim:2] = a * c - b * s
+        y[1:rotary_dim:2] = b * c + a * s
+    else:
+        a, b = y[:half].copy(), y[half:rotary_dim].copy()
+        y[:half] = a * c - b * s
+        y[half:rotary_dim] = b * c + a * s
+    return y
+
+
+def qkv_prologue(q: np.ndarray, k: np.ndarray, v: np.ndarray, act: str, token_pos: np.ndarray,
+                 q_norm_weight: Optional[np.ndarray] = None,
+                 k_norm_weight: Optional[np.ndarray] = None, eps: float = 1e-6,
+                 cos_cache: Optional[np.ndarray] = None, sin_cache: Optional[np.ndarray] = None,
+                 rotary_dim: int = 0, interleaved: bool = False,
+                 position_ids: Optional[np.ndarray] = None, rotary_offset: int = 0):
+    """Per token and head: RMSNorm (if its weight is given), then RoPE (if the
+    caches are given) of q and k; v passes through.  Inputs and outputs are
+    encoded in `act`.  Returns (q_out, k_out, v_out, status)."""
+    T = q.shape[0]
+    status = 0
+    qo = decode(q, act).copy()
+    ko = decode(k, act).copy()
+    rope = cos_cache is not None and rotary_dim > 0
+    max_pos = cos_cache.shape[0] if rope else 0
+    for t in range(T):
+        pos = int(position_ids[t]) if position_ids is not None else int(token_pos[t]) + int(rotary_offset)
+        rot_ok = rope and 0 <= pos < max_pos
+        if rope and not rot_ok:
+            status |= ST_BOUNDS
+        for x, w in ((qo, q_norm_weight), (ko, k_norm_weight)):
+            for h in range(x.shape[1]):
+                r = x[t, h]
+                if w is not None:
+                    r = rms_norm(r, w, eps)
+                if rot_ok:
+                    r = rotate(r, cos_cache[pos], sin_cache[pos], rotary_dim, interleaved)
+                x[t, h] = r
+    return encode(qo, act), encode(ko, act), np.array(v, copy=True), status
+
+
+# ---------------------------------------------------------------------------
 # 2. KV append scatter
 # ---------------------------------------------------------------------------
 
@@ -302,10 +407,21 @@ def run_step(wl, tokens: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray
     a = wl.arrays
     meta = prepare_metadata(a["cu_seqlens_q"], a["past_seqlens"], a["block_table"], wl.T,
                             wl.max_seqlen_q, wl.max_seqlen_k, wl.block_size, wl.NB)
-    kc, vc = append_kv(a["k_new"], a["v_new"], wl.act, a["k_cache"], a["v_cache"], wl.cache,
+    q, k_new, v_new = a["q"], a["k_new"], a["v_new"]
+    pro = getattr(wl, "prologue", None)
+    if pro:
+        if pro.get("packed"):
+            q, k_new, v_new = split_packed(a["qkv"], wl.H_q, wl.H_kv)
+        q, k_new, v_new, st = qkv_prologue(
+            q, k_new, v_new, wl.act, meta["token_pos"], a.get("q_norm_weight"),
+            a.get("k_norm_weight"), pro.get("eps", 1e-6), a.get("cos_cache"), a.get("sin_cache"),
+            pro.get("rotary_dim", 0), pro.get("interleaved", False), a.get("position_ids"),
+            pro.get("rotary_offset", 0))
+        meta = dict(meta, status=meta["status"] | st)
+    kc, vc = append_kv(k_new, v_new, wl.act, a["k_cache"], a["v_cache"], wl.cache,
                        meta["slot_mapping"], a.get("k_scale"), a.get("v_scale"))
     sel = a.get("selected_idx")
-    res = attention(a["q"], wl.act, kc, vc, wl.cache, a["block_table"], meta, H_kv=wl.H_kv,
+    res = attention(q, wl.act, kc, vc, wl.cache, a["block_table"], meta, H_kv=wl.H_kv,
                     window=wl.window, selected_idx=sel, sel_per_request=wl.sel_per_request,
                     sel_target=1 if wl.sel_mode == "aux" else 0, aux_k=a.get("aux_k"),
                     aux_v=a.get("aux_v"), aux_seqlens=a.get("aux_seqlens"),
@@ -314,5 +430,7 @@ def run_step(wl, tokens: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray
     res["meta"] = meta
     res["k_cache"] = kc
     res["v_cache"] = vc
+    if pro:
+        res["q_out"] = q
     res["status"] = res["status"] | meta["status"]
     return res

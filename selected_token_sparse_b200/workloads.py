@@ -95,6 +95,9 @@ class Workload:
     seed: int
     arrays: Dict[str, np.ndarray] = dataclasses.field(default_factory=dict)
     dtypes: Dict[str, str] = dataclasses.field(default_factory=dict)
+    # optional QKV prologue ahead of the append: packed (bool), qk_norm (bool),
+    # eps, rotary_dim, interleaved (bool), max_pos, pos_ids (bool), rotary_offset
+    prologue: Optional[Dict] = None
 
     @property
     def T(self) -> int:
@@ -129,7 +132,7 @@ def make_workload(*, name="custom", act="f16", cache=None, B=2, H_q=8, H_kv=2, D
                   sel_per_request=1, sel_width=0, sel_valid=None, sel_sorted=False,
                   sel_tail_pad=0, aux_cap=0, aux_lens=None, has_sinks=True, scale=0.0,
                   int8_history=False, kv_scale_range=(0.01, 0.05), spare_blocks=0,
-                  seed=0) -> Workload:
+                  prologue: Optional[Dict] = None, seed=0) -> Workload:
     """Draw one seeded workload.
 
     Lengths: request b has ``past[b]`` resident tokens and ``q_lens[b]`` new
@@ -224,11 +227,37 @@ def make_workload(*, name="custom", act="f16", cache=None, B=2, H_q=8, H_kv=2, D
                 sel[r, h, :nv] = idx
         arrays["selected_idx"] = sel
         dtypes["selected_idx"] = "i32"
+    pro = None
+    if prologue:
+        # drawn from a stream of its own, so the arrays above do not change
+        pro = dict(prologue)
+        prng = np.random.default_rng(seed + 7919)
+        if pro.get("packed"):
+            arrays["qkv"] = np.concatenate([arrays["q"], arrays["k_new"], arrays["v_new"]], axis=1)
+            dtypes["qkv"] = act
+        if pro.get("qk_norm"):
+            arrays["q_norm_weight"] = prng.uniform(0.5, 1.5, size=D).astype(np.float32)
+            arrays["k_norm_weight"] = prng.uniform(0.5, 1.5, size=D).astype(np.float32)
+            dtypes["q_norm_weight"] = dtypes["k_norm_weight"] = "f32"
+        rd = int(pro.get("rotary_dim", 0))
+        if rd:
+            max_pos = int(pro.get("max_pos", (max(totals) if totals else 0) + 64))
+            pro["max_pos"] = max_pos
+            inv_freq = float(pro.get("base", 10000.0)) ** (-np.arange(0, rd, 2, dtype=np.float64) / rd)
+            angle = np.arange(max_pos, dtype=np.float64)[:, None] * inv_freq[None, :]
+            arrays["cos_cache"] = np.cos(angle).astype(np.float32)
+            arrays["sin_cache"] = np.sin(angle).astype(np.float32)
+            dtypes["cos_cache"] = dtypes["sin_cache"] = "f32"
+        if pro.get("pos_ids"):
+            shift = int(pro.get("pos_shift", 3))
+            pos = [past[b] + i + shift for b in range(B) for i in range(q_lens[b])]
+            arrays["position_ids"] = np.asarray(pos, dtype=np.int32).reshape(T)
+            dtypes["position_ids"] = "i32"
     wl = Workload(name=name, act=act, cache=cache, B=B, H_q=H_q, H_kv=H_kv, D=D,
                   block_size=block_size, q_lens=q_lens, past=past, window=window,
                   sel_mode=sel_mode, sel_per_request=sel_per_request, sel_width=sel_width,
                   aux_cap=aux_cap, has_sinks=has_sinks, scale=scale, seed=seed,
-                  arrays=arrays, dtypes=dtypes)
+                  arrays=arrays, dtypes=dtypes, prologue=pro)
     return wl
 
 

@@ -37,6 +37,15 @@ MUTATIONS = [
     ("aux length bound ignored", "aux_pos = sel[(sel >= 0) & (sel < int(aux_seqlens[b]))]",
      "aux_pos = sel[(sel >= 0)]"),
     ("lse without the max", "lse[t, h] = m + math.log(l)", "lse[t, h] = math.log(l)"),
+    ("rotation sign flipped", "y[:half] = a * c - b * s", "y[:half] = a * c + b * s"),
+    ("interleaved pair order swapped", "a, b = y[0:rotary_dim:2].copy(), y[1:rotary_dim:2].copy()",
+     "b, a = y[0:rotary_dim:2].copy(), y[1:rotary_dim:2].copy()"),
+    ("RMS over the sum, not the mean", "ms = np.mean(x * x, axis=-1, keepdims=True)",
+     "ms = np.sum(x * x, axis=-1, keepdims=True)"),
+    ("RMSNorm eps dropped", "np.sqrt(ms + float(eps))", "np.sqrt(ms)"),
+    ("rotary offset ignored", "int(token_pos[t]) + int(rotary_offset)", "int(token_pos[t])"),
+    ("bf16 ties away from even", "(((c >> 16) & 1) == 0) & (((best >> 16) & 1) == 1)",
+     "(((c >> 16) & 1) == 1) & (((best >> 16) & 1) == 0)"),
 ]
 
 

@@ -497,3 +497,142 @@ def test_bad_index_flag_and_skip():
     assert r["status"] == O.ST_BAD_IDX
     ok = lw.run(selected_idx=np.array([[[3, 5]]], np.int32), sel_per_request=1, sel_target=0)
     np.testing.assert_array_equal(r["out"], ok["out"])
+
+
+# ---------------------------------------------------------------------------
+# QKV prologue: RMSNorm, rotary embedding, rounding to the activation dtype
+# ---------------------------------------------------------------------------
+
+def test_rms_norm_worked_example():
+    # [3, 4]: mean square 12.5, so [3, 4] / sqrt(12.5) scaled by [1, 2]
+    got = O.rms_norm(np.array([3.0, 4.0]), np.array([1.0, 2.0]), 0.0)
+    r = math.sqrt(12.5)
+    np.testing.assert_allclose(got, [3.0 / r, 8.0 / r], rtol=0, atol=1e-15)
+
+
+def test_rms_norm_matches_torch_and_eps():
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((5, 64))
+    w = rng.uniform(0.5, 1.5, 64)
+    for eps in (0.0, 1e-6, 0.5):
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,), torch.from_numpy(w), eps)
+        np.testing.assert_allclose(O.rms_norm(x, w, eps), ref.numpy(), rtol=1e-13, atol=1e-14)
+    # scale invariance without eps
+    np.testing.assert_allclose(O.rms_norm(7.5 * x, w, 0.0), O.rms_norm(x, w, 0.0), rtol=1e-13)
+
+
+def test_rotate_quarter_turn():
+    x = np.array([1.0, 2.0, 3.0, 4.0, 5.0])
+    c, s = np.zeros(2), np.ones(2)
+    # half-split pairs (0, 2), (1, 3): (a, b) -> (-b, a); channel 4 is past rotary_dim
+    np.testing.assert_array_equal(O.rotate(x, c, s, 4, False), [-3.0, -4.0, 1.0, 2.0, 5.0])
+    # interleaved pairs (0, 1), (2, 3)
+    np.testing.assert_array_equal(O.rotate(x, c, s, 4, True), [-2.0, 1.0, -4.0, 3.0, 5.0])
+
+
+def test_rotate_zero_angle_and_partial_tail():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal(64)
+    np.testing.assert_array_equal(O.rotate(x, np.ones(16), np.zeros(16), 32, True), x)
+    y = O.rotate(x, *np.split(rng.standard_normal(32), 2), 32, False)
+    np.testing.assert_array_equal(y[32:], x[32:])
+
+
+def _theta(pos, rd, base=10000.0):
+    inv = base ** (-np.arange(0, rd, 2) / rd)
+    return np.cos(pos * inv), np.sin(pos * inv)
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_rotate_as_complex_multiplication(interleaved):
+    """Each channel pair (a, b) is the complex number a + ib times exp(i theta)."""
+    rng = np.random.default_rng(13)
+    rd, x = 48, rng.standard_normal(64)
+    c, s = _theta(37, rd)
+    if interleaved:
+        a, b = x[0:rd:2], x[1:rd:2]
+    else:
+        a, b = x[:rd // 2], x[rd // 2:rd]
+    z = (a + 1j * b) * np.exp(1j * np.arctan2(s, c))
+    y = O.rotate(x, c, s, rd, interleaved)
+    ya, yb = (y[0:rd:2], y[1:rd:2]) if interleaved else (y[:rd // 2], y[rd // 2:rd])
+    np.testing.assert_allclose(ya, z.real, atol=1e-13)
+    np.testing.assert_allclose(yb, z.imag, atol=1e-13)
+
+
+def test_rope_relative_position_and_norm():
+    rng = np.random.default_rng(14)
+    rd = 64
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    dots = []
+    for p in (5, 40, 300):
+        qr = O.rotate(q, *_theta(p + 9, rd), rd, False)
+        kr = O.rotate(k, *_theta(p, rd), rd, False)
+        np.testing.assert_allclose(np.linalg.norm(qr), np.linalg.norm(q), rtol=1e-13)
+        dots.append(float(qr @ kr))
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-11)
+
+
+def test_interleaved_is_half_split_of_permuted_channels():
+    rng = np.random.default_rng(15)
+    rd, x = 32, rng.standard_normal(64)
+    c, s = _theta(21, rd)
+    perm = np.concatenate([np.arange(0, rd, 2), np.arange(1, rd, 2), np.arange(rd, 64)])
+    # interleaved on x == half-split on x[perm], read back through the permutation
+    got = O.rotate(x, c, s, rd, True)
+    via = np.empty(64)
+    via[perm] = O.rotate(x[perm], c, s, rd, False)
+    np.testing.assert_allclose(got, via, atol=1e-14)
+
+
+def test_encode_rounds_to_nearest_even():
+    # bf16 spacing at 1 is 2^-7: 1 + 2^-8 is a tie (to 1.0, the even code);
+    # 1 + 2^-8 + 2^-9 rounds up; -2.5e-3 and pi round to their bf16 neighbours
+    x = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 2.0 ** -8 + 2.0 ** -9, 1.0 + 3 * 2.0 ** -8])
+    np.testing.assert_array_equal(O.encode(x, "bf16"), [0x3F80, 0x3F80, 0x3F81, 0x3F82])
+    h = O.encode(np.array([1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11]), "f16")
+    np.testing.assert_array_equal(h.view(np.uint16), [0x3C00, 0x3C02])
+
+
+def _prologue_wl(**pro):
+    from selected_token_sparse_b200 import workloads as W
+    return W.make_workload(act="f16", B=2, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[3, 2],
+                           past=[7, 20], window=16, prologue=pro, seed=21)
+
+
+def test_prologue_without_norm_or_rope_is_identity():
+    wl = _prologue_wl(packed=True)
+    q, k, v = O.split_packed(wl["qkv"], wl.H_q, wl.H_kv)
+    meta = O.prepare_metadata(wl["cu_seqlens_q"], wl["past_seqlens"], wl["block_table"], wl.T,
+                              wl.max_seqlen_q, wl.max_seqlen_k, wl.block_size, wl.NB)
+    qo, ko, vo, st = O.qkv_prologue(q, k, v, "f16", meta["token_pos"])
+    assert st == 0
+    for a, b in ((qo, wl["q"]), (ko, wl["k_new"]), (vo, wl["v_new"])):
+        np.testing.assert_array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_prologue_position_ids_equal_offset():
+    """Explicit positions p + 3 give what the metadata positions with offset 3 give."""
+    a = O.run_step(_prologue_wl(qk_norm=True, rotary_dim=32, interleaved=True, pos_ids=True,
+                                pos_shift=3))
+    b = O.run_step(_prologue_wl(qk_norm=True, rotary_dim=32, interleaved=True, rotary_offset=3))
+    np.testing.assert_array_equal(a["q_out"].view(np.uint16), b["q_out"].view(np.uint16))
+    np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=0)
+
+
+def test_prologue_rotation_uses_the_token_position():
+    """q_out of a token equals RMSNorm then rotation at past + index, rounded."""
+    wl = _prologue_wl(qk_norm=True, rotary_dim=64, interleaved=False)
+    r = O.run_step(wl)
+    t, h = 4, 1                        # request 1, second token: position 20 + 1
+    x = O.decode(wl["q"][t, h], "f16")
+    y = O.rotate(O.rms_norm(x, wl["q_norm_weight"], 1e-6), wl["cos_cache"][21], wl["sin_cache"][21],
+                 64, False)
+    np.testing.assert_array_equal(r["q_out"][t, h], y.astype(np.float16))
+
+
+def test_prologue_out_of_range_position_flags_bounds():
+    wl = _prologue_wl(rotary_dim=32, pos_ids=True, pos_shift=10 ** 6)
+    r = O.run_step(wl)
+    assert r["status"] & O.ST_BOUNDS
+    np.testing.assert_array_equal(r["q_out"].view(np.uint16), wl["q"].view(np.uint16))
