@@ -282,12 +282,7 @@ def run_ours(args):
         insts.append(pipeline.Step(wl, d, num_splits=args.splits, mode=args.mode))
     del base
     step0 = insts[0]
-    a0 = spa.attention_args(step0.d["q"], step0.d["k_cache"], step0.d["v_cache"],
-                            step0.d["block_table"], dict(step0.meta,
-                                                         cu_seqlens_q=step0.d["cu_seqlens_q"]),
-                            max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
-                            out=step0.out, num_splits=args.splits, **step0.kw)
-    plan = spa.attention_plan(a0)
+    plan = spa.attention_plan(step0.args)
     launches_per_step = step0.launches()
     # one launch per step: the fused step kernel is the whole step
     single = launches_per_step == 1
@@ -314,12 +309,7 @@ def run_ours(args):
 
     def attn_only(st):
         def f():
-            a = spa.attention_args(st.d["q"], st.d["k_cache"], st.d["v_cache"],
-                                   st.d["block_table"], dict(st.meta, cu_seqlens_q=st.d["cu_seqlens_q"]),
-                                   max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
-                                   out=st.out, lse=None, num_splits=args.splits, status=st.status,
-                                   **st.kw)
-            spa.run_attention(a, st.workspace)
+            spa.run_attention(st.args, st.workspace)   # the step's own attention call
         return f
 
     ga_one = [capture(attn_only(st)) for st in insts]
@@ -373,8 +363,10 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         host = pipeline.to_device(wl, pin=True)
-        names = [n for n in ("q", "k_new", "v_new", "cu_seqlens_q", "past_seqlens", "block_table",
-                             "selected_idx") if n in host]
+        packed = bool(getattr(wl, "prologue", None) and wl.prologue.get("packed"))
+        inputs = (("qkv",) if packed else ("q", "k_new", "v_new")) + (
+            "cu_seqlens_q", "past_seqlens", "block_table", "selected_idx", "position_ids")
+        names = [n for n in inputs if n in host]
         h2d = sum(host[n].numel() * host[n].element_size() for n in names)
         out_host = torch.empty(step0.out.shape, dtype=step0.out.dtype, pin_memory=True)
         d2h = out_host.numel() * out_host.element_size()

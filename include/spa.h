@@ -267,6 +267,69 @@ int spa_prepare_append_attention(const spa_attention_args_t* a, const int32_t* p
 int spa_prepare_append_attention_launches(const spa_attention_args_t* a);
 
 /*
+ * spa_prepare_qkv_append -- steps 1 and 2 with the QKV prologue between them,
+ * in one launch: the metadata of spa_prepare_metadata, then per (token, head)
+ * row of q and k an optional RMSNorm and an optional rotary embedding, then q
+ * written for the attention and k / v appended as spa_append_kv does.
+ * Source: "[WebGPU] Add DynamicSparseAttention", Description -- QKV and cache
+ * (packed and unpacked QKV), Position processing (QK RMSNorm; partial and
+ * interleaved RoPE; rotary offsets and explicit position IDs); "[WebGPU] Add
+ * SparsePagedAttention", Description (packed-QKV split and RoPE ahead of the
+ * block-table scatter).  Per row x of a q or k head:
+ *   x <- x / sqrt(mean(x^2) + norm_eps) * w             (w = q_ / k_norm_weight)
+ *   x <- RoPE on channels [0, rotary_dim): pairs (i, i + rotary_dim/2), or
+ *        (2i, 2i+1) when rotary_interleaved: (a, b) -> (a c - b s, b c + a s)
+ *        with c, s = cos_cache, sin_cache[position, i]
+ *   position = position_ids[t] if given, else token_pos[t] + rotary_offset;
+ *   outside [0, max_pos) the row is not rotated and SPA_ST_BOUNDS is set.
+ * Results are rounded to `act` (nearest even); k and v are then appended
+ * (INT8: q8 = clamp(rint(x / scale), -128, 127) of the rounded x).
+ */
+typedef struct {
+  size_t struct_size;            /* sizeof(spa_qkv_args_t) */
+  /* step 1, as spa_prepare_metadata (the five arrays are outputs) */
+  const int32_t* cu_seqlens_q;   /* [B + 1] */
+  const int32_t* past_seqlens;   /* [B] */
+  const int32_t* block_table;    /* [B, MB] */
+  int32_t B, T, max_seqlen_q, max_seqlen_k, MB, block_size, num_blocks;
+  int32_t* seqlens_q;
+  int32_t* seqlen_k;
+  int32_t* token_batch;
+  int32_t* token_pos;
+  int32_t* slot_mapping;
+  /* the rows */
+  int32_t act;                   /* SPA_F32 / SPA_F16 / SPA_BF16 */
+  int32_t H_q, H_kv, D;          /* D = 64 or 128 */
+  const void* qkv;               /* packed [T, H_q + 2 H_kv, D]: q, then k, then v heads; or NULL */
+  const void* q;                 /* [T, H_q, D]  \                                  */
+  const void* k;                 /* [T, H_kv, D]  } when qkv is NULL                 */
+  const void* v;                 /* [T, H_kv, D] /                                   */
+  /* prologue */
+  const float* q_norm_weight;    /* [D] or NULL (no q norm) */
+  const float* k_norm_weight;    /* [D] or NULL (no k norm) */
+  float norm_eps;
+  const float* cos_cache;        /* [max_pos, rotary_dim / 2] or NULL (no rotation) */
+  const float* sin_cache;        /* [max_pos, rotary_dim / 2] */
+  int32_t max_pos, rotary_dim, rotary_interleaved;   /* rotary_dim even, <= D */
+  const int32_t* position_ids;   /* [T] or NULL */
+  int32_t rotary_offset;
+  /* outputs */
+  void* q_out;                   /* [T, H_q, D] act */
+  void* k_cache;                 /* [num_blocks, block_size, H_kv, D] */
+  void* v_cache;
+  int32_t cache;                 /* act or SPA_I8 */
+  const float* k_scale;          /* [H_kv, D] iff SPA_I8 */
+  const float* v_scale;
+  int32_t* status;
+} spa_qkv_args_t;
+
+/* Errors: SPA_ERR_INVALID_ARG for a NULL required pointer, a bad dtype pair,
+   D not 64 / 128, an odd or oversized rotary_dim, a row pointer not 16-byte
+   aligned, or inconsistent sizes; SPA_ERR_UNSUPPORTED for B > 16384.  B = 0 or
+   T = 0 is valid. */
+int spa_prepare_qkv_append(const spa_qkv_args_t* a, spa_stream_t stream);
+
+/*
  * spa_attention_noalloc -- spa_attention for callers that cannot allocate
  * device memory.  The pages have no counterpart: this entry point exists for
  * callers of this library that cannot provide a workspace -- code running

@@ -30,6 +30,7 @@ int tc_supported(int act, int cache, int D, int max_rows);
 int tc_key_tile();
 int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream);
 int launch_step_mma(const AttnParams& p, int act, int max_rows, cudaStream_t stream);
+int launch_prepare_qkv_append(const QkvParams& P, int act, int cache, cudaStream_t stream);
 int mma_step_fits(int D, int max_rows, int B);
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream);
 int prefill_supported(const spa_attention_args_t* a);
@@ -398,6 +399,78 @@ int spa_prepare_append_attention_launches(const spa_attention_args_t* a) {
   Plan pl;
   if ((rc = make_plan(a, &pl)) != SPA_OK) return rc;
   return step_fusable(a, pl) ? 1 : 1 + launches_of(pl);
+}
+
+int spa_prepare_qkv_append(const spa_qkv_args_t* a, spa_stream_t stream) {
+  if (!a || a->struct_size < sizeof(spa_qkv_args_t)) return SPA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->T < 0 || a->MB < 0 || a->block_size <= 0 || a->num_blocks < 0) return SPA_ERR_INVALID_ARG;
+  if (a->B > 16384) return SPA_ERR_UNSUPPORTED;
+  if ((long long)a->num_blocks * a->block_size >= (1LL << 31)) return SPA_ERR_INVALID_ARG;
+  if (!act_ok(a->act) || !(a->cache == a->act || a->cache == SPA_I8)) return SPA_ERR_INVALID_ARG;
+  if (a->H_q <= 0 || a->H_kv <= 0 || a->H_q % a->H_kv != 0) return SPA_ERR_INVALID_ARG;
+  if (a->D != 64 && a->D != 128) return SPA_ERR_INVALID_ARG;
+  if (a->cache == SPA_I8 && (!a->k_scale || !a->v_scale)) return SPA_ERR_INVALID_ARG;
+  if (!a->cu_seqlens_q) return SPA_ERR_INVALID_ARG;
+  if (a->B > 0 && (!a->past_seqlens || !a->seqlens_q || !a->seqlen_k || (a->MB > 0 && !a->block_table)))
+    return SPA_ERR_INVALID_ARG;
+  if (a->cos_cache) {
+    if (!a->sin_cache || a->rotary_dim <= 0 || (a->rotary_dim & 1) || a->rotary_dim > a->D || a->max_pos <= 0)
+      return SPA_ERR_INVALID_ARG;
+  }
+  if (a->T > 0) {
+    if (!a->token_batch || !a->token_pos || !a->slot_mapping || !a->q_out || !a->k_cache || !a->v_cache)
+      return SPA_ERR_INVALID_ARG;
+    if (!a->qkv && (!a->q || !a->k || !a->v)) return SPA_ERR_INVALID_ARG;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(a->qkv) | reinterpret_cast<uintptr_t>(a->q) |
+                         reinterpret_cast<uintptr_t>(a->k) | reinterpret_cast<uintptr_t>(a->v) |
+                         reinterpret_cast<uintptr_t>(a->q_out) | reinterpret_cast<uintptr_t>(a->k_cache) |
+                         reinterpret_cast<uintptr_t>(a->v_cache);
+    if (al & 15) return SPA_ERR_INVALID_ARG;
+  }
+  QkvParams P;
+  memset(&P, 0, sizeof(P));
+  P.cu = a->cu_seqlens_q;
+  P.past = a->past_seqlens;
+  P.block_table = a->block_table;
+  P.B = a->B;
+  P.T = a->T;
+  P.max_q = a->max_seqlen_q;
+  P.max_k = a->max_seqlen_k;
+  P.MB = a->MB;
+  P.bs = a->block_size;
+  P.NB = a->num_blocks;
+  P.seqlens_q = a->seqlens_q;
+  P.seqlen_k = a->seqlen_k;
+  P.token_batch = a->token_batch;
+  P.token_pos = a->token_pos;
+  P.slot_mapping = a->slot_mapping;
+  P.H_q = a->H_q;
+  P.H_kv = a->H_kv;
+  P.D = a->D;
+  P.qkv = a->qkv;
+  P.q = a->q;
+  P.k = a->k;
+  P.v = a->v;
+  P.q_norm = a->q_norm_weight;
+  P.k_norm = a->k_norm_weight;
+  P.eps = a->norm_eps;
+  P.cos_cache = a->cos_cache;
+  P.sin_cache = a->sin_cache;
+  P.max_pos = a->max_pos;
+  P.rotary_dim = a->cos_cache ? a->rotary_dim : 0;
+  P.interleaved = a->rotary_interleaved != 0;
+  P.position_ids = a->position_ids;
+  P.rotary_offset = a->rotary_offset;
+  P.q_out = a->q_out;
+  P.k_cache = a->k_cache;
+  P.v_cache = a->v_cache;
+  P.k_scale = a->k_scale;
+  P.v_scale = a->v_scale;
+  P.status = a->status;
+  if (a->B == 0 && a->T == 0) return SPA_OK;
+  int rc = launch_prepare_qkv_append(P, a->act, a->cache, (cudaStream_t)stream);
+  if (rc != SPA_OK) return rc;
+  return check_launch();
 }
 
 int spa_attention_plan(const spa_attention_args_t* a, int32_t* num_splits, int32_t* num_launches,

@@ -60,6 +60,38 @@ struct AttnParams {
   int cluster_merge;     // 1: the splits of a unit are one cluster, merged in shared memory
 };
 
+// Parameters of the fused metadata + QKV prologue + append kernel.
+struct QkvParams {
+  const int32_t* cu;
+  const int32_t* past;
+  const int32_t* block_table;
+  int B, T, max_q, max_k, MB, bs, NB;
+  int32_t* seqlens_q;
+  int32_t* seqlen_k;
+  int32_t* token_batch;
+  int32_t* token_pos;
+  int32_t* slot_mapping;
+  int H_q, H_kv, D;
+  const void* qkv;   // packed, or nullptr
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* q_norm;
+  const float* k_norm;
+  float eps;
+  const float* cos_cache;
+  const float* sin_cache;
+  int max_pos, rotary_dim, interleaved;
+  const int32_t* position_ids;
+  int rotary_offset;
+  void* q_out;
+  void* k_cache;
+  void* v_cache;
+  const float* k_scale;
+  const float* v_scale;
+  int32_t* status;
+};
+
 // Programmatic dependent launch: let the next kernel in the stream be
 // scheduled early, and wait for the previous one before touching memory.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }

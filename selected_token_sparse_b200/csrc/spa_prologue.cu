@@ -1,0 +1,188 @@
+// Steps 1 and 2 with the QKV prologue in between, in one launch: metadata,
+// then for every (token, head) row of q, k and v the prologue, then q is
+// written for the attention and k / v are appended to the paged cache.
+//
+// Prologue ("[WebGPU] Add DynamicSparseAttention", Description: QKV and cache
+// -- packed and unpacked QKV; Position processing -- QK RMSNorm, partial and
+// interleaved RoPE, rotary offsets and explicit position IDs; "[WebGPU] Add
+// SparsePagedAttention", Description -- packed-QKV split and RoPE ahead of the
+// block-table scatter):
+//   x  = the row of head h of q or k (packed [T, H_q + 2 H_kv, D]: q heads,
+//        then k heads, then v heads; or separate q / k / v tensors);
+//   x <- x / sqrt(mean(x^2) + eps) * w                 (when w is given)
+//   x <- RoPE(x, position)  on the first rotary_dim channels, pairs
+//        (i, i + rotary_dim/2) or (2i, 2i+1): (a, b) -> (a c - b s, b c + a s),
+//        c / s = cos_cache / sin_cache[position, i]   (when the caches are given)
+//   position = position_ids[t], or the token's position + rotary_offset; a
+//        position outside [0, max_pos) leaves the row unrotated (BOUNDS).
+// q leaves rounded to the activation dtype; k and v are rounded to it and
+// then appended exactly as spa_append_kv does (copy, or INT8 per-channel
+// quantisation of the rounded value).  v has no prologue.
+//
+// One warp per (token, head) row: lane l holds channels [l E, l E + E),
+// E = D / 32; the sum of squares is a warp reduction; a rotation reads its
+// pair partner through a per-warp row in shared memory.
+#include "spa_attn.cuh"
+#include "spa_meta.cuh"
+
+namespace spa {
+
+constexpr int kProThreads = 256;
+
+
+template <typename T>
+__device__ __forceinline__ T from_f32_rn(float x) {
+  return from_f32<T>(x);
+}
+
+template <typename ActT, typename CacheT, int E>
+__global__ void __launch_bounds__(kProThreads)
+prepare_qkv_append_kernel(const QkvParams P) {
+  extern __shared__ int32_t pro_smem[];   // cs [B + 1], past [B], then per-warp rows [8][D]
+  int32_t* cs = pro_smem;
+  int32_t* past_s = cs + P.B + 1;
+  float* rows = reinterpret_cast<float*>(past_s + P.B + ((2 * P.B + 1) & 1));   // 8-byte aligned
+  constexpr int D = E * 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* xrow = rows + warp * D;
+  pdl_wait();
+  pdl_trigger();
+  for (int b = threadIdx.x; b < P.B; b += blockDim.x) past_s[b] = P.past[b];
+  build_cs<kProThreads>(P.cu, P.B, P.T, cs);
+  int bits = 0;
+  if (blockIdx.x == 0)
+    bits |= per_request(P.cu, past_s, cs, P.B, P.T, P.max_q, P.max_k, P.seqlens_q, P.seqlen_k);
+  const int NH = P.H_q + 2 * P.H_kv;
+  const bool rope = P.cos_cache != nullptr && P.rotary_dim > 0;
+  const int rd = P.rotary_dim, half = rd / 2;
+  const long long rows_total = (long long)P.T * NH;
+  for (long long r = (long long)blockIdx.x * (kProThreads / 32) + warp; r < rows_total;
+       r += (long long)gridDim.x * (kProThreads / 32)) {
+    const int t = (int)(r / NH), hh = (int)(r % NH);
+    int tb = 0;
+    const TokenMeta m = token_meta(t, cs, P.B, past_s, P.block_table, P.MB, P.bs, P.NB, tb);
+    if (hh == 0 && lane == 0) {
+      bits |= tb;
+      P.token_batch[t] = m.b;
+      P.token_pos[t] = m.pos;
+      P.slot_mapping[t] = m.slot;
+    }
+    const int kind = hh < P.H_q ? 0 : (hh < P.H_q + P.H_kv ? 1 : 2);   // q, k, v
+    const int h = kind == 0 ? hh : (kind == 1 ? hh - P.H_q : hh - P.H_q - P.H_kv);
+    if (kind != 0 && m.slot < 0) continue;   // nothing to append
+    const ActT* src;
+    if (P.qkv) {
+      src = static_cast<const ActT*>(P.qkv) + ((long long)t * NH + hh) * D;
+    } else {
+      const void* base = kind == 0 ? P.q : (kind == 1 ? P.k : P.v);
+      const int H = kind == 0 ? P.H_q : P.H_kv;
+      src = static_cast<const ActT*>(base) + ((long long)t * H + h) * D;
+    }
+    float x[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] = to_f32(src[lane * E + e]);
+    if (kind != 2) {
+      const float* w = kind == 0 ? P.q_norm : P.k_norm;
+      if (w != nullptr) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = 1.0f / sqrtf(ss / (float)D + P.eps);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] = x[e] * inv * w[lane * E + e];
+      }
+      if (rope) {
+        const int pos = P.position_ids ? P.position_ids[t] : m.pos + P.rotary_offset;
+        if (pos >= 0 && pos < P.max_pos) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) xrow[lane * E + e] = x[e];
+          __syncwarp();
+          const float* cr = P.cos_cache + (long long)pos * half;
+          const float* sr = P.sin_cache + (long long)pos * half;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const int d = lane * E + e;
+            if (d >= rd) continue;
+            int i, partner;
+            bool first;
+            if (P.interleaved) {
+              i = d >> 1;
+              first = (d & 1) == 0;
+              partner = d ^ 1;
+            } else {
+              first = d < half;
+              i = first ? d : d - half;
+              partner = first ? d + half : d - half;
+            }
+            const float c = cr[i], s = sr[i], y = xrow[partner];
+            x[e] = first ? (x[e] * c - y * s) : (x[e] * c + y * s);
+          }
+          __syncwarp();
+        } else {
+          bits |= kStBounds;
+        }
+      }
+    }
+    if (kind == 0) {
+      ActT* dst = static_cast<ActT*>(P.q_out) + ((long long)t * P.H_q + h) * D;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dst[lane * E + e] = from_f32_rn<ActT>(x[e]);
+      continue;
+    }
+    // append: the value rounded to the activation dtype, copied or quantised
+    const long long drow = ((long long)m.slot * P.H_kv + h) * D;
+    if constexpr (sizeof(CacheT) != 1) {
+      CacheT* dst = static_cast<CacheT*>(kind == 1 ? P.k_cache : P.v_cache) + drow;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dst[lane * E + e] = from_f32_rn<CacheT>(x[e]);
+    } else {
+      const float* sc = (kind == 1 ? P.k_scale : P.v_scale) + (long long)h * D;
+      int8_t* dst = static_cast<int8_t*>(kind == 1 ? P.k_cache : P.v_cache) + drow;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float xr = to_f32(from_f32_rn<ActT>(x[e]));
+        float q8 = rintf(__fdiv_rn(xr, sc[lane * E + e]));
+        q8 = fminf(fmaxf(q8, -128.0f), 127.0f);
+        dst[lane * E + e] = static_cast<int8_t>(static_cast<int>(q8));
+      }
+    }
+  }
+  flag(P.status, bits);
+}
+
+size_t prologue_smem_bytes(int B, int D) {
+  return sizeof(int32_t) * (size_t)(2 * B + 2) + sizeof(float) * (size_t)(kProThreads / 32) * D;
+}
+
+template <typename ActT, typename CacheT>
+static int launch_pro_t(const QkvParams& P, cudaStream_t stream) {
+  const int NH = P.H_q + 2 * P.H_kv;
+  const long long rows = (long long)P.T * NH;
+  long long grid = (rows + (kProThreads / 32) - 1) / (kProThreads / 32);
+  if (grid < 1) grid = 1;
+  if (grid > 148 * 16) grid = 148 * 16;
+  const size_t smem = prologue_smem_bytes(P.B, P.D);
+  if (P.D == 64) {
+    auto kern = prepare_qkv_append_kernel<ActT, CacheT, 2>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kProThreads), smem, stream, P);
+  }
+  auto kern = prepare_qkv_append_kernel<ActT, CacheT, 4>;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kProThreads), smem, stream, P);
+}
+
+int launch_prepare_qkv_append(const QkvParams& P, int act, int cache, cudaStream_t stream) {
+  if (cache == SPA_I8) {
+    if (act == SPA_F32) return launch_pro_t<float, int8_t>(P, stream);
+    if (act == SPA_F16) return launch_pro_t<__half, int8_t>(P, stream);
+    return launch_pro_t<__nv_bfloat16, int8_t>(P, stream);
+  }
+  if (act == SPA_F32) return launch_pro_t<float, float>(P, stream);
+  if (act == SPA_F16) return launch_pro_t<__half, __half>(P, stream);
+  return launch_pro_t<__nv_bfloat16, __nv_bfloat16>(P, stream);
+}
+
+}  // namespace spa

@@ -47,7 +47,9 @@ class Step:
 
     mode "step": spa_prepare_append_attention (one launch where the path
     allows it); "prepare_append": spa_prepare_append_kv then spa_attention;
-    "staged": spa_prepare_metadata, spa_append_kv, spa_attention.
+    "staged": spa_prepare_metadata, spa_append_kv, spa_attention.  A workload
+    with a QKV prologue runs spa_prepare_qkv_append (metadata, prologue,
+    append) and then spa_attention on the prologue's q, whatever the mode.
     """
 
     def __init__(self, wl, d: Dict[str, torch.Tensor], num_splits: int = 0,
@@ -67,7 +69,25 @@ class Step:
         self.num_splits = num_splits
         self.kw = attention_kwargs(wl, d)
         meta = dict(self.meta, cu_seqlens_q=d["cu_seqlens_q"], status=self.status)
-        self.args = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], d["block_table"], meta,
+        self.pro = getattr(wl, "prologue", None)
+        q_att = d["q"]
+        if self.pro:
+            self.q_pro = torch.empty_like(d["q"])
+            q_att = self.q_pro
+            packed = bool(self.pro.get("packed"))
+            self.qargs = spa.qkv_args(
+                d["cu_seqlens_q"], d["past_seqlens"], d["block_table"], T, wl.max_seqlen_q,
+                wl.max_seqlen_k, self.meta, H_q=wl.H_q, q_out=self.q_pro, k_cache=d["k_cache"],
+                v_cache=d["v_cache"], qkv=d["qkv"] if packed else None,
+                q=None if packed else d["q"], k=None if packed else d["k_new"],
+                v=None if packed else d["v_new"], q_norm_weight=d.get("q_norm_weight"),
+                k_norm_weight=d.get("k_norm_weight"), norm_eps=self.pro.get("eps", 1e-6),
+                cos_cache=d.get("cos_cache"), sin_cache=d.get("sin_cache"),
+                rotary_dim=self.pro.get("rotary_dim", 0),
+                rotary_interleaved=self.pro.get("interleaved", False),
+                position_ids=d.get("position_ids"), rotary_offset=self.pro.get("rotary_offset", 0),
+                k_scale=d.get("k_scale"), v_scale=d.get("v_scale"), status=self.status)
+        self.args = spa.attention_args(q_att, d["k_cache"], d["v_cache"], d["block_table"], meta,
                                        max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
                                        out=self.out, lse=self.lse, num_splits=num_splits,
                                        status=self.status, **self.kw)
@@ -75,12 +95,18 @@ class Step:
 
     def launches(self) -> int:
         """Kernel launches one call makes."""
+        if self.pro:
+            return 1 + spa.attention_plan(self.args)["launches"]
         if self.mode == "step":
             return spa.prepare_append_attention_launches(self.args)
         return (1 if self.mode == "prepare_append" else 2) + spa.attention_plan(self.args)["launches"]
 
     def __call__(self):
         wl, d = self.wl, self.d
+        if self.pro:
+            spa.run_prepare_qkv_append(self.qargs, d["q"].device)
+            spa.run_attention(self.args, self.workspace)
+            return self.out
         if self.mode == "step":
             spa.run_prepare_append_attention(self.args, d["past_seqlens"], d["k_new"], d["v_new"],
                                              self.meta["slot_mapping"], self.workspace)
@@ -115,4 +141,6 @@ def run_step(wl, device="cuda", num_splits: int = 0, want_lse: bool = True, mode
         res["lse"] = st.lse.cpu().numpy().astype(np.float64)
     res["k_cache"] = d["k_cache"].cpu()
     res["v_cache"] = d["v_cache"].cpu()
+    if st.pro:
+        res["q_out"] = st.q_pro.cpu()
     return res

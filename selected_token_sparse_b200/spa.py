@@ -21,8 +21,10 @@ SPA_F32, SPA_F16, SPA_BF16, SPA_I8 = 0, 1, 2, 3
 SPA_OK, SPA_ERR_INVALID_ARG, SPA_ERR_UNSUPPORTED, SPA_ERR_WORKSPACE, SPA_ERR_CUDA = 0, -1, -2, -3, -4
 ST_BAD_CU, ST_CAPACITY, ST_BAD_BLOCK, ST_BOUNDS, ST_BAD_IDX = 0x1, 0x2, 0x4, 0x8, 0x10
 
-EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_prepare_append_kv", "spa_attention",
-            "spa_attention_workspace_size", "spa_attention_plan", "spa_error_string")
+EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_prepare_append_kv", "spa_prepare_qkv_append",
+            "spa_attention", "spa_attention_workspace_size", "spa_attention_plan",
+            "spa_prepare_append_attention", "spa_prepare_append_attention_launches",
+            "spa_attention_noalloc", "spa_error_string")
 
 _DT = {torch.float32: SPA_F32, torch.float16: SPA_F16, torch.bfloat16: SPA_BF16, torch.int8: SPA_I8}
 
@@ -48,6 +50,26 @@ class AttentionArgs(ctypes.Structure):
         ("aux_k", _vp), ("aux_v", _vp), ("aux_cap", _i32), ("aux_seqlens", _vp),
         ("sinks", _vp), ("scale", ctypes.c_float), ("lse", _vp),
         ("num_splits", _i32), ("status", _vp),
+    ]
+
+
+class QkvArgs(ctypes.Structure):
+    """Mirror of spa_qkv_args_t (include/spa.h)."""
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("cu_seqlens_q", _vp), ("past_seqlens", _vp), ("block_table", _vp),
+        ("B", _i32), ("T", _i32), ("max_seqlen_q", _i32), ("max_seqlen_k", _i32), ("MB", _i32),
+        ("block_size", _i32), ("num_blocks", _i32),
+        ("seqlens_q", _vp), ("seqlen_k", _vp), ("token_batch", _vp), ("token_pos", _vp),
+        ("slot_mapping", _vp),
+        ("act", _i32), ("H_q", _i32), ("H_kv", _i32), ("D", _i32),
+        ("qkv", _vp), ("q", _vp), ("k", _vp), ("v", _vp),
+        ("q_norm_weight", _vp), ("k_norm_weight", _vp), ("norm_eps", ctypes.c_float),
+        ("cos_cache", _vp), ("sin_cache", _vp),
+        ("max_pos", _i32), ("rotary_dim", _i32), ("rotary_interleaved", _i32),
+        ("position_ids", _vp), ("rotary_offset", _i32),
+        ("q_out", _vp), ("k_cache", _vp), ("v_cache", _vp), ("cache", _i32),
+        ("k_scale", _vp), ("v_scale", _vp), ("status", _vp),
     ]
 
 
@@ -83,6 +105,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                  ctypes.c_size_t, _vp]
     lib.spa_prepare_append_attention_launches.restype = ctypes.c_int
     lib.spa_prepare_append_attention_launches.argtypes = [ctypes.POINTER(AttentionArgs)]
+    lib.spa_prepare_qkv_append.restype = ctypes.c_int
+    lib.spa_prepare_qkv_append.argtypes = [ctypes.POINTER(QkvArgs), _vp]
     lib.spa_error_string.restype = ctypes.c_char_p
     lib.spa_error_string.argtypes = [ctypes.c_int]
     return lib
@@ -195,6 +219,50 @@ def prepare_append_kv(cu_seqlens_q: torch.Tensor, past_seqlens: torch.Tensor,
     _check(rc, "spa_prepare_append_kv")
     out["cu_seqlens_q"] = cu_seqlens_q
     return out
+
+
+def qkv_args(cu_seqlens_q: torch.Tensor, past_seqlens: torch.Tensor, block_table: torch.Tensor, T: int,
+             max_seqlen_q: int, max_seqlen_k: int, meta: Dict[str, torch.Tensor], *, H_q: int,
+             q_out: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+             qkv: Optional[torch.Tensor] = None, q: Optional[torch.Tensor] = None,
+             k: Optional[torch.Tensor] = None, v: Optional[torch.Tensor] = None,
+             q_norm_weight: Optional[torch.Tensor] = None, k_norm_weight: Optional[torch.Tensor] = None,
+             norm_eps: float = 1e-6, cos_cache: Optional[torch.Tensor] = None,
+             sin_cache: Optional[torch.Tensor] = None, rotary_dim: int = 0, rotary_interleaved: bool = False,
+             position_ids: Optional[torch.Tensor] = None, rotary_offset: int = 0,
+             k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
+             status: Optional[torch.Tensor] = None) -> QkvArgs:
+    """Arguments of spa_prepare_qkv_append (steps 1, prologue, 2); `meta` holds the
+    five metadata output arrays."""
+    NB, bs, H_kv, D = k_cache.shape
+    a = QkvArgs()
+    a.struct_size = ctypes.sizeof(QkvArgs)
+    a.cu_seqlens_q, a.past_seqlens, a.block_table = _ptr(cu_seqlens_q), _ptr(past_seqlens), _ptr(block_table)
+    a.B, a.T = cu_seqlens_q.numel() - 1, T
+    a.max_seqlen_q, a.max_seqlen_k = max_seqlen_q, max_seqlen_k
+    a.MB = block_table.shape[1] if block_table.dim() == 2 else 0
+    a.block_size, a.num_blocks = bs, NB
+    a.seqlens_q, a.seqlen_k = _ptr(meta["seqlens_q"]), _ptr(meta["seqlen_k"])
+    a.token_batch, a.token_pos, a.slot_mapping = (_ptr(meta["token_batch"]), _ptr(meta["token_pos"]),
+                                                  _ptr(meta["slot_mapping"]))
+    a.act = _DT[q_out.dtype]
+    a.H_q, a.H_kv, a.D = H_q, H_kv, D
+    a.qkv, a.q, a.k, a.v = _ptr(qkv), _ptr(q), _ptr(k), _ptr(v)
+    a.q_norm_weight, a.k_norm_weight, a.norm_eps = _ptr(q_norm_weight), _ptr(k_norm_weight), float(norm_eps)
+    a.cos_cache, a.sin_cache = _ptr(cos_cache), _ptr(sin_cache)
+    a.max_pos = cos_cache.shape[0] if cos_cache is not None else 0
+    a.rotary_dim = rotary_dim if cos_cache is not None else 0
+    a.rotary_interleaved = 1 if rotary_interleaved else 0
+    a.position_ids, a.rotary_offset = _ptr(position_ids), rotary_offset
+    a.q_out, a.k_cache, a.v_cache, a.cache = _ptr(q_out), _ptr(k_cache), _ptr(v_cache), _DT[k_cache.dtype]
+    a.k_scale, a.v_scale = _ptr(k_scale), _ptr(v_scale)
+    a.status = _ptr(status)
+    return a
+
+
+def run_prepare_qkv_append(args: QkvArgs, device) -> None:
+    """Enqueue spa_prepare_qkv_append for prepared arguments on the current stream."""
+    _check(lib().spa_prepare_qkv_append(ctypes.byref(args), _stream(device)), "spa_prepare_qkv_append")
 
 
 def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

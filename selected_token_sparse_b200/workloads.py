@@ -342,8 +342,27 @@ def windowed_chunked_prefill_f16(seed: int = 5, small: bool = False) -> Workload
                          block_size=16, q_lens=q_lens, past=past, window=128, has_sinks=True, seed=seed)
 
 
+# Workloads that run the QKV prologue ahead of the append.
+PROLOGUE_WORKLOADS = ("qkv_prologue_selected_decode_bf16",)
+
+
+def qkv_prologue_selected_decode_bf16(seed: int = 6, small: bool = False) -> Workload:
+    """Selected-token decode fed by the QKV prologue: packed QKV, QK RMSNorm and
+    rotary embedding over all D channels (half-split pairs) ahead of the append;
+    B=16, H_q=32, H_kv=4, D=128, cache length 8192 paged in blocks of 64, 1024
+    sorted selected indices per (request, kv head) with 5% -1 padding, sinks, bf16."""
+    B = 3 if small else 16
+    L = 700 if small else 8192
+    W_sel = 100 if small else 1024
+    return make_workload(name="qkv_prologue_selected_decode_bf16", act="bf16", B=B, H_q=32, H_kv=4,
+                         D=128, block_size=64, q_lens=[1] * B, past=[L - 1] * B, sel_mode="main",
+                         sel_per_request=1, sel_width=W_sel, sel_sorted=True,
+                         sel_tail_pad=W_sel // 20, has_sinks=True,
+                         prologue=dict(packed=True, qk_norm=True, rotary_dim=128), seed=seed)
+
+
 def by_name(name: str, small: bool = False, seed: Optional[int] = None) -> Workload:
-    fn = {n: globals()[n] for n in WORKLOADS}[name]
+    fn = {n: globals()[n] for n in WORKLOADS + PROLOGUE_WORKLOADS}[name]
     if seed is None:
         return fn(small=small)
     return fn(seed=seed, small=small)

@@ -71,3 +71,22 @@ def test_workspace_size_for_invalid_args_is_zero(lib):
     a.is_causal = 0
     assert lib.spa_attention_workspace_size(ctypes.byref(a)) == 0
     assert lib.spa_attention(ctypes.byref(a), None, 0, None) == spa.SPA_ERR_UNSUPPORTED
+
+
+def test_qkv_struct_layout_matches_header(tmp_path):
+    fields = [f[0] for f in spa.QkvArgs._fields_]
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "spa.h"', "int main(void) {",
+            'printf("size %zu\\n", sizeof(spa_qkv_args_t));']
+    for f in fields:
+        prog.append(f'printf("{f} %zu\\n", offsetof(spa_qkv_args_t, {f}));')
+    prog.append("return 0; }")
+    c = tmp_path / "layout_qkv.c"
+    c.write_text("\n".join(prog))
+    exe = tmp_path / "layout_qkv"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)],
+                   check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    assert int(got["size"]) == ctypes.sizeof(spa.QkvArgs)
+    for f in fields:
+        assert int(got[f]) == getattr(spa.QkvArgs, f).offset, f
