@@ -47,17 +47,32 @@ prepare_qkv_append_kernel(const QkvParams P) {
   float* xrow = rows + warp * D;
   pdl_wait();
   pdl_trigger();
+  const int NH = P.H_q + 2 * P.H_kv;
+  const long long rows_total = (long long)P.T * NH;
+  // source row (token t, head hh) of the packed or separate q / k / v
+  auto row_src = [&](int t, int hh) -> const ActT* {
+    if (P.qkv) return static_cast<const ActT*>(P.qkv) + ((long long)t * NH + hh) * D;
+    const int kind = hh < P.H_q ? 0 : (hh < P.H_q + P.H_kv ? 1 : 2);
+    const int h = kind == 0 ? hh : (kind == 1 ? hh - P.H_q : hh - P.H_q - P.H_kv);
+    const void* base = kind == 0 ? P.q : (kind == 1 ? P.k : P.v);
+    return static_cast<const ActT*>(base) + ((long long)t * (kind == 0 ? P.H_q : P.H_kv) + h) * D;
+  };
+  // the warp's first row is loaded before the metadata is known
+  const long long r0 = (long long)blockIdx.x * (kProThreads / 32) + warp;
+  ActT x0[E];
+  if (r0 < rows_total) {
+    const ActT* src = row_src((int)(r0 / NH), (int)(r0 % NH));
+#pragma unroll
+    for (int e = 0; e < E; ++e) x0[e] = src[lane * E + e];
+  }
   for (int b = threadIdx.x; b < P.B; b += blockDim.x) past_s[b] = P.past[b];
   build_cs<kProThreads>(P.cu, P.B, P.T, cs);
   int bits = 0;
   if (blockIdx.x == 0)
     bits |= per_request(P.cu, past_s, cs, P.B, P.T, P.max_q, P.max_k, P.seqlens_q, P.seqlen_k);
-  const int NH = P.H_q + 2 * P.H_kv;
   const bool rope = P.cos_cache != nullptr && P.rotary_dim > 0;
   const int rd = P.rotary_dim, half = rd / 2;
-  const long long rows_total = (long long)P.T * NH;
-  for (long long r = (long long)blockIdx.x * (kProThreads / 32) + warp; r < rows_total;
-       r += (long long)gridDim.x * (kProThreads / 32)) {
+  for (long long r = r0; r < rows_total; r += (long long)gridDim.x * (kProThreads / 32)) {
     const int t = (int)(r / NH), hh = (int)(r % NH);
     int tb = 0;
     const TokenMeta m = token_meta(t, cs, P.B, past_s, P.block_table, P.MB, P.bs, P.NB, tb);
@@ -70,17 +85,15 @@ prepare_qkv_append_kernel(const QkvParams P) {
     const int kind = hh < P.H_q ? 0 : (hh < P.H_q + P.H_kv ? 1 : 2);   // q, k, v
     const int h = kind == 0 ? hh : (kind == 1 ? hh - P.H_q : hh - P.H_q - P.H_kv);
     if (kind != 0 && m.slot < 0) continue;   // nothing to append
-    const ActT* src;
-    if (P.qkv) {
-      src = static_cast<const ActT*>(P.qkv) + ((long long)t * NH + hh) * D;
-    } else {
-      const void* base = kind == 0 ? P.q : (kind == 1 ? P.k : P.v);
-      const int H = kind == 0 ? P.H_q : P.H_kv;
-      src = static_cast<const ActT*>(base) + ((long long)t * H + h) * D;
-    }
     float x[E];
+    if (r == r0) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) x[e] = to_f32(src[lane * E + e]);
+      for (int e = 0; e < E; ++e) x[e] = to_f32(x0[e]);
+    } else {
+      const ActT* src = row_src(t, hh);
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = to_f32(src[lane * E + e]);
+    }
     if (kind != 2) {
       const float* w = kind == 0 ? P.q_norm : P.k_norm;
       if (w != nullptr) {
