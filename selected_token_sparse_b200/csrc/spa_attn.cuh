@@ -356,74 +356,68 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, 
 // unit form one cluster (rank = split); each has left its partial state at
 // the same shared-memory offsets: o [rows][D + 4] fp32 (row stride D + 4) and
 // (m, l) [rows][2], log2 units.  After a cluster barrier, CTA k merges rows
-// k, k + S, k + 2S, ... with the sink exactly as merge_rows does (pass 1: one
-// thread per row; pass 2: one thread per 4 output columns), reading the peers'
-// shared memory.  The caller ends with another cluster barrier so that no CTA
-// leaves while its state is being read.
+// k, k + S, k + 2S, ... with the sink as merge_rows does, in one pass: each
+// thread takes 4 output columns of a row, reads every split's (m, l) and
+// partial columns from the peers' shared memory at once, and forms the
+// weights itself.  The caller ends with another cluster barrier so that no
+// CTA leaves while its state is being read.
 constexpr int kClusterMaxSplits = 8;
 
 template <typename ActT, int D>
 __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, int nq, int h_kv,
                                                    const float* part_o, const float* part_ml) {
-  __shared__ float sW[kMergeRows][kClusterMaxSplits];
-  __shared__ float sInv[kMergeRows];
-  constexpr int C4 = D / 4, PS = D + 4;
+  constexpr int C4 = D / 4, PS = D + 4, IPT = 1;   // items of a thread whose loads are in flight together
   const int S = p.num_splits, k = (int)cluster_rank();
   const int R = nq * p.G;
   const int mine = R > k ? (R - k + S - 1) / S : 0;   // rows k, k + S, ...
-  for (int i0 = 0; i0 < mine; i0 += kMergeRows) {
-    const int n = min(kMergeRows, mine - i0);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const int r = k + (i0 + i) * S;
-      const int h = h_kv * p.G + r % p.G;
-      const long long row = (long long)(t0 + r / p.G) * p.H_q + h;
-      const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
-      float2 ml[kClusterMaxSplits];
-      float M = sink2;
+  const int n_items = mine * C4;
+  for (int base = threadIdx.x; base < n_items; base += IPT * blockDim.x) {
+    float2 ml[IPT][kClusterMaxSplits];
+    float4 a[IPT][kClusterMaxSplits];
+    float sink2[IPT];
+#pragma unroll
+    for (int t = 0; t < IPT; ++t) {
+      const int it = base + t * blockDim.x;
+      const int r = k + (it / C4) * S, c = (it % C4) * 4;
+      sink2[t] = (p.sinks && it < n_items) ? ld_early(p.sinks + h_kv * p.G + r % p.G) * kLog2e : -INFINITY;
 #pragma unroll
       for (int s = 0; s < kClusterMaxSplits; ++s) {
-        ml[s] = make_float2(-INFINITY, 0.f);
-        if (s < S) ml[s] = ld_peer2(peer_smem(part_ml + 2 * r, s));
-        M = fmaxf(M, ml[s].x);
+        ml[t][s] = make_float2(-INFINITY, 0.f);
+        a[t][s] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s < S && it < n_items) {
+          ml[t][s] = ld_peer2(peer_smem(part_ml + 2 * r, s));
+          a[t][s] = ld_peer4(peer_smem(part_o + r * PS + c, s));
+        }
       }
+    }
+#pragma unroll
+    for (int t = 0; t < IPT; ++t) {
+      const int it = base + t * blockDim.x;
+      if (it >= n_items) continue;
+      const int r = k + (it / C4) * S, c = (it % C4) * 4;
+      const long long row = (long long)(t0 + r / p.G) * p.H_q + h_kv * p.G + r % p.G;
+      float M = sink2[t];
+#pragma unroll
+      for (int s = 0; s < kClusterMaxSplits; ++s) M = fmaxf(M, ml[t][s].x);
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
       float inv = 0.f, lse = -INFINITY;
       if (M != -INFINITY) {
-        float Lsum = (sink2 == -INFINITY) ? 0.f : exp2f(sink2 - M);
+        float Lsum = (sink2[t] == -INFINITY) ? 0.f : exp2f(sink2[t] - M);
 #pragma unroll
         for (int s = 0; s < kClusterMaxSplits; ++s) {
-          const float w = (ml[s].x == -INFINITY) ? 0.f : exp2f(ml[s].x - M);
-          sW[i][s] = w;
-          Lsum += w * ml[s].y;
+          const float w = (ml[t][s].x == -INFINITY) ? 0.f : exp2f(ml[t][s].x - M);
+          Lsum += w * ml[t][s].y;
+          o.x = fmaf(w, a[t][s].x, o.x);
+          o.y = fmaf(w, a[t][s].y, o.y);
+          o.z = fmaf(w, a[t][s].z, o.z);
+          o.w = fmaf(w, a[t][s].w, o.w);
         }
         inv = 1.0f / Lsum;
         lse = (M + log2f(Lsum)) * kLn2;
-      } else {
-#pragma unroll
-        for (int s = 0; s < kClusterMaxSplits; ++s) sW[i][s] = 0.f;
       }
-      sInv[i] = inv;
-      if (p.lse) p.lse[row] = lse;
-    }
-    __syncthreads();
-    for (int it = threadIdx.x; it < n * C4; it += blockDim.x) {
-      const int i = it / C4, c = (it % C4) * 4;
-      const int r = k + (i0 + i) * S;
-      const long long row = (long long)(t0 + r / p.G) * p.H_q + h_kv * p.G + r % p.G;
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int s = 0; s < kClusterMaxSplits; ++s) {
-        if (s >= S) break;
-        const float w = sW[i][s];
-        const float4 a = ld_peer4(peer_smem(part_o + r * PS + c, s));
-        o.x = fmaf(w, a.x, o.x);
-        o.y = fmaf(w, a.y, o.y);
-        o.z = fmaf(w, a.z, o.z);
-        o.w = fmaf(w, a.w, o.w);
-      }
-      const float inv = sInv[i];
       store4<ActT>(static_cast<ActT*>(p.out) + row * D + c, o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      if (c == 0 && p.lse) p.lse[row] = lse;
     }
-    __syncthreads();
   }
 }
 

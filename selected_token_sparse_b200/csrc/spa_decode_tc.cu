@@ -3,28 +3,33 @@
 // fifth-generation tensor cores.
 //
 // With tens of rows per kv head every gathered K/V row feeds a 96- or
-// 128-row contraction, so the unit is one M = 128 tcgen05 tile, and the CTA
-// splits into two roles that overlap:
+// 128-row contraction, so the unit is one M = 128 tcgen05 tile.  The CTA
+// runs three roles that overlap:
 //
 //   * producer warps (4): resolve the candidates (window positions, selected
 //     or auxiliary slots) through the block table with every guard, gather
-//     64-key tiles with cp.async, and place them as fp16 / bf16 K and V tiles
+//     64-key tiles, and place them as fp16 / bf16 K and V tiles
 //     (128-byte-swizzled; V is the MN-major B operand of PV, the same bytes)
-//     in a two-stage ring; INT8 rows go through a raw staging ring and are
-//     converted to exact fp16 integers.  A tile's "full" barrier is released
+//     in a three-stage ring.  Rows are gathered with cp.async (16-bit rows
+//     straight into place; INT8 rows into a raw staging ring, converted to
+//     exact fp16 integers).  A tile's "full" barrier is released
 //     when it is in place; its "empty" barrier is committed by the MMAs that
-//     read it, so the next tile is prepared while this one is computed;
-//   * consumer warps (8, two per TMEM lane quadrant, each half of a tile's
-//     keys): the unit's rows (token i, head g) -> row i*G + g of a Q tile in
-//     shared memory (INT8 caches fold the key scale into q, split into fp16
-//     high and low tiles, so S = Q_hi K^T + Q_lo K^T carries ~22 bits);
-//     S = Q K^T into TMEM, softmax from TMEM (mask by key position: causal /
-//     window for the main cache, always visible for auxiliary entries; a
-//     lazily raised max in log2 units), P written over S, O += P V (A from
-//     TMEM); O scaled by the value scale (INT8), then normalised with the sink
-//     and written (one split) or merged with the unit's other splits (a
+//     read it, so the next tiles are prepared while this one is computed;
+//   * softmax warps (4, one thread per TMEM lane = one row of the unit:
+//     token i, head g -> row i*G + g): the row's q goes into tensor memory
+//     (INT8 caches fold the key scale into q, split into fp16 high and low
+//     parts, so S = Q_hi K^T + Q_lo K^T carries ~22 bits); per tile, the
+//     row's 64 scores from TMEM, masked by key position (causal / window for
+//     the main cache, always visible for auxiliary entries), a lazily raised
+//     max in log2 units, P into one of two TMEM buffers of its own; at the
+//     end O is scaled by the value scale (INT8), normalised with the sink and
+//     written (one split) or merged with the unit's other splits (a
 //     thread-block cluster through distributed shared memory, else the
-//     workspace).
+//     workspace);
+//   * an MMA warp (one thread): S = Q K^T into one of two TMEM buffers, the
+//     next tile's S ahead of this tile's PV so that it is computed while the
+//     softmax runs, and O += P V (A from TMEM) once the four softmax warps
+//     have placed P.
 //
 // Sources: "[WebGPU] Add DynamicSparseAttention" (Attention: selected and
 // local-plus-auxiliary modes, joint FP32 stable softmax with optional sink),
@@ -41,13 +46,17 @@ namespace spa {
 using namespace sm100;
 
 constexpr int kTcKT = 64;                       // keys per tile (MMA N)
-constexpr int kTcCons = 256;                    // consumer threads (8 warps)
+constexpr int kTcStages = 3;                    // K/V tiles in the ring
+constexpr int kTcCons = 128;                    // softmax threads (4 warps, one per row)
 constexpr int kTcProd = 128;                    // producer threads (4 warps)
-constexpr int kTcThreads = kTcCons + kTcProd;
-constexpr int kTcBarCons = 1, kTcBarProd = 2;   // named barriers of the two roles
+constexpr int kTcMmaTid = kTcCons + kTcProd;    // the MMA-issuing thread (its own warp)
+constexpr int kTcThreads = kTcCons + kTcProd + 32;
+constexpr int kTcBarProd = 2;                   // named barrier of the producers
 constexpr int kTcCandTiles = 8;                 // tiles whose candidates are resolved at once
 constexpr int kTcCand = kTcCandTiles * kTcKT;
-constexpr uint32_t kTcTmemCols = 256;           // S [0, 64) | O [128, 128 + D)
+// tensor memory columns: S[2] | O | P[2] (packed 16-bit pairs) | Q_hi | Q_lo
+constexpr uint32_t kTcColS = 0, kTcColO = 128, kTcColP = 256, kTcColQ = 320;
+constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcWaitLimit = 1u << 20;
 
 int tc_key_tile() { return kTcKT; }
@@ -57,29 +66,29 @@ struct TcCfg {
   static constexpr bool kInt8 = sizeof(CacheT) == 1;
   using MT = typename std::conditional<kInt8, __half, ActT>::type;
   static constexpr int NCH = D / 64;
-  static constexpr int QTILE = NCH * 128 * 128;       // 128 rows x D, 16-bit, swizzled
   static constexpr int KCHUNK = kTcKT * 128;          // one 64-column chunk of a 64-row tile
   static constexpr int KTILE = NCH * KCHUNK;          // 64 rows x D, 16-bit, swizzled
   static constexpr int ROW_BYTES = D * (int)sizeof(CacheT);
   static constexpr int RAW = kTcKT * ROW_BYTES;       // one staged INT8 K or V tile
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_QLO = OFF_Q + QTILE;
-  static constexpr int OFF_CONV = OFF_QLO + (kInt8 ? QTILE : 0);    // [2 stages][K, V]
-  static constexpr int OFF_RAW = OFF_CONV + 4 * KTILE;              // INT8: [2 stages][K, V]
-  static constexpr int OFF_KVIS = OFF_RAW + (kInt8 ? 4 * RAW : 0);  // [2][64] visible row intervals
-  static constexpr int OFF_TVIS = OFF_KVIS + 2 * kTcKT * 8;         // [2] tile seen by every row
-  static constexpr int OFF_CAND = OFF_TVIS + 16;                    // [2 chunks] offsets + positions
-  static constexpr int OFF_RED = OFF_CAND + 2 * kTcCand * 12;       // [2][128] row max, [2][128] sum
-  static constexpr int OFF_SCALE = OFF_RED + 4 * 128 * 4;           // INT8: ks, vs
-  static constexpr int OFF_BAR = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);  // s, o, full[2], empty[2]
-  static constexpr int OFF_MISC = OFF_BAR + 6 * 8;                  // tmem holder, abort flag
-  static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int SMEM = BYTES + 1024;
-  // cluster split merge: partial o [128][D + 4] and (m, l) [128][2], fp32, over
-  // Q and the K/V ring once every tile is consumed
+  static constexpr int RAW_ST = kInt8 ? 2 : 0;        // raw stages (INT8)
+  static constexpr int OFF_CONV = 0;                                   // [stage][K, V]
+  static constexpr int OFF_RAW = OFF_CONV + kTcStages * 2 * KTILE;     // INT8: [raw stage][K, V]
+  static constexpr int END_RING = OFF_RAW + RAW_ST * 2 * RAW;
+  // cluster split merge: partial o [128][D + 4] and (m, l) [128][2], fp32,
+  // over the rings once every tile is consumed
   static constexpr int OFF_PART = 0;
   static constexpr int PART_ML = OFF_PART + 128 * (D + 4) * 4;
-  static_assert(PART_ML + 128 * 2 * 4 <= OFF_KVIS, "partial state must fit over Q and the K/V ring");
+  static constexpr int END_PART = PART_ML + 128 * 2 * 4;
+  static constexpr int OFF_KVIS = END_RING > END_PART ? END_RING : END_PART;  // [stage][64] row intervals
+  static constexpr int OFF_TVIS = OFF_KVIS + kTcStages * kTcKT * 8;           // [stage] tile seen by every row
+  static constexpr int OFF_CAND = OFF_TVIS + 16;                    // [2 chunks] offsets + positions
+  static constexpr int OFF_SCALE = OFF_CAND + 2 * kTcCand * 12;     // INT8: ks, vs
+  static constexpr int NBAR = 2 * kTcStages + 7;   // full, empty, s[2], o[2], p[2], q
+  static constexpr int OFF_BAR = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;                  // tmem holder, abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  // at least 120 KB, so one CTA holds an SM and its 512 TMEM columns
+  static constexpr int SMEM = BYTES + 1024 > 120 * 1024 ? BYTES + 1024 : 120 * 1024;
 };
 
 // byte offset of 16-byte unit u (0 .. D/8-1) of row r in a ROWS-row swizzled tile
@@ -131,6 +140,24 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
   return r;
 }
 
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+  static_assert(N == 16 || N == 32, "columns");
+  if constexpr (N == 32) tmem_st32(taddr, r);
+  else tmem_st16(taddr, r);
+}
+
 template <typename ActT, typename CacheT, int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const AttnParams p) {
@@ -139,17 +166,17 @@ decode_tc_kernel(const AttnParams p) {
   constexpr uint32_t FMT = std::is_same<MT, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = idesc_f16(FMT, 128, kTcKT, 0);
   constexpr uint32_t IDESC_O = idesc_f16(FMT, 128, D, 1);
-  constexpr int KT = kTcKT;
-  constexpr int HK = KT / 2, HD = D / 2;   // key columns / O columns per consumer half
+  constexpr int KT = kTcKT, NST = kTcStages;
   constexpr int CPR = C::ROW_BYTES / 16;   // 16-byte chunks per gathered row
+  constexpr uint32_t QCOLS = D / 2;        // TMEM columns of one Q part (two 16-bit values each)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = tid >= kTcCons;
+  const bool softmax = tid < kTcCons;
+  const bool producer = !softmax && tid < kTcCons + kTcProd;
   const int ptid = tid - kTcCons;             // producer thread index
-  const int quad = warp & 3, half = (warp >> 2) & 1;
-  const int row = quad * 32 + lane;           // consumer: the S / O row (TMEM lane)
+  const int row = tid;                        // softmax: the S / O row (TMEM lane)
   __shared__ int last_flag;
   pdl_wait();
   pdl_trigger();
@@ -170,32 +197,25 @@ decode_tc_kernel(const AttnParams p) {
   // query positions of the unit's rows: [p_lo, p_hi]
   const int p_lo = has_rows ? U.p_first : 0, p_hi = has_rows ? U.p_last : -1;
 
-  unsigned char* sQ = smem + C::OFF_Q;
-  unsigned char* sQlo = smem + C::OFF_QLO;
   int2* kvis_s = reinterpret_cast<int2*>(smem + C::OFF_KVIS);
   int* tvis_s = reinterpret_cast<int*>(smem + C::OFF_TVIS);
   // candidate chunks are double-buffered: resolving chunk c + 1 leaves the
   // tiles of chunk c still in flight untouched
   long long* cand_off = reinterpret_cast<long long*>(smem + C::OFF_CAND);
   int* cand_kpos = reinterpret_cast<int*>(smem + C::OFF_CAND + 2 * kTcCand * 8);
-  float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);
-  float* red_l = red_max + 2 * 128;
   float* ksc = reinterpret_cast<float*>(smem + C::OFF_SCALE);
   float* vsc = ksc + D;
-  uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* bar_o = bar_s + 1;
-  uint64_t* bar_full = bar_s + 2;    // [2] tile in place (one producer arrival)
-  uint64_t* bar_empty = bar_s + 4;   // [2] tile's MMAs complete (tcgen05.commit)
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);   // [NST] tile in place
+  uint64_t* bar_empty = bar_full + NST;   // [NST] tile's MMAs complete (tcgen05.commit)
+  uint64_t* bar_s = bar_empty + NST;      // [2] S of tile j in buffer j % 2 complete
+  uint64_t* bar_o = bar_s + 2;            // [2] PV of tile j (P buffer j % 2) complete
+  uint64_t* bar_p = bar_o + 2;            // [2] P of tile j placed by the four softmax warps
+  uint64_t* bar_q = bar_p + 2;            // Q in tensor memory (four softmax warps)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
 
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_full + i, 1);
-      mbar_init(bar_empty + i, 1);
-    }
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar_full + i, i >= 2 * NST + 4 ? kTcCons / 32 : 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -210,20 +230,18 @@ decode_tc_kernel(const AttnParams p) {
     }
   }
   int bits = 0;
-  // consumer: Q rows (row r = token r / G, head r % G) in coalesced 16-byte
-  // units, in flight across the set-up
-  constexpr int QU = D / 8;
-  constexpr int QPER = 128 * QU / kTcCons;
-  uint4 qv[QPER];
+  // softmax: Q row `row` (token row / G, head row % G), in flight across the set-up
+  constexpr int QV = D / 8;
+  uint4 qv[QV];
   float sink_raw = -INFINITY;
-  if (!producer) {
-    const ActT* q = static_cast<const ActT*>(p.q);
+  if (softmax) {
 #pragma unroll
-    for (int k = 0; k < QPER; ++k) {
-      const int i = tid + k * kTcCons, r = i / QU, u = i % QU;
-      qv[k] = make_uint4(0, 0, 0, 0);
-      if (r < R)
-        qv[k] = *reinterpret_cast<const uint4*>(q + ((long long)(t0 + r / G) * p.H_q + h_kv * G + r % G) * D + u * 8);
+    for (int k = 0; k < QV; ++k) qv[k] = make_uint4(0, 0, 0, 0);
+    if (row < R) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          static_cast<const ActT*>(p.q) + ((long long)(t0 + row / G) * p.H_q + h_kv * G + row % G) * D);
+#pragma unroll
+      for (int k = 0; k < QV; ++k) qv[k] = src[k];
     }
     // the epilogue's sink logit of row `row`
     if (p.sinks && p.num_splits == 1 && row < R) sink_raw = ld_early(p.sinks + h_kv * G + row % G);
@@ -270,9 +288,12 @@ decode_tc_kernel(const AttnParams p) {
     };
     // cp.async copies of tile j: into the raw ring (INT8) or straight into the
     // swizzled K / V stage (16-bit caches)
+    constexpr int NIT = KT * CPR * 2 / kTcProd;   // 16-byte chunks per producer thread and tile
+    static_assert(KT * CPR * 2 % kTcProd == 0, "chunks per thread");
     auto issue = [&](int j) {
-      const int st = j & 1;
-      for (int e = ptid; e < KT * CPR * 2; e += kTcProd) {
+#pragma unroll 8
+      for (int k = 0; k < NIT; ++k) {
+        const int e = ptid + k * kTcProd;
         const bool isv = e >= KT * CPR;
         const int ee = isv ? e - KT * CPR : e;
         const int r = ee / CPR, ch = ee % CPR;
@@ -284,9 +305,9 @@ decode_tc_kernel(const AttnParams p) {
         const CacheT* src = okr ? base + off + ch * (16 / sizeof(CacheT)) : kc;
         unsigned char* dst;
         if constexpr (C::kInt8) {
-          dst = smem + C::OFF_RAW + (st * 2 + (isv ? 1 : 0)) * C::RAW + r * C::ROW_BYTES + ch * 16;
+          dst = smem + C::OFF_RAW + ((j & 1) * 2 + (isv ? 1 : 0)) * C::RAW + r * C::ROW_BYTES + ch * 16;
         } else {
-          dst = smem + C::OFF_CONV + (st * 2 + (isv ? 1 : 0)) * C::KTILE + sw_off<KT>(r, ch);
+          dst = smem + C::OFF_CONV + ((j % NST) * 2 + (isv ? 1 : 0)) * C::KTILE + sw_off<KT>(r, ch);
         }
         cp_async_16(dst, src, okr);
       }
@@ -296,7 +317,7 @@ decode_tc_kernel(const AttnParams p) {
     // or j .. with no window); returns whether every key this thread placed
     // is visible to every row of the unit
     auto place_vis = [&](int j) -> bool {
-      const int st = j & 1;
+      const int st = j % NST;
       bool all_vis = true;
       for (int r = ptid; r < KT; r += kTcProd) {
         const int kp = cand_kpos[cslot(j, r)];
@@ -315,15 +336,16 @@ decode_tc_kernel(const AttnParams p) {
       return all_vis;
     };
     bool ok = true;
-    auto wait_empty = [&](int j) {   // the MMAs of tile j - 2 (same stage) are complete
-      if (j >= 2 && ok) ok = mbar_wait(bar_empty + (j & 1), ((j >> 1) - 1) & 1, kTcWaitLimit, abort_flag);
+    auto wait_empty = [&](int j) {   // the MMAs of tile j - NST (same stage) are complete
+      if (j >= NST && ok)
+        ok = mbar_wait(bar_empty + j % NST, ((j / NST) - 1) & 1, kTcWaitLimit, abort_flag);
     };
     auto publish = [&](int j, bool all_vis) {   // tile j in place: release its full barrier
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       const bool tv = bar_red_and(all_vis, kTcBarProd, kTcProd);
       if (ptid == 0) {
-        tvis_s[j & 1] = tv ? 1 : 0;
-        mbar_arrive(bar_full + (j & 1));
+        tvis_s[j % NST] = tv ? 1 : 0;
+        mbar_arrive(bar_full + j % NST);
       }
     };
     if (ntiles > 0) resolve_chunk(0);
@@ -348,21 +370,29 @@ decode_tc_kernel(const AttnParams p) {
           ok = false;
           break;
         }
-        const int st = j & 1;
-        unsigned char* kcv = smem + C::OFF_CONV + st * 2 * C::KTILE;
+        unsigned char* kcv = smem + C::OFF_CONV + (j % NST) * 2 * C::KTILE;
         unsigned char* vcv = kcv + C::KTILE;
-        const unsigned char* rawp = smem + C::OFF_RAW + st * 2 * C::RAW;
-#pragma unroll 2
-        for (int e = ptid; e < KT * CPR * 2; e += kTcProd) {
+        const unsigned char* rawp = smem + C::OFF_RAW + (j & 1) * 2 * C::RAW;
+        // every raw chunk of this thread is read before any is converted
+        uint4 rv[NIT];
+#pragma unroll
+        for (int k = 0; k < NIT; ++k) {
+          const int e = ptid + k * kTcProd;
+          const bool isv = e >= KT * CPR;
+          const int ee = isv ? e - KT * CPR : e;
+          rv[k] = *reinterpret_cast<const uint4*>(rawp + (isv ? C::RAW : 0) + (ee / CPR) * C::ROW_BYTES + (ee % CPR) * 16);
+        }
+#pragma unroll
+        for (int k = 0; k < NIT; ++k) {
+          const int e = ptid + k * kTcProd;
           const bool isv = e >= KT * CPR;
           const int ee = isv ? e - KT * CPR : e;
           const int r = ee / CPR, ch = ee % CPR;
-          const uint4 rv = *reinterpret_cast<const uint4*>(rawp + (isv ? C::RAW : 0) + r * C::ROW_BYTES + ch * 16);
           uint4 h0, h1;
-          i8x4_to_h2x2(rv.x, h0.x, h0.y);
-          i8x4_to_h2x2(rv.y, h0.z, h0.w);
-          i8x4_to_h2x2(rv.z, h1.x, h1.y);
-          i8x4_to_h2x2(rv.w, h1.z, h1.w);
+          i8x4_to_h2x2(rv[k].x, h0.x, h0.y);
+          i8x4_to_h2x2(rv[k].y, h0.z, h0.w);
+          i8x4_to_h2x2(rv[k].z, h1.x, h1.y);
+          i8x4_to_h2x2(rv[k].w, h1.z, h1.w);
           unsigned char* dst = isv ? vcv : kcv;
           *reinterpret_cast<uint4*>(dst + sw_off<KT>(r, 2 * ch)) = h0;
           *reinterpret_cast<uint4*>(dst + sw_off<KT>(r, 2 * ch + 1)) = h1;
@@ -370,17 +400,20 @@ decode_tc_kernel(const AttnParams p) {
         publish(j, place_vis(j));
       }
     } else {
-      // two tiles in flight; tile j + 2 goes into tile j's stage once its MMAs are done
-      for (int j = 0; j < 2 && j < ntiles; ++j) {
+      // NST tiles in flight; tile j + NST goes into tile j's stage once its MMAs are done
+      for (int j = 0; j < NST && j < ntiles; ++j) {
         issue(j);
         cp_async_commit();
       }
       for (int j = 0; j < ntiles && ok; ++j) {
-        if (j + 1 < ntiles) cp_async_wait<1>();
+        // groups committed after tile j's: min(j + NST - 1, ntiles - 1) - j
+        const int newer = min(j + NST - 1, ntiles - 1) - j;
+        if (newer >= 2) cp_async_wait<2>();
+        else if (newer == 1) cp_async_wait<1>();
         else cp_async_wait<0>();
         bar_sync(kTcBarProd, kTcProd);   // tile j landed (every producer's copies)
         publish(j, place_vis(j));
-        const int n = j + 2;
+        const int n = j + NST;
         if (n < ntiles) {
           if (n % kTcCandTiles == 0) {
             bar_sync(kTcBarProd, kTcProd);
@@ -401,81 +434,131 @@ decode_tc_kernel(const AttnParams p) {
     if (!ok) *abort_flag = 1;
   }
 
-  float m_used = -INFINITY, l_sum = 0.f;
-  const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-  const uint32_t tS = tmem + lane_off;
-  const uint32_t tO = tmem + 128 + lane_off + half * HD;
-  bool lost = false;
-  if (!producer) {
-    // ---- Q tile in swizzled shared memory; INT8 caches fold the key scale
-    // into q and split it into fp16 high and low tiles
+  // S of tile n into buffer n % 2: A = Q from tensor memory, B = the tile's
+  // K rows (K-major, 128-byte swizzle)
+  auto issue_s = [&](int n) {
+    const unsigned char* kt = smem + C::OFF_CONV + (n % NST) * 2 * C::KTILE;
+    const uint32_t dS = tmem + kTcColS + (n & 1) * KT;
 #pragma unroll
-    for (int k = 0; k < QPER; ++k) {
-      const int i = tid + k * kTcCons, r = i / QU, u = i % QU;
-      if constexpr (!C::kInt8) {
-        *reinterpret_cast<uint4*>(sQ + sw_off<128>(r, u)) = qv[k];
-      } else {
-        const ActT* x8 = reinterpret_cast<const ActT*>(&qv[k]);
-        alignas(16) __half h8[8], l8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float x = to_f32(x8[e]) * ksc[u * 8 + e];
-          h8[e] = __float2half_rn(x);
-          l8[e] = __float2half_rn(x - __half2float(h8[e]));
-        }
-        *reinterpret_cast<uint4*>(sQ + sw_off<128>(r, u)) = *reinterpret_cast<const uint4*>(h8);
-        *reinterpret_cast<uint4*>(sQlo + sw_off<128>(r, u)) = *reinterpret_cast<const uint4*>(l8);
-      }
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c = kk / 4, koff = (kk % 4) * 32;
+      const uint64_t bd = smem_desc_sw128(smem_u32(kt + c * C::KCHUNK + koff), 16, 1024);
+      mma_ts(dS, tmem + kTcColQ + kk * 8, bd, IDESC_S, kk > 0 ? 1u : 0u);
+      if constexpr (C::kInt8) mma_ts(dS, tmem + kTcColQ + QCOLS + kk * 8, bd, IDESC_S, 1u);
     }
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    bar_sync(kTcBarCons, kTcCons);
+    tc_commit(bar_s + (n & 1));
+  };
+  if (tid == kTcMmaTid && ntiles > 0) {
+    // =================== MMA thread ===================
+    // order: S(0), then per tile j: S(j + 1), PV(j).  S(j + 1) overwrites the
+    // scores of tile j - 1, which the softmax warps read before placing P(j - 1),
+    // which PV(j - 1) waited for.
+    bool ok = mbar_wait(bar_q, 0, kTcWaitLimit, abort_flag) && mbar_wait(bar_full, 0, kTcWaitLimit, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+    }
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int st = j % NST, sb = j & 1;
+      if (j + 1 < ntiles) {
+        ok = mbar_wait(bar_full + (j + 1) % NST, ((j + 1) / NST) & 1, kTcWaitLimit, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(j + 1);
+      }
+      ok = mbar_wait(bar_p + sb, (j >> 1) & 1, kTcWaitLimit, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const unsigned char* vt = smem + C::OFF_CONV + st * 2 * C::KTILE + C::KTILE;
+#pragma unroll
+      for (int kk = 0; kk < KT / 16; ++kk) {
+        const uint64_t bd = smem_desc_sw128(smem_u32(vt + kk * 2048), C::KCHUNK, 1024);
+        mma_ts(tmem + kTcColO, tmem + kTcColP + sb * (KT / 2) + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(bar_o + sb);
+      tc_commit(bar_empty + st);   // the stage is free once S and PV of this tile complete
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  float m_used = -INFINITY, l_sum = 0.f;
+  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+  const uint32_t tO = tmem + kTcColO + lane_off;
+  if (softmax) {
+    // ---- Q row `row` -> tensor memory (the A operand of S); INT8 caches fold
+    // the key scale into q and split it into fp16 high and low parts
+    {
+      // 32 columns (64 values) at a time
+#pragma unroll
+      for (int c = 0; c < (int)QCOLS; c += 32) {
+        uint32_t qh[32];
+        if constexpr (!C::kInt8) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 u = qv[c / 4 + k];
+            qh[4 * k + 0] = u.x;
+            qh[4 * k + 1] = u.y;
+            qh[4 * k + 2] = u.z;
+            qh[4 * k + 3] = u.w;
+          }
+          tmem_st32(tmem + lane_off + kTcColQ + c, qh);
+        } else {
+          uint32_t ql[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const ActT* x8 = reinterpret_cast<const ActT*>(&qv[c / 4 + k]);
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int d = (c / 4 + k) * 8 + e;
+              const float x0 = to_f32(x8[e]) * ksc[d];
+              const float x1 = to_f32(x8[e + 1]) * ksc[d + 1];
+              const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+              const __half l0 = __float2half_rn(x0 - __half2float(h0));
+              const __half l1 = __float2half_rn(x1 - __half2float(h1));
+              __half2 hh = __halves2half2(h0, h1), ll = __halves2half2(l0, l1);
+              qh[4 * k + e / 2] = *reinterpret_cast<uint32_t*>(&hh);
+              ql[4 * k + e / 2] = *reinterpret_cast<uint32_t*>(&ll);
+            }
+          }
+          tmem_st32(tmem + lane_off + kTcColQ + c, qh);
+          tmem_st32(tmem + lane_off + kTcColQ + QCOLS + c, ql);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_q);
+    }
     const float sl2 = p.scale_log2;
     const int prow = (row < R && has_rows) ? U.p_first + row / G : -1;
+    bool lost = false;
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
-      bool got = mbar_wait(bar_full + st, (j >> 1) & 1, kTcWaitLimit, abort_flag);
-      if (bar_red_or(!got, kTcBarCons, kTcCons)) {
-        lost = true;
-        break;
-      }
-      const unsigned char* kt = smem + C::OFF_CONV + st * 2 * C::KTILE;
-      const unsigned char* vt = kt + C::KTILE;
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int c = kk / 4, koff = (kk % 4) * 32;
-          const uint64_t bd = smem_desc_sw128(smem_u32(kt + c * C::KCHUNK + koff), 16, 1024);
-          mma_ss(tmem, smem_desc_sw128(smem_u32(sQ + c * 16384 + koff), 16, 1024), bd, IDESC_S,
-                 kk > 0 ? 1u : 0u);
-          if constexpr (C::kInt8)
-            mma_ss(tmem, smem_desc_sw128(smem_u32(sQlo + c * 16384 + koff), 16, 1024), bd, IDESC_S, 1u);
-        }
-        tc_commit(bar_s);
-      }
-      got = mbar_wait(bar_s, j & 1, kTcWaitLimit, abort_flag);
-      if (bar_red_or(!got, kTcBarCons, kTcCons)) {
+      const int st = j % NST, sb = j & 1;
+      // S(j) complete; the tile's visibility flags were placed before its full barrier
+      const bool got = mbar_wait(bar_s + sb, (j >> 1) & 1, kTcWaitLimit, abort_flag) &&
+                       mbar_wait(bar_full + st, (j / NST) & 1, kTcWaitLimit, abort_flag);
+      if (__any_sync(0xffffffffu, !got)) {
         lost = true;
         break;
       }
       tc_fence_after();
-      // ---- softmax of row `row` over this half's 32 keys of the tile; the two
-      // halves exchange their maxima through shared memory
+      // ---- softmax of row `row` over the tile's 64 keys
       const bool tile_vis = tvis_s[st] != 0;
-      uint32_t v[HK];
-      tmem_ld32(tS + half * HK, v);
+      uint32_t v[KT];
+      tmem_ld32(tmem + kTcColS + lane_off + sb * KT, v);
+      tmem_ld32(tmem + kTcColS + lane_off + sb * KT + 32, v + 32);
       tmem_wait_ld();
       float mx0 = -INFINITY, mx1 = -INFINITY;
       if (tile_vis) {
 #pragma unroll
-        for (int e = 0; e < HK; e += 2) {
+        for (int e = 0; e < KT; e += 2) {
           mx0 = fmaxf(mx0, __uint_as_float(v[e]));
           mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
         }
       } else {
-        const int4* kv4 = reinterpret_cast<const int4*>(kvis_s + st * KT + half * HK);
+        const int4* kv4 = reinterpret_cast<const int4*>(kvis_s + st * KT);
 #pragma unroll
-        for (int e = 0; e < HK; e += 2) {
+        for (int e = 0; e < KT; e += 2) {
           const int4 w = kv4[e / 2];
           const float x0 = (prow >= w.x && prow <= w.y) ? __uint_as_float(v[e]) : -INFINITY;
           const float x1 = (prow >= w.z && prow <= w.w) ? __uint_as_float(v[e + 1]) : -INFINITY;
@@ -485,16 +568,17 @@ decode_tc_kernel(const AttnParams p) {
           mx1 = fmaxf(mx1, x1);
         }
       }
-      red_max[half * 128 + row] = fmaxf(mx0, mx1);
-      bar_sync(kTcBarCons, kTcCons);
-      const float mx = fmaxf(red_max[row], red_max[128 + row]) * sl2;
+      const float mx = fmaxf(mx0, mx1) * sl2;
       const bool need = mx > m_used + 8.0f;
       const float m_new = need ? mx : m_used;
       const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2a(m_used - m_new)) : 1.f;
       if (j > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
+        // O is rescaled in place once the previous tile's PV is complete
+        if (!mbar_wait(bar_o + ((j - 1) & 1), ((j - 1) >> 1) & 1, kTcWaitLimit, abort_flag)) *abort_flag = 1;
+        tc_fence_after();
         uint32_t o[32];
 #pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
@@ -505,53 +589,44 @@ decode_tc_kernel(const AttnParams p) {
       m_used = m_new;
       const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
       float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[HK / 2];
+      uint32_t pk[KT / 2];
 #pragma unroll
-      for (int e = 0; e < HK; e += 2) {
+      for (int e = 0; e < KT; e += 2) {
         const float pa = ex2a(fmaf(__uint_as_float(v[e]), sl2, nm));
         const float pb = ex2a(fmaf(__uint_as_float(v[e + 1]), sl2, nm));
         ls0 += pa;
         ls1 += pb;
         pk[e / 2] = pk_pair<MT>(pa, pb);
       }
-      // packed P of keys [half*32, half*32 + 32) -> columns [half*16, half*16 + 16);
-      // every S column was read into registers before the barrier above
-      tmem_st16(tS + half * (HK / 2), pk);
       l_sum = l_sum * alpha + (ls0 + ls1);
+      // P buffer sb was last read by the PV of tile j - 2
+      if (j >= 2) {
+        if (!mbar_wait(bar_o + sb, ((j - 2) >> 1) & 1, kTcWaitLimit, abort_flag)) *abort_flag = 1;
+        tc_fence_after();
+      }
+      // packed P of the 64 keys -> the buffer's 32 columns
+      tmem_st32(tmem + kTcColP + lane_off + sb * (KT / 2), pk);
       tmem_wait_st();
       tc_fence_before();
-      bar_sync(kTcBarCons, kTcCons);
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(smem_u32(vt + kk * 2048), C::KCHUNK, 1024);
-          mma_ts(tmem + 128, tmem + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar_o);
-        tc_commit(bar_empty + st);   // the stage is free once S and PV of this tile complete
-      }
-      // the next S overwrites P, and the O rescale needs PV done
-      got = mbar_wait(bar_o, j & 1, kTcWaitLimit, abort_flag);
-      if (bar_red_or(!got, kTcBarCons, kTcCons)) {
-        lost = true;
-        break;
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p + sb);
+    }
+    // O is complete once the last tile's PV is
+    if (!lost && ntiles > 0) {
+      if (!mbar_wait(bar_o + ((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, kTcWaitLimit, abort_flag))
+        *abort_flag = 1;
       tc_fence_after();
     }
     if (lost) *abort_flag = 1;
-    red_l[half * 128 + row] = l_sum;
-    bar_sync(kTcBarCons, kTcCons);
-    l_sum = red_l[row] + red_l[128 + row];
   }
   // every role is done with the rings (the producers drained their copies)
   __syncthreads();
-  lost = *abort_flag != 0;
+  const bool lost = *abort_flag != 0;
   if (lost) bits |= SPA_ST_TIMEOUT;
 
-  // ---- epilogue (consumers): row `row`, this half's D/2 columns; O (x value
-  // scale) -> output or partial state
-  if (!producer) {
+  // ---- epilogue (softmax warps): row `row`; O (x value scale) -> output or
+  // partial state
+  if (softmax) {
     const bool have_o = ntiles > 0 && !lost;
     const int tt = t0 + row / max(G, 1), h = h_kv * G + row % G;
     const long long orow = (long long)tt * p.H_q + h;
@@ -564,7 +639,7 @@ decode_tc_kernel(const AttnParams p) {
       f = a * inv_l;
     }
 #pragma unroll 1
-    for (int c = 0; c < HD / 32; ++c) {
+    for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
       if (have_o) {
         tmem_ld32(tO + c * 32, o);
@@ -574,7 +649,7 @@ decode_tc_kernel(const AttnParams p) {
         for (int e = 0; e < 32; ++e) o[e] = 0u;
       }
       if (!mine) continue;
-      const int col = half * HD + c * 32;
+      const int col = c * 32;
       float ov[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) ov[e] = __uint_as_float(o[e]) * (C::kInt8 ? vsc[col + e] : 1.f);
@@ -594,7 +669,7 @@ decode_tc_kernel(const AttnParams p) {
         for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(acc + e) = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
       }
     }
-    if (mine && half == 0) {
+    if (mine) {
       if (p.num_splits == 1) {
         if (p.lse) p.lse[orow] = lse;
       } else if (p.cluster_merge) {
