@@ -78,15 +78,10 @@ append_int8_kernel(const ActT* __restrict__ k_new, const ActT* __restrict__ v_ne
     }
     const ActT* src = (is_v ? v_new : k_new) + row * D + c * 16;
     const float* sc = (is_v ? v_scale : k_scale) + (long long)h * D + c * 16;
-    alignas(16) int8_t q[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      float r = rintf(__fdiv_rn(to_f32(src[e]), sc[e]));
-      r = fminf(fmaxf(r, -128.0f), 127.0f);
-      q[e] = static_cast<int8_t>(static_cast<int>(r));
-    }
+    Group16<ActT> g;
+    g.load(src);
     int8_t* dst = (is_v ? v_cache : k_cache) + ((long long)slot * H_kv + h) * D + c * 16;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(q);
+    *reinterpret_cast<uint4*>(dst) = quant_group16<ActT>(g.v, sc);
   }
   flag(status, bits);
 }

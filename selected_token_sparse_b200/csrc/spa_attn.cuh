@@ -355,7 +355,7 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, 
 // Split merge through distributed shared memory.  The num_splits CTAs of a
 // unit form one cluster (rank = split); each has left its partial state at
 // the same shared-memory offsets: o [rows][D + 4] fp32 (row stride D + 4) and
-// (m, l) [rows][2], log2 units.  After a cluster barrier, CTA k merges rows
+// (m, l, sink * log2(e), 0) [rows][4], log2 units.  After a cluster barrier, CTA k merges rows
 // k, k + S, k + 2S, ... with the sink as merge_rows does, in one pass: each
 // thread takes 4 output columns of a row, reads every split's (m, l) and
 // partial columns from the peers' shared memory at once, and forms the
@@ -363,29 +363,31 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, 
 // CTA leaves while its state is being read.
 constexpr int kClusterMaxSplits = 8;
 
-template <typename ActT, int D>
+// SMAX bounds the split count; IPT items of a thread have their peer loads in
+// flight together (a peer load is a round trip through the cluster network).
+template <typename ActT, int D, int SMAX, int IPT>
 __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, int nq, int h_kv,
                                                    const float* part_o, const float* part_ml) {
-  constexpr int C4 = D / 4, PS = D + 4, IPT = 1;   // items of a thread whose loads are in flight together
+  constexpr int C4 = D / 4, PS = D + 4;
   const int S = p.num_splits, k = (int)cluster_rank();
   const int R = nq * p.G;
   const int mine = R > k ? (R - k + S - 1) / S : 0;   // rows k, k + S, ...
   const int n_items = mine * C4;
   for (int base = threadIdx.x; base < n_items; base += IPT * blockDim.x) {
-    float2 ml[IPT][kClusterMaxSplits];
-    float4 a[IPT][kClusterMaxSplits];
+    float2 ml[IPT][SMAX];
+    float4 a[IPT][SMAX];
     float sink2[IPT];
 #pragma unroll
     for (int t = 0; t < IPT; ++t) {
       const int it = base + t * blockDim.x;
       const int r = k + (it / C4) * S, c = (it % C4) * 4;
-      sink2[t] = (p.sinks && it < n_items) ? ld_early(p.sinks + h_kv * p.G + r % p.G) * kLog2e : -INFINITY;
+      sink2[t] = it < n_items ? part_ml[4 * r + 2] : -INFINITY;   // the same in every split
 #pragma unroll
-      for (int s = 0; s < kClusterMaxSplits; ++s) {
+      for (int s = 0; s < SMAX; ++s) {
         ml[t][s] = make_float2(-INFINITY, 0.f);
         a[t][s] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (s < S && it < n_items) {
-          ml[t][s] = ld_peer2(peer_smem(part_ml + 2 * r, s));
+          ml[t][s] = ld_peer2(peer_smem(part_ml + 4 * r, s));
           a[t][s] = ld_peer4(peer_smem(part_o + r * PS + c, s));
         }
       }
@@ -398,13 +400,13 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, 
       const long long row = (long long)(t0 + r / p.G) * p.H_q + h_kv * p.G + r % p.G;
       float M = sink2[t];
 #pragma unroll
-      for (int s = 0; s < kClusterMaxSplits; ++s) M = fmaxf(M, ml[t][s].x);
+      for (int s = 0; s < SMAX; ++s) M = fmaxf(M, ml[t][s].x);
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
       float inv = 0.f, lse = -INFINITY;
       if (M != -INFINITY) {
         float Lsum = (sink2[t] == -INFINITY) ? 0.f : exp2f(sink2[t] - M);
 #pragma unroll
-        for (int s = 0; s < kClusterMaxSplits; ++s) {
+        for (int s = 0; s < SMAX; ++s) {
           const float w = (ml[t][s].x == -INFINITY) ? 0.f : exp2f(ml[t][s].x - M);
           Lsum += w * ml[t][s].y;
           o.x = fmaf(w, a[t][s].x, o.x);

@@ -29,6 +29,32 @@ __device__ __forceinline__ void flag(int32_t* status, int bits) {
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// INT8 K/V quantisation of one group of 16 channels: q8 = clamp(rint(x / scale),
+// -128, 127) with an IEEE fp32 division, the 16 bytes packed in channel order.
+// `x` holds the group's values as they were loaded (16-byte vectors).
+template <typename ActT>
+__device__ __forceinline__ uint4 quant_group16(const uint4* x, const float* __restrict__ sc) {
+  const ActT* v = reinterpret_cast<const ActT*>(x);
+  alignas(16) int8_t q[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float r = rintf(__fdiv_rn(to_f32(v[e]), sc[e]));
+    r = fminf(fmaxf(r, -128.0f), 127.0f);
+    q[e] = static_cast<int8_t>(static_cast<int>(r));
+  }
+  return *reinterpret_cast<const uint4*>(q);
+}
+// The 16-byte vectors of a group of 16 values (16-byte aligned).
+template <typename ActT>
+struct Group16 {
+  static constexpr int NV = 16 * (int)sizeof(ActT) / 16;
+  uint4 v[NV];
+  __device__ __forceinline__ void load(const ActT* src) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[i] = reinterpret_cast<const uint4*>(src)[i];
+  }
+};
 __device__ __forceinline__ float to_f32(int8_t x) { return static_cast<float>(x); }
 
 // Round-to-nearest-even conversion of an fp32 value to the output encoding.

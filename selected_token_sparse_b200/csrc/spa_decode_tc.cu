@@ -74,11 +74,11 @@ struct TcCfg {
   static constexpr int OFF_CONV = 0;                                   // [stage][K, V]
   static constexpr int OFF_RAW = OFF_CONV + kTcStages * 2 * KTILE;     // INT8: [raw stage][K, V]
   static constexpr int END_RING = OFF_RAW + RAW_ST * 2 * RAW;
-  // cluster split merge: partial o [128][D + 4] and (m, l) [128][2], fp32,
-  // over the rings once every tile is consumed
+  // cluster split merge: partial o [128][D + 4] and (m, l, sink, 0) [128][4],
+  // fp32, over the rings once every tile is consumed
   static constexpr int OFF_PART = 0;
   static constexpr int PART_ML = OFF_PART + 128 * (D + 4) * 4;
-  static constexpr int END_PART = PART_ML + 128 * 2 * 4;
+  static constexpr int END_PART = PART_ML + 128 * 4 * 4;
   static constexpr int OFF_KVIS = END_RING > END_PART ? END_RING : END_PART;  // [stage][64] row intervals
   static constexpr int OFF_TVIS = OFF_KVIS + kTcStages * kTcKT * 8;           // [stage] tile seen by every row
   static constexpr int OFF_CAND = OFF_TVIS + 16;                    // [2 chunks] offsets + positions
@@ -243,8 +243,8 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
       for (int k = 0; k < QV; ++k) qv[k] = src[k];
     }
-    // the epilogue's sink logit of row `row`
-    if (p.sinks && p.num_splits == 1 && row < R) sink_raw = ld_early(p.sinks + h_kv * G + row % G);
+    // the epilogue's (or the cluster merge's) sink logit of row `row`
+    if (p.sinks && (p.num_splits == 1 || p.cluster_merge) && row < R) sink_raw = ld_early(p.sinks + h_kv * G + row % G);
   }
   tc_fence_before();
   __syncthreads();
@@ -673,7 +673,8 @@ decode_tc_kernel(const AttnParams p) {
       if (p.num_splits == 1) {
         if (p.lse) p.lse[orow] = lse;
       } else if (p.cluster_merge) {
-        *reinterpret_cast<float2*>(smem + C::PART_ML + row * 8) = make_float2(m_used, l_sum);
+        *reinterpret_cast<float4*>(smem + C::PART_ML + row * 16) =
+            make_float4(m_used, l_sum, p.sinks ? sink_raw * kLog2e : -INFINITY, 0.f);
       } else {
         const long long wrow = (long long)split * p.T * p.H_q + orow;
         p.ws_ml[wrow * 2 + 0] = m_used;
@@ -691,8 +692,10 @@ decode_tc_kernel(const AttnParams p) {
   if (p.num_splits > 1) {
     if (p.cluster_merge) {
       cluster_sync();
-      cluster_merge_rows<ActT, D>(p, t0, nq, h_kv, reinterpret_cast<const float*>(smem + C::OFF_PART),
-                                  reinterpret_cast<const float*>(smem + C::PART_ML));
+      const float* po = reinterpret_cast<const float*>(smem + C::OFF_PART);
+      const float* pml = reinterpret_cast<const float*>(smem + C::PART_ML);
+      if (p.num_splits <= 4) cluster_merge_rows<ActT, D, 4, 3>(p, t0, nq, h_kv, po, pml);
+      else cluster_merge_rows<ActT, D, kClusterMaxSplits, 1>(p, t0, nq, h_kv, po, pml);
       cluster_sync();
     } else {
       finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);

@@ -53,7 +53,7 @@ __device__ __forceinline__ void append_token_rows(const ActT* __restrict__ k_new
                                                   CacheT* __restrict__ k_cache, CacheT* __restrict__ v_cache,
                                                   const float* __restrict__ k_scale,
                                                   const float* __restrict__ v_scale, int t, int slot,
-                                                  int H_kv, int D, int lane) {
+                                                  int H_kv, int D, int lane, int first = 0) {
   const long long src_row = (long long)t * H_kv * D;
   const long long dst_row = (long long)slot * H_kv * D;
   if constexpr (sizeof(CacheT) != 1) {
@@ -69,30 +69,24 @@ __device__ __forceinline__ void append_token_rows(const ActT* __restrict__ k_new
       vd[i] = vs[i];
     }
   } else {
-    // q8 = clamp(rint(x / scale), -128, 127) per channel, 16 channels per lane step
+    // q8 = clamp(rint(x / scale), -128, 127) per channel, 16 channels per lane
+    // step; items below `first` were done by the caller
     const int ngrp = H_kv * D / 16;
-    for (int i = lane; i < 2 * ngrp; i += 32) {
+    for (int i = first + lane; i < 2 * ngrp; i += 32) {
       const bool isv = i >= ngrp;
-      const int gi = isv ? i - ngrp : i;
-      const int e0 = gi * 16;                  // element offset within the token's H_kv*D row
-      const int h = e0 / D, d0 = e0 % D;
-      const ActT* src = (isv ? v_new : k_new) + src_row + e0;
-      const float* sc = (isv ? v_scale : k_scale) + (long long)h * D + d0;
-      alignas(16) int8_t qv[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        float r = rintf(__fdiv_rn(to_f32(src[e]), sc[e]));
-        r = fminf(fmaxf(r, -128.0f), 127.0f);
-        qv[e] = static_cast<int8_t>(static_cast<int>(r));
-      }
+      const int e0 = (isv ? i - ngrp : i) * 16;   // element offset within the token's H_kv*D row
+      Group16<ActT> g;
+      g.load((isv ? v_new : k_new) + src_row + e0);
       int8_t* dst = reinterpret_cast<int8_t*>(isv ? v_cache : k_cache) + dst_row + e0;
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(qv);
+      *reinterpret_cast<uint4*>(dst) = quant_group16<ActT>(g.v, (isv ? v_scale : k_scale) + e0);
     }
   }
 }
 
-// 16-byte vectors of a token's K (and V) rows each lane loads before the
-// metadata is known (16-bit caches), so the copy does not wait for them
+// 16-byte vectors (16-bit caches) or 16-channel groups (INT8 caches) of a
+// token's K and V rows each lane loads before the metadata is known, so the
+// copy does not wait for them; INT8 groups are quantised while the token's
+// block-table entry is in flight
 constexpr int kAppendPre = 2;
 
 template <typename ActT, typename CacheT>
@@ -131,13 +125,41 @@ prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict_
       }
     }
   }
+  const int ngrp = H_kv * D / 16;   // INT8: 16-channel groups of a K (or V) row
+  Group16<ActT> gpre[kAppendPre];
+  uint4 qpre[kAppendPre];
+  if constexpr (!kCopy) {
+    if (t_first < T) {
+#pragma unroll
+      for (int i = 0; i < kAppendPre; ++i) {
+        const int it = lane + 32 * i;
+        if (it < 2 * ngrp) {
+          const bool isv = it >= ngrp;
+          gpre[i].load((isv ? v_new : k_new) + (long long)t_first * H_kv * D + (isv ? it - ngrp : it) * 16);
+        }
+      }
+    }
+  }
   for (int b = threadIdx.x; b < B; b += blockDim.x) past_s[b] = past[b];
   build_cs<kMetaThreads>(cu, B, T, cs);   // ends with a block barrier: past_s is visible too
   if (blockIdx.x == 0) flag(status, per_request(cu, past_s, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
   int bits = 0;
   for (int t = t_first; t < T; t += gridDim.x * wpb) {
     int tb = 0;  // every lane computes the same metadata; lane 0 reports and writes it
-    const TokenMeta m = token_meta(t, cs, B, past_s, block_table, MB, bs, num_blocks, tb);
+    const TokenLoad tl = token_meta_load(t, cs, B, past_s, block_table, MB, bs);
+    if constexpr (!kCopy) {
+      if (t == t_first) {
+#pragma unroll
+        for (int i = 0; i < kAppendPre; ++i) {
+          const int it = lane + 32 * i;
+          if (it < 2 * ngrp) {
+            const bool isv = it >= ngrp;
+            qpre[i] = quant_group16<ActT>(gpre[i].v, (isv ? v_scale : k_scale) + (isv ? it - ngrp : it) * 16);
+          }
+        }
+      }
+    }
+    const TokenMeta m = token_meta_finish(tl, MB, bs, num_blocks, tb);
     if (lane == 0) {
       bits |= tb;
       token_batch[t] = m.b;
@@ -163,6 +185,23 @@ prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict_
           kd[v] = ks[v];
           vd[v] = vs[v];
         }
+        continue;
+      }
+    }
+    if constexpr (!kCopy) {
+      if (t == t_first) {
+#pragma unroll
+        for (int i = 0; i < kAppendPre; ++i) {
+          const int it = lane + 32 * i;
+          if (it < 2 * ngrp) {
+            const bool isv = it >= ngrp;
+            int8_t* dst = reinterpret_cast<int8_t*>(isv ? v_cache : k_cache) + (long long)m.slot * H_kv * D +
+                          (isv ? it - ngrp : it) * 16;
+            *reinterpret_cast<uint4*>(dst) = qpre[i];
+          }
+        }
+        append_token_rows<ActT, CacheT>(k_new, v_new, k_cache, v_cache, k_scale, v_scale, t, m.slot, H_kv, D,
+                                        lane, 32 * kAppendPre);
         continue;
       }
     }
