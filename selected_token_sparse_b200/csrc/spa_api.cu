@@ -193,11 +193,9 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   p->split_len = pl.split_len;
   p->status = a->status;
   // the splits of a unit merge through distributed shared memory when they
-  // fit one cluster and the kernel runs one CTA per SM (tcgen05 decode);
-  // otherwise through the workspace.  Measured: the cluster merge takes the
-  // INT8 multi-row decode from 30.5 to 21.4 us, while the warp-MMA kernel
-  // (two or more CTAs per SM) got slower under cluster scheduling.
-  p->cluster_merge = pl.kind == kPlanTc && pl.num_splits > 1 && pl.num_splits <= 8;
+  // fit one cluster (tensor-core decode kernels); otherwise through the
+  // workspace, where the CTA that finishes last merges
+  p->cluster_merge = (pl.kind == kPlanTc || pl.kind == kPlanMma) && pl.num_splits > 1 && pl.num_splits <= 8;
   if (pl.num_splits > 1) {
     p->ws_acc = static_cast<float*>(ws);
     p->ws_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.ws_acc_bytes);

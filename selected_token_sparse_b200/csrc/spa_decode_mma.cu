@@ -119,8 +119,13 @@ struct MmaCfg {
   // the cross-warp merge reuses the K/V ring once every tile is consumed
   static constexpr int OFF_RED = OFF_RAW;
   static constexpr int RED_BYTES = (KW > 1) ? NW * 32 * (D / 2 + 4) * 4 : 0;
-  static constexpr int SMEM = (OFF_RED + RED_BYTES > END) ? OFF_RED + RED_BYTES : END;
-  static_assert(OFF_RED + RED_BYTES <= OFF_KPOS, "merge buffer must not reach the scales / positions");
+  // cluster split merge: the CTA's partial o [ROWS][D + 4] and (m, l, sink,
+  // 0) [ROWS][4], fp32, after the cross-warp buffer
+  static constexpr int OFF_PART = OFF_RED + RED_BYTES;
+  static constexpr int PART_ML = OFF_PART + ROWS * (D + 4) * 4;
+  static constexpr int END_PART = PART_ML + ROWS * 16;
+  static constexpr int SMEM = (END_PART > END) ? END_PART : END;
+  static_assert(END_PART <= OFF_KPOS, "merge buffers must not reach the scales / positions");
 };
 
 // FUSED: one launch of the whole step (16-bit caches).  Every CTA rebuilds
@@ -373,7 +378,7 @@ decode_mma_kernel(const AttnParams p) {
   const int r1 = r0 + 8;
   // the epilogue's sink logits, in flight from here
   float sink_raw[2] = {-INFINITY, -INFINITY};
-  if (p.sinks && p.num_splits == 1) {
+  if (p.sinks && (p.num_splits == 1 || p.cluster_merge)) {
     if (r0 < R) sink_raw[0] = ld_early(p.sinks + h_kv * G + r0 % G);
     if (r1 < R) sink_raw[1] = ld_early(p.sinks + h_kv * G + r1 % G);
   }
@@ -630,6 +635,16 @@ decode_mma_kernel(const AttnParams p) {
         *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(fo[nn][hrow * 2 + 0] * f, fo[nn][hrow * 2 + 1] * f);
       }
       if (wk == 0 && (lane & 3) == 0 && p.lse) p.lse[row] = lse;
+    } else if (p.cluster_merge) {
+      float* po = reinterpret_cast<float*>(smem + C::OFF_PART) + r * (D + 4);
+#pragma unroll
+      for (int nn = 0; nn < NPW; ++nn) {
+        const int d = (n_lo + nn) * 8 + (lane & 3) * 2;
+        *reinterpret_cast<float2*>(po + d) = make_float2(fo[nn][hrow * 2], fo[nn][hrow * 2 + 1]);
+      }
+      if (wk == 0 && (lane & 3) == 0)
+        *reinterpret_cast<float4*>(smem + C::PART_ML + r * 16) =
+            make_float4(mf[hrow], lf[hrow], p.sinks ? sink_raw[hrow] * kLog2e : -INFINITY, 0.f);
     } else {
       const long long wrow = (long long)split * p.T * p.H_q + row;
       float* acc = p.ws_acc + wrow * D;
@@ -663,7 +678,19 @@ decode_mma_kernel(const AttnParams p) {
     }
   }
   flag(p.status, bits);
-  if (p.num_splits > 1) finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
+  if (p.num_splits > 1) {
+    if (p.cluster_merge) {
+      // the unit's splits are one cluster: merge through distributed shared memory
+      cluster_sync();
+      const float* po = reinterpret_cast<const float*>(smem + C::OFF_PART);
+      const float* pml = reinterpret_cast<const float*>(smem + C::PART_ML);
+      if (p.num_splits <= 4) cluster_merge_rows<ActT, D, 4, 2>(p, t0, nq, h_kv, po, pml);
+      else cluster_merge_rows<ActT, D, kClusterMaxSplits, 1>(p, t0, nq, h_kv, po, pml);
+      cluster_sync();
+    } else {
+      finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -688,6 +715,7 @@ static int launch_rt(const AttnParams& p, cudaStream_t stream) {
   if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
   dim3 grid(units, p.num_splits);
+  if (p.cluster_merge) return launch_pdl_cluster_y(kern, grid, dim3(C::NT), smem, stream, p.num_splits, p);
   return launch_pdl(kern, grid, dim3(C::NT), smem, stream, p);
 }
 
