@@ -177,6 +177,23 @@ decode_mma_kernel(const AttnParams p) {
       app_data = fused_load_row_vector<CacheT>(p, blockIdx.x / p.H_kv, blockIdx.x % p.H_kv, tid, NV);
   }
 
+  // Per-request selection rows: the unit's request and kv head follow from the
+  // block index, so the first chunk's selection entries can be in flight
+  // while the unit's metadata is read (and their block-table entries right
+  // after); resolve_chunk(0) then only applies the guards.
+  constexpr int RPT = (kMmaCandChunk + NT - 1) / NT;
+  const bool pre = p.group_by_request && p.sel != nullptr && p.sel_target == 0 && p.sel_per_request;
+  int pre_raw[RPT], pre_blk[RPT];
+  if (pre) {
+    const int32_t* selrow = p.sel + (long long)blockIdx.x * p.sel_width;   // (request, kv head) = block index
+    const int cb = blockIdx.y * p.split_len, ce = min(cb + p.split_len, p.sel_width);
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int i = tid + k * NT;
+      pre_raw[k] = (i < kMmaCandChunk && cb + i < ce) ? ld_early(selrow + cb + i) : -1;
+    }
+  }
+
   Unit U;
   bool has_rows;
   int bits = 0;
@@ -205,6 +222,14 @@ decode_mma_kernel(const AttnParams p) {
   } else {
     has_rows = decode_unit(p, blockIdx.x, U);
     if (p.group_by_request && !has_rows) return;
+  }
+  if (pre) {
+    const int b = blockIdx.x / p.H_kv;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int raw = pre_raw[k];
+      pre_blk[k] = (raw >= 0 && raw / p.bs < p.MB) ? ld_early(p.block_table + (long long)b * p.MB + raw / p.bs) : -1;
+    }
   }
   const int split = blockIdx.y;
   const int G = p.G;
@@ -275,17 +300,25 @@ decode_mma_kernel(const AttnParams p) {
   int* cand_kpos = reinterpret_cast<int*>(smem + C::OFF_CAND + kMmaCandChunk * 8);
   auto resolve_chunk = [&](int first_tile) {
     // every stage's loads of this thread's candidates are in flight together
-    constexpr int RPT = (kMmaCandChunk + NT - 1) / NT;
     int raw[RPT], blk[RPT];
+    if (pre && first_tile == 0) {
+      // the prefetched entries; cand_finish rejects what cand_stage2 would have
 #pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
-      raw[k] = (i < kMmaCandChunk && cand < c_end) ? cand_stage1(p, U, cand) : -1;
-    }
+      for (int k = 0; k < RPT; ++k) {
+        raw[k] = pre_raw[k];
+        blk[k] = pre_blk[k];
+      }
+    } else {
 #pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
-      blk[k] = (i < kMmaCandChunk && cand < c_end) ? cand_stage2(p, U, cand, raw[k]) : -1;
+      for (int k = 0; k < RPT; ++k) {
+        const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
+        raw[k] = (i < kMmaCandChunk && cand < c_end) ? cand_stage1(p, U, cand) : -1;
+      }
+#pragma unroll
+      for (int k = 0; k < RPT; ++k) {
+        const int i = tid + k * NT, cand = c_begin + first_tile * KT + i;
+        blk[k] = (i < kMmaCandChunk && cand < c_end) ? cand_stage2(p, U, cand, raw[k]) : -1;
+      }
     }
 #pragma unroll
     for (int k = 0; k < RPT; ++k) {
