@@ -30,6 +30,8 @@ int tc_supported(int act, int cache, int D, int max_rows);
 int tc_key_tile();
 int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream);
 int launch_step_mma(const AttnParams& p, int act, int max_rows, cudaStream_t stream);
+int launch_step_tc(const AttnParams& p, int act, int cache, cudaStream_t stream);
+int tc_step_fits(int D, int cache, int B);
 int launch_prepare_qkv_append(const QkvParams& P, int act, int cache, cudaStream_t stream);
 int mma_step_fits(int D, int max_rows, int B);
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream);
@@ -224,7 +226,9 @@ int launches_of(const Plan&) { return 1; }
 // The fused step runs as one launch when the plan picks the warp-MMA kernel
 // on a cache of the activation dtype and the metadata fits shared memory.
 static bool step_fusable(const spa_attention_args_t* a, const Plan& pl) {
-  return pl.kind == kPlanMma && a->cache == a->act && a->B <= 4096 && mma_step_fits(a->D, pl.max_rows, a->B);
+  if (a->B > 4096) return false;
+  if (pl.kind == kPlanTc) return tc_step_fits(a->D, a->cache, a->B) != 0;
+  return pl.kind == kPlanMma && a->cache == a->act && mma_step_fits(a->D, pl.max_rows, a->B);
 }
 
 const char* cuda_message() { return g_cuda_msg; }
@@ -386,7 +390,8 @@ int spa_prepare_append_attention(const spa_attention_args_t* a, const int32_t* p
   p.slot_out = slot_mapping;
   p.max_seqlen_q = a->max_seqlen_q;
   p.max_seqlen_k = a->max_seqlen_k;
-  if ((rc = launch_step_mma(p, a->act, pl.max_rows, st)) != SPA_OK) return rc;
+  rc = pl.kind == kPlanTc ? launch_step_tc(p, a->act, a->cache, st) : launch_step_mma(p, a->act, pl.max_rows, st);
+  if (rc != SPA_OK) return rc;
   return check_launch();
 }
 

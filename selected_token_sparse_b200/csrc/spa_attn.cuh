@@ -111,11 +111,24 @@ struct Unit {
   int new_lo, new_hi, new_t0;
 };
 
+// First packed token of request b under the sanitised cumulative lengths
+// (the non-decreasing sequence clamped to [0, T] that token ownership follows):
+// when request b has tokens and the raw lengths agree with its sanitised
+// length, cu[b] is that start; otherwise (malformed lengths only) it is the
+// sum of the sanitised lengths of the requests before b.
+__device__ __forceinline__ int sanitised_start(const AttnParams& p, int b) {
+  const int c0 = p.cu[b], c1 = p.cu[b + 1], q = p.seqlens_q[b];
+  if (q > 0 && (long long)c1 - c0 == q) return c0;
+  int s = 0;
+  for (int i = 0; i < b; ++i) s += max(p.seqlens_q[i], 0);
+  return s;
+}
+
 // Step-1 metadata as the attention kernels read it: the arrays written by the
 // metadata entry points.
 struct StagedMeta {
   const AttnParams& p;
-  __device__ __forceinline__ int cu(int g) const { return p.cu[g]; }
+  __device__ __forceinline__ int cu(int g) const { return sanitised_start(p, g); }
   __device__ __forceinline__ int seqlens_q(int b) const { return p.seqlens_q[b]; }
   __device__ __forceinline__ int seqlen_k(int b) const { return p.seqlen_k[b]; }
   __device__ __forceinline__ void token(int t, int& b, int& pos) const {

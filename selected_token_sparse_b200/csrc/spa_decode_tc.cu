@@ -39,6 +39,7 @@
 #include <type_traits>
 
 #include "spa_attn.cuh"
+#include "spa_meta.cuh"
 #include "spa_sm100.cuh"
 
 namespace spa {
@@ -58,6 +59,7 @@ constexpr int kTcCand = kTcCandTiles * kTcKT;
 constexpr uint32_t kTcColS = 0, kTcColO = 128, kTcColP = 256, kTcColQ = 320;
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcWaitLimit = 1u << 20;
+constexpr int kTcStageTok = 64;   // fused INT8 step: tokens of a request whose new rows are staged
 
 int tc_key_tile() { return kTcKT; }
 
@@ -86,7 +88,7 @@ struct TcCfg {
   static constexpr int NBAR = 2 * kTcStages + 7;   // full, empty, s[2], o[2], p[2], q
   static constexpr int OFF_BAR = OFF_SCALE + (kInt8 ? 2 * D * 4 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;                  // tmem holder, abort flag
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int BYTES = (OFF_MISC + 16 + 15) & ~15;   // what follows (fused step) is 16-byte aligned
   // at least 120 KB, so one CTA holds an SM and its 512 TMEM columns
   static constexpr int SMEM = BYTES + 1024 > 120 * 1024 ? BYTES + 1024 : 120 * 1024;
 };
@@ -158,7 +160,14 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
   else tmem_st16(taddr, r);
 }
 
-template <typename ActT, typename CacheT, int D>
+// FUSED: one launch of the whole step.  Every CTA rebuilds the sanitised
+// cumulative lengths and reads the past lengths into shared memory (after the
+// kernel's own layout), decodes its unit from them with the metadata
+// kernels' helpers, reads candidates at this step's new positions from k_new
+// / v_new (INT8: quantised exactly as the append quantises them), and the
+// producer warps of split 0 write the unit's share of the step-1/2 outputs
+// once their gather is done.
+template <typename ActT, typename CacheT, int D, bool FUSED>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const AttnParams p) {
   using C = TcCfg<ActT, CacheT, D>;
@@ -182,8 +191,38 @@ decode_tc_kernel(const AttnParams p) {
   pdl_trigger();
 
   Unit U;
-  const bool has_rows = decode_unit(p, blockIdx.x, U);
-  if (p.group_by_request && !has_rows) return;
+  bool has_rows;
+  int bits = 0;
+  int32_t* cs_s = nullptr;
+  int32_t* past_s = nullptr;
+  int8_t* stage_s = nullptr;   // fused INT8 step: [token][K, V][D] quantised new rows
+  if constexpr (FUSED) {
+    cs_s = reinterpret_cast<int32_t*>(smem + C::BYTES);
+    past_s = cs_s + p.B + 1;
+    stage_s = reinterpret_cast<int8_t*>(smem + C::BYTES + ((sizeof(int32_t) * (2 * p.B + 1) + 15) & ~size_t(15)));
+    for (int b = tid; b < p.B; b += kTcThreads) past_s[b] = p.past[b];
+    build_cs<kTcThreads>(p.cu, p.B, p.T, cs_s);   // ends with a block barrier
+    has_rows = decode_unit_with(p, FusedMeta{p.cu, cs_s, past_s, p.B}, blockIdx.x, U);
+    if (has_rows) {
+      U.new_lo = max(past_s[U.b], 0);
+      U.new_hi = U.new_lo + (cs_s[U.b + 1] - cs_s[U.b]);
+      U.new_t0 = cs_s[U.b];
+    }
+    if (p.group_by_request && !has_rows) {
+      // no attention rows: split 0 still writes the request's outputs and appends
+      if (blockIdx.y == 0) {
+        const int b = blockIdx.x / p.H_kv, hk = blockIdx.x % p.H_kv;
+        if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits, tid, kTcThreads);
+        fused_append_rows<ActT, CacheT>(p, cs_s, past_s, cs_s[b], cs_s[b + 1], hk, p.k_scale + hk * D,
+                                        p.v_scale + hk * D, tid, kTcThreads, bits);
+      }
+      flag(p.status, bits);
+      return;
+    }
+  } else {
+    has_rows = decode_unit(p, blockIdx.x, U);
+    if (p.group_by_request && !has_rows) return;
+  }
   const int split = blockIdx.y;
   const int G = p.G;
   const int nq = p.group_by_request ? U.nq : 1;
@@ -196,6 +235,8 @@ decode_tc_kernel(const AttnParams p) {
   const int ntiles = c_end > c_begin ? (c_end - c_begin + KT - 1) / KT : 0;
   // query positions of the unit's rows: [p_lo, p_hi]
   const int p_lo = has_rows ? U.p_first : 0, p_hi = has_rows ? U.p_last : -1;
+  // fused INT8 step: the request's new rows fit the staging area
+  const bool staged_new = FUSED && C::kInt8 && has_rows && U.new_hi - U.new_lo <= kTcStageTok;
 
   int2* kvis_s = reinterpret_cast<int2*>(smem + C::OFF_KVIS);
   int* tvis_s = reinterpret_cast<int*>(smem + C::OFF_TVIS);
@@ -229,7 +270,6 @@ decode_tc_kernel(const AttnParams p) {
       vsc[d] = p.v_scale[h_kv * D + d];
     }
   }
-  int bits = 0;
   // softmax: Q row `row` (token row / G, head row % G), in flight across the set-up
   constexpr int QV = D / 8;
   uint4 qv[QV];
@@ -282,6 +322,11 @@ decode_tc_kernel(const AttnParams p) {
         bool from_aux = false;
         long long off = -1;
         if (cand < c_end) off = cand_finish(p, U, cand, raw[k], blk[k], kp, from_aux, bits);
+        if constexpr (FUSED) {
+          // this step's tokens: read the row the append writes from its source
+          if (off >= 0 && kp >= U.new_lo && kp < U.new_hi)
+            off = (((long long)(U.new_t0 + kp - U.new_lo) * p.H_kv + U.h_kv) * D) | kNewRow;
+        }
         cand_off[buf + i] = off;
         cand_kpos[buf + i] = kp;
       }
@@ -291,6 +336,7 @@ decode_tc_kernel(const AttnParams p) {
     constexpr int NIT = KT * CPR * 2 / kTcProd;   // 16-byte chunks per producer thread and tile
     static_assert(KT * CPR * 2 % kTcProd == 0, "chunks per thread");
     auto issue = [&](int j) {
+      bool any_new = false;   // fused INT8 step: rows of this step's tokens, quantised below
 #pragma unroll 8
       for (int k = 0; k < NIT; ++k) {
         const int e = ptid + k * kTcProd;
@@ -298,10 +344,21 @@ decode_tc_kernel(const AttnParams p) {
         const int ee = isv ? e - KT * CPR : e;
         const int r = ee / CPR, ch = ee % CPR;
         const int ci = cslot(j, r);
-        const long long off = cand_off[ci];
+        long long off = cand_off[ci];
         const int kp = cand_kpos[ci];
         const bool okr = off >= 0;
         const CacheT* base = isv ? (kp == kPosAux ? av : vc) : (kp == kPosAux ? ak : kc);
+        if constexpr (FUSED) {
+          if (okr && (off & kNewRow)) {
+            if constexpr (C::kInt8) {
+              any_new = true;
+              continue;
+            } else {
+              off &= ~kNewRow;
+              base = static_cast<const CacheT*>(isv ? p.v_new : p.k_new);
+            }
+          }
+        }
         const CacheT* src = okr ? base + off + ch * (16 / sizeof(CacheT)) : kc;
         unsigned char* dst;
         if constexpr (C::kInt8) {
@@ -310,6 +367,32 @@ decode_tc_kernel(const AttnParams p) {
           dst = smem + C::OFF_CONV + ((j % NST) * 2 + (isv ? 1 : 0)) * C::KTILE + sw_off<KT>(r, ch);
         }
         cp_async_16(dst, src, okr);
+      }
+      if constexpr (FUSED && C::kInt8) {
+        if (any_new) {
+          // each such 16-byte chunk is 16 channels of a k_new / v_new row:
+          // copied from the staged rows, or quantised here with this kv
+          // head's scales when the request has too many new tokens to stage
+          for (int k = 0; k < NIT; ++k) {
+            const int e = ptid + k * kTcProd;
+            const bool isv = e >= KT * CPR;
+            const int ee = isv ? e - KT * CPR : e;
+            const int r = ee / CPR, ch = ee % CPR;
+            const long long off = cand_off[cslot(j, r)];
+            if (off < 0 || !(off & kNewRow)) continue;
+            uint4 q8;
+            if (staged_new) {
+              const int tj = cand_kpos[cslot(j, r)] - U.new_lo;
+              q8 = *reinterpret_cast<const uint4*>(stage_s + (tj * 2 + (isv ? 1 : 0)) * D + ch * 16);
+            } else {
+              Group16<ActT> g;
+              g.load(static_cast<const ActT*>(isv ? p.v_new : p.k_new) + (off & ~kNewRow) + ch * 16);
+              q8 = quant_group16<ActT>(g.v, (isv ? vsc : ksc) + ch * 16);
+            }
+            *reinterpret_cast<uint4*>(smem + C::OFF_RAW + ((j & 1) * 2 + (isv ? 1 : 0)) * C::RAW +
+                                      r * C::ROW_BYTES + ch * 16) = q8;
+          }
+        }
       }
     };
     // each key's interval [a, b] of query positions that see it (auxiliary
@@ -348,7 +431,61 @@ decode_tc_kernel(const AttnParams p) {
         mbar_arrive(bar_full + j % NST);
       }
     };
+    // fused INT8 step: the request's new rows (this step's tokens, kv head
+    // h_kv) are loaded with the first candidates' loads, quantised once into
+    // the staging area, and split 0 appends them to the cache from there
+    constexpr int PRE = 1;
+    const int per_tok = 2 * (D / 16);
+    const int n_new = (FUSED && C::kInt8 && staged_new) ? (U.new_hi - U.new_lo) * per_tok : 0;
+    Group16<ActT> pre_g[PRE];
+    TokenLoad pre_tl[PRE];
+    if constexpr (FUSED && C::kInt8) {
+#pragma unroll
+      for (int k = 0; k < PRE; ++k) {
+        const int idx = ptid + k * kTcProd;
+        if (idx < n_new) {
+          const int t = U.new_t0 + idx / per_tok, it = idx % per_tok;
+          const bool isv = it >= D / 16;
+          pre_g[k].load(static_cast<const ActT*>(isv ? p.v_new : p.k_new) + ((long long)t * p.H_kv + h_kv) * D +
+                        (isv ? it - D / 16 : it) * 16);
+          if (split == 0) pre_tl[k] = token_meta_load(t, cs_s, p.B, past_s, p.block_table, p.MB, p.bs);
+        }
+      }
+    }
     if (ntiles > 0) resolve_chunk(0);
+    if constexpr (FUSED && C::kInt8) {
+      for (int idx = ptid; idx < n_new; idx += kTcProd) {
+        const int k = (idx - ptid) / kTcProd;
+        const int tj = idx / per_tok, it = idx % per_tok;
+        const int t = U.new_t0 + tj;
+        const bool isv = it >= D / 16;
+        const int g = isv ? it - D / 16 : it;
+        Group16<ActT> x;
+        TokenLoad tl;
+        if (k < PRE) {
+          x = pre_g[k < PRE ? k : 0];
+          if (split == 0) tl = pre_tl[k < PRE ? k : 0];
+        } else {
+          x.load(static_cast<const ActT*>(isv ? p.v_new : p.k_new) + ((long long)t * p.H_kv + h_kv) * D + g * 16);
+          if (split == 0) tl = token_meta_load(t, cs_s, p.B, past_s, p.block_table, p.MB, p.bs);
+        }
+        const uint4 q8 = quant_group16<ActT>(x.v, (isv ? vsc : ksc) + g * 16);
+        *reinterpret_cast<uint4*>(stage_s + (tj * 2 + (isv ? 1 : 0)) * D + g * 16) = q8;
+        if (split == 0) {
+          int tb = 0;
+          const TokenMeta m = token_meta_finish(tl, p.MB, p.bs, p.NB, tb);
+          if (it == 0 && h_kv == 0) {
+            bits |= tb;
+            p.token_batch_out[t] = m.b;
+            p.token_pos_out[t] = m.pos;
+            p.slot_out[t] = m.slot;
+          }
+          if (m.slot >= 0)
+            *reinterpret_cast<uint4*>(static_cast<int8_t*>(const_cast<void*>(isv ? p.v_cache : p.k_cache)) +
+                                      ((long long)m.slot * p.H_kv + h_kv) * D + g * 16) = q8;
+        }
+      }
+    }
     bar_sync(kTcBarProd, kTcProd);
     if constexpr (C::kInt8) {
       if (ntiles > 0) issue(0);
@@ -432,6 +569,20 @@ decode_tc_kernel(const AttnParams p) {
     }
     cp_async_wait<0>();   // no copy outlives the CTA's use of the ring
     if (!ok) *abort_flag = 1;
+    if constexpr (FUSED) {
+      // steps 1-2 of the unit's tokens, off the attention's critical path
+      if (split == 0) {
+        if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits, ptid, kTcProd);
+        int t_lo = blockIdx.x / p.H_kv, t_hi = t_lo + 1;
+        if (p.group_by_request) {
+          t_lo = cs_s[t_lo];
+          t_hi = cs_s[blockIdx.x / p.H_kv + 1];
+        }
+        // staged INT8 rows were appended at the start
+        if (!(C::kInt8 && staged_new && p.group_by_request))
+          fused_append_rows<ActT, CacheT>(p, cs_s, past_s, t_lo, t_hi, h_kv, ksc, vsc, ptid, kTcProd, bits);
+      }
+    }
   }
 
   // S of tile n into buffer n % 2: A = Q from tensor memory, B = the tile's
@@ -710,28 +861,58 @@ int tc_supported(int act, int cache, int D, int max_rows) {
   return max_rows > 32 && max_rows <= 128;
 }
 
-template <typename ActT, typename CacheT, int D>
+// Shared memory the fused step adds: cumulative lengths [B + 1] and past
+// lengths [B], then (INT8) the staged new rows [kTcStageTok][K, V][D].
+static size_t tc_fused_extra_smem(int B, int cache, int D) {
+  return ((sizeof(int32_t) * (size_t)(2 * B + 1) + 15) & ~size_t(15)) +
+         (cache == SPA_I8 ? (size_t)kTcStageTok * 2 * D : 0);
+}
+
+template <typename ActT, typename CacheT, int D, bool FUSED>
 static int launch_tc_t(const AttnParams& p, cudaStream_t stream) {
   using C = TcCfg<ActT, CacheT, D>;
   static_assert(C::SMEM <= 227 * 1024, "shared memory");
-  auto kern = decode_tc_kernel<ActT, CacheT, D>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static_assert(C::SMEM >= C::BYTES + 1024, "the fused step's arrays follow the aligned layout");
+  static_assert(C::BYTES % 16 == 0, "the staged rows are 16-byte vectors");
+  auto kern = decode_tc_kernel<ActT, CacheT, D, FUSED>;
+  const size_t smem = C::SMEM + (FUSED ? tc_fused_extra_smem(p.B, C::kInt8 ? SPA_I8 : SPA_F16, D) : 0);
+  if (smem > 227 * 1024) return SPA_ERR_UNSUPPORTED;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int units = p.group_by_request ? p.B * p.H_kv : p.T * p.H_kv;
   if (p.cluster_merge)
-    return launch_pdl_cluster_y(kern, dim3(units, p.num_splits), dim3(kTcThreads), C::SMEM, stream, p.num_splits, p);
-  return launch_pdl(kern, dim3(units, p.num_splits), dim3(kTcThreads), C::SMEM, stream, p);
+    return launch_pdl_cluster_y(kern, dim3(units, p.num_splits), dim3(kTcThreads), smem, stream, p.num_splits, p);
+  return launch_pdl(kern, dim3(units, p.num_splits), dim3(kTcThreads), smem, stream, p);
+}
+
+template <bool FUSED>
+static int launch_tc_any(const AttnParams& p, int act, int cache, cudaStream_t stream) {
+  if (act == SPA_F16) {
+    if (cache == SPA_I8) return p.D == 64 ? launch_tc_t<__half, int8_t, 64, FUSED>(p, stream)
+                                          : launch_tc_t<__half, int8_t, 128, FUSED>(p, stream);
+    return p.D == 64 ? launch_tc_t<__half, __half, 64, FUSED>(p, stream)
+                     : launch_tc_t<__half, __half, 128, FUSED>(p, stream);
+  }
+  if (cache == SPA_I8) return p.D == 64 ? launch_tc_t<__nv_bfloat16, int8_t, 64, FUSED>(p, stream)
+                                        : launch_tc_t<__nv_bfloat16, int8_t, 128, FUSED>(p, stream);
+  return p.D == 64 ? launch_tc_t<__nv_bfloat16, __nv_bfloat16, 64, FUSED>(p, stream)
+                   : launch_tc_t<__nv_bfloat16, __nv_bfloat16, 128, FUSED>(p, stream);
 }
 
 int launch_attention_tc(const AttnParams& p, int act, int cache, cudaStream_t stream) {
-  if (act == SPA_F16) {
-    if (cache == SPA_I8) return p.D == 64 ? launch_tc_t<__half, int8_t, 64>(p, stream)
-                                          : launch_tc_t<__half, int8_t, 128>(p, stream);
-    return p.D == 64 ? launch_tc_t<__half, __half, 64>(p, stream) : launch_tc_t<__half, __half, 128>(p, stream);
-  }
-  if (cache == SPA_I8) return p.D == 64 ? launch_tc_t<__nv_bfloat16, int8_t, 64>(p, stream)
-                                        : launch_tc_t<__nv_bfloat16, int8_t, 128>(p, stream);
-  return p.D == 64 ? launch_tc_t<__nv_bfloat16, __nv_bfloat16, 64>(p, stream)
-                   : launch_tc_t<__nv_bfloat16, __nv_bfloat16, 128>(p, stream);
+  return launch_tc_any<false>(p, act, cache, stream);
+}
+
+// The whole step in one launch.
+int launch_step_tc(const AttnParams& p, int act, int cache, cudaStream_t stream) {
+  return launch_tc_any<true>(p, act, cache, stream);
+}
+
+// Whether the fused step fits one CTA's shared memory.
+int tc_step_fits(int D, int cache, int B) {
+  size_t base;
+  if (cache == SPA_I8) base = D == 64 ? TcCfg<__half, int8_t, 64>::SMEM : TcCfg<__half, int8_t, 128>::SMEM;
+  else base = D == 64 ? TcCfg<__half, __half, 64>::SMEM : TcCfg<__half, __half, 128>::SMEM;
+  return base + tc_fused_extra_smem(B, cache, D) <= 227 * 1024;
 }
 
 }  // namespace spa

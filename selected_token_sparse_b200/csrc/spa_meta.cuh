@@ -52,15 +52,17 @@ __device__ __forceinline__ int32_t request_seqlen_k(int past, int q_len) {
 }
 
 // Per-request outputs and the request-level status bits (block 0 only).
+// Threads ti = 0 .. nthr - 1 of the block share the work.
 __device__ __forceinline__ int per_request(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
                                            const int32_t* cs, int B, int T, int max_q, int max_k,
-                                           int32_t* __restrict__ seqlens_q, int32_t* __restrict__ seqlen_k) {
+                                           int32_t* __restrict__ seqlens_q, int32_t* __restrict__ seqlen_k,
+                                           int ti, int nthr) {
   int bits = 0;
-  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
+  for (int b = ti; b <= B; b += nthr) {
     if (cu[b] != cs[b]) bits |= kStBadCu;
     if (b == B && cs[B] != T) bits |= kStBadCu;
   }
-  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+  for (int b = ti; b < B; b += nthr) {
     int pb = past[b];
     if (pb < 0) {
       bits |= kStBadCu;
@@ -73,6 +75,11 @@ __device__ __forceinline__ int per_request(const int32_t* __restrict__ cu, const
     if (q_len > max_q || total > (long long)max_k) bits |= kStBounds;
   }
   return bits;
+}
+__device__ __forceinline__ int per_request(const int32_t* __restrict__ cu, const int32_t* __restrict__ past,
+                                           const int32_t* cs, int B, int T, int max_q, int max_k,
+                                           int32_t* __restrict__ seqlens_q, int32_t* __restrict__ seqlen_k) {
+  return per_request(cu, past, cs, B, T, max_q, max_k, seqlens_q, seqlen_k, threadIdx.x, blockDim.x);
 }
 
 struct TokenMeta {
@@ -144,7 +151,7 @@ struct FusedMeta {
   const int32_t* cs;
   const int32_t* past;
   int B;
-  __device__ __forceinline__ int cu(int g) const { return cu_raw[g]; }
+  __device__ __forceinline__ int cu(int g) const { return cs[g]; }   // request g's first token
   __device__ __forceinline__ int seqlens_q(int b) const { return cs[b + 1] - cs[b]; }
   __device__ __forceinline__ int seqlen_k(int b) const { return request_seqlen_k(past[b], cs[b + 1] - cs[b]); }
   __device__ __forceinline__ void token(int t, int& b, int& pos) const { token_owner(t, cs, B, past, b, pos); }
@@ -159,16 +166,20 @@ constexpr long long kNewRow = 1LL << 62;
 // Request-level part (CTA 0 of split 0): the per-request outputs and, with
 // request-grouped units, the metadata of tokens no request owns.
 __device__ __forceinline__ void fused_request_outputs(const AttnParams& p, const int32_t* cs, const int32_t* past,
-                                                      int& bits) {
+                                                      int& bits, int ti, int nthr) {
   bits |= per_request(p.cu, past, cs, p.B, p.T, p.max_seqlen_q, p.max_seqlen_k, p.seqlens_q_out,
-                      p.seqlen_k_out);
+                      p.seqlen_k_out, ti, nthr);
   if (p.group_by_request) {
-    for (int t = cs[p.B] + threadIdx.x; t < p.T; t += blockDim.x) {
+    for (int t = cs[p.B] + ti; t < p.T; t += nthr) {
       p.token_batch_out[t] = -1;
       p.token_pos_out[t] = -1;
       p.slot_out[t] = -1;
     }
   }
+}
+__device__ __forceinline__ void fused_request_outputs(const AttnParams& p, const int32_t* cs, const int32_t* past,
+                                                      int& bits) {
+  fused_request_outputs(p, cs, past, bits, threadIdx.x, blockDim.x);
 }
 
 // Token-level part for token t and kv head h_kv (split 0): the token's
@@ -214,6 +225,45 @@ __device__ __forceinline__ void fused_append_tokens(const AttnParams& p, const i
     if (m.slot < 0) continue;
     for (int v = threadIdx.x; v < 2 * nv; v += blockDim.x)
       fused_store_row_vector<T16>(p, m.slot, h_kv, v, nv, fused_load_row_vector<T16>(p, t, h_kv, v, nv));
+  }
+}
+
+// Tokens [t_lo, t_hi) of a unit for kv head h_kv, by threads ti = 0 .. nthr - 1:
+// each (token, item) pair finds the token's slot (the thread with item 0 of a
+// token writes its metadata, from kv head 0) and stores one item of the rows
+// -- a 16-byte vector copied (16-bit caches) or a 16-channel group quantised
+// with the shared group quantiser (INT8 caches; `ksc` / `vsc` are this kv
+// head's scales), so the cache holds what the append kernels write.
+template <typename ActT, typename CacheT>
+__device__ __forceinline__ void fused_append_rows(const AttnParams& p, const int32_t* cs, const int32_t* past,
+                                                 int t_lo, int t_hi, int h_kv, const float* ksc, const float* vsc,
+                                                 int ti, int nthr, int& bits) {
+  constexpr bool kI8 = sizeof(CacheT) == 1;
+  const int per_row = kI8 ? p.D / 16 : p.D * (int)sizeof(CacheT) / 16;
+  const int per_tok = 2 * per_row;
+  const int n = max(t_hi - t_lo, 0) * per_tok;
+  for (int idx = ti; idx < n; idx += nthr) {
+    const int t = t_lo + idx / per_tok, it = idx % per_tok;
+    int tb = 0;
+    const TokenMeta m = token_meta(t, cs, p.B, past, p.block_table, p.MB, p.bs, p.NB, tb);
+    if (it == 0 && h_kv == 0) {
+      bits |= tb;
+      p.token_batch_out[t] = m.b;
+      p.token_pos_out[t] = m.pos;
+      p.slot_out[t] = m.slot;
+    }
+    if (m.slot < 0) continue;
+    if constexpr (kI8) {
+      const bool isv = it >= per_row;
+      const int g = isv ? it - per_row : it;
+      Group16<ActT> x;
+      x.load(static_cast<const ActT*>(isv ? p.v_new : p.k_new) + ((long long)t * p.H_kv + h_kv) * p.D + g * 16);
+      int8_t* dst = static_cast<int8_t*>(const_cast<void*>(isv ? p.v_cache : p.k_cache)) +
+                    ((long long)m.slot * p.H_kv + h_kv) * p.D + g * 16;
+      *reinterpret_cast<uint4*>(dst) = quant_group16<ActT>(x.v, (isv ? vsc : ksc) + g * 16);
+    } else {
+      fused_store_row_vector<CacheT>(p, m.slot, h_kv, it, per_row, fused_load_row_vector<CacheT>(p, t, h_kv, it, per_row));
+    }
   }
 }
 

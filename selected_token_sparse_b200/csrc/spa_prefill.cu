@@ -160,7 +160,7 @@ __device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_pai
   g.b = rem / p.H_q;
   g.h = rem - g.b * p.H_q;
   const int pair = n_pairs - 1 - pz;
-  g.t_begin = clampi(p.cu[g.b], 0, p.T);
+  g.t_begin = clampi(sanitised_start(p, g.b), 0, p.T);
   g.q_len = clampi(p.seqlens_q[g.b], 0, p.T - g.t_begin);
   g.q0[0] = pair * 2 * kPfBM;
   g.q0[1] = g.q0[0] + kPfBM;
