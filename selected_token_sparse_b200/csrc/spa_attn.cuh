@@ -400,8 +400,13 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, 
         ml[t][s] = make_float2(-INFINITY, 0.f);
         a[t][s] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (s < S && it < n_items) {
-          ml[t][s] = ld_peer2(peer_smem(part_ml + 4 * r, s));
-          a[t][s] = ld_peer4(peer_smem(part_o + r * PS + c, s));
+          if (s == k) {   // this CTA's own state: a local read
+            ml[t][s] = *reinterpret_cast<const float2*>(part_ml + 4 * r);
+            a[t][s] = *reinterpret_cast<const float4*>(part_o + r * PS + c);
+          } else {
+            ml[t][s] = ld_peer2(peer_smem(part_ml + 4 * r, s));
+            a[t][s] = ld_peer4(peer_smem(part_o + r * PS + c, s));
+          }
         }
       }
     }
