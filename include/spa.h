@@ -225,8 +225,10 @@ size_t spa_attention_workspace_size(const spa_attention_args_t* a);
  * before its first use: it holds per-unit split tickets that every call
  * leaves at zero again (the partial states around them need no
  * initialisation).  Calls that share a workspace must be ordered on one
- * stream.  The whole operation is one kernel launch: the last CTA to finish
- * a unit's splits merges them.
+ * stream.  The whole operation is one kernel launch: on the tensor-core
+ * decode kernels the (at most 8) splits of a unit form one thread-block
+ * cluster and merge through distributed shared memory; otherwise the last
+ * CTA to finish a unit's splits merges them from the workspace.
  */
 int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
                   spa_stream_t stream);
@@ -238,10 +240,12 @@ int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspa
  * Source: "[WebGPU] Add SparsePagedAttention", File summaries (prepare the
  * token metadata, scatter the current K/V into the cache, then attend) --
  * here one kernel launch when the plan picks the warp-MMA decode kernel on a
- * 16-bit cache of the activation dtype (each CTA derives its unit's metadata
- * from cu_seqlens_q and past_seqlens in shared memory, writes its share of
- * the metadata and of the appended rows, and reads this step's own new rows
- * from k_new / v_new); otherwise the two launches of the staged sequence.
+ * 16-bit cache of the activation dtype, or the tcgen05 decode kernel on a
+ * 16-bit or INT8 cache (each CTA derives its unit's metadata from
+ * cu_seqlens_q and past_seqlens in shared memory, writes its share of the
+ * metadata and of the appended rows, and reads this step's own new rows from
+ * k_new / v_new -- INT8 rows quantised exactly as the append quantises
+ * them); otherwise the two launches of the staged sequence.
  *   a               the attention arguments; a->seqlens_q, a->seqlen_k,
  *                   a->token_batch and a->token_pos are OUTPUTS here (the
  *                   step-1 arrays, written with spa_prepare_metadata's
