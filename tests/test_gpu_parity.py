@@ -264,6 +264,12 @@ STEP_CASES = {
                            past=[100, 9, 3], window=64),
     "tc_int8_malformed_cu": dict(act="f16", cache="i8", B=3, H_q=48, H_kv=4, D=128, block_size=16,
                                  q_lens=[4, 3, 6], past=[20, 5, 40], window=8, spare_blocks=2),
+    # more new tokens than the staging area holds: quantised where a tile needs them
+    "tc_int8_many_new_tokens": dict(act="f16", cache="i8", B=2, H_q=2, H_kv=2, D=128, block_size=16,
+                                    q_lens=[80, 70], past=[30, 0]),
+    # 64 q heads per kv head: one token per unit (per-token units on tcgen05)
+    "tc_int8_per_token_units": dict(act="bf16", cache="i8", B=2, H_q=64, H_kv=1, D=64, block_size=16,
+                                    q_lens=[3, 2], past=[40, 9], window=16),
 }
 
 
