@@ -202,8 +202,7 @@ decode_mma_kernel(const AttnParams p) {
   if constexpr (FUSED) {
     cs_s = reinterpret_cast<int32_t*>(smem + C::SMEM);
     past_s = cs_s + p.B + 1;
-    for (int b = tid; b < p.B; b += NT) past_s[b] = p.past[b];
-    build_cs<NT>(p.cu, p.B, p.T, cs_s);   // ends with a block barrier
+    build_cs<NT>(p.cu, p.B, p.T, cs_s, p.past, past_s);   // ends with a block barrier
     has_rows = decode_unit_with(p, FusedMeta{p.cu, cs_s, past_s, p.B}, blockIdx.x, U);
     if (has_rows) {
       U.new_lo = max(past_s[U.b], 0);

@@ -200,8 +200,7 @@ decode_tc_kernel(const AttnParams p) {
     cs_s = reinterpret_cast<int32_t*>(smem + C::BYTES);
     past_s = cs_s + p.B + 1;
     stage_s = reinterpret_cast<int8_t*>(smem + C::BYTES + ((sizeof(int32_t) * (2 * p.B + 1) + 15) & ~size_t(15)));
-    for (int b = tid; b < p.B; b += kTcThreads) past_s[b] = p.past[b];
-    build_cs<kTcThreads>(p.cu, p.B, p.T, cs_s);   // ends with a block barrier
+    build_cs<kTcThreads>(p.cu, p.B, p.T, cs_s, p.past, past_s);   // ends with a block barrier
     has_rows = decode_unit_with(p, FusedMeta{p.cu, cs_s, past_s, p.B}, blockIdx.x, U);
     if (has_rows) {
       U.new_lo = max(past_s[U.b], 0);

@@ -12,11 +12,16 @@
 namespace spa {
 
 // Sanitised cumulative lengths into cs[0..B] (all threads of the block).
+// With `past`, the past lengths are copied into past_s[0..B) as well; their
+// first loads are issued ahead of the cumulative lengths' so that both are in
+// flight together, and the copy is visible once this returns.
 template <int NT>
-__device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, int T, int32_t* cs) {
+__device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, int T, int32_t* cs,
+                                         const int32_t* __restrict__ past = nullptr, int32_t* past_s = nullptr) {
   __shared__ int32_t warp_max[NT / 32];
   __shared__ int32_t chunk_carry[NT];
   const int tid = threadIdx.x;
+  const int pv0 = (past != nullptr && tid < B) ? ld_early(past + tid) : 0;
   const int n = B + 1;
   // contiguous chunk per thread: local prefix max, then a scan over chunk maxima
   const int per = (n + NT - 1) / NT;
@@ -36,6 +41,10 @@ __device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, 
     if (lane >= o) x = max(x, y);
   }
   if (lane == 31) warp_max[warp] = x;
+  if (past != nullptr) {
+    if (tid < B) past_s[tid] = pv0;
+    for (int b = tid + NT; b < B; b += NT) past_s[b] = past[b];
+  }
   __syncthreads();
   int prev_warps = 0;
   for (int w = 0; w < warp; ++w) prev_warps = max(prev_warps, warp_max[w]);

@@ -140,8 +140,7 @@ prepare_append_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict_
       }
     }
   }
-  for (int b = threadIdx.x; b < B; b += blockDim.x) past_s[b] = past[b];
-  build_cs<kMetaThreads>(cu, B, T, cs);   // ends with a block barrier: past_s is visible too
+  build_cs<kMetaThreads>(cu, B, T, cs, past, past_s);   // ends with a block barrier: past_s is visible too
   if (blockIdx.x == 0) flag(status, per_request(cu, past_s, cs, B, T, max_q, max_k, seqlens_q, seqlen_k));
   int bits = 0;
   for (int t = t_first; t < T; t += gridDim.x * wpb) {

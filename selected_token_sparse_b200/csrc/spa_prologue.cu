@@ -65,8 +65,7 @@ prepare_qkv_append_kernel(const QkvParams P) {
 #pragma unroll
     for (int e = 0; e < E; ++e) x0[e] = src[lane * E + e];
   }
-  for (int b = threadIdx.x; b < P.B; b += blockDim.x) past_s[b] = P.past[b];
-  build_cs<kProThreads>(P.cu, P.B, P.T, cs);
+  build_cs<kProThreads>(P.cu, P.B, P.T, cs, P.past, past_s);
   int bits = 0;
   if (blockIdx.x == 0)
     bits |= per_request(P.cu, past_s, cs, P.B, P.T, P.max_q, P.max_k, P.seqlens_q, P.seqlen_k);
