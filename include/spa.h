@@ -204,7 +204,8 @@ typedef struct spa_attention_args {
   int32_t* status;    /* OR-ed status bits */
 } spa_attention_args_t;
 
-/* Bytes of workspace spa_attention needs for these arguments (0 if none).
+/* Bytes of workspace spa_attention needs for these arguments (0 if none: one
+   split per unit, or splits that merge inside a thread-block cluster).
    Returns 0 as well for invalid arguments; spa_attention then reports the error. */
 size_t spa_attention_workspace_size(const spa_attention_args_t* a);
 
@@ -346,10 +347,15 @@ int spa_prepare_qkv_append(const spa_qkv_args_t* a, spa_stream_t stream);
  * and no allocating routine.
  *   - A call whose plan needs more scratch than SPA_NOALLOC_SCRATCH_BYTES
  *     (spa_attention_workspace_size() of the same arguments) returns
- *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.
+ *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.  Plans whose splits merge
+ *     inside a thread-block cluster need no scratch at all.
  *   - The first call on each device resolves the array's device address (with
  *     that device current); make that first call before any stream capture.
- *     If the address cannot be resolved the call returns SPA_ERR_CUDA.
+ *     Every later call made outside a capture resolves it again; a call made
+ *     during a capture reuses the address of the last uncaptured call on the
+ *     device, so after a context reset (cudaDeviceReset) make one call
+ *     outside a capture before capturing again.  If the address cannot be
+ *     resolved the call returns SPA_ERR_CUDA.
  *   - Every call on a device shares the array and sees what the previous call
  *     left in it; the values that must start at zero are cleared on `stream`
  *     before the kernel runs (one memset).  Calls that may overlap on the GPU

@@ -140,7 +140,12 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   pl->num_splits = (int)splits;
   pl->split_len = (int)std::min<long long>(per_tiles * KT, 0x7fffffffLL);
   pl->units = (int)units;
-  if (pl->num_splits > 1) {
+  // the splits of a unit merge through distributed shared memory when they
+  // fit one cluster (tensor-core decode kernels) and need no workspace;
+  // otherwise through the workspace, where the CTA that finishes last merges
+  pl->cluster_merge = (pl->kind == kPlanTc || pl->kind == kPlanMma) && pl->num_splits > 1 &&
+                      pl->num_splits <= 8;
+  if (pl->num_splits > 1 && !pl->cluster_merge) {
     const size_t rows = (size_t)a->T * a->H_q;
     pl->ws_acc_bytes = align256(rows * a->D * sizeof(float) * pl->num_splits);
     pl->ws_ml_bytes = align256(rows * 2 * sizeof(float) * pl->num_splits);
@@ -194,11 +199,8 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   p->num_splits = pl.num_splits;
   p->split_len = pl.split_len;
   p->status = a->status;
-  // the splits of a unit merge through distributed shared memory when they
-  // fit one cluster (tensor-core decode kernels); otherwise through the
-  // workspace, where the CTA that finishes last merges
-  p->cluster_merge = (pl.kind == kPlanTc || pl.kind == kPlanMma) && pl.num_splits > 1 && pl.num_splits <= 8;
-  if (pl.num_splits > 1) {
+  p->cluster_merge = pl.cluster_merge;
+  if (pl.num_splits > 1 && !pl.cluster_merge) {
     p->ws_acc = static_cast<float*>(ws);
     p->ws_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.ws_acc_bytes);
     p->ws_count = reinterpret_cast<int*>(static_cast<char*>(ws) + pl.ws_acc_bytes + pl.ws_ml_bytes);

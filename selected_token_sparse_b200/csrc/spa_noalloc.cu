@@ -12,9 +12,10 @@
 // The scratch is a file-scope __device__ array of SPA_NOALLOC_SCRATCH_BYTES;
 // every GPU that loads the library holds it until the process exits.  Host
 // code never uses the array's name as a device address: the first call on
-// each device, with that device current, resolves the address once with
+// each device, with that device current, resolves the address with
 // cudaGetSymbolAddress (so that first call should come before any stream
-// capture), and every call passes that pointer to the kernel.  All calls on a
+// capture; every later call outside a capture resolves it again), and every
+// call passes that pointer to the kernel.  All calls on a
 // device share the array and find the previous call's contents in it: the
 // tickets that must start at zero are cleared on the stream before each
 // launch, and calls that overlap on the GPU (other streams, other threads)
@@ -36,14 +37,27 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// Device address of the scratch array on the current device (set-up once).
-int scratch_address(void** out) {
+// Device address of the scratch array on the current device.  It is resolved
+// with that device current on the first call, and again on every call made
+// while `stream` is not being captured, so that a call after a context reset
+// (cudaDeviceReset reloads the module, and the array may move) uses the new
+// address.  A call made during a capture uses the address the last uncaptured
+// call on this device resolved.
+int scratch_address(cudaStream_t stream, void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SPA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SPA_ERR_CUDA;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    cs = cudaStreamCaptureStatusActive;  // unknown: do not resolve during a possible capture
+  }
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || cs == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
@@ -66,7 +80,7 @@ extern "C" int spa_attention_noalloc(const spa_attention_args_t* a, spa_stream_t
   const size_t need = pl.ws_acc_bytes + pl.ws_ml_bytes + pl.ws_count_bytes;
   if (need > SPA_NOALLOC_SCRATCH_BYTES) return SPA_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
-  if ((rc = scratch_address(&scratch)) != SPA_OK) return rc;
+  if ((rc = scratch_address((cudaStream_t)stream, &scratch)) != SPA_OK) return rc;
   if (pl.ws_count_bytes > 0) {
     // split tickets start at zero; the bytes may hold an earlier call's partials
     unsigned char* tickets = static_cast<unsigned char*>(scratch) + pl.ws_acc_bytes + pl.ws_ml_bytes;

@@ -44,6 +44,12 @@ MUTATIONS = [
      "ms = np.sum(x * x, axis=-1, keepdims=True)"),
     ("RMSNorm eps dropped", "np.sqrt(ms + float(eps))", "np.sqrt(ms)"),
     ("rotary offset ignored", "int(token_pos[t]) + int(rotary_offset)", "int(token_pos[t])"),
+    ("bf16 decode without the shift", "bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << 16",
+     "bits = np.asarray(x, dtype=np.uint16).astype(np.uint32)"),
+    ("bf16 decode shifted by 15", "bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << 16",
+     "bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << 15"),
+    ("bf16 bits read as float16", "return bits.view(np.float32).astype(np.float64)",
+     "return np.asarray(x, dtype=np.uint16).view(np.float16).astype(np.float64)"),
     ("bf16 ties away from even", "(((c >> 16) & 1) == 0) & (((best >> 16) & 1) == 1)",
      "(((c >> 16) & 1) == 1) & (((best >> 16) & 1) == 0)"),
 ]

@@ -594,6 +594,30 @@ def test_encode_rounds_to_nearest_even():
     np.testing.assert_array_equal(h.view(np.uint16), [0x3C00, 0x3C02])
 
 
+def test_bf16_decode_bit_patterns():
+    """bf16 codes read by hand from the format (1 sign, 8 exponent, 7 fraction
+    bits, bias 127): the value is the code placed in the upper half of a
+    binary32 word."""
+    codes = np.array([0x3F80, 0xC040, 0x0001, 0x4049, 0x3F81, 0x7F7F, 0x8000, 0x0080, 0x7F80, 0xFF80],
+                     dtype=np.uint16)
+    want = [1.0, -3.0, 2.0 ** -133, 3.140625, 1.0 + 2.0 ** -7, (2.0 - 2.0 ** -7) * 2.0 ** 127, -0.0,
+            2.0 ** -126, math.inf, -math.inf]
+    got = O.decode(codes, "bf16")
+    assert got.dtype == np.float64
+    np.testing.assert_array_equal(got, want)
+    assert math.copysign(1.0, got[6]) == -1.0
+
+
+def test_bf16_decode_encode_round_trip():
+    """Every non-NaN bf16 code decodes to a value that encodes back to itself."""
+    codes = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    exp = (codes.astype(np.uint32) >> 7) & 0xFF
+    frac = codes.astype(np.uint32) & 0x7F
+    keep = ~((exp == 0xFF) & (frac != 0))
+    codes = codes[keep]
+    np.testing.assert_array_equal(O.encode(O.decode(codes, "bf16"), "bf16"), codes)
+
+
 def _prologue_wl(**pro):
     from selected_token_sparse_b200 import workloads as W
     return W.make_workload(act="f16", B=2, H_q=4, H_kv=2, D=64, block_size=16, q_lens=[3, 2],
