@@ -1,16 +1,21 @@
 """Benchmark of the hot path: metadata prepare + KV append + sparse attention.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--only]
 
-A step is one pass of the whole path (spa_prepare_metadata, spa_append_kv,
-spa_attention) over one batch of the GPT-OSS-like paged decode workload
-(B=32, S_q=1, H_q=64, H_kv=8, D=64, block 16, lengths U[512, 8192], causal
-window 128, learned sinks, fp16).  Inputs are resident in HBM when the timed
-region starts; the step cycles through enough independent cache instances
-that the attended bytes of one cycle exceed twice the L2, so every step
-reads its keys from HBM.  Steps are replayed from CUDA graphs and timed with
-CUDA events on the launching stream.
+A step is one pass of the whole path (metadata prepare, KV append,
+attention) over one batch of a workload.  The headline workload is the
+GPT-OSS-like paged decode (B=32, S_q=1, H_q=64, H_kv=8, D=64, block 16,
+lengths U[512, 8192], causal window 128, learned sinks, fp16); unless
+--only is given, every other named workload (tiny fp32 decode,
+selected-token bf16 decode, local-plus-selected INT8 decode, ragged prefill,
+windowed chunked prefill, the QKV-prologue decode) is measured the same way
+and listed under "workloads" in the same JSON line.  Inputs are resident in
+HBM when the timed region starts; each step reads a different one of enough
+independent device instances that the attended bytes of one cycle exceed
+twice the L2, so every step reads its keys from HBM.  The K timed steps
+are captured as one CUDA graph (one per 1000 steps) and timed with CUDA
+events on the launching stream.
 
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no data
 collective); the time is the maximum over ranks.
@@ -45,33 +50,40 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # bookkeeping shared by both arms
 # ---------------------------------------------------------------------------
 
-def attended_kv_bytes(wl) -> int:
+def _token_set(wl, tokens):
+    return set(range(wl.T)) if tokens is None else {int(t) for t in tokens}
+
+
+def attended_kv_bytes(wl, tokens=None) -> int:
     """Algorithmic attended K+V bytes of one step: for every (request, kv
-    head), the union over the request's query tokens of the attended keys,
-    times D times the cache element size, for K and V."""
+    head), the union over the request's query tokens (those in ``tokens``
+    when given) of the attended keys, times D times the cache element size,
+    for K and V."""
     elt = {"f32": 4, "f16": 2, "bf16": 2, "i8": 1}[wl.cache]
+    keep = _token_set(wl, tokens)
     total = 0
     a = wl.arrays
+    cu = [int(x) for x in a["cu_seqlens_q"]]
     for b in range(wl.B):
         q, p0 = wl.q_lens[b], wl.past[b]
-        if q == 0:
+        toks = [t for t in range(cu[b], cu[b + 1]) if t in keep]
+        if q == 0 or not toks:
             continue
         L = p0 + q
         for h in range(wl.H_kv):
             n = 0
             if wl.sel_mode == "main":
-                rows = [b] if wl.sel_per_request else list(range(int(a["cu_seqlens_q"][b]),
-                                                                 int(a["cu_seqlens_q"][b + 1])))
+                rows = [b] if wl.sel_per_request else toks
                 s = set()
                 for r in rows:
                     s |= {int(i) for i in a["selected_idx"][r, h] if 0 <= i < L}
                 n = len(s)
             else:
-                lo = max(0, p0 - wl.window + 1) if wl.window > 0 else 0
-                n = L - lo
+                ps = [p0 + t - cu[b] for t in toks]
+                lo = max(0, min(ps) - wl.window + 1) if wl.window > 0 else 0
+                n = max(ps) + 1 - lo
                 if wl.sel_mode == "aux":
-                    rows = [b] if wl.sel_per_request else list(range(int(a["cu_seqlens_q"][b]),
-                                                                     int(a["cu_seqlens_q"][b + 1])))
+                    rows = [b] if wl.sel_per_request else toks
                     s = set()
                     for r in rows:
                         s |= {int(i) for i in a["selected_idx"][r, h] if 0 <= i < int(a["aux_seqlens"][b])}
@@ -80,16 +92,55 @@ def attended_kv_bytes(wl) -> int:
     return total
 
 
-def attention_flops(wl) -> int:
-    """Algorithmic FLOPs of QK^T and PV over the attended (causal) pairs."""
+def attention_flops(wl, tokens=None) -> int:
+    """Algorithmic FLOPs of QK^T and PV over the attended (causal) pairs of
+    the query tokens (those in ``tokens`` when given)."""
+    keep = _token_set(wl, tokens)
     pairs = 0
+    t = 0
     for b in range(wl.B):
         q, p0 = wl.q_lens[b], wl.past[b]
         for i in range(q):
-            p = p0 + i
-            lo = max(0, p - wl.window + 1) if wl.window > 0 else 0
-            pairs += p - lo + 1
+            if t in keep:
+                p = p0 + i
+                lo = max(0, p - wl.window + 1) if wl.window > 0 else 0
+                pairs += p - lo + 1
+            t += 1
     return 4 * wl.D * wl.H_q * pairs
+
+
+def is_prefill(wl) -> bool:
+    return wl.max_seqlen_q > 16 and wl.sel_mode is None
+
+
+def work_of(wl, tokens=None):
+    """(amount, unit scale, unit) of the metric for a step over ``tokens``:
+    attended K+V bytes in GB/s for decode, attention FLOPs in TFLOP/s for
+    prefill."""
+    if is_prefill(wl):
+        return attention_flops(wl, tokens), 1e12, "TFLOP/s"
+    return attended_kv_bytes(wl, tokens), 1e9, "GB/s"
+
+
+L2_NOTE = ("inputs larger than L2: each step reads a different one of several independent device "
+           "copies of the workload, whose attended bytes per cycle exceed twice the L2")
+
+
+def workload_config(wl, world: int) -> dict:
+    """The `config` object of a JSON line: the workload, identical in both arms."""
+    return {"workload": wl.name, "B": wl.B, "S_q": wl.max_seqlen_q, "T": wl.T, "H_q": wl.H_q,
+            "H_kv": wl.H_kv, "D": wl.D, "block_size": wl.block_size, "window": wl.window,
+            "max_seqlen_k": wl.max_seqlen_k, "selection": wl.sel_mode, "sel_width": wl.sel_width,
+            "sinks": wl.has_sinks, "act": wl.act, "cache": wl.cache,
+            "prologue": bool(getattr(wl, "prologue", None)),
+            "parallelism": f"dp{world}" if world > 1 else "single", "l2": L2_NOTE}
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def load_peaks():
@@ -228,55 +279,131 @@ class ClockSampler:
 # the CPU baseline (fp64 oracle)
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(wl, budget_s: float = 12.0, max_steps: int = 1000, min_steps: int = 1):
-    """Time the oracle as it stands on the host: whole steps of the workload
-    until the budget is spent.  Returns (seconds per step, steps, cores)."""
+def oracle_sample(wl, budget_s: float):
+    """Token sample of one oracle step that takes about budget_s / 3 on this
+    host: every token when a whole step fits, else evenly spaced tokens (the
+    metadata and the append always run in full).  The step's fixed cost and
+    its cost per token are estimated from steps over one and over four
+    tokens.  Returns the token list, or None for whole steps."""
     from oracle import spa_oracle as O
+
+    def spaced(n):
+        return [int(x) for x in np.linspace(0, wl.T - 1, n).round().astype(int)]
+
+    def seconds(tokens):
+        t0 = time.perf_counter()
+        O.run_step(wl, tokens=tokens)
+        return time.perf_counter() - t0
+
+    if wl.T <= 4:
+        return None
+    seconds(spaced(1))                       # first touch of the arrays
+    t1 = seconds(spaced(1))
+    t4 = seconds(spaced(4))
+    per_tok = max((t4 - t1) / 3.0, 1e-6)
+    fixed = max(t1 - per_tok, 0.0)
+    n = int((budget_s / 3.0 - fixed) / per_tok)
+    if n >= wl.T:
+        return None
+    return spaced(max(1, n))
+
+
+def cpu_baseline(wl, budget_s: float = 10.0, max_steps: int = 1000):
+    """Time the oracle as it stands on the host: steps of the workload (each
+    over a bounded token sample) until the budget is spent.  Returns the
+    cpu_baseline object."""
+    from oracle import spa_oracle as O
+    tokens = oracle_sample(wl, budget_s)
     n = 0
     t0, c0 = time.perf_counter(), time.process_time()
-    while n < min_steps or (time.perf_counter() - t0 < budget_s and n < max_steps):
-        O.run_step(wl)
+    while n < 1 or (time.perf_counter() - t0 < budget_s and n < max_steps):
+        O.run_step(wl, tokens=tokens)
         n += 1
     wall = time.perf_counter() - t0
-    cpu = time.process_time() - c0
-    cores = max(1, int(round(cpu / wall)))
-    return wall / n, n, cores
+    cores = max(1, int(round((time.process_time() - c0) / wall)))
+    amount, scale, unit = work_of(wl, tokens)
+    sample = (f"{n} whole step(s)" if tokens is None else
+              f"{n} step(s) over {len(tokens)} of {wl.T} query tokens (metadata and append in full)")
+    return {"value": amount / (wall / n) / scale, "unit": unit, "cores": cores,
+            "host_cores": host_cores(), "kind": "oracle",
+            "sample": sample + " of the same workload, fp64 numpy oracle, single-threaded"}
 
 
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args):
+GRAPH_CHUNK = 1000   # steps per captured graph; K steps replay ceil(K / chunk) graphs
+
+
+class Graphs:
+    """K consecutive steps captured as few CUDA graphs as possible (one when
+    K <= GRAPH_CHUNK), each step on the next device instance in turn."""
+
+    def __init__(self, stream, step_fns, k: int, start: int = 0):
+        import torch
+        self.graphs = []
+        R = len(step_fns)
+        i = start
+        left = k
+        while left > 0:
+            n = min(left, GRAPH_CHUNK)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(n):
+                    step_fns[(i + j) % R]()
+            self.graphs.append(g)
+            i += n
+            left -= n
+
+    def replay(self):
+        for g in self.graphs:
+            g.replay()
+
+
+def timed(dev, stream, graphs: Graphs, sampler=None):
+    """Device time (ms) of one replay of `graphs`, bracketed by a barrier and a
+    synchronize on both sides; the maximum over ranks."""
     import torch
-    import torch.distributed as dist
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    if sampler is not None:
+        sampler.__enter__()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        graphs.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if sampler is not None:
+        sampler.__exit__(None, None, None)
+    barrier(dev)
+    return reduce_max(ev0.elapsed_time(ev1), dev)
+
+
+def measure(name, args, dev, rank, world, headline: bool):
+    """Time K steps of one workload (and its dominant kernel); returns the
+    per-workload result object."""
+    import torch
 
     from selected_token_sparse_b200 import pipeline, spa, workloads as W
 
-    rank, world, local = dist_env()
-    if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
-                                timeout=__import__("datetime").timedelta(seconds=120))
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
-    seed_off = 100 * rank
-    wl = W.by_name(args.workload, seed=None if rank == 0 else 1 + seed_off)
-    alg_bytes = attended_kv_bytes(wl)
-    flops = attention_flops(wl)
-    is_prefill = wl.max_seqlen_q > 16 and wl.sel_mode is None
+    # rank 0 draws the named workload's own seed; other ranks draw other batches
+    wl = W.by_name(name) if rank == 0 else W.by_name(name, seed=1000 * rank + len(name))
+    amount, scale, unit = work_of(wl)
+    prefill = is_prefill(wl)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    K = args.steps if headline else min(args.steps, GRAPH_CHUNK)
+    Wm = args.warmup if headline else min(args.warmup, 50)
 
     # independent device instances so that a cycle's attended bytes exceed 2x L2
     base = pipeline.to_device(wl, dev)
-    per_inst = alg_bytes + sum(base[k].numel() * base[k].element_size()
-                               for k in ("q", "k_new", "v_new"))
+    per_inst = (attended_kv_bytes(wl) if not prefill else 0) + sum(
+        base[k].numel() * base[k].element_size() for k in ("q", "k_new", "v_new") if k in base)
     R = args.instances or max(2, min(64, math.ceil(2 * l2 / max(per_inst, 1))))
-    if is_prefill:
-        R = args.instances or 2
     insts = []
     for i in range(R):
-        d = {k: (v.clone() if k in ("k_cache", "v_cache", "q", "k_new", "v_new", "block_table",
+        d = {k: (v.clone() if k in ("k_cache", "v_cache", "q", "k_new", "v_new", "qkv", "block_table",
                                    "cu_seqlens_q", "past_seqlens", "selected_idx") else v)
              for k, v in base.items()}
         insts.append(pipeline.Step(wl, d, num_splits=args.splits, mode=args.mode))
@@ -284,7 +411,6 @@ def run_ours(args):
     step0 = insts[0]
     plan = spa.attention_plan(step0.args)
     launches_per_step = step0.launches()
-    # one launch per step: the fused step kernel is the whole step
     single = launches_per_step == 1
     kind_name = {0: "decode_scalar", 1: "decode_mma", 2: "prefill_tcgen05", 3: "decode_tc"}[plan["kind"]]
     if single:
@@ -297,180 +423,165 @@ def run_ours(args):
             st()
     torch.cuda.synchronize(dev)
 
-    # CUDA graphs: one per instance, plus one chaining all instances
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            fn()
-        return g
-
-    g_one = [capture(st) for st in insts]
-    g_all = capture(lambda: [st() for st in insts])
-
-    def attn_only(st):
-        def f():
-            spa.run_attention(st.args, st.workspace)   # the step's own attention call
-        return f
-
-    ga_one = [capture(attn_only(st)) for st in insts]
-    ga_all = capture(lambda: [attn_only(st)() for st in insts])
-
-    def replay(graph_all, graph_one, k):
-        q, r = divmod(k, R)
-        for _ in range(q):
-            graph_all.replay()
-        for i in range(r):
-            graph_one[i].replay()
-
-    K, Wm = args.steps, args.warmup
+    g_warm = Graphs(stream, insts, Wm)
+    g_steps = Graphs(stream, insts, K, start=Wm)
     with torch.cuda.stream(stream):
-        replay(g_all, g_one, Wm)
+        g_warm.replay()
     torch.cuda.synchronize(dev)
-
-    # ---- timed region: exactly K steps
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clk:
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            replay(g_all, g_one, K)
-            ev1.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(dev)
-    ms = ev0.elapsed_time(ev1)
-    ms = reduce_max(ms, dev)
+    clk = ClockSampler(dev.index)
+    ms = timed(dev, stream, g_steps, clk)
     ms_per_step = ms / K
+    del g_steps
 
-    # ---- dominant kernel alone (same rotation), for the roofline; a fused
-    # step is one launch, so the timed steps above time that kernel
+    # the dominant kernel: a one-launch step is that kernel; otherwise the
+    # step's attention launch alone, over the same rotation
     if single:
         attn_ms = ms_per_step
     else:
-        with torch.cuda.stream(stream):
-            replay(ga_all, ga_one, Wm)
-        torch.cuda.synchronize(dev)
+        attn = [lambda st=st: spa.run_attention(st.args, st.workspace) for st in insts]
         ka = max(K, R)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga_warm = Graphs(stream, attn, Wm)
+        ga = Graphs(stream, attn, ka, start=Wm)
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            replay(ga_all, ga_one, ka)
-            e1.record(stream)
+            ga_warm.replay()
         torch.cuda.synchronize(dev)
-        attn_ms = e0.elapsed_time(e1) / ka
+        attn_ms = timed(dev, stream, ga) / ka
+        del ga, ga_warm
+    del g_warm
 
-    # ---- end to end through the Python API with host buffers
     e2e = None
-    if not args.no_e2e:
-        host = pipeline.to_device(wl, pin=True)
-        packed = bool(getattr(wl, "prologue", None) and wl.prologue.get("packed"))
-        inputs = (("qkv",) if packed else ("q", "k_new", "v_new")) + (
-            "cu_seqlens_q", "past_seqlens", "block_table", "selected_idx", "position_ids")
-        names = [n for n in inputs if n in host]
-        # a step's inputs travel as ONE host->device copy: they sit in one pinned
-        # host buffer and, on the device, in one buffer whose 256-byte-aligned
-        # slices are the tensors the step reads (the caches stay per instance)
-        offs, total = {}, 0
-        for n in names:
-            offs[n] = total
-            total += (host[n].numel() * host[n].element_size() + 255) // 256 * 256
-        hbuf = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-        for n in names:
-            nb = host[n].numel() * host[n].element_size()
-            hbuf[offs[n]:offs[n] + nb].copy_(host[n].contiguous().view(-1).view(torch.uint8))
-        e2e_insts = []
-        for st in insts:
-            dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
-            d2 = dict(st.d)
-            for n in names:
-                nb = host[n].numel() * host[n].element_size()
-                d2[n] = dbuf[offs[n]:offs[n] + nb].view(host[n].dtype).view(host[n].shape)
-                d2[n].copy_(st.d[n])
-            e2e_insts.append((dbuf, pipeline.Step(wl, d2, num_splits=args.splits, want_lse=False,
-                                                  mode=args.mode)))
-        h2d = total
-        out_host = torch.empty(step0.out.shape, dtype=step0.out.dtype, pin_memory=True)
-        d2h = out_host.numel() * out_host.element_size()
-        ke = min(K, 2000)
-
-        def e2e_step(i):
-            dbuf, st = e2e_insts[i % R]
-            dbuf.copy_(hbuf, non_blocking=True)
-            st()
-            out_host.copy_(st.out, non_blocking=True)
-
-        with torch.cuda.stream(stream):
-            for i in range(min(Wm, 50)):
-                e2e_step(i)
-        torch.cuda.synchronize(dev)
-        barrier(dev)
-        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            x0.record(stream)
-            for i in range(ke):
-                e2e_step(i)
-            x1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = reduce_max(x0.elapsed_time(x1), dev) / ke
-        if is_prefill:
-            e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s"}
-        else:
-            e2e = {"value": world * alg_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s"}
-        e2e.update({"h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "ms_per_step": e2e_ms, "steps": ke})
+    if headline and not args.no_e2e:
+        e2e = measure_e2e(wl, args, dev, stream, insts, amount, scale, unit, world)
 
     status = int(insts[0].status.item())
     hbm, bf16, bf16_sus, peak_src = load_peaks()
-    if is_prefill:
-        achieved = flops / (attn_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                "frac": achieved / bf16, "peak_source": f"{peak_src} bf16 dense (fp16 same rate)"}
-        value = world * flops / (ms_per_step * 1e-3) / 1e12
-        unit = "TFLOP/s"
+    achieved = amount / (attn_ms * 1e-3) / scale
+    if prefill:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": unit,
+                "frac": achieved / bf16, "peak_source": f"{peak_src} bf16 dense burst (fp16 same rate)"}
     else:
-        achieved = alg_bytes / (attn_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": unit,
                 "frac": achieved / hbm, "peak_source": f"{peak_src} HBM copy"}
-        value = world * alg_bytes / (ms_per_step * 1e-3) / 1e9
-        unit = "GB/s"
     entry = "spa_prepare_append_attention" if single else "spa_attention"
     roof.update({"kernel": f"{entry} ({kind_name}, 1 launch, {plan['num_splits']} split(s))",
-                 "us_per_launch": attn_ms * 1e3,
-                 "algorithmic_per_launch": flops if is_prefill else alg_bytes,
-                 "traffic": recorded_traffic(kind_name, args.workload)})
-
+                 "us_per_launch": attn_ms * 1e3, "algorithmic_per_launch": amount,
+                 "traffic": recorded_traffic(kind_name, name)})
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sec, n, cores = cpu_baseline(wl)
-        cv = (flops / sec / 1e12) if is_prefill else (alg_bytes / sec / 1e9)
-        cpu = {"value": cv, "unit": unit, "cores": cores, "kind": "oracle",
-               "sample": f"{n} whole step(s) of the same workload (metadata, append, attention "
-                         f"for all {wl.T} tokens), fp64 numpy oracle"}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K,
-        "warmup": Wm, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": wl.act, "data": "synthetic",
-        "config": {"workload": args.workload, "B": wl.B, "S_q": wl.max_seqlen_q, "H_q": wl.H_q,
-                   "H_kv": wl.H_kv, "D": wl.D, "block_size": wl.block_size, "window": wl.window,
-                   "max_seqlen_k": wl.max_seqlen_k, "sinks": wl.has_sinks, "cache": wl.cache,
-                   "parallelism": f"dp{world}" if world > 1 else "single",
+        cpu = cpu_baseline(wl, budget_s=10.0 if headline else 3.0)
+    res = {"workload": name, "dtype": wl.act, "value": world * amount / (ms_per_step * 1e-3) / scale, "unit": unit,
+           "ms_per_step": ms_per_step, "steps": K, "warmup": Wm,
+           "tokens_per_s": world * wl.T / (ms_per_step * 1e-3),
+           "algorithmic_per_step": amount, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+           "gpu_launches": K * launches_per_step, "launches_per_step": launches_per_step,
+           "num_splits": plan["num_splits"], "clocks": clk.summary(), "status": status,
+           "config": workload_config(wl, world),
+           "run": {"instances": R,
                    "l2": f"rotating {R} device instances, attended+q/k/v bytes per cycle "
                          f"{R * per_inst / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB",
-                   "timing": "CUDA graphs of whole steps, CUDA events on the launching stream",
-                   "step_entry": {"step": "spa_prepare_append_attention",
-                                  "prepare_append": "spa_prepare_append_kv + spa_attention",
-                                  "staged": "spa_prepare_metadata + spa_append_kv + spa_attention"}[args.mode],
-                   "launches_per_step": launches_per_step,
-                   "num_splits": plan["num_splits"]},
-        "tokens_per_s": world * wl.T / (ms_per_step * 1e-3),
-        "attended_kv_bytes_per_step": alg_bytes,
-        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": K * launches_per_step,
-        "clocks": clk.summary(), "status": status,
+                   "timing": f"{K} steps captured in {math.ceil(K / GRAPH_CHUNK)} CUDA graph(s), "
+                             "CUDA events on the launching stream",
+                   "step_entry": ("spa_prepare_qkv_append + spa_attention" if getattr(wl, "prologue", None) else
+                                  {"step": "spa_prepare_append_attention",
+                                   "prepare_append": "spa_prepare_append_kv + spa_attention",
+                                   "staged": "spa_prepare_metadata + spa_append_kv + spa_attention"}[args.mode])}}
+    del insts
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_e2e(wl, args, dev, stream, insts, amount, scale, unit, world):
+    """The metric end to end through the Python API: every step copies its
+    inputs from pinned host memory to the device and reads the output back."""
+    import torch
+
+    from selected_token_sparse_b200 import pipeline
+    R = len(insts)
+    host = pipeline.to_device(wl, pin=True)
+    packed = bool(getattr(wl, "prologue", None) and wl.prologue.get("packed"))
+    inputs = (("qkv",) if packed else ("q", "k_new", "v_new")) + (
+        "cu_seqlens_q", "past_seqlens", "block_table", "selected_idx", "position_ids")
+    names = [n for n in inputs if n in host]
+    # a step's inputs travel as ONE host->device copy: they sit in one pinned
+    # host buffer and, on the device, in one buffer whose 256-byte-aligned
+    # slices are the tensors the step reads (the caches stay per instance)
+    offs, total = {}, 0
+    for n in names:
+        offs[n] = total
+        total += (host[n].numel() * host[n].element_size() + 255) // 256 * 256
+    hbuf = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    for n in names:
+        nb = host[n].numel() * host[n].element_size()
+        hbuf[offs[n]:offs[n] + nb].copy_(host[n].contiguous().view(-1).view(torch.uint8))
+    e2e_insts = []
+    for st in insts:
+        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        d2 = dict(st.d)
+        for n in names:
+            nb = host[n].numel() * host[n].element_size()
+            d2[n] = dbuf[offs[n]:offs[n] + nb].view(host[n].dtype).view(host[n].shape)
+            d2[n].copy_(st.d[n])
+        e2e_insts.append((dbuf, pipeline.Step(wl, d2, num_splits=args.splits, want_lse=False,
+                                              mode=args.mode)))
+    out_host = torch.empty(insts[0].out.shape, dtype=insts[0].out.dtype, pin_memory=True)
+    d2h = out_host.numel() * out_host.element_size()
+    ke = min(args.steps, 2000)
+
+    def e2e_step(i):
+        dbuf, st = e2e_insts[i % R]
+        dbuf.copy_(hbuf, non_blocking=True)
+        st()
+        out_host.copy_(st.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(min(args.warmup, 50)):
+            e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        x0.record(stream)
+        for i in range(ke):
+            e2e_step(i)
+        x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(x0.elapsed_time(x1), dev) / ke
+    return {"value": world * amount / (e2e_ms * 1e-3) / scale, "unit": unit,
+            "h2d_bytes_per_step": int(total), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": e2e_ms, "steps": ke}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from selected_token_sparse_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    names = [args.workload]
+    if not args.only:
+        names += [n for n in W.WORKLOADS + W.PROLOGUE_WORKLOADS if n != args.workload]
+    results = [measure(n, args, dev, rank, world, headline=(i == 0)) for i, n in enumerate(names)]
+    h = results[0]
+    line = {
+        "metric": METRIC, "value": h["value"], "unit": h["unit"], "n_gpus": world, "steps": h["steps"],
+        "warmup": h["warmup"], "ms_per_step": h["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": h["dtype"], "data": "synthetic",
+        "config": h["config"], "tokens_per_s": h["tokens_per_s"],
+        "algorithmic_per_step": h["algorithmic_per_step"],
+        "roofline": h["roofline"], "cpu_baseline": h["cpu_baseline"], "e2e": h["e2e"],
+        "gpu_launches": h["gpu_launches"], "clocks": h["clocks"], "status": h["status"],
+        "run": h["run"],
+        "workloads": [{k: v for k, v in r.items() if k != "e2e"} for r in results],
     }
     if world > 1:
-        del g_one, g_all, ga_one, ga_all
         dist.barrier(device_ids=[dev.index])
         dist.destroy_process_group()
     if rank == 0:
@@ -488,17 +599,8 @@ def run_reference(args):
     from oracle import spa_oracle as O
     from selected_token_sparse_b200 import workloads as W
     wl = W.by_name(args.workload)
-    alg_bytes = attended_kv_bytes(wl)
-    flops = attention_flops(wl)
-    is_prefill = wl.max_seqlen_q > 16 and wl.sel_mode is None
     budget = 120.0 / max(1, args.steps + args.warmup)     # seconds per step
-    # whole steps when they fit the per-step budget, otherwise a token sample
-    t0 = time.perf_counter()
-    O.run_step(wl)
-    full = time.perf_counter() - t0
-    frac = 1.0 if full <= budget else max(budget / full, 1.0 / wl.T)
-    ntok = max(1, int(round(frac * wl.T)))
-    tokens = None if ntok >= wl.T else list(np.linspace(0, wl.T - 1, ntok).astype(int))
+    tokens = oracle_sample(wl, 3.0 * budget)
     for _ in range(args.warmup):
         O.run_step(wl, tokens=tokens)
     c0 = time.process_time()
@@ -507,20 +609,17 @@ def run_reference(args):
         O.run_step(wl, tokens=tokens)
     wall = time.perf_counter() - t0
     cores = max(1, int(round((time.process_time() - c0) / wall)))
-    share = 1.0 if tokens is None else len(tokens) / wl.T
+    amount, scale, unit = work_of(wl, tokens)
     sec = wall / args.steps
-    if is_prefill:
-        value, unit = share * flops / sec / 1e12, "TFLOP/s"
-    else:
-        value, unit = share * alg_bytes / sec / 1e9, "GB/s"
+    value = amount / sec / scale
     sample = ("whole steps" if tokens is None else
-              f"{len(tokens)} of {wl.T} tokens per step (metadata and append in full)")
+              f"{len(tokens)} of {wl.T} query tokens per step (metadata and append in full)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload},
-            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "data": "synthetic", "config": workload_config(wl, world),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "host_cores": host_cores(),
+                             "kind": "oracle", "sample": sample + ", fp64 numpy oracle, single-threaded"},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -531,7 +630,8 @@ def main():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, help="the headline workload")
+    ap.add_argument("--only", action="store_true", help="measure the headline workload only")
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--splits", type=int, default=0, help="key splits per unit (0 = automatic)")
     ap.add_argument("--mode", choices=["step", "prepare_append", "staged"], default="step",
@@ -542,6 +642,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.steps < 1:
+        args.steps = 1
     if args.impl == "reference":
         run_reference(args)
     else:

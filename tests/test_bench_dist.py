@@ -69,3 +69,36 @@ def test_attention_flops_causal():
                          past=[0, 4], seed=0)
     pairs = (1 + 2 + 3) + (5 + 6)
     assert bench.attention_flops(wl) == 4 * 8 * 2 * pairs
+
+
+def test_attended_bytes_of_a_token_subset():
+    # two requests of 3 tokens each, window 4: request 0 tokens at 10, 11, 12
+    wl = W.make_workload(act="f16", B=2, H_q=2, H_kv=1, D=64, block_size=16, q_lens=[3, 3],
+                         past=[10, 2], window=4, seed=0)
+    row = 64 * 2 * 2
+    # all tokens: request 0 keys 7..12 (6), request 1 keys 0..4 (5)
+    assert bench.attended_kv_bytes(wl) == (6 + 5) * row
+    # token 1 alone (position 11): keys 8..11
+    assert bench.attended_kv_bytes(wl, tokens=[1]) == 4 * row
+    # token 3 (request 1, position 2): keys 0..2
+    assert bench.attended_kv_bytes(wl, tokens=[1, 3]) == (4 + 3) * row
+    assert bench.attention_flops(wl, tokens=[0]) == 4 * 64 * 2 * 4
+
+
+def test_reference_arm_prints_our_config(capsys):
+    """The reference arm (the oracle on the host) reports the same config object
+    as our arm would for the same workload."""
+    import json
+    import sys
+    argv = sys.argv
+    sys.argv = ["bench.py", "--impl", "reference", "--workload", "tiny_decode_f32", "--steps", "1",
+                "--warmup", "3"]
+    try:
+        bench.main()
+    finally:
+        sys.argv = argv
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.workload_config(W.by_name("tiny_decode_f32"), 1)
+    assert line["cpu_baseline"]["host_cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
