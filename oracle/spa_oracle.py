@@ -7,6 +7,11 @@ its Python binding) never calls it and shares no code with it.
 It is a plain, slow restatement of what the pages define, written in the order
 the pages describe the pipeline:
 
+  0. selection producer -- onnxruntime PR #33472, Key Changes
+     (PackedSparseAttentionIndexer: QSA TopK selection) and experiments note
+     (compact TopK keeps stable keys, causal tails, capacity padding and
+     overflow handling): the top_k keys of per-key scores, as selected
+     indices for step 3.
   1. metadata prepare  -- "[WebGPU] Add PagedAttention metadata and GPT-OSS
      support" (onnxruntime PR #32277), Description and Changes (exact
      per-request seqlen_k / seqlens_q derived on device), review item T1
@@ -77,6 +82,41 @@ def decode(x: np.ndarray, dtype: str) -> np.ndarray:
         bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << 16
         return bits.view(np.float32).astype(np.float64)
     raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# 0. selection producer (TopK over per-key scores)
+# ---------------------------------------------------------------------------
+#
+# onnxruntime PR #33472, Key Changes (PackedSparseAttentionIndexer: QSA block
+# scoring and hierarchical / compact TopK selection feeding the selected
+# indices of DynamicSparseAttention) and the experiments note on compact TopK
+# (it keeps stable keys, causal tails, capacity stride / padding and overflow
+# handling).  The pages never define the score itself, so the scores are an
+# input here.  Readings:
+#   * a row's eligible keys are j <= bound (the causal tail: a request's
+#     last position, seqlen_k = total - 1, or a token's own position) with a
+#     score that is neither NaN nor -inf (-inf masks a key);
+#   * the top_k eligible keys by score are kept; equal scores keep the lower
+#     key index first (stable);
+#   * the kept indices are written in increasing order at the start of the
+#     row, and the rest of the row (its capacity, sel_width) is -1;
+#   * fewer eligible keys than top_k: all of them are kept (no overflow).
+
+def select_topk(scores: np.ndarray, bound: np.ndarray, top_k: int, sel_width: int) -> np.ndarray:
+    """selected_idx [R, H, sel_width] of fp32 scores [R, H, N] with per-row bounds [R]."""
+    scores = np.asarray(scores, dtype=np.float32)
+    R, H, N = scores.shape
+    out = np.full((R, H, sel_width), -1, dtype=np.int32)
+    for r in range(R):
+        last = min(int(bound[r]), N - 1)
+        for h in range(H):
+            row = [float(v) for v in scores[r, h]]
+            eligible = [j for j in range(last + 1) if not math.isnan(row[j]) and row[j] != -math.inf]
+            ranked = sorted(eligible, key=lambda j: (-row[j], j))
+            kept = sorted(ranked[:top_k])
+            out[r, h, :len(kept)] = kept
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -50,6 +50,14 @@ MUTATIONS = [
      "bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << 15"),
     ("bf16 bits read as float16", "return bits.view(np.float32).astype(np.float64)",
      "return np.asarray(x, dtype=np.uint16).view(np.float16).astype(np.float64)"),
+    ("topk ties keep the higher index", "key=lambda j: (-row[j], j)", "key=lambda j: (-row[j], -j)"),
+    ("topk bound exclusive", "for j in range(last + 1) if not", "for j in range(last) if not"),
+    ("topk -inf eligible", "not math.isnan(row[j]) and row[j] != -math.inf]", "not math.isnan(row[j])]"),
+    ("topk kept in rank order", "kept = sorted(ranked[:top_k])", "kept = ranked[:top_k]"),
+    ("topk padded with zeros", "out = np.full((R, H, sel_width), -1, dtype=np.int32)",
+     "out = np.full((R, H, sel_width), 0, dtype=np.int32)"),
+    ("topk smallest scores", "ranked = sorted(eligible, key=lambda j: (-row[j], j))",
+     "ranked = sorted(eligible, key=lambda j: (row[j], j))"),
     ("bf16 ties away from even", "(((c >> 16) & 1) == 0) & (((best >> 16) & 1) == 1)",
      "(((c >> 16) & 1) == 1) & (((best >> 16) & 1) == 0)"),
 ]

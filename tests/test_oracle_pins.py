@@ -660,3 +660,66 @@ def test_prologue_out_of_range_position_flags_bounds():
     r = O.run_step(wl)
     assert r["status"] & O.ST_BOUNDS
     np.testing.assert_array_equal(r["q_out"].view(np.uint16), wl["q"].view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# selection producer (TopK over per-key scores)
+# ---------------------------------------------------------------------------
+
+def test_topk_worked_examples():
+    g = load("topk_worked.json")
+    for c in g["cases"]:
+        got = O.select_topk(np.array(c["scores"], dtype=np.float32), np.array(c["bound"]), c["top_k"],
+                            c["sel_width"])
+        np.testing.assert_array_equal(got, np.array(c["expected"]), err_msg=c["name"])
+
+
+def _topk_by_dominance(row, last, k):
+    """The unique set S of min(k, E) eligible keys such that every kept key
+    beats every eligible key left out (higher score, or an equal score and a
+    lower index), found by enumerating all subsets of a tiny row."""
+    import itertools
+    elig = [j for j in range(min(last, len(row) - 1) + 1) if not math.isnan(row[j]) and row[j] != -math.inf]
+    n = min(k, len(elig))
+    found = []
+    for S in itertools.combinations(elig, n):
+        rest = [j for j in elig if j not in S]
+        if all(row[i] > row[j] or (row[i] == row[j] and i < j) for i in S for j in rest):
+            found.append(list(S))
+    assert len(found) == 1
+    return found[0]
+
+
+def test_topk_brute_force_dominance():
+    rng = np.random.default_rng(7)
+    for trial in range(300):
+        n = int(rng.integers(1, 9))
+        # few distinct values, so that ties are common; some masked keys
+        row = rng.integers(-2, 3, size=n).astype(np.float32)
+        row[rng.random(n) < 0.15] = -np.inf
+        row[rng.random(n) < 0.1] = np.nan
+        last = int(rng.integers(-1, n + 2))
+        k = int(rng.integers(1, n + 2))
+        W = k + int(rng.integers(0, 3))
+        got = O.select_topk(row.reshape(1, 1, n), np.array([last]), k, W)[0, 0]
+        want = _topk_by_dominance([float(v) for v in row], last, k)
+        np.testing.assert_array_equal(got[:len(want)], want)
+        assert (got[len(want):] == -1).all()
+
+
+def test_topk_matches_stable_lexsort():
+    """numpy's lexsort (score descending, then index) gives the same kept set
+    on a larger row; the kept indices come out increasing."""
+    rng = np.random.default_rng(8)
+    R, H, N = 3, 2, 500
+    scores = np.round(rng.standard_normal((R, H, N)), 1).astype(np.float32)   # many ties
+    bound = np.array([499, 250, 37])
+    got = O.select_topk(scores, bound, 60, 64)
+    for r in range(R):
+        for h in range(H):
+            idx = np.arange(bound[r] + 1)
+            order = np.lexsort((idx, -scores[r, h, :bound[r] + 1].astype(np.float64)))
+            want = np.sort(order[:60])
+            np.testing.assert_array_equal(got[r, h, :len(want)], want)
+            assert (got[r, h, len(want):] == -1).all()
+            assert (np.diff(got[r, h, :len(want)]) > 0).all()
