@@ -360,6 +360,26 @@ class Graphs:
         for g in self.graphs:
             g.replay()
 
+    def upload(self, stream) -> bool:
+        """Upload the instantiated graphs to the device ahead of their first
+        replay, so that the timed replay does not pay for it."""
+        try:
+            from cuda.bindings import driver as cu
+            for g in self.graphs:
+                err, = cu.cuGraphUpload(cu.CUgraphExec(int(g.raw_cuda_graph_exec())),
+                                        cu.CUstream(int(stream.cuda_stream)))
+                if err != cu.CUresult.CUDA_SUCCESS:
+                    return False
+            return True
+        except Exception:
+            return False
+
+
+# Cycles the GPU spins (torch.cuda._sleep) ahead of the first timing event,
+# so that the host has submitted the graphs before the event is recorded:
+# the events then bracket device execution only (about 100 us at 1.9 GHz).
+LEAD_CYCLES = 200_000
+
 
 def timed(dev, stream, graphs: Graphs, sampler=None):
     """Device time (ms) of one replay of `graphs`, bracketed by a barrier and a
@@ -371,6 +391,7 @@ def timed(dev, stream, graphs: Graphs, sampler=None):
     if sampler is not None:
         sampler.__enter__()
     with torch.cuda.stream(stream):
+        torch.cuda._sleep(LEAD_CYCLES)
         ev0.record(stream)
         graphs.replay()
         ev1.record(stream)
@@ -427,6 +448,7 @@ def measure(name, args, dev, rank, world, headline: bool):
     g_steps = Graphs(stream, insts, K, start=Wm)
     with torch.cuda.stream(stream):
         g_warm.replay()
+    uploaded = g_steps.upload(stream)
     torch.cuda.synchronize(dev)
     clk = ClockSampler(dev.index)
     ms = timed(dev, stream, g_steps, clk)
@@ -444,6 +466,7 @@ def measure(name, args, dev, rank, world, headline: bool):
         ga = Graphs(stream, attn, ka, start=Wm)
         with torch.cuda.stream(stream):
             ga_warm.replay()
+        ga.upload(stream)
         torch.cuda.synchronize(dev)
         attn_ms = timed(dev, stream, ga) / ka
         del ga, ga_warm
@@ -479,13 +502,84 @@ def measure(name, args, dev, rank, world, headline: bool):
            "run": {"instances": R,
                    "l2": f"rotating {R} device instances, attended+q/k/v bytes per cycle "
                          f"{R * per_inst / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB",
-                   "timing": f"{K} steps captured in {math.ceil(K / GRAPH_CHUNK)} CUDA graph(s), "
-                             "CUDA events on the launching stream",
+                   "timing": f"{K} steps captured in {math.ceil(K / GRAPH_CHUNK)} CUDA graph(s)"
+                             f"{' uploaded before the timed replay' if uploaded else ''}; CUDA events on the "
+                             "launching stream, recorded after a GPU-side lead so that they bracket device "
+                             "execution",
                    "step_entry": ("spa_prepare_qkv_append + spa_attention" if getattr(wl, "prologue", None) else
                                   {"step": "spa_prepare_append_attention",
                                    "prepare_append": "spa_prepare_append_kv + spa_attention",
                                    "staged": "spa_prepare_metadata + spa_append_kv + spa_attention"}[args.mode])}}
     del insts
+    torch.cuda.empty_cache()
+    return res
+
+
+def select_bytes(sw) -> int:
+    """Algorithmic bytes of one selection-producer launch: every candidate
+    score read once (keys 0..bound of each row) and every output slot written."""
+    cand = sum(min(int(b), sw.n_keys - 1) + 1 for b in sw.bound if b >= 0)
+    return 4 * sw.H * cand + 4 * sw.R * sw.H * sw.sel_width
+
+
+def measure_select(name, args, dev, rank, world):
+    """Time K launches of the selection producer (spa_select_topk) over
+    rotating device copies of its scores."""
+    import torch
+
+    from selected_token_sparse_b200 import spa, workloads as W
+    sw = getattr(W, name)() if rank == 0 else getattr(W, name)(seed=1000 * rank + 7)
+    amount = select_bytes(sw)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = args.instances or max(2, min(64, math.ceil(2 * l2 / amount)))
+    K = min(args.steps, GRAPH_CHUNK)
+    Wm = min(args.warmup, 50)
+    sc0 = torch.from_numpy(sw.scores).to(dev)
+    bound = torch.from_numpy(sw.bound).to(dev)
+    scores = [sc0.clone() for _ in range(R)]
+    del sc0
+    outs = [torch.empty(sw.R, sw.H, sw.sel_width, dtype=torch.int32, device=dev) for _ in range(R)]
+    fns = [lambda i=i: spa.select_topk(scores[i], bound, sw.top_k, sw.sel_width, out=outs[i]) for i in range(R)]
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for f in fns:
+            f()
+    torch.cuda.synchronize(dev)
+    g_warm = Graphs(stream, fns, Wm)
+    g = Graphs(stream, fns, K, start=Wm)
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+    g.upload(stream)
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(dev.index)
+    ms = timed(dev, stream, g, clk) / K
+    hbm, _, _, peak_src = load_peaks()
+    achieved = amount / (ms * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import spa_oracle as O
+        n, t0, c0 = 0, time.perf_counter(), time.process_time()
+        while n < 1 or time.perf_counter() - t0 < 3.0:
+            O.select_topk(sw.scores, sw.bound, sw.top_k, sw.sel_width)
+            n += 1
+        wall = time.perf_counter() - t0
+        cpu = {"value": amount / (wall / n) / 1e9, "unit": "GB/s",
+               "cores": max(1, int(round((time.process_time() - c0) / wall))), "host_cores": host_cores(),
+               "kind": "oracle", "sample": f"{n} whole call(s) of the same workload, numpy/Python oracle"}
+    res = {"workload": name, "dtype": "f32", "value": world * amount / (ms * 1e-3) / 1e9, "unit": "GB/s",
+           "ms_per_step": ms, "steps": K, "warmup": Wm, "algorithmic_per_step": amount,
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                        "peak_source": f"{peak_src} HBM copy", "kernel": "spa_select_topk (select_topk_kernel, 1 launch)",
+                        "us_per_launch": ms * 1e3, "algorithmic_per_launch": amount,
+                        "traffic": recorded_traffic("select_topk", name)},
+           "cpu_baseline": cpu, "gpu_launches": K, "launches_per_step": 1, "num_splits": 1,
+           "clocks": clk.summary(), "status": 0,
+           "config": {"workload": name, "R": sw.R, "H_kv": sw.H, "n_keys": sw.n_keys, "top_k": sw.top_k,
+                      "sel_width": sw.sel_width, "scores": "f32 N(0,1)",
+                      "parallelism": f"dp{world}" if world > 1 else "single", "l2": L2_NOTE},
+           "run": {"instances": R, "timing": f"{K} launches captured in one CUDA graph; CUDA events"}}
+    del g, g_warm, scores, outs
     torch.cuda.empty_cache()
     return res
 
@@ -568,6 +662,8 @@ def run_ours(args):
     if not args.only:
         names += [n for n in W.WORKLOADS + W.PROLOGUE_WORKLOADS if n != args.workload]
     results = [measure(n, args, dev, rank, world, headline=(i == 0)) for i, n in enumerate(names)]
+    if not args.only:
+        results += [measure_select(n, args, dev, rank, world) for n in W.SELECTION_WORKLOADS]
     h = results[0]
     line = {
         "metric": METRIC, "value": h["value"], "unit": h["unit"], "n_gpus": world, "steps": h["steps"],

@@ -67,6 +67,37 @@ typedef enum {
 #define SPA_ST_TIMEOUT 0x20   /* a bounded on-chip wait expired; the affected outputs are unspecified */
 
 /*
+ * spa_select_topk -- the selection producer ahead of step 3: for every row r
+ * (a request, or a query token) and kv head h, the top_k keys of the per-key
+ * scores, written as the -1 padded selected-index row that spa_attention's
+ * selected mode reads (selected_idx with sel_target = 0).
+ * Source: onnxruntime PR #33472, Key Changes (PackedSparseAttentionIndexer:
+ * QSA scoring and hierarchical / compact TopK selection) and its experiments
+ * note (the compact TopK keeps stable keys, causal tails, capacity stride /
+ * padding and overflow handling).  The pages do not define the score, so it
+ * is an input.
+ *
+ *   scores [R, H, n_keys]  fp32 score of key j of row r under kv head h.
+ *   bound [R]              last eligible key of row r (the causal tail):
+ *                          seqlen_k of spa_prepare_metadata for per-request
+ *                          rows, token_pos for per-token rows; keys beyond it,
+ *                          or beyond n_keys - 1, are never selected; a
+ *                          negative bound gives an empty row.
+ *   top_k, sel_width       [host] keys kept per row, 0 <= top_k <= sel_width;
+ *                          sel_width is the row capacity of the output.
+ *   selected_idx [R, H, sel_width] (output) the kept keys in increasing order,
+ *                          then -1 up to sel_width.
+ * A key is eligible when its score is neither NaN nor -inf (-inf masks a
+ * key); -0 and +0 are equal.  The kept keys are the min(top_k, eligible)
+ * largest scores; among equal scores the lower key index is kept first, so
+ * the result is unique and bit-exact.  Errors: SPA_ERR_INVALID_ARG for
+ * negative sizes, H <= 0, sel_width <= 0, top_k > sel_width or a NULL
+ * required pointer.  R = 0 is valid.  One kernel launch.
+ */
+int spa_select_topk(const float* scores, int32_t R, int32_t H, int32_t n_keys, const int32_t* bound,
+                    int32_t top_k, int32_t sel_width, int32_t* selected_idx, spa_stream_t stream);
+
+/*
  * spa_prepare_metadata -- step 1, exact per-request and per-token metadata on
  * the device, replacing a device-to-host readback per layer.
  * Source: "[WebGPU] Add PagedAttention metadata and GPT-OSS support",

@@ -66,6 +66,23 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 // cp.async: 16-byte global -> shared copy, zero-filled when src_bytes == 0.
+// Residual of a 16-bit pair: given x, y and their rounding to T packed in `hi`
+// (x in the low half), the pair (x - T(x), y - T(y)) rounded to T.  A product
+// P V with 16-bit P is run as P_hi V + P_lo V where P's own rounding would
+// show in the output -- bf16 P (8 bits: a row dominated by one key carries
+// that key's 2^-9 rounding), and fp16 P against integer-valued INT8 V (values
+// up to 127 before the scale) -- so that P keeps about twice its bits.
+template <typename T> __device__ __forceinline__ uint32_t residual_pair(float x, float y, uint32_t hi);
+template <> __device__ __forceinline__ uint32_t residual_pair<__nv_bfloat16>(float x, float y, uint32_t hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(x - __uint_as_float(hi << 16), y - __uint_as_float(hi & 0xffff0000u));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+template <> __device__ __forceinline__ uint32_t residual_pair<__half>(float x, float y, uint32_t hi) {
+  const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+  __half2 v = __floats2half2_rn(x - h.x, y - h.y);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ void cp_async_16(void* smem, const void* gmem, bool valid) {
   uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
   int src_bytes = valid ? 16 : 0;

@@ -552,6 +552,15 @@ decode_mma_kernel(const AttnParams p) {
       a[1] = pack2<MT>(s[2 * kk][2], s[2 * kk][3]);
       a[2] = pack2<MT>(s[2 * kk + 1][0], s[2 * kk + 1][1]);
       a[3] = pack2<MT>(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      // bf16 P, and fp16 P against INT8 V, run as P_hi V + P_lo V (see residual_pair)
+      constexpr bool kPLo = MmaName<MT>::bf16 || C::kInt8;
+      uint32_t al[4];
+      if constexpr (kPLo) {
+        al[0] = residual_pair<MT>(s[2 * kk][0], s[2 * kk][1], a[0]);
+        al[1] = residual_pair<MT>(s[2 * kk][2], s[2 * kk][3], a[1]);
+        al[2] = residual_pair<MT>(s[2 * kk + 1][0], s[2 * kk + 1][1], a[2]);
+        al[3] = residual_pair<MT>(s[2 * kk + 1][2], s[2 * kk + 1][3], a[3]);
+      }
 #pragma unroll
       for (int n = 0; n < D / 8; n += 2) {
         uint32_t b[4];
@@ -560,6 +569,10 @@ decode_mma_kernel(const AttnParams p) {
         ldsm_x4_t(b, vs + swz(vrow, n + (mi >> 1), CPR));
         mma16816<MT>(o[n], a, b);
         mma16816<MT>(o[n + 1], a, b + 2);
+        if constexpr (kPLo) {
+          mma16816<MT>(o[n], al, b);
+          mma16816<MT>(o[n + 1], al, b + 2);
+        }
       }
     }
     __syncthreads();

@@ -55,8 +55,9 @@ constexpr int kTcThreads = kTcCons + kTcProd + 32;
 constexpr int kTcBarProd = 2;                   // named barrier of the producers
 constexpr int kTcCandTiles = 8;                 // tiles whose candidates are resolved at once
 constexpr int kTcCand = kTcCandTiles * kTcKT;
-// tensor memory columns: S[2] | O | P[2] (packed 16-bit pairs) | Q_hi | Q_lo
-constexpr uint32_t kTcColS = 0, kTcColO = 128, kTcColP = 256, kTcColQ = 320;
+// tensor memory columns: S[2] | O | P[2] (packed 16-bit pairs) | Q_hi | Q_lo |
+// P_lo[2] (P residuals for bf16 P and INT8 caches; see residual_pair)
+constexpr uint32_t kTcColS = 0, kTcColO = 128, kTcColP = 256, kTcColQ = 320, kTcColPlo = 448;
 constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcWaitLimit = 1u << 20;
 constexpr int kTcStageTok = 64;   // fused INT8 step: tokens of a request whose new rows are staged
@@ -67,6 +68,8 @@ template <typename ActT, typename CacheT, int D>
 struct TcCfg {
   static constexpr bool kInt8 = sizeof(CacheT) == 1;
   using MT = typename std::conditional<kInt8, __half, ActT>::type;
+  // P as P_hi + P_lo (residual_pair): bf16 P, or fp16 P against INT8 V
+  static constexpr bool kPLo = kInt8 || std::is_same<MT, __nv_bfloat16>::value;
   static constexpr int NCH = D / 64;
   static constexpr int KCHUNK = kTcKT * 128;          // one 64-column chunk of a 64-row tile
   static constexpr int KTILE = NCH * KCHUNK;          // 64 rows x D, 16-bit, swizzled
@@ -624,6 +627,7 @@ decode_tc_kernel(const AttnParams p) {
       for (int kk = 0; kk < KT / 16; ++kk) {
         const uint64_t bd = smem_desc_sw128(smem_u32(vt + kk * 2048), C::KCHUNK, 1024);
         mma_ts(tmem + kTcColO, tmem + kTcColP + sb * (KT / 2) + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        if constexpr (C::kPLo) mma_ts(tmem + kTcColO, tmem + kTcColPlo + sb * (KT / 2) + kk * 8, bd, IDESC_O, 1u);
       }
       tc_commit(bar_o + sb);
       tc_commit(bar_empty + st);   // the stage is free once S and PV of this tile complete
@@ -739,7 +743,8 @@ decode_tc_kernel(const AttnParams p) {
       m_used = m_new;
       const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
       float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[KT / 2];
+      constexpr bool kLo = C::kPLo;
+      uint32_t pk[KT / 2], pl[kLo ? KT / 2 : 1];
 #pragma unroll
       for (int e = 0; e < KT; e += 2) {
         const float pa = ex2a(fmaf(__uint_as_float(v[e]), sl2, nm));
@@ -747,6 +752,7 @@ decode_tc_kernel(const AttnParams p) {
         ls0 += pa;
         ls1 += pb;
         pk[e / 2] = pk_pair<MT>(pa, pb);
+        if constexpr (kLo) pl[e / 2] = residual_pair<MT>(pa, pb, pk[e / 2]);
       }
       l_sum = l_sum * alpha + (ls0 + ls1);
       // P buffer sb was last read by the PV of tile j - 2
@@ -756,6 +762,7 @@ decode_tc_kernel(const AttnParams p) {
       }
       // packed P of the 64 keys -> the buffer's 32 columns
       tmem_st32(tmem + kTcColP + lane_off + sb * (KT / 2), pk);
+      if constexpr (kLo) tmem_st32(tmem + kTcColPlo + lane_off + sb * (KT / 2), pl);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

@@ -95,6 +95,10 @@ __device__ __forceinline__ uint32_t pack_pair<__nv_bfloat16>(float lo, float hi)
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// bf16 P runs as P_hi V + P_lo V (residual_pair); fp16 P keeps 11 bits
+template <typename T>
+constexpr bool kPfLo = std::is_same<T, __nv_bfloat16>::value;
+
 struct PfGeom {
   int b, h, h_kv, t_begin, q_len, past, L, k_lo, k_hi, ntiles;
   int q0[2], rows[2];   // per q tile: first row within the request, rows present (0 = absent)
@@ -367,7 +371,13 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 #pragma unroll
             for (int kk = 0; kk < kPfBN / 16; ++kk) {
               const uint64_t bd = smem_desc_sw128(smem_u32(sV + st * C::TILE + kk * 2048), C::CHUNK, 1024);
-              mma_ts(tO, tP + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+              if constexpr (kPfLo<T>) {   // P_hi and P_lo of 64-key halves (see the softmax)
+                const uint32_t col = (kk / 4) * 64 + (kk % 4) * 8;
+                mma_ts(tO, tP + col, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_ts(tO, tP + col + 32, bd, IDESC_O, 1u);
+              } else {
+                mma_ts(tO, tP + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+              }
             }
             tc_commit(bar_o + t);
             ++o_iss[t];
@@ -518,10 +528,12 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         // pass 2: P = 2^(s*scale - m) for 64 keys at a time, packed in pairs into
         // the TMEM columns that held those keys' scores (already read)
         // hidden keys (masked tiles) give p = 0
+        // bf16: P_hi and P_lo (residual_pair) of keys hh*64 .. hh*64+63 go
+        // to the 64 columns that held those keys' scores
         float ls = 0.f;
 #pragma unroll
         for (int hh = 0; hh < kPfBN / 64; ++hh) {
-          uint32_t pk[32];
+          uint32_t pk[32], pl[kPfLo<T> ? 32 : 1];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t v[32];
@@ -535,9 +547,15 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
               const float pb = ((m >> (e + 1)) & 1u) ? ex2(fmaf(u2f(v[e + 1]), sl2, nm)) : 0.f;
               ls += pa + pb;
               pk[half * 16 + e / 2] = pack_pair<T>(pa, pb);
+              if constexpr (kPfLo<T>) pl[half * 16 + e / 2] = residual_pair<T>(pa, pb, pk[half * 16 + e / 2]);
             }
           }
-          tmem_st32(tS + hh * 32, pk);
+          if constexpr (kPfLo<T>) {
+            tmem_st32(tS + hh * 64, pk);
+            tmem_st32(tS + hh * 64 + 32, pl);
+          } else {
+            tmem_st32(tS + hh * 32, pk);
+          }
         }
         l_sum += ls;
         tmem_wait_st();

@@ -1,0 +1,231 @@
+// Selection producer: the top_k keys of per-key scores, as the -1 padded,
+// increasing selected-index rows that the attention's selected mode reads.
+//
+// Source: onnxruntime PR #33472, Key Changes (PackedSparseAttentionIndexer:
+// QSA scoring and hierarchical / compact TopK selection ahead of
+// DynamicSparseAttention) and its experiments note (the compact TopK keeps
+// stable keys, causal tails, capacity stride / padding and overflow
+// handling).  The pages do not define the score; it is an input.
+//
+// One CTA of 1024 threads per (row, kv head):
+//   1. the row's candidate scores (keys 0..bound) are read once, coalesced,
+//      and kept in shared memory as order-preserving 32-bit keys (NaN and
+//      -inf, which are never selected, become 0; -0 becomes +0);
+//   2. when more than top_k keys are eligible, a radix select over four
+//      8-bit digits (a 256-bin shared histogram per digit, warp-aggregated
+//      increments) finds the exact k-th largest key T and how many keys equal
+//      to T are still to be taken -- the first ones by index (stable);
+//   3. a compaction over contiguous per-warp segments (ballot / popc counts,
+//      one scan over the 32 warps) writes every kept index at its rank among
+//      the kept ones, so the row comes out in increasing index order;
+//   4. the rest of the row, up to its capacity sel_width, is -1.
+// Rows longer than the shared-memory capacity read their scores again from
+// global memory (L2) in every pass instead.
+#include "spa_attn.cuh"
+
+namespace spa {
+
+int check_launch_public();
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelStageKeys = 48 * 1024;   // keys kept in shared memory (192 KB)
+
+// Order-preserving key of a score: larger score, larger key; 0 = not eligible.
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;                       // -0 ties with +0
+  if ((u & 0x7fffffffu) > 0x7f800000u) return 0u;     // NaN
+  if (u == 0xff800000u) return 0u;                    // -inf masks the key
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 0x00800000 for eligible keys
+}
+
+struct SelShared {
+  uint32_t hist[256];
+  int warp_gt[kSelWarps];
+  int warp_eq[kSelWarps];
+  int red[kSelWarps];
+  int digit, above, in_bin;
+};
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const int32_t* __restrict__ bound,
+                   int top_k, int sel_width, int32_t* __restrict__ out, int staged) {
+  extern __shared__ uint32_t sel_keys[];
+  __shared__ SelShared sh;
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long row = blockIdx.x;
+  const int r = (int)(row / H);
+  const float* src = scores + row * (long long)n_keys;
+  int32_t* dst = out + row * (long long)sel_width;
+  const int last = min(bound[r], n_keys - 1);
+  const int n = last + 1 > 0 ? last + 1 : 0;   // candidate keys 0 .. last
+
+  auto key_at = [&](int j) -> uint32_t { return staged ? sel_keys[j] : score_key(__ldg(src + j)); };
+
+  // 1. stage the keys and count the eligible ones
+  int elig = 0;
+  for (int j0 = 0; j0 < n; j0 += 8 * kSelThreads) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * kSelThreads + tid;
+      v[u] = j < n ? __ldg(src + j) : __int_as_float(0xff800000);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * kSelThreads + tid;
+      const uint32_t k = score_key(v[u]);
+      elig += k != 0u;
+      if (staged && j < n) sel_keys[j] = k;
+    }
+  }
+  elig = __reduce_add_sync(0xffffffffu, elig);
+  if (lane == 0) sh.red[warp] = elig;
+  __syncthreads();
+  if (warp == 0) {
+    const int e = __reduce_add_sync(0xffffffffu, sh.red[lane]);
+    if (lane == 0) sh.red[0] = e;
+  }
+  __syncthreads();
+  const int E = sh.red[0];
+
+  // 2. the threshold: keep keys > T, plus the first need_eq keys equal to T
+  uint32_t T = 0u;
+  int need_eq = 0;
+  if (E > top_k && top_k > 0) {
+    uint32_t prefix = 0u, pmask = 0u;
+    int k_rem = top_k;
+    bool exact = true;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0u;
+      __syncthreads();
+      for (int j0 = 0; j0 < n; j0 += kSelThreads) {
+        const int j = j0 + tid;
+        const uint32_t k = j < n ? key_at(j) : 0u;
+        const bool m = k != 0u && (k & pmask) == prefix;
+        const unsigned active = __ballot_sync(0xffffffffu, m);
+        if (m) {
+          const uint32_t d = (k >> shift) & 255u;
+          const unsigned peers = __match_any_sync(active, d);
+          if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[d], (uint32_t)__popc(peers));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l holds bins 255 - 8l ... 248 - 8l (largest digits first)
+        uint32_t c[8];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          c[i] = sh.hist[255 - lane * 8 - i];
+          sum += (int)c[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int excl = incl - sum;
+        if (excl < k_rem && k_rem <= incl) {
+          int cum = excl;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (cum + (int)c[i] >= k_rem) {
+              sh.digit = 255 - lane * 8 - i;
+              sh.above = cum;
+              sh.in_bin = (int)c[i];
+              break;
+            }
+            cum += (int)c[i];
+          }
+        }
+      }
+      __syncthreads();
+      const int d = sh.digit;
+      k_rem -= sh.above;
+      prefix |= (uint32_t)d << shift;
+      pmask |= 255u << shift;
+      if (sh.in_bin == k_rem) {   // every key of this bin is kept: no tie to split
+        T = prefix - 1u;          // keys with this prefix are >= prefix
+        need_eq = 0;
+        exact = false;
+        break;
+      }
+      __syncthreads();            // sh.* is rewritten by the next pass
+    }
+    if (exact) {
+      T = prefix;
+      need_eq = k_rem;
+    }
+  }
+  const int kept = E < top_k ? E : top_k;
+
+  // 3. compaction in index order over contiguous per-warp segments
+  const int seg = ((n + kSelWarps - 1) / kSelWarps + 31) & ~31;
+  const int beg = warp * seg, end = min(beg + seg, n);
+  int gt_w = 0, eq_w = 0;
+  if (kept > 0) {
+    for (int j0 = beg; j0 < end; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t k = j < end ? key_at(j) : 0u;
+      gt_w += __popc(__ballot_sync(0xffffffffu, k > T));
+      eq_w += __popc(__ballot_sync(0xffffffffu, need_eq > 0 && k == T));
+    }
+  }
+  if (lane == 0) {
+    sh.warp_gt[warp] = gt_w;
+    sh.warp_eq[warp] = eq_w;
+  }
+  __syncthreads();
+  if (kept > 0) {
+    int gt_before = 0, eq_before = 0;
+    for (int w = 0; w < warp; ++w) {
+      gt_before += sh.warp_gt[w];
+      eq_before += sh.warp_eq[w];
+    }
+    int pos = gt_before + min(eq_before, need_eq);
+    int eq_seen = eq_before;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j0 = beg; j0 < end; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t k = j < end ? key_at(j) : 0u;
+      const bool is_eq = need_eq > 0 && k == T;
+      const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = k > T || (is_eq && eq_seen + __popc(eqm & lt) < need_eq);
+      const unsigned tm = __ballot_sync(0xffffffffu, take);
+      if (take) dst[pos + __popc(tm & lt)] = j;
+      pos += __popc(tm);
+      eq_seen += __popc(eqm);
+    }
+  }
+  // 4. padding up to the row's capacity
+  for (int i = kept + tid; i < sel_width; i += kSelThreads) dst[i] = -1;
+}
+
+}  // namespace spa
+
+using namespace spa;
+
+extern "C" int spa_select_topk(const float* scores, int32_t R, int32_t H, int32_t n_keys, const int32_t* bound,
+                               int32_t top_k, int32_t sel_width, int32_t* selected_idx, spa_stream_t stream) {
+  if (R < 0 || H <= 0 || n_keys < 0 || top_k < 0 || sel_width <= 0 || top_k > sel_width)
+    return SPA_ERR_INVALID_ARG;
+  if ((long long)R * H > 0x7fffffffLL) return SPA_ERR_INVALID_ARG;
+  if (R == 0) return SPA_OK;
+  if (!selected_idx || !bound || (n_keys > 0 && !scores)) return SPA_ERR_INVALID_ARG;
+  const int staged = n_keys <= kSelStageKeys ? 1 : 0;
+  const size_t smem = staged ? (size_t)(n_keys > 0 ? n_keys : 1) * sizeof(uint32_t) : 0;
+  if (staged && smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSelStageKeys * (int)sizeof(uint32_t)) != cudaSuccess)
+      return check_launch_public();
+  }
+  const int rc = launch_pdl(select_topk_kernel, dim3((unsigned)(R * H)), dim3(kSelThreads), smem,
+                            (cudaStream_t)stream, scores, H, n_keys, bound, top_k, sel_width, selected_idx, staged);
+  if (rc != SPA_OK) return rc;
+  return check_launch_public();
+}

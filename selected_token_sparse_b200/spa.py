@@ -24,7 +24,7 @@ ST_BAD_CU, ST_CAPACITY, ST_BAD_BLOCK, ST_BOUNDS, ST_BAD_IDX = 0x1, 0x2, 0x4, 0x8
 EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_prepare_append_kv", "spa_prepare_qkv_append",
             "spa_attention", "spa_attention_workspace_size", "spa_attention_plan",
             "spa_prepare_append_attention", "spa_prepare_append_attention_launches",
-            "spa_attention_noalloc", "spa_error_string")
+            "spa_attention_noalloc", "spa_select_topk", "spa_error_string")
 
 _DT = {torch.float32: SPA_F32, torch.float16: SPA_F16, torch.bfloat16: SPA_BF16, torch.int8: SPA_I8}
 
@@ -107,6 +107,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spa_prepare_append_attention_launches.argtypes = [ctypes.POINTER(AttentionArgs)]
     lib.spa_prepare_qkv_append.restype = ctypes.c_int
     lib.spa_prepare_qkv_append.argtypes = [ctypes.POINTER(QkvArgs), _vp]
+    lib.spa_select_topk.restype = ctypes.c_int
+    lib.spa_select_topk.argtypes = [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _vp]
     lib.spa_error_string.restype = ctypes.c_char_p
     lib.spa_error_string.argtypes = [ctypes.c_int]
     return lib
@@ -370,3 +372,19 @@ def attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                              _stream(q.device))
     _check(rc, "spa_attention")
     return out, lse
+
+
+def select_topk(scores: torch.Tensor, bound: torch.Tensor, top_k: int, sel_width: int,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Selection producer: the top_k keys of fp32 scores [R, H, n_keys] per row,
+    keys 0..bound[r] eligible; returns selected_idx [R, H, sel_width] (increasing,
+    -1 padded), the layout spa_attention's selected mode reads."""
+    R, H, N = scores.shape
+    if scores.dtype != torch.float32 or bound.dtype != torch.int32:
+        raise ValueError("select_topk takes fp32 scores and int32 bounds")
+    if out is None:
+        out = torch.empty(R, H, sel_width, dtype=torch.int32, device=scores.device)
+    rc = lib().spa_select_topk(_ptr(scores), R, H, N, _ptr(bound), int(top_k), int(sel_width), _ptr(out),
+                               _stream(scores.device))
+    _check(rc, "spa_select_topk")
+    return out

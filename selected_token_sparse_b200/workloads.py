@@ -361,6 +361,33 @@ def qkv_prologue_selected_decode_bf16(seed: int = 6, small: bool = False) -> Wor
                          prologue=dict(packed=True, qk_norm=True, rotary_dim=128), seed=seed)
 
 
+# Inputs of the selection producer (TopK over per-key scores).
+@dataclasses.dataclass
+class SelectionWorkload:
+    name: str
+    R: int
+    H: int
+    n_keys: int
+    top_k: int
+    sel_width: int
+    scores: np.ndarray            # [R, H, n_keys] fp32
+    bound: np.ndarray             # [R] int32: last eligible key of each row
+
+
+SELECTION_WORKLOADS = ("topk_selection_f32",)
+
+
+def topk_selection_f32(seed: int = 7, small: bool = False) -> SelectionWorkload:
+    """Scores for the selected-token decode shape: 16 requests x 4 kv heads x
+    32768 keys, N(0, 1) fp32, every key of a request eligible (bound = 32767);
+    1946 kept in rows of capacity 2048 (the decode workload's 5% padding)."""
+    R, H, N, W = (2, 4, 1000, 200) if small else (16, 4, 32768, 2048)
+    rng = np.random.default_rng(seed)
+    scores = rng.standard_normal((R, H, N)).astype(np.float32)
+    return SelectionWorkload(name="topk_selection_f32", R=R, H=H, n_keys=N, top_k=W - W // 20, sel_width=W,
+                             scores=scores, bound=np.full(R, N - 1, dtype=np.int32))
+
+
 def by_name(name: str, small: bool = False, seed: Optional[int] = None) -> Workload:
     fn = {n: globals()[n] for n in WORKLOADS + PROLOGUE_WORKLOADS}[name]
     if seed is None:

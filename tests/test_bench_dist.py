@@ -102,3 +102,10 @@ def test_reference_arm_prints_our_config(capsys):
     assert line["config"] == bench.workload_config(W.by_name("tiny_decode_f32"), 1)
     assert line["cpu_baseline"]["host_cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_select_bytes():
+    sw = W.topk_selection_f32(small=True)
+    sw.bound[:] = [9, -1]
+    # row 0: keys 0..9 of H heads read; every output slot written
+    assert bench.select_bytes(sw) == 4 * sw.H * 10 + 4 * sw.R * sw.H * sw.sel_width
