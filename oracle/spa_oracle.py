@@ -36,6 +36,9 @@ the pages describe the pipeline:
      (FP32 partial softmax state merged in a finalize stage).  The combine is
      exact in real arithmetic, so the oracle computes the single-pass
      definition: softmax over the whole attended set plus the sink.
+  5b. sequence-sharded split-KV -- the same finalize merge over shards of a
+     sequence split across devices: attention() over one shard's key range
+     (kv_range) without the sink, then merge_partials() with the sink once.
 
 Readings where the pages are silent (all listed in the design notes):
   * KV cache layout [num_blocks, block_size, H_kv, D]; slot = block*bs + offset.
@@ -333,8 +336,12 @@ def append_kv(k_new: np.ndarray, v_new: np.ndarray, act: str, k_cache: np.ndarra
 def attended_keys(t: int, h_kv: int, meta: Dict[str, np.ndarray], block_table: np.ndarray,
                   block_size: int, num_blocks: int, window: int,
                   selected_idx: Optional[np.ndarray], sel_per_request: int, sel_target: int,
-                  aux_seqlens: Optional[np.ndarray]):
+                  aux_seqlens: Optional[np.ndarray], kv_range: Optional[np.ndarray] = None):
     """The attended set of token t under kv head h_kv.
+
+    With ``kv_range`` ([B, 2]) only the main-cache positions lo <= j < hi of
+    the token's request are kept (one shard of a sequence split across
+    devices); they are dropped before any block-table lookup.
 
     Returns (blocks, offsets, aux_pos, status): the physical main-cache rows
     (block id, row within block) and the auxiliary positions of request b,
@@ -361,6 +368,8 @@ def attended_keys(t: int, h_kv: int, meta: Dict[str, np.ndarray], block_table: n
         # causal local window (or dense causal when the window is off)
         lo = max(0, p - window + 1) if window > 0 else 0
         main_pos = np.arange(lo, p + 1, dtype=np.int64)
+    if kv_range is not None:
+        main_pos = main_pos[(main_pos >= int(kv_range[b][0])) & (main_pos < int(kv_range[b][1]))]
     if sel is not None and sel_target == 1:
         aux_pos = sel[(sel >= 0) & (sel < int(aux_seqlens[b]))]
     else:
@@ -385,7 +394,8 @@ def attention(q: np.ndarray, act: str, k_cache: np.ndarray, v_cache: np.ndarray,
               aux_seqlens: Optional[np.ndarray] = None, sinks: Optional[np.ndarray] = None,
               scale: float = 0.0, k_scale: Optional[np.ndarray] = None,
               v_scale: Optional[np.ndarray] = None,
-              tokens: Optional[Iterable[int]] = None) -> Dict[str, np.ndarray]:
+              tokens: Optional[Iterable[int]] = None,
+              kv_range: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Output o[T, H_q, D] (float64) and lse[T, H_q] of the attention step.
 
     For token t at position p in request b and q head h (kv head h // G):
@@ -409,7 +419,7 @@ def attention(q: np.ndarray, act: str, k_cache: np.ndarray, v_cache: np.ndarray,
         for h_kv in range(H_kv):
             blk, off, aux_pos, st = attended_keys(
                 t, h_kv, meta, block_table, bs, NB, window, selected_idx,
-                sel_per_request, sel_target, aux_seqlens)
+                sel_per_request, sel_target, aux_seqlens, kv_range)
             status |= st
             K = decode(k_cache[blk, off, h_kv], cache)           # [n_main, D]
             V = decode(v_cache[blk, off, h_kv], cache)
@@ -433,6 +443,42 @@ def attention(q: np.ndarray, act: str, k_cache: np.ndarray, v_cache: np.ndarray,
                 out[t, h] = (e @ V) / l
                 lse[t, h] = m + math.log(l)
     return {"out": out, "lse": lse, "status": status}
+
+
+# ---------------------------------------------------------------------------
+# 5b. sequence-sharded split-KV: merge of per-shard partial states
+# ---------------------------------------------------------------------------
+#
+# "[WebGPU] Add SparsePagedAttention", File summaries: the main and the
+# auxiliary pass each leave a partial FP32 softmax state, and a finalize stage
+# merges them and applies the sink.  A sequence split across devices is the
+# same merge over shards: shard r attends only its key range (attention()
+# with kv_range and no sink) and leaves o_r (normalised over its keys, 0 when
+# it has none) and lse_r = m_r + log(l_r) (-inf when it has none).  Then
+#   M   = max(sink, max_r lse_r)
+#   L   = exp(sink - M) + sum_r exp(lse_r - M)
+#   out = sum_r exp(lse_r - M) o_r / L,   lse = M + log(L)
+# (out = 0 and lse = -inf when M = -inf): the sink is counted once.
+
+def merge_partials(outs: np.ndarray, lses: np.ndarray, sinks: Optional[np.ndarray]):
+    """Merge R shards' partial states outs [R, T, H_q, D], lses [R, T, H_q]
+    with the per-head sinks [H_q] (or none).  Returns (out, lse) in float64."""
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    R, T, H_q, D = outs.shape
+    out = np.zeros((T, H_q, D))
+    lse = np.full((T, H_q), -math.inf)
+    for t in range(T):
+        for h in range(H_q):
+            sink = -math.inf if sinks is None else float(sinks[h])
+            M = max([sink] + [float(lses[r, t, h]) for r in range(R)])
+            if M == -math.inf:
+                continue
+            w = [math.exp(float(lses[r, t, h]) - M) for r in range(R)]
+            L = math.exp(sink - M) + sum(w)
+            out[t, h] = sum(w[r] * outs[r, t, h] for r in range(R)) / L
+            lse[t, h] = M + math.log(L)
+    return out, lse
 
 
 # ---------------------------------------------------------------------------

@@ -58,6 +58,12 @@ MUTATIONS = [
      "out = np.full((R, H, sel_width), 0, dtype=np.int32)"),
     ("topk smallest scores", "ranked = sorted(eligible, key=lambda j: (-row[j], j))",
      "ranked = sorted(eligible, key=lambda j: (row[j], j))"),
+    ("shard range inclusive of hi", "(main_pos < int(kv_range[b][1]))]", "(main_pos <= int(kv_range[b][1]))]"),
+    ("merge drops the sink", "L = math.exp(sink - M) + sum(w)", "L = sum(w)"),
+    ("merge counts the sink per shard", "L = math.exp(sink - M) + sum(w)", "L = R * math.exp(sink - M) + sum(w)"),
+    ("merge lse without log L", "lse[t, h] = M + math.log(L)", "lse[t, h] = M"),
+    ("merge ignores the sink in the max", "M = max([sink] + [float(lses[r, t, h]) for r in range(R)])",
+     "M = max([float(lses[r, t, h]) for r in range(R)])"),
     ("bf16 ties away from even", "(((c >> 16) & 1) == 0) & (((best >> 16) & 1) == 1)",
      "(((c >> 16) & 1) == 1) & (((best >> 16) & 1) == 0)"),
 ]

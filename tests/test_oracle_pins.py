@@ -723,3 +723,66 @@ def test_topk_matches_stable_lexsort():
             np.testing.assert_array_equal(got[r, h, :len(want)], want)
             assert (got[r, h, len(want):] == -1).all()
             assert (np.diff(got[r, h, :len(want)]) > 0).all()
+
+
+# ---------------------------------------------------------------------------
+# sequence-sharded split-KV: shard partials and their merge
+# ---------------------------------------------------------------------------
+
+def _ranges(lw, cuts):
+    """kv_range [B, 2] of shard `cuts` = (lo, hi) for every request."""
+    return np.array([[lo, hi] for lo, hi in cuts], dtype=np.int64)
+
+
+def test_shard_partial_vs_sdpa_without_sink():
+    """A shard's partial is plain softmax attention over the keys of its range
+    (no sink): SDPA with the causal mask restricted to the range."""
+    lw = Logical([3, 1], [40, 70], H_q=4, H_kv=2, D=64, bs=16, seed=31)
+    rng = [(10, 30), (45, 71)]
+    r = lw.run(window=0, kv_range=_ranges(lw, rng))
+    for b in range(lw.B):
+        lo, hi = rng[b]
+        cols = torch.arange(lw.L[b])
+        mask = lw.causal_mask(b) & ((cols >= lo) & (cols < hi))[None, :]
+        want = lw.sdpa(b, mask)
+        t0 = int(lw.cu[b])
+        np.testing.assert_allclose(r["out"][t0:t0 + lw.q_lens[b]], want, atol=1e-12)
+
+
+def test_merged_shards_equal_unsharded_sdpa_with_sink():
+    """Partials over a partition of the keys (one shard empty for some rows),
+    merged with the sink once, equal SDPA over all keys with the sink as an
+    extra key."""
+    lw = Logical([2, 1, 3], [50, 9, 100], H_q=6, H_kv=3, D=64, bs=16, seed=32)
+    sinks = np.random.default_rng(5).standard_normal(6)
+    cuts = [[(0, 20), (0, 4), (0, 0)], [(20, 45), (4, 10), (0, 60)], [(45, 1000), (10, 1000), (60, 1000)]]
+    parts = [lw.run(window=0, kv_range=_ranges(lw, c)) for c in cuts]
+    out, lse = O.merge_partials(np.stack([p["out"] for p in parts]), np.stack([p["lse"] for p in parts]), sinks)
+    for b in range(lw.B):
+        want = lw.sdpa(b, lw.causal_mask(b), sinks=sinks)
+        t0 = int(lw.cu[b])
+        np.testing.assert_allclose(out[t0:t0 + lw.q_lens[b]], want, atol=1e-12)
+    whole = lw.run(window=0, sinks=sinks)
+    np.testing.assert_allclose(lse, whole["lse"], atol=1e-12)
+
+
+def test_merge_closed_forms():
+    """One shard and no sink: the merge returns the shard's state.  All shards
+    empty: 0 and -inf.  A sink alone over one shard rescales by l / (l + e^sink)."""
+    rng = np.random.default_rng(6)
+    o = rng.standard_normal((1, 2, 3, 8))
+    l = rng.standard_normal((1, 2, 3))
+    out, lse = O.merge_partials(o, l, None)
+    np.testing.assert_allclose(out, o[0], atol=1e-15)
+    np.testing.assert_allclose(lse, l[0], atol=1e-15)
+    out, lse = O.merge_partials(np.zeros((2, 1, 1, 4)), np.full((2, 1, 1), -np.inf), None)
+    assert (out == 0).all() and np.isneginf(lse).all()
+    # every shard empty but a finite sink: the denominator is the sink alone
+    out, lse = O.merge_partials(np.zeros((2, 1, 1, 4)), np.full((2, 1, 1), -np.inf), np.array([0.3]))
+    assert (out == 0).all()
+    np.testing.assert_allclose(lse, [[0.3]], atol=1e-15)
+    sink = np.array([0.7, -1.0, 2.0])
+    out, lse = O.merge_partials(o, l, sink)
+    f = np.exp(l[0]) / (np.exp(l[0]) + np.exp(sink)[None, :])
+    np.testing.assert_allclose(out, o[0] * f[..., None], atol=1e-12)
+    np.testing.assert_allclose(lse, np.log(np.exp(l[0]) + np.exp(sink)[None, :]), atol=1e-12)
