@@ -645,6 +645,79 @@ def measure_e2e(wl, args, dev, stream, insts, amount, scale, unit, world):
             "ms_per_step": e2e_ms, "steps": ke}
 
 
+def measure_seq_shard(args, dev, rank, world):
+    """One batch's keys split across the ranks by position (sequence-sharded
+    split-KV): every rank attends its kv_range (partial state, no sink), the
+    states are all-gathered over NCCL and merged with the sink.  Strong
+    scaling: the total work is the same batch at every N."""
+    import torch
+
+    from selected_token_sparse_b200 import pipeline, shard, spa, workloads as W
+    wl = W.by_name(args.workload)        # the same requests on every rank
+    amount, scale, unit = work_of(wl)
+    a = wl.arrays
+    lengths = [p + q for p, q in zip(wl.past, wl.q_lens)]
+    rng = shard.sequence_ranges(lengths, world, rank, wl.block_size)
+    d = pipeline.to_device(wl, dev)
+    st = pipeline.Step(wl, d, want_lse=True)
+    st()                                 # metadata and append (every rank; the new rows land in its cache)
+    torch.cuda.synchronize(dev)
+    bt = torch.from_numpy(shard.shard_block_table(a["block_table"], rng, wl.block_size)).to(dev)
+    meta = dict(st.meta, cu_seqlens_q=d["cu_seqlens_q"])
+    po = torch.empty(wl.T, wl.H_q, wl.D, dtype=torch.float32, device=dev)
+    pl = torch.empty(wl.T, wl.H_q, dtype=torch.float32, device=dev)
+    kw = dict(st.kw)
+    if wl.sel_mode == "aux" and rank != 0:
+        kw.update(selected_idx=None, sel_target=0, aux_k=None, aux_v=None, aux_seqlens=None)
+    rng_d = torch.from_numpy(rng).to(dev)    # the arguments hold its address for every step
+    args_p = spa.attention_args(d["q"], d["k_cache"], d["v_cache"], bt, meta, max_seqlen_q=wl.max_seqlen_q,
+                                max_seqlen_k=wl.max_seqlen_k, out=po, lse=pl, num_splits=args.splits,
+                                status=st.status, kv_range=rng_d, partial=True, **kw)
+    ws = spa.new_workspace(spa.workspace_size(args_p), dev)
+    out = torch.empty_like(st.out)
+    lse = torch.empty(wl.T, wl.H_q, dtype=torch.float32, device=dev)
+    gpo = torch.empty(world, *po.shape, dtype=po.dtype, device=dev)
+    gpl = torch.empty(world, *pl.shape, dtype=pl.dtype, device=dev)
+
+    def step():
+        spa.run_attention(args_p, ws)
+        if world > 1:
+            import torch.distributed as dist
+            dist.all_gather_into_tensor(gpo, po)
+            dist.all_gather_into_tensor(gpl, pl)
+            spa.merge_partials(gpo, gpl, d.get("sinks"), out, lse)
+        else:
+            spa.merge_partials(po.unsqueeze(0), pl.unsqueeze(0), d.get("sinks"), out, lse)
+
+    stream = torch.cuda.current_stream(dev)
+    K, Wm = args.steps, args.warmup
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(dev.index)
+    with clk:
+        ev0.record(stream)
+        for _ in range(K):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dev)
+    ms = reduce_max(ev0.elapsed_time(ev1), dev) / K
+    status = int(st.status.item())
+    hbm, _, _, peak_src = load_peaks()
+    return {"workload": wl.name, "dtype": wl.act, "value": amount / (ms * 1e-3) / scale, "unit": unit,
+            "ms_per_step": ms, "steps": K, "warmup": Wm, "tokens_per_s": wl.T / (ms * 1e-3),
+            "algorithmic_per_step": amount, "status": status, "clocks": clk.summary(),
+            "scaling": "strong", "gpu_launches": K * 2,
+            "config": dict(workload_config(wl, world), parallelism=f"sequence-sharded split-KV over {world} rank(s)"),
+            "run": {"timing": "eager launches (partial attention, NCCL all-gather of the partial states, merge); "
+                              "CUDA events on the current stream, maximum over ranks",
+                    "roofline_per_rank_bytes": amount / world, "hbm_peak": hbm, "peak_source": peak_src}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -658,6 +731,20 @@ def run_ours(args):
                                 timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
+    if args.seq_shard:
+        r = measure_seq_shard(args, dev, rank, world)
+        line = {"metric": METRIC, "value": r["value"], "unit": r["unit"], "n_gpus": world, "steps": r["steps"],
+                "warmup": r["warmup"], "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": r["dtype"], "data": "synthetic",
+                "config": r["config"], "tokens_per_s": r["tokens_per_s"], "gpu_launches": r["gpu_launches"],
+                "clocks": r["clocks"], "status": r["status"], "run": r["run"], "roofline": None,
+                "cpu_baseline": None, "e2e": None}
+        if world > 1:
+            dist.barrier(device_ids=[dev.index])
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     names = [args.workload]
     if not args.only:
         names += [n for n in W.WORKLOADS + W.PROLOGUE_WORKLOADS if n != args.workload]
@@ -733,6 +820,8 @@ def main():
     ap.add_argument("--mode", choices=["step", "prepare_append", "staged"], default="step",
                     help="entry points of one step: the fused step call, prepare+append then attention, "
                          "or the three staged calls")
+    ap.add_argument("--seq-shard", action="store_true",
+                    help="split one batch's keys across the ranks (partial states, all-gather, merge)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -233,6 +233,28 @@ typedef struct spa_attention_args {
   float* lse;         /* [T, H_q] optional: log of the softmax denominator incl. the sink */
   int32_t num_splits; /* 0 = automatic; otherwise the number of key splits per unit */
   int32_t* status;    /* OR-ed status bits */
+  /* One shard of a sequence split across devices ("[WebGPU] Add
+     SparsePagedAttention", File summaries: partial FP32 softmax states merged
+     by a finalize stage that applies the sink).
+     kv_range [B, 2]: main-cache positions lo <= j < hi of request b that this
+       call attends (NULL = all).  Keys outside the range are dropped before
+       any block-table lookup, so a shard's block table may leave the other
+       shards' blocks unmapped (-1) without setting a status bit.  Auxiliary
+       entries are not affected.
+     partial = 1: the call leaves the shard's partial state for
+       spa_merge_partials instead of the output: `out` is FP32 [T, H_q, D],
+       the softmax over the shard's attended keys WITHOUT the sink (0 when it
+       has none); `lse` is required and holds its log-sum-exp (-inf when
+       none); `sinks` is ignored (the merge applies it once). */
+  const int32_t* kv_range;
+  int32_t partial;
+  /* Test hook of the failure detection, 0 in normal use: 1 makes the
+     tcgen05 prefill kernel drop one barrier arrival per CTA (on a barrier
+     that guards no copy and no MMA) and poll for it only briefly, so that the
+     bounded wait expires: every CTA drains its copies and MMAs, frees its
+     tensor memory and returns, and SPA_ST_TIMEOUT is set.  Other kernels
+     ignore it. */
+  int32_t test_expire_wait;
 } spa_attention_args_t;
 
 /* Bytes of workspace spa_attention needs for these arguments (0 if none: one
@@ -264,6 +286,27 @@ size_t spa_attention_workspace_size(const spa_attention_args_t* a);
  */
 int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
                   spa_stream_t stream);
+
+/*
+ * spa_merge_partials -- the merge of a sequence split across R devices: the
+ * partial states that R spa_attention calls with partial = 1 left (each over
+ * its kv_range of the same requests), gathered into one buffer, combined by
+ * log-sum-exp with the sink counted once.
+ * Source: "[WebGPU] Add SparsePagedAttention", File summaries (main and
+ * auxiliary partial FP32 softmax states; finalize merge with the sink).
+ *   part_out [R, T, H_q, D] fp32 (16-byte aligned), part_lse [R, T, H_q] fp32:
+ *                   shard r's out and lse.
+ *   sinks [H_q]     learned sink logits, or NULL (no sink).
+ *   act             dtype of `out` (SPA_F32 / SPA_F16 / SPA_BF16).
+ *   out [T, H_q, D], lse [T, H_q] (optional): for each row
+ *     M = max(sink, max_r lse_r), L = e^(sink - M) + sum_r e^(lse_r - M),
+ *     out = sum_r e^(lse_r - M) out_r / L, lse = M + ln L;
+ *     out = 0, lse = -inf when every shard is empty and there is no sink.
+ * Errors: SPA_ERR_INVALID_ARG for R <= 0, D not 64 / 128, a bad dtype or a
+ * NULL / misaligned required pointer.  T = 0 is valid.  One kernel launch.
+ */
+int spa_merge_partials(const float* part_out, const float* part_lse, int32_t R, int32_t T, int32_t H_q,
+                       int32_t D, const float* sinks, int32_t act, void* out, float* lse, spa_stream_t stream);
 
 /*
  * spa_prepare_append_attention -- steps 1 to 5 as one call: the outputs of

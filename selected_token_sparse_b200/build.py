@@ -58,6 +58,33 @@ def _compile(src: str, force: bool, verbose: bool, ptxas_v: bool) -> str:
     return obj
 
 
+PROBE_DIR = os.path.join(BUILD, "probe")
+PROBE_LIB = os.path.join(PROBE_DIR, "libspa_probe.so")
+
+
+def build_probe(verbose: bool = False) -> str:
+    """The phase-probe variant of the library (-DSPA_PHASE_PROBE: kernels stamp
+    %globaltimer at phase boundaries), built beside the objects, never into
+    the package.  Used by selected_token_sparse_b200.phase_probe."""
+    os.makedirs(PROBE_DIR, exist_ok=True)
+    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+    def one(src):
+        obj = os.path.join(PROBE_DIR, os.path.basename(src) + ".o")
+        cmd = [nvcc()] + ARCH + FLAGS + ["-DSPA_PHASE_PROBE", "-c", src, "-o", obj]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
+        return obj
+
+    with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
+        objs = list(ex.map(one, srcs))
+    r = subprocess.run([nvcc()] + ARCH + ["-shared", "-o", PROBE_LIB] + objs, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+    return PROBE_LIB
+
+
 def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
@@ -79,5 +106,6 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register / shared-memory use")
+    ap.add_argument("--probe", action="store_true", help="build the phase-probe library instead")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_v))
+    print(build_probe(a.verbose) if a.probe else build(a.force, a.verbose, a.ptxas_v))

@@ -81,6 +81,8 @@ int validate_attention(const spa_attention_args_t* a) {
       return SPA_ERR_INVALID_ARG;
   }
   if (!std::isfinite(a->scale) || a->scale < 0.f) return SPA_ERR_INVALID_ARG;
+  if (a->partial != 0 && a->partial != 1) return SPA_ERR_INVALID_ARG;
+  if (a->partial && !a->lse) return SPA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->out) |
        reinterpret_cast<uintptr_t>(a->k_cache) | reinterpret_cast<uintptr_t>(a->v_cache)) & 15)
     return SPA_ERR_INVALID_ARG;
@@ -190,7 +192,10 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   p->aux_v = a->aux_v;
   p->aux_cap = a->aux_cap;
   p->aux_len = a->aux_seqlens;
-  p->sinks = a->sinks;
+  p->sinks = a->partial ? nullptr : a->sinks;   // a shard's partial leaves the sink to the merge
+  p->kv_range = a->kv_range;
+  p->out_f32 = a->partial;
+  p->test_expire_wait = a->test_expire_wait != 0;
   const float scale = a->scale == 0.f ? (float)(1.0 / std::sqrt((double)a->D)) : a->scale;
   p->scale_log2 = scale * kLog2e;
   p->group_by_request = pl.group_by_request;

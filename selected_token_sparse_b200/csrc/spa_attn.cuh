@@ -58,6 +58,15 @@ struct AttnParams {
   int max_seqlen_q;      // host bounds for the step-1 status bits
   int max_seqlen_k;
   int cluster_merge;     // 1: the splits of a unit are one cluster, merged in shared memory
+  // one shard of a sequence split across devices: main-cache keys lo <= j < hi
+  // of request b ([B, 2], or nullptr for all); out_f32: `out` is fp32 (the
+  // shard's partial output; the host passes no sink then)
+  const int32_t* kv_range;
+  int out_f32;
+  // test hook (0 in normal use): the tcgen05 prefill kernel drops one arrival
+  // on a barrier that guards no copy or MMA, so that the bounded wait for it
+  // expires and the CTA takes its abort path (SPA_ST_TIMEOUT)
+  int test_expire_wait;
 };
 
 // Parameters of the fused metadata + QKV prologue + append kernel.
@@ -109,6 +118,7 @@ struct Unit {
   // fused step only: positions [new_lo, new_hi) are this step's tokens of the
   // request, whose K/V rows are read from k_new / v_new (token new_t0 + j - new_lo)
   int new_lo, new_hi, new_t0;
+  int rlo, rhi;           // main-cache key range of this shard (0, INT_MAX: all)
 };
 
 // First packed token of request b under the sanitised cumulative lengths
@@ -162,6 +172,12 @@ __device__ __forceinline__ bool decode_unit_with(const AttnParams& p, const Meta
     U.p_first = tpos;
   }
   U.p_last = U.p_first + U.nq - 1;
+  U.rlo = 0;
+  U.rhi = INT_MAX;
+  if (p.kv_range) {
+    U.rlo = max(p.kv_range[2 * U.b], 0);
+    U.rhi = p.kv_range[2 * U.b + 1];
+  }
   U.sel_main = p.sel != nullptr && p.sel_target == 0;
   U.sel_aux = p.sel != nullptr && p.sel_target == 1;
   U.selrow = p.sel ? p.sel + ((long long)(p.sel_per_request ? U.b : U.t0) * p.H_kv + U.h_kv) * p.sel_width
@@ -170,8 +186,8 @@ __device__ __forceinline__ bool decode_unit_with(const AttnParams& p, const Meta
   if (U.sel_main) {
     U.n_main = p.sel_width;
   } else {
-    U.lo = p.window > 0 ? max(0, U.p_first - p.window + 1) : 0;
-    const int hi = min(U.p_last + 1, U.L);
+    U.lo = max(p.window > 0 ? max(0, U.p_first - p.window + 1) : 0, U.rlo);
+    const int hi = min(min(U.p_last + 1, U.L), U.rhi);
     U.n_main = max(hi - U.lo, 0);
   }
   U.n_aux = U.sel_aux ? p.sel_width : 0;
@@ -197,7 +213,7 @@ __device__ __forceinline__ int cand_stage1(const AttnParams& p, const Unit& U, i
 
 __device__ __forceinline__ int cand_stage2(const AttnParams& p, const Unit& U, int c, int raw) {
   if (c >= U.n_main) return -1;
-  if (U.sel_main && (raw < 0 || raw >= U.L)) return -1;
+  if (U.sel_main && (raw < 0 || raw >= U.L || raw < U.rlo || raw >= U.rhi)) return -1;
   const int lb = raw / p.bs;
   if (lb >= p.MB) return -1;
   return p.block_table[(long long)U.b * p.MB + lb];
@@ -214,6 +230,7 @@ __device__ __forceinline__ long long cand_finish(const AttnParams& p, const Unit
         bits |= kStBadIdx;
         return -1;
       }
+      if (raw < U.rlo || raw >= U.rhi) return -1;   // another shard's key
     }
     const int j = raw;
     if (j / p.bs >= p.MB) {
@@ -284,6 +301,14 @@ __device__ __forceinline__ void store4(ActT* dst, float a, float b, float c, flo
     ActT v[4] = {from_f32<ActT>(a), from_f32<ActT>(b), from_f32<ActT>(c), from_f32<ActT>(d)};
     *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(v);
   }
+}
+
+// Four output columns at element offset `off` of `out`: in the activation
+// dtype, or fp32 for a shard's partial output.
+template <typename ActT>
+__device__ __forceinline__ void store_out4(const AttnParams& p, long long off, float a, float b, float c, float d) {
+  if (p.out_f32) *reinterpret_cast<float4*>(static_cast<float*>(p.out) + off) = make_float4(a, b, c, d);
+  else store4<ActT>(static_cast<ActT*>(p.out) + off, a, b, c, d);
 }
 
 template <typename ActT, int D>
@@ -357,8 +382,7 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, 
       for (int j = 0; j < 4; ++j) {
         if (base + j * (int)blockDim.x >= n_items) continue;
         const float inv = sInv[ii[j] / C4];
-        store4<ActT>(static_cast<ActT*>(p.out) + rw[j] * D + (ii[j] % C4) * 4, o[j].x * inv, o[j].y * inv,
-                     o[j].z * inv, o[j].w * inv);
+        store_out4<ActT>(p, rw[j] * D + (ii[j] % C4) * 4, o[j].x * inv, o[j].y * inv, o[j].z * inv, o[j].w * inv);
       }
     }
     __syncthreads();
@@ -435,7 +459,7 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, 
         inv = 1.0f / Lsum;
         lse = (M + log2f(Lsum)) * kLn2;
       }
-      store4<ActT>(static_cast<ActT*>(p.out) + row * D + c, o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      store_out4<ActT>(p, row * D + c, o.x * inv, o.y * inv, o.z * inv, o.w * inv);
       if (c == 0 && p.lse) p.lse[row] = lse;
     }
   }

@@ -30,6 +30,24 @@
 
 namespace spa {
 
+#ifdef SPA_PHASE_PROBE
+// Phase probe, compiled only into the separate probe library (build.py
+// --probe): thread 0 of every CTA stamps %globaltimer at the phase boundaries
+// below; the host reads the stamps of the last launch back.
+constexpr int kProbeCtas = 8192, kProbeSlots = 16;
+static __device__ unsigned long long g_phase_mma[kProbeCtas * kProbeSlots];
+__device__ __forceinline__ void phase_stamp(int i) {
+  const int c = blockIdx.y * gridDim.x + blockIdx.x;
+  if (threadIdx.x != 0 || c >= kProbeCtas) return;
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  g_phase_mma[c * kProbeSlots + i] = t;
+}
+#define SPA_PHASE(i) phase_stamp(i)
+#else
+#define SPA_PHASE(i) ((void)0)
+#endif
+
 constexpr int kMmaCandChunk = 512;   // candidates resolved at once
 
 // Keys per tile: one 128-key tile (one softmax pass, four 32-key warp slices)
@@ -146,8 +164,10 @@ decode_mma_kernel(const AttnParams p) {
   const int wr = warp % RT;   // row tile of this warp
   const int wk = warp / RT;   // key slice of this warp
   __shared__ int last_flag;
+  SPA_PHASE(0);
   pdl_wait();
   pdl_trigger();
+  SPA_PHASE(1);
 
   // Q rows of the unit in 16-byte chunks (row r = token r / G, head r % G).
   // A per-token unit knows its token from the block index, so its loads are
@@ -230,6 +250,7 @@ decode_mma_kernel(const AttnParams p) {
       pre_blk[k] = (raw >= 0 && raw / p.bs < p.MB) ? ld_early(p.block_table + (long long)b * p.MB + raw / p.bs) : -1;
     }
   }
+  SPA_PHASE(2);
   const int split = blockIdx.y;
   const int G = p.G;
   const int nq = p.group_by_request ? U.nq : 1;
@@ -373,8 +394,10 @@ decode_mma_kernel(const AttnParams p) {
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   uint32_t qf[C::kInt8 ? 1 : D / 16][4];
 
+  SPA_PHASE(3);
   if (ntiles > 0) resolve_chunk(0);
   __syncthreads();
+  SPA_PHASE(4);
 #pragma unroll
   for (int s = 0; s < kMmaStages - 1; ++s) {
     if (s < ntiles) issue(s);
@@ -418,6 +441,7 @@ decode_mma_kernel(const AttnParams p) {
   const int prow1 = r1 < R ? prow_s[r1 / G] : -1;
   const float sl2 = p.scale_log2;
 
+  SPA_PHASE(5);
   for (int it = 0; it < ntiles; ++it) {
     const int nxt = it + kMmaStages - 1;
     if (nxt < ntiles && nxt % kMmaCandTiles == 0) {
@@ -579,6 +603,7 @@ decode_mma_kernel(const AttnParams p) {
   }
   cp_async_wait<0>();
   __syncthreads();
+  SPA_PHASE(6);
 
   // row sums across the quad
 #pragma unroll
@@ -674,10 +699,14 @@ decode_mma_kernel(const AttnParams p) {
       finalize_row(mf[hrow], lf[hrow], sink2, a, inv_l, lse);
       const float f = a * inv_l;
       ActT* out = static_cast<ActT*>(p.out) + row * D;
+      float* out32 = static_cast<float*>(p.out) + row * D;
 #pragma unroll
       for (int nn = 0; nn < NPW; ++nn) {
         const int d = (n_lo + nn) * 8 + (lane & 3) * 2;
-        *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(fo[nn][hrow * 2 + 0] * f, fo[nn][hrow * 2 + 1] * f);
+        if (p.out_f32)
+          *reinterpret_cast<float2*>(out32 + d) = make_float2(fo[nn][hrow * 2 + 0] * f, fo[nn][hrow * 2 + 1] * f);
+        else
+          *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(fo[nn][hrow * 2 + 0] * f, fo[nn][hrow * 2 + 1] * f);
       }
       if (wk == 0 && (lane & 3) == 0 && p.lse) p.lse[row] = lse;
     } else if (p.cluster_merge) {
@@ -705,6 +734,7 @@ decode_mma_kernel(const AttnParams p) {
     }
   }
 
+  SPA_PHASE(7);
   // fused step: the rest of steps 1-2 (off the attention's critical path)
   if constexpr (FUSED) {
     if (split == 0) {
@@ -723,6 +753,7 @@ decode_mma_kernel(const AttnParams p) {
     }
   }
   flag(p.status, bits);
+  SPA_PHASE(8);
   if (p.num_splits > 1) {
     if (p.cluster_merge) {
       // the unit's splits are one cluster: merge through distributed shared memory
@@ -736,6 +767,7 @@ decode_mma_kernel(const AttnParams p) {
       finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
     }
   }
+  SPA_PHASE(9);
 }
 
 // ---------------------------------------------------------------------------
@@ -822,3 +854,16 @@ int launch_step_mma(const AttnParams& p, int act, int max_rows, cudaStream_t str
 }
 
 }  // namespace spa
+
+#ifdef SPA_PHASE_PROBE
+// Probe library only: copy / clear the phase stamps of decode_mma_kernel.
+extern "C" int spa_probe_read_mma(void* host, size_t bytes) {
+  if (bytes > sizeof(spa::g_phase_mma)) bytes = sizeof(spa::g_phase_mma);
+  return (int)cudaMemcpyFromSymbol(host, spa::g_phase_mma, bytes);
+}
+extern "C" int spa_probe_clear_mma() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, spa::g_phase_mma) != cudaSuccess) return -1;
+  return (int)cudaMemset(p, 0, sizeof(spa::g_phase_mma));
+}
+#endif

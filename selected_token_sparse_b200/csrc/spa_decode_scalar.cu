@@ -195,7 +195,9 @@ decode_scalar_kernel(const AttnParams p) {
         const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
         float a, inv_l, lse;
         finalize_row(m_s[r], l_s[r], sink2, a, inv_l, lse);
-        out[((long long)t * p.H_q + h) * D + d] = from_f32<ActT>(acc[i] * a * inv_l);
+        const long long oi = ((long long)t * p.H_q + h) * D + d;
+        if (p.out_f32) static_cast<float*>(p.out)[oi] = acc[i] * a * inv_l;
+        else out[oi] = from_f32<ActT>(acc[i] * a * inv_l);
         if (d == 0 && p.lse) p.lse[(long long)t * p.H_q + h] = lse;
       }
     }

@@ -607,9 +607,11 @@ decode_tc_kernel(const AttnParams p) {
     // scores of tile j - 1, which the softmax warps read before placing P(j - 1),
     // which PV(j - 1) waited for.
     bool ok = mbar_wait(bar_q, 0, kTcWaitLimit, abort_flag) && mbar_wait(bar_full, 0, kTcWaitLimit, abort_flag);
+    int s_iss = 0, pv_iss = 0;   // S and PV groups issued (each committed to its buffer's barrier)
     if (ok) {
       tc_fence_after();
       issue_s(0);
+      ++s_iss;
     }
     for (int j = 0; j < ntiles && ok; ++j) {
       const int st = j % NST, sb = j & 1;
@@ -618,6 +620,7 @@ decode_tc_kernel(const AttnParams p) {
         if (!ok) break;
         tc_fence_after();
         issue_s(j + 1);
+        ++s_iss;
       }
       ok = mbar_wait(bar_p + sb, (j >> 1) & 1, kTcWaitLimit, abort_flag);
       if (!ok) break;
@@ -631,8 +634,15 @@ decode_tc_kernel(const AttnParams p) {
       }
       tc_commit(bar_o + sb);
       tc_commit(bar_empty + st);   // the stage is free once S and PV of this tile complete
+      ++pv_iss;
     }
-    if (!ok) *abort_flag = 1;
+    if (!ok) {
+      *abort_flag = 1;
+      // the MMAs already issued complete before the tensor memory is freed
+      // (bounded; the latest commit on a barrier covers every earlier MMA)
+      if (s_iss > 0) mbar_wait(bar_s + ((s_iss - 1) & 1), ((s_iss - 1) >> 1) & 1, kTcWaitLimit);
+      if (pv_iss > 0) mbar_wait(bar_o + ((pv_iss - 1) & 1), ((pv_iss - 1) >> 1) & 1, kTcWaitLimit);
+    }
   }
 
   float m_used = -INFINITY, l_sum = 0.f;
@@ -813,9 +823,15 @@ decode_tc_kernel(const AttnParams p) {
       if (p.num_splits == 1) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) ov[e] *= f;
-        uint4* out = reinterpret_cast<uint4*>(static_cast<ActT*>(p.out) + orow * D + col);
+        if (p.out_f32) {
+          float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * D + col);
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) out[e / 8] = pack8<ActT>(ov + e);
+          for (int e = 0; e < 32; e += 4) out[e / 4] = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
+        } else {
+          uint4* out = reinterpret_cast<uint4*>(static_cast<ActT*>(p.out) + orow * D + col);
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) out[e / 8] = pack8<ActT>(ov + e);
+        }
       } else if (p.cluster_merge) {
         float* po = reinterpret_cast<float*>(smem + C::OFF_PART) + row * (D + 4) + col;
 #pragma unroll

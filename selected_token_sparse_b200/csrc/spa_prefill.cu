@@ -101,6 +101,8 @@ constexpr bool kPfLo = std::is_same<T, __nv_bfloat16>::value;
 
 struct PfGeom {
   int b, h, h_kv, t_begin, q_len, past, L, k_lo, k_hi, ntiles;
+  int k_first;   // first key any row of the item attends (k_lo is it rounded down to a tile)
+  int rlo;       // first key of this shard's range (0: all)
   int q0[2], rows[2];   // per q tile: first row within the request, rows present (0 = absent)
 };
 
@@ -137,7 +139,7 @@ __device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g
   for (int i = 0; i < 8; ++i) {
     if (i >= nbox) break;
     const int key0 = kb + i * box_rows;
-    const bool needed = key0 < g.k_hi;
+    const bool needed = key0 < g.k_hi && key0 + box_rows > g.k_first;   // some key of the box is attended
     const int lb = key0 / p.bs;
     int blk = -1;
     if (lb >= p.MB) {
@@ -177,9 +179,15 @@ __device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_pai
   const int last_row = g.rows[1] > 0 ? g.q0[1] + g.rows[1] - 1 : g.q0[0] + g.rows[0] - 1;
   const int p_first = g.past + g.q0[0];
   const int p_last = g.past + last_row;
-  g.k_lo = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
-  g.k_lo = (g.k_lo / kPfBN) * kPfBN;
-  g.k_hi = min(p_last + 1, g.L);
+  g.rlo = 0;
+  int rhi = INT_MAX;
+  if (p.kv_range) {
+    g.rlo = max(p.kv_range[2 * g.b], 0);
+    rhi = p.kv_range[2 * g.b + 1];
+  }
+  g.k_first = max(p.window > 0 ? max(0, p_first - p.window + 1) : 0, g.rlo);
+  g.k_lo = (g.k_first / kPfBN) * kPfBN;
+  g.k_hi = min(min(p_last + 1, g.L), rhi);
   g.ntiles = g.k_hi > g.k_lo ? (g.k_hi - g.k_lo + kPfBN - 1) / kPfBN : 0;
   g.ntiles = min(g.ntiles, max_tiles);
   return true;
@@ -246,6 +254,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   int bits = 0;
+  int kv_issued = 0;   // K/V tiles the producer has issued (its thread only)
+  // test hook: the MMA thread's waits for P give up after a few polls, and
+  // softmax warp 0 drops its first arrival (see AttnParams::test_expire_wait)
+  const uint32_t p_wait_limit = p.test_expire_wait ? 256u : kPfWaitLimit;
 
   // the next item, from `item` on, with key tiles (others need no tensor work)
   auto next_work = [&](int& item, PfGeom& gg) {
@@ -270,7 +282,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           if (!ok) break;
           pf_issue_kv(p, g, &tm_k, &tm_v, sK + st * C::TILE, sV + st * C::TILE, bar_kf + st, bar_vf + st,
                       g.k_lo + j * kPfBN, box_rows, C::NCH, bits, C::TX_TILE);
-          ++c;
+          kv_issued = ++c;
         }
         item += gridDim.x;
       }
@@ -357,7 +369,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           bool k_next = false;
           ok = mbar_wait(bar_vf + st, ph, kPfWaitLimit, abort_flag);
           for (int t = 0; t < ntq && ok; ++t) {
-            ok = mbar_wait(bar_p + t, p_seen[t] & 1, kPfWaitLimit, abort_flag);
+            ok = mbar_wait(bar_p + t, p_seen[t] & 1, p_wait_limit, abort_flag);
             if (ok) ++p_seen[t];
             // the first PV of an item overwrites O_t: the previous epilogue must have read it
             while (ok && j == 0 && e_seen[t] < e_due[t]) {
@@ -462,12 +474,12 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         if (j + 1 < g.ntiles) blk_next = pf_block_id(p, g.b, kb + kPfBN, lane, nbox, box_shift);
         const bool all_mapped = boxmask == (1u << nbox) - 1u;
         const bool full = all_mapped && kb + kPfBN - 1 <= p_lo && kb + kPfBN <= g.k_hi &&
-                          (p.window <= 0 || kb > p_hi - p.window);
+                          (p.window <= 0 || kb > p_hi - p.window) && kb >= g.rlo;
         // visibility of key column c (only consulted on tiles that need a mask):
         // the row's causal / window / end-of-keys limits as a column interval
         // [c_lo, c_hi), and the mapped-block bitmask
         const int c_hi = min(min(prow + 1, g.k_hi) - kb, kPfBN);
-        const int c_lo = p.window > 0 ? max(prow - p.window + 1 - kb, 0) : 0;
+        const int c_lo = max(p.window > 0 ? max(prow - p.window + 1 - kb, 0) : 0, g.rlo - kb);
         // visibility of the 32 columns of chunk c4 as a bitmask: the row's
         // causal / window / end-of-keys interval and the mapped blocks
         auto chunk_bits = [&](int c4) -> uint32_t {
@@ -561,7 +573,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_p + t);
+        const bool drop = p.test_expire_wait && warp == 0 && j == 0 && item == (int)blockIdx.x;
+        if (lane == 0 && !drop) mbar_arrive(bar_p + t);
       }
       if (!ok) break;
       // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
@@ -593,7 +606,13 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-          if (mine) {
+            if (mine && p.out_f32) {
+            float* o32 = static_cast<float*>(p.out) + orow * D + c * 32;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(o32 + e) =
+                  make_float4(u2f(o[e]) * f, u2f(o[e + 1]) * f, u2f(o[e + 2]) * f, u2f(o[e + 3]) * f);
+          } else if (mine) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint4 v;
@@ -615,7 +634,17 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     if (!ok) *abort_flag = 1;
   }
   __syncthreads();
-  if (*abort_flag) bits |= SPA_ST_TIMEOUT;
+  if (*abort_flag) {
+    bits |= SPA_ST_TIMEOUT;
+    // another role gave up: the producer's last two K/V tiles may still be in
+    // flight although it finished issuing normally; they land before the CTA
+    // leaves (bounded; the latest phase of each stage is unambiguous)
+    if (warp == 9 && lane == 0)
+      for (int k = kv_issued >= 2 ? kv_issued - 2 : 0; k < kv_issued; ++k) {
+        mbar_wait(bar_kf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
+        mbar_wait(bar_vf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
+      }
+  }
   flag(p.status, bits);
   tc_fence_before();
   __syncthreads();

@@ -12,9 +12,9 @@
 //      and kept in shared memory as order-preserving 32-bit keys (NaN and
 //      -inf, which are never selected, become 0; -0 becomes +0);
 //   2. when more than top_k keys are eligible, a radix select over four
-//      8-bit digits (a 256-bin shared histogram per digit, warp-aggregated
-//      increments) finds the exact k-th largest key T and how many keys equal
-//      to T are still to be taken -- the first ones by index (stable);
+//      8-bit digits (a 256-bin shared histogram per digit) finds the exact
+//      k-th largest key T and how many keys equal to T are still to be taken
+//      -- the first ones by index (stable);
 //   3. a compaction over contiguous per-warp segments (ballot / popc counts,
 //      one scan over the 32 warps) writes every kept index at its rank among
 //      the kept ones, so the row comes out in increasing index order;
@@ -50,7 +50,7 @@ struct SelShared {
 
 __global__ void __launch_bounds__(kSelThreads, 1)
 select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const int32_t* __restrict__ bound,
-                   int top_k, int sel_width, int32_t* __restrict__ out, int staged) {
+                   int top_k, int sel_width, int32_t* __restrict__ out, int staged, int vec) {
   extern __shared__ uint32_t sel_keys[];
   __shared__ SelShared sh;
   pdl_wait();
@@ -65,21 +65,49 @@ select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const in
 
   auto key_at = [&](int j) -> uint32_t { return staged ? sel_keys[j] : score_key(__ldg(src + j)); };
 
-  // 1. stage the keys and count the eligible ones
+  // 1. stage the keys and count the eligible ones.  Rows whose start is
+  // 16-byte aligned are read with 16-byte vectors, eight in flight per thread
+  // (a 32768-key row in one batch).
   int elig = 0;
-  for (int j0 = 0; j0 < n; j0 += 8 * kSelThreads) {
-    float v[8];
+  if (vec) {
+    const float4* src4 = reinterpret_cast<const float4*>(src);
+    const int n4 = (n + 3) >> 2;
+    for (int i0 = 0; i0 < n4; i0 += 8 * kSelThreads) {
+      float4 v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * kSelThreads + tid;
-      v[u] = j < n ? __ldg(src + j) : __int_as_float(0xff800000);
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kSelThreads + tid;
+        v[u] = i < n4 ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kSelThreads + tid;
+        if (i >= n4) continue;
+        const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t k[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          k[e] = 4 * i + e < n ? score_key(x[e]) : 0u;   // keys beyond the bound are not candidates
+          elig += k[e] != 0u;
+        }
+        if (staged) *reinterpret_cast<uint4*>(sel_keys + 4 * i) = make_uint4(k[0], k[1], k[2], k[3]);
+      }
     }
+  } else {
+    for (int j0 = 0; j0 < n; j0 += 8 * kSelThreads) {
+      float v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u * kSelThreads + tid;
-      const uint32_t k = score_key(v[u]);
-      elig += k != 0u;
-      if (staged && j < n) sel_keys[j] = k;
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * kSelThreads + tid;
+        v[u] = j < n ? __ldg(src + j) : __int_as_float(0xff800000);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * kSelThreads + tid;
+        const uint32_t k = score_key(v[u]);
+        elig += k != 0u;
+        if (staged && j < n) sel_keys[j] = k;
+      }
     }
   }
   elig = __reduce_add_sync(0xffffffffu, elig);
@@ -105,13 +133,7 @@ select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const in
       for (int j0 = 0; j0 < n; j0 += kSelThreads) {
         const int j = j0 + tid;
         const uint32_t k = j < n ? key_at(j) : 0u;
-        const bool m = k != 0u && (k & pmask) == prefix;
-        const unsigned active = __ballot_sync(0xffffffffu, m);
-        if (m) {
-          const uint32_t d = (k >> shift) & 255u;
-          const unsigned peers = __match_any_sync(active, d);
-          if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[d], (uint32_t)__popc(peers));
-        }
+        if (k != 0u && (k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
       }
       __syncthreads();
       if (warp == 0) {
@@ -218,14 +240,17 @@ extern "C" int spa_select_topk(const float* scores, int32_t R, int32_t H, int32_
   if (R == 0) return SPA_OK;
   if (!selected_idx || !bound || (n_keys > 0 && !scores)) return SPA_ERR_INVALID_ARG;
   const int staged = n_keys <= kSelStageKeys ? 1 : 0;
-  const size_t smem = staged ? (size_t)(n_keys > 0 ? n_keys : 1) * sizeof(uint32_t) : 0;
+  // whole-row 16-byte vectors: every row starts 16-byte aligned
+  const int vec = (n_keys % 4 == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) ? 1 : 0;
+  const size_t smem = staged ? (size_t)(n_keys > 0 ? ((n_keys + 3) & ~3) : 4) * sizeof(uint32_t) : 0;
   if (staged && smem > 48 * 1024) {
     if (cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSelStageKeys * (int)sizeof(uint32_t)) != cudaSuccess)
       return check_launch_public();
   }
   const int rc = launch_pdl(select_topk_kernel, dim3((unsigned)(R * H)), dim3(kSelThreads), smem,
-                            (cudaStream_t)stream, scores, H, n_keys, bound, top_k, sel_width, selected_idx, staged);
+                            (cudaStream_t)stream, scores, H, n_keys, bound, top_k, sel_width, selected_idx, staged,
+                            vec);
   if (rc != SPA_OK) return rc;
   return check_launch_public();
 }

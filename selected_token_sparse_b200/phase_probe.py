@@ -1,0 +1,106 @@
+"""Warm, in-graph phase breakdown of the warp-MMA decode kernel.
+
+    python -m selected_token_sparse_b200.phase_probe [--workload NAME] [--lib PATH]
+
+Builds (or loads) the probe variant of libspa (build.py --probe: the same
+sources compiled with -DSPA_PHASE_PROBE, where thread 0 of every CTA stamps
+%globaltimer at the kernel's phase boundaries), captures K steps of the
+workload over rotating device instances in one CUDA graph, replays it twice
+(warm), clears the stamps, replays it once more and reads back the stamps of
+the graph's last step -- a step that ran right after another one, as in the
+benchmark.  Prints the median / p90 duration of each phase over the CTAs.
+
+Phase stamps of decode_mma_kernel:
+  0 entry (before griddepcontrol.wait)   1 predecessor complete (wait released)
+  2 unit decoded (metadata, fused scan)  3 Q staged, before the candidates
+  4 first candidate chunk resolved       5 first K/V stages issued
+  6 key loop done (all copies landed)    7 output / partial state written
+  8 fused metadata + append tail done    9 split merge done (CTA end)
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import math
+import os
+
+import numpy as np
+import torch
+
+from . import build, pipeline, spa, workloads as W
+
+PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumulative-length scan)"),
+          (2, 3, "Q rows to shared memory"), (3, 4, "candidates: block ids, row offsets"),
+          (4, 5, "issue the first K/V stages"), (5, 6, "key loop (copies, QK, softmax, PV)"),
+          (6, 7, "epilogue: normalise, write output"), (7, 8, "fused metadata / append tail"),
+          (8, 9, "split merge"), (1, 9, "CTA after the wait"), (0, 9, "CTA incl. the wait")]
+
+
+def run(workload: str, lib_path: str, steps: int = 64):
+    lib = spa.load_library(lib_path)
+    lib.spa_probe_read_mma.restype = ctypes.c_int
+    lib.spa_probe_read_mma.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
+    lib.spa_probe_clear_mma.restype = ctypes.c_int
+    spa._LIB = lib
+    wl = W.by_name(workload)
+    base = pipeline.to_device(wl)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    per = sum(base[k].numel() * base[k].element_size() for k in ("k_cache", "v_cache"))
+    R = max(2, min(16, math.ceil(2 * l2 / per) + 1))
+    insts = []
+    for _ in range(R):
+        d = {k: (v.clone() if k in ("k_cache", "v_cache", "q", "k_new", "v_new", "block_table", "cu_seqlens_q",
+                                   "past_seqlens", "selected_idx") else v) for k, v in base.items()}
+        insts.append(pipeline.Step(wl, d))
+    assert spa.attention_plan(insts[0].args)["kind"] == 1, "the workload does not run the warp-MMA kernel"
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for st in insts:
+            st()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            insts[i % R]()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert lib.spa_probe_clear_mma() == 0
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    buf = np.zeros(8192 * 16, dtype=np.uint64)
+    assert lib.spa_probe_read_mma(buf.ctypes.data, buf.nbytes) == 0
+    P = buf.reshape(8192, 16).astype(np.int64)
+    P = P[P[:, 0] > 0]
+    lines = [f"workload {workload}: {len(P)} CTAs of the graph's last step ({steps} steps, {R} instances)",
+             f"CTA span (first entry to last end): {(P[:, 9].max() - P[:, 0].min()) / 1e3:.2f} us; "
+             f"from the first wait release: {(P[:, 9].max() - P[:, 1].min()) / 1e3:.2f} us",
+             "", "| phase | median us | p90 us | max us |", "|---|---|---|---|"]
+    for a, b, name in PHASES:
+        ok = (P[:, a] > 0) & (P[:, b] > 0)
+        if ok.any():
+            x = (P[ok, b] - P[ok, a]) / 1e3
+            lines.append(f"| {a}->{b} {name} | {np.median(x):.2f} | {np.percentile(x, 90):.2f} | {x.max():.2f} |")
+    t0 = P[:, 1].min()
+    lines += ["", "stamp offsets from the first wait release (us), percentiles 0 / 50 / 100:"]
+    for k in range(10):
+        ok = P[:, k] > 0
+        if ok.any():
+            q = np.percentile((P[ok, k] - t0) / 1e3, [0, 50, 100])
+            lines.append(f"  stamp {k}: {q[0]:.2f} / {q[1]:.2f} / {q[2]:.2f}")
+    return "\n".join(lines)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="gptoss_paged_decode_f16")
+    ap.add_argument("--lib", default=None, help="probe library (default: build it with build.py --probe)")
+    ap.add_argument("--steps", type=int, default=64)
+    a = ap.parse_args()
+    lib = a.lib or (build.PROBE_LIB if os.path.exists(build.PROBE_LIB) else build.build_probe())
+    print(run(a.workload, lib, a.steps))
+
+
+if __name__ == "__main__":
+    main()

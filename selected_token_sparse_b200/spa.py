@@ -24,7 +24,7 @@ ST_BAD_CU, ST_CAPACITY, ST_BAD_BLOCK, ST_BOUNDS, ST_BAD_IDX = 0x1, 0x2, 0x4, 0x8
 EXPORTED = ("spa_prepare_metadata", "spa_append_kv", "spa_prepare_append_kv", "spa_prepare_qkv_append",
             "spa_attention", "spa_attention_workspace_size", "spa_attention_plan",
             "spa_prepare_append_attention", "spa_prepare_append_attention_launches",
-            "spa_attention_noalloc", "spa_select_topk", "spa_error_string")
+            "spa_attention_noalloc", "spa_select_topk", "spa_merge_partials", "spa_error_string")
 
 _DT = {torch.float32: SPA_F32, torch.float16: SPA_F16, torch.bfloat16: SPA_BF16, torch.int8: SPA_I8}
 
@@ -50,6 +50,7 @@ class AttentionArgs(ctypes.Structure):
         ("aux_k", _vp), ("aux_v", _vp), ("aux_cap", _i32), ("aux_seqlens", _vp),
         ("sinks", _vp), ("scale", ctypes.c_float), ("lse", _vp),
         ("num_splits", _i32), ("status", _vp),
+        ("kv_range", _vp), ("partial", _i32), ("test_expire_wait", _i32),
     ]
 
 
@@ -107,6 +108,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.spa_prepare_append_attention_launches.argtypes = [ctypes.POINTER(AttentionArgs)]
     lib.spa_prepare_qkv_append.restype = ctypes.c_int
     lib.spa_prepare_qkv_append.argtypes = [ctypes.POINTER(QkvArgs), _vp]
+    lib.spa_merge_partials.restype = ctypes.c_int
+    lib.spa_merge_partials.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp]
     lib.spa_select_topk.restype = ctypes.c_int
     lib.spa_select_topk.argtypes = [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _vp]
     lib.spa_error_string.restype = ctypes.c_char_p
@@ -277,7 +280,10 @@ def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
                    sinks: Optional[torch.Tensor] = None, scale: float = 0.0,
                    k_scale: Optional[torch.Tensor] = None, v_scale: Optional[torch.Tensor] = None,
                    num_splits: int = 0, status: Optional[torch.Tensor] = None,
-                   is_causal: int = 1) -> AttentionArgs:
+                   is_causal: int = 1, kv_range: Optional[torch.Tensor] = None,
+                   partial: bool = False) -> AttentionArgs:
+    """Argument struct of spa_attention.  It holds raw device addresses: every
+    tensor passed here must stay alive for as long as the struct is used."""
     T, H_q, D = q.shape
     a = AttentionArgs()
     a.struct_size = ctypes.sizeof(AttentionArgs)
@@ -301,6 +307,8 @@ def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     a.sinks, a.scale, a.lse = _ptr(sinks), float(scale), _ptr(lse)
     a.num_splits = num_splits
     a.status = _ptr(status if status is not None else meta.get("status"))
+    a.kv_range = _ptr(kv_range)
+    a.partial = 1 if partial else 0
     return a
 
 
@@ -387,4 +395,16 @@ def select_topk(scores: torch.Tensor, bound: torch.Tensor, top_k: int, sel_width
     rc = lib().spa_select_topk(_ptr(scores), R, H, N, _ptr(bound), int(top_k), int(sel_width), _ptr(out),
                                _stream(scores.device))
     _check(rc, "spa_select_topk")
+    return out
+
+
+def merge_partials(part_out: torch.Tensor, part_lse: torch.Tensor, sinks: Optional[torch.Tensor],
+                   out: torch.Tensor, lse: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Merge R shards' partial states part_out [R, T, H_q, D] fp32 and
+    part_lse [R, T, H_q] (spa_attention with partial=1 over each shard's
+    kv_range) into out [T, H_q, D] (its own dtype), the sink counted once."""
+    R, T, H_q, D = part_out.shape
+    rc = lib().spa_merge_partials(_ptr(part_out), _ptr(part_lse), R, T, H_q, D, _ptr(sinks), _DT[out.dtype],
+                                  _ptr(out), _ptr(lse), _stream(out.device))
+    _check(rc, "spa_merge_partials")
     return out
