@@ -46,6 +46,24 @@ namespace spa {
 
 using namespace sm100;
 
+#ifdef SPA_PHASE_PROBE
+// Phase probe, compiled only into the separate probe library (build.py
+// --probe): the given thread of every CTA stamps %globaltimer at a phase
+// boundary; the host reads the stamps of the last launch back.
+constexpr int kTcProbeCtas = 4096, kTcProbeSlots = 16;
+static __device__ unsigned long long g_phase_tc[kTcProbeCtas * kTcProbeSlots];
+__device__ __forceinline__ void tc_phase_stamp(int i, int t) {
+  const int c = blockIdx.y * gridDim.x + blockIdx.x;
+  if ((int)threadIdx.x != t || c >= kTcProbeCtas) return;
+  unsigned long long v;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(v));
+  g_phase_tc[c * kTcProbeSlots + i] = v;
+}
+#define SPA_PHASE_T(i, t) tc_phase_stamp(i, t)
+#else
+#define SPA_PHASE_T(i, t) ((void)0)
+#endif
+
 constexpr int kTcKT = 64;                       // keys per tile (MMA N)
 constexpr int kTcStages = 3;                    // K/V tiles in the ring
 constexpr int kTcCons = 128;                    // softmax threads (4 warps, one per row)
@@ -190,8 +208,27 @@ decode_tc_kernel(const AttnParams p) {
   const int ptid = tid - kTcCons;             // producer thread index
   const int row = tid;                        // softmax: the S / O row (TMEM lane)
   __shared__ int last_flag;
+  SPA_PHASE_T(0, 0);
   pdl_wait();
   pdl_trigger();
+  SPA_PHASE_T(1, 0);
+
+  // Issued before the metadata is known: the lengths every warp scans by
+  // itself (fused step, B + 1 <= 64: build_cs_warp, no block barrier that
+  // would wait for loads in flight) and the INT8 scales of the kv head.
+  const bool warp_scan = FUSED && p.B + 1 <= 64;
+  int pc0 = 0, pc1 = 0, pp0 = 0, pp1 = 0;
+  if (warp_scan) {
+    pc0 = (lane >= 1 && lane <= p.B) ? ld_early(p.cu + lane) : 0;
+    pc1 = lane + 32 <= p.B ? ld_early(p.cu + lane + 32) : 0;
+    pp0 = lane < p.B ? ld_early(p.past + lane) : 0;
+    pp1 = lane + 32 < p.B ? ld_early(p.past + lane + 32) : 0;
+  }
+  float ks_r = 0.f, vs_r = 0.f;
+  if (C::kInt8 && tid < D) {
+    ks_r = ld_early(p.k_scale + (blockIdx.x % p.H_kv) * D + tid);
+    vs_r = ld_early(p.v_scale + (blockIdx.x % p.H_kv) * D + tid);
+  }
 
   Unit U;
   bool has_rows;
@@ -203,7 +240,8 @@ decode_tc_kernel(const AttnParams p) {
     cs_s = reinterpret_cast<int32_t*>(smem + C::BYTES);
     past_s = cs_s + p.B + 1;
     stage_s = reinterpret_cast<int8_t*>(smem + C::BYTES + ((sizeof(int32_t) * (2 * p.B + 1) + 15) & ~size_t(15)));
-    build_cs<kTcThreads>(p.cu, p.B, p.T, cs_s, p.past, past_s);   // ends with a block barrier
+    if (warp_scan) build_cs_warp(p.B, p.T, cs_s, past_s, pc0, pc1, pp0, pp1);
+    else build_cs<kTcThreads>(p.cu, p.B, p.T, cs_s, p.past, past_s);   // ends with a block barrier
     has_rows = decode_unit_with(p, FusedMeta{p.cu, cs_s, past_s, p.B}, blockIdx.x, U);
     if (has_rows) {
       U.new_lo = max(past_s[U.b], 0);
@@ -225,6 +263,7 @@ decode_tc_kernel(const AttnParams p) {
     has_rows = decode_unit(p, blockIdx.x, U);
     if (p.group_by_request && !has_rows) return;
   }
+  SPA_PHASE_T(2, 0);
   const int split = blockIdx.y;
   const int G = p.G;
   const int nq = p.group_by_request ? U.nq : 1;
@@ -266,13 +305,17 @@ decode_tc_kernel(const AttnParams p) {
     tmem_alloc(tmem_holder, kTcTmemCols);
     tmem_relinquish();
   }
-  if constexpr (C::kInt8) {
-    for (int d = tid; d < D; d += kTcThreads) {
-      ksc[d] = p.k_scale[h_kv * D + d];
-      vsc[d] = p.v_scale[h_kv * D + d];
-    }
+  if (C::kInt8 && tid < D) {
+    ksc[tid] = ks_r;
+    vsc[tid] = vs_r;
   }
-  // softmax: Q row `row` (token row / G, head row % G), in flight across the set-up
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // softmax: Q row `row` (token row / G, head row % G), loaded after the
+  // set-up barrier (which would otherwise wait for it: the producers' path
+  // is the critical one; the softmax warps wait for S(0) long after)
   constexpr int QV = D / 8;
   uint4 qv[QV];
   float sink_raw = -INFINITY;
@@ -288,10 +331,6 @@ decode_tc_kernel(const AttnParams p) {
     // the epilogue's (or the cluster merge's) sink logit of row `row`
     if (p.sinks && (p.num_splits == 1 || p.cluster_merge) && row < R) sink_raw = ld_early(p.sinks + h_kv * G + row % G);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
 
   if (producer) {
     // =================== producers: candidates, gather, conversion ===================
@@ -454,7 +493,9 @@ decode_tc_kernel(const AttnParams p) {
         }
       }
     }
+    SPA_PHASE_T(3, kTcCons);
     if (ntiles > 0) resolve_chunk(0);
+    SPA_PHASE_T(4, kTcCons);
     if constexpr (FUSED && C::kInt8) {
       for (int idx = ptid; idx < n_new; idx += kTcProd) {
         const int k = (idx - ptid) / kTcProd;
@@ -537,6 +578,7 @@ decode_tc_kernel(const AttnParams p) {
           *reinterpret_cast<uint4*>(dst + sw_off<KT>(r, 2 * ch + 1)) = h1;
         }
         publish(j, place_vis(j));
+        if (j == 0) SPA_PHASE_T(5, kTcCons);
       }
     } else {
       // NST tiles in flight; tile j + NST goes into tile j's stage once its MMAs are done
@@ -552,6 +594,7 @@ decode_tc_kernel(const AttnParams p) {
         else cp_async_wait<0>();
         bar_sync(kTcBarProd, kTcProd);   // tile j landed (every producer's copies)
         publish(j, place_vis(j));
+        if (j == 0) SPA_PHASE_T(5, kTcCons);
         const int n = j + NST;
         if (n < ntiles) {
           if (n % kTcCandTiles == 0) {
@@ -693,6 +736,7 @@ decode_tc_kernel(const AttnParams p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_q);
     }
+    SPA_PHASE_T(6, 0);
     const float sl2 = p.scale_log2;
     const int prow = (row < R && has_rows) ? U.p_first + row / G : -1;
     bool lost = false;
@@ -705,6 +749,7 @@ decode_tc_kernel(const AttnParams p) {
         lost = true;
         break;
       }
+      if (j == 0) SPA_PHASE_T(7, 0);
       tc_fence_after();
       // ---- softmax of row `row` over the tile's 64 keys
       const bool tile_vis = tvis_s[st] != 0;
@@ -785,6 +830,7 @@ decode_tc_kernel(const AttnParams p) {
       tc_fence_after();
     }
     if (lost) *abort_flag = 1;
+    SPA_PHASE_T(8, 0);
   }
   // every role is done with the rings (the producers drained their copies)
   __syncthreads();
@@ -855,6 +901,7 @@ decode_tc_kernel(const AttnParams p) {
       }
     }
   }
+  SPA_PHASE_T(9, 0);
   flag(p.status, bits);
   tc_fence_before();
   __syncthreads();
@@ -874,6 +921,7 @@ decode_tc_kernel(const AttnParams p) {
       finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
     }
   }
+  SPA_PHASE_T(10, 0);
 }
 
 int tc_supported(int act, int cache, int D, int max_rows) {
@@ -938,3 +986,16 @@ int tc_step_fits(int D, int cache, int B) {
 }
 
 }  // namespace spa
+
+#ifdef SPA_PHASE_PROBE
+// Probe library only: copy / clear the phase stamps of decode_tc_kernel.
+extern "C" int spa_probe_read_tc(void* host, size_t bytes) {
+  if (bytes > sizeof(spa::g_phase_tc)) bytes = sizeof(spa::g_phase_tc);
+  return (int)cudaMemcpyFromSymbol(host, spa::g_phase_tc, bytes);
+}
+extern "C" int spa_probe_clear_tc() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, spa::g_phase_tc) != cudaSuccess) return -1;
+  return (int)cudaMemset(p, 0, sizeof(spa::g_phase_tc));
+}
+#endif

@@ -55,6 +55,36 @@ __device__ __forceinline__ void build_cs(const int32_t* __restrict__ cu, int B, 
   __syncthreads();
 }
 
+// build_cs without a block barrier, for B + 1 <= 64: every warp computes the
+// clamped cumulative lengths (a shuffle prefix maximum) and copies the past
+// lengths itself, and writes them to shared memory (all warps write the same
+// values; each reads back only after its own writes).  The caller loaded
+// cu[lane], cu[lane + 32] (entries <= B, entry 0 unused) and past[lane],
+// past[lane + 32] (entries < B).  Loads still in flight when it runs are not
+// waited for, as a block barrier would.
+__device__ __forceinline__ void build_cs_warp(int B, int T, int32_t* cs, int32_t* past_s, int cu0, int cu1,
+                                              int p0, int p1) {
+  const int lane = threadIdx.x & 31;
+  const int i0 = lane, i1 = lane + 32;
+  int x0 = (i0 == 0 || i0 > B) ? 0 : cu0;
+  int x1 = i1 > B ? 0 : cu1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y0 = __shfl_up_sync(0xffffffffu, x0, o);
+    const int y1 = __shfl_up_sync(0xffffffffu, x1, o);
+    if (lane >= o) {
+      x0 = max(x0, y0);
+      x1 = max(x1, y1);
+    }
+  }
+  x1 = max(x1, __shfl_sync(0xffffffffu, x0, 31));
+  if (i0 <= B) cs[i0] = min(x0, T);
+  if (i1 <= B) cs[i1] = min(x1, T);
+  if (i0 < B) past_s[i0] = p0;
+  if (i1 < B) past_s[i1] = p1;
+  __syncwarp();
+}
+
 // seqlen_k of a request: past + q_len - 1 (past < 0 counts as 0), as int32.
 __device__ __forceinline__ int32_t request_seqlen_k(int past, int q_len) {
   return (int32_t)((long long)max(past, 0) + q_len - 1);

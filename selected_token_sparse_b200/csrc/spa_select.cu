@@ -11,10 +11,10 @@
 //   1. the row's candidate scores (keys 0..bound) are read once, coalesced,
 //      and kept in shared memory as order-preserving 32-bit keys (NaN and
 //      -inf, which are never selected, become 0; -0 becomes +0);
-//   2. when more than top_k keys are eligible, a radix select over four
-//      8-bit digits (a 256-bin shared histogram per digit) finds the exact
-//      k-th largest key T and how many keys equal to T are still to be taken
-//      -- the first ones by index (stable);
+//   2. when more than top_k keys are eligible, a radix select over three
+//      digits of 11, 11 and 10 bits (a 2048-bin shared histogram per digit)
+//      finds the exact k-th largest key T and how many keys equal to T are
+//      still to be taken -- the first ones by index (stable);
 //   3. a compaction over contiguous per-warp segments (ballot / popc counts,
 //      one scan over the 32 warps) writes every kept index at its rank among
 //      the kept ones, so the row comes out in increasing index order;
@@ -40,8 +40,10 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 0x00800000 for eligible keys
 }
 
+constexpr int kSelBins = 2048;   // radix digits of 11, 11 and 10 bits
+
 struct SelShared {
-  uint32_t hist[256];
+  uint32_t hist[kSelBins];
   int warp_gt[kSelWarps];
   int warp_eq[kSelWarps];
   int red[kSelWarps];
@@ -127,42 +129,49 @@ select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const in
     uint32_t prefix = 0u, pmask = 0u;
     int k_rem = top_k;
     bool exact = true;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kSelThreads) sh.hist[i] = 0u;
+    // digits: bits 31..21, 20..10, 9..0 (the first spreads the sign, the
+    // exponent and two mantissa bits over 2048 bins)
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+      const int nbins = (int)dmask + 1;
+      for (int i = tid; i < nbins; i += kSelThreads) sh.hist[i] = 0u;
       __syncthreads();
       for (int j0 = 0; j0 < n; j0 += kSelThreads) {
         const int j = j0 + tid;
         const uint32_t k = j < n ? key_at(j) : 0u;
-        if (k != 0u && (k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+        if (k != 0u && (k & pmask) == prefix) atomicAdd(&sh.hist[(k >> shift) & dmask], 1u);
       }
       __syncthreads();
-      if (warp == 0) {
-        // lane l holds bins 255 - 8l ... 248 - 8l (largest digits first)
-        uint32_t c[8];
-        int sum = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          c[i] = sh.hist[255 - lane * 8 - i];
-          sum += (int)c[i];
-        }
-        int incl = sum;
+      {
+        // block-wide: thread t holds the bins nbins-1-bpt*t ... (largest
+        // digits first); an inclusive scan over the threads finds the bin
+        // where the count of larger keys reaches k_rem
+        const int bpt = nbins / kSelThreads;   // 2 or 1
+        const int b0 = nbins - 1 - tid * bpt;
+        const int c0 = (int)sh.hist[b0];
+        const int c1 = bpt == 2 ? (int)sh.hist[b0 - 1] : 0;
+        int incl = c0 + c1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += y;
         }
-        const int excl = incl - sum;
+        if (lane == 31) sh.red[warp] = incl;
+        __syncthreads();
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += sh.red[w];
+        incl += before;
+        const int excl = incl - c0 - c1;
         if (excl < k_rem && k_rem <= incl) {
-          int cum = excl;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (cum + (int)c[i] >= k_rem) {
-              sh.digit = 255 - lane * 8 - i;
-              sh.above = cum;
-              sh.in_bin = (int)c[i];
-              break;
-            }
-            cum += (int)c[i];
+          if (excl + c0 >= k_rem) {
+            sh.digit = b0;
+            sh.above = excl;
+            sh.in_bin = c0;
+          } else {
+            sh.digit = b0 - 1;
+            sh.above = excl + c0;
+            sh.in_bin = c1;
           }
         }
       }
@@ -170,7 +179,7 @@ select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const in
       const int d = sh.digit;
       k_rem -= sh.above;
       prefix |= (uint32_t)d << shift;
-      pmask |= 255u << shift;
+      pmask |= dmask << shift;
       if (sh.in_bin == k_rem) {   // every key of this bin is kept: no tie to split
         T = prefix - 1u;          // keys with this prefix are >= prefix
         need_eq = 0;

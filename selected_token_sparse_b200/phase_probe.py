@@ -1,4 +1,4 @@
-"""Warm, in-graph phase breakdown of the warp-MMA decode kernel.
+"""Warm, in-graph phase breakdown of the decode kernels (warp-MMA and tcgen05).
 
     python -m selected_token_sparse_b200.phase_probe [--workload NAME] [--lib PATH]
 
@@ -10,7 +10,8 @@ workload over rotating device instances in one CUDA graph, replays it twice
 the graph's last step -- a step that ran right after another one, as in the
 benchmark.  Prints the median / p90 duration of each phase over the CTAs.
 
-Phase stamps of decode_mma_kernel:
+Phase stamps of decode_mma_kernel (those of decode_tc_kernel are listed in
+TC_PHASES below):
   0 entry (before griddepcontrol.wait)   1 predecessor complete (wait released)
   2 unit decoded (metadata, fused scan)  3 Q staged, before the candidates
   4 first candidate chunk resolved       5 first K/V stages issued
@@ -29,6 +30,13 @@ import torch
 
 from . import build, pipeline, spa, workloads as W
 
+TC_PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumulative-length scan)"),
+             (2, 3, "producers: to their first candidates"), (3, 4, "producers: candidates of chunk 0"),
+             (4, 5, "producers: INT8 staging, tile 0 copied, converted, published"),
+             (2, 6, "softmax warps: Q (x key scale, hi / lo) into tensor memory"),
+             (6, 7, "softmax warps: wait for S(0)"), (7, 8, "key loop (S, softmax, PV per tile)"),
+             (8, 9, "epilogue: normalise, write output / partial"), (9, 10, "split merge"),
+             (1, 10, "CTA after the wait"), (0, 10, "CTA incl. the wait")]
 PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumulative-length scan)"),
           (2, 3, "Q rows to shared memory"), (3, 4, "candidates: block ids, row offsets"),
           (4, 5, "issue the first K/V stages"), (5, 6, "key loop (copies, QK, softmax, PV)"),
@@ -38,9 +46,10 @@ PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumul
 
 def run(workload: str, lib_path: str, steps: int = 64):
     lib = spa.load_library(lib_path)
-    lib.spa_probe_read_mma.restype = ctypes.c_int
-    lib.spa_probe_read_mma.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
-    lib.spa_probe_clear_mma.restype = ctypes.c_int
+    for k in ("mma", "tc"):
+        getattr(lib, f"spa_probe_read_{k}").restype = ctypes.c_int
+        getattr(lib, f"spa_probe_read_{k}").argtypes = [ctypes.c_void_p, ctypes.c_size_t]
+        getattr(lib, f"spa_probe_clear_{k}").restype = ctypes.c_int
     spa._LIB = lib
     wl = W.by_name(workload)
     base = pipeline.to_device(wl)
@@ -52,7 +61,11 @@ def run(workload: str, lib_path: str, steps: int = 64):
         d = {k: (v.clone() if k in ("k_cache", "v_cache", "q", "k_new", "v_new", "block_table", "cu_seqlens_q",
                                    "past_seqlens", "selected_idx") else v) for k, v in base.items()}
         insts.append(pipeline.Step(wl, d))
-    assert spa.attention_plan(insts[0].args)["kind"] == 1, "the workload does not run the warp-MMA kernel"
+    kind = spa.attention_plan(insts[0].args)["kind"]
+    assert kind in (1, 3), "the workload runs neither the warp-MMA nor the tcgen05 decode kernel"
+    tag, phases, last, nct = ("mma", PHASES, 9, 8192) if kind == 1 else ("tc", TC_PHASES, 10, 4096)
+    clear = getattr(lib, f"spa_probe_clear_{tag}")
+    read = getattr(lib, f"spa_probe_read_{tag}")
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         for st in insts:
@@ -65,26 +78,27 @@ def run(workload: str, lib_path: str, steps: int = 64):
     for _ in range(2):
         g.replay()
     torch.cuda.synchronize()
-    assert lib.spa_probe_clear_mma() == 0
+    assert clear() == 0
     torch.cuda.synchronize()
     g.replay()
     torch.cuda.synchronize()
-    buf = np.zeros(8192 * 16, dtype=np.uint64)
-    assert lib.spa_probe_read_mma(buf.ctypes.data, buf.nbytes) == 0
-    P = buf.reshape(8192, 16).astype(np.int64)
+    buf = np.zeros(nct * 16, dtype=np.uint64)
+    assert read(buf.ctypes.data, buf.nbytes) == 0
+    P = buf.reshape(nct, 16).astype(np.int64)
     P = P[P[:, 0] > 0]
-    lines = [f"workload {workload}: {len(P)} CTAs of the graph's last step ({steps} steps, {R} instances)",
-             f"CTA span (first entry to last end): {(P[:, 9].max() - P[:, 0].min()) / 1e3:.2f} us; "
-             f"from the first wait release: {(P[:, 9].max() - P[:, 1].min()) / 1e3:.2f} us",
+    lines = [f"workload {workload} ({tag} kernel): {len(P)} CTAs of the graph's last step ({steps} steps, "
+             f"{R} instances)",
+             f"CTA span (first entry to last end): {(P[:, last].max() - P[:, 0].min()) / 1e3:.2f} us; "
+             f"from the first wait release: {(P[:, last].max() - P[:, 1].min()) / 1e3:.2f} us",
              "", "| phase | median us | p90 us | max us |", "|---|---|---|---|"]
-    for a, b, name in PHASES:
+    for a, b, name in phases:
         ok = (P[:, a] > 0) & (P[:, b] > 0)
         if ok.any():
             x = (P[ok, b] - P[ok, a]) / 1e3
             lines.append(f"| {a}->{b} {name} | {np.median(x):.2f} | {np.percentile(x, 90):.2f} | {x.max():.2f} |")
     t0 = P[:, 1].min()
     lines += ["", "stamp offsets from the first wait release (us), percentiles 0 / 50 / 100:"]
-    for k in range(10):
+    for k in range(last + 1):
         ok = P[:, k] > 0
         if ok.any():
             q = np.percentile((P[ok, k] - t0) / 1e3, [0, 50, 100])
