@@ -237,6 +237,311 @@ select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const in
   for (int i = kept + tid; i < sel_width; i += kSelThreads) dst[i] = -1;
 }
 
+// ---------------------------------------------------------------------------
+// Rows that fit shared memory with 16-byte aligned scores.  Every warp owns a
+// contiguous segment of the row (a multiple of 128 keys; each lane takes 4
+// consecutive keys per step, so a warp step is 128 keys in index order).
+// After the histogram of the first digit, only the keys of the threshold bin
+// can change the answer: they go (key, index) to a candidate buffer, and the
+// two remaining digits are resolved on that buffer alone.  The per-warp
+// counts the final write needs are gathered on the way (keys above the bin in
+// the candidate pass, the buffer's keys once the threshold is exact), so the
+// row is read from shared memory three more times after staging: the first
+// histogram, the candidate pass and the write pass.  When the threshold bin
+// is larger than the buffer (e.g. all scores equal), the remaining digits and
+// the counts run over the whole row instead.
+constexpr int kFastStageKeys = 40 * 1024;   // keys staged (160 KB)
+constexpr int kFastCand = 4096;             // candidate buffer entries (32 KB)
+
+struct FastShared {
+  uint32_t hist[kSelBins];
+  int warp_el[kSelWarps];
+  int warp_gt[kSelWarps];
+  int warp_eq[kSelWarps];
+  int red[kSelWarps];
+  int digit, above, in_bin, nbuf;
+};
+
+// inclusive and exclusive warp prefix sums of x
+__device__ __forceinline__ int warp_excl_scan(int x, int lane, int& total) {
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  total = __shfl_sync(0xffffffffu, incl, 31);
+  return incl - x;
+}
+
+// Block-wide search of the histogram bin where the count of larger keys
+// reaches k_rem (bins ordered from the largest digit); results in fs.
+__device__ __forceinline__ void find_digit(FastShared& fs, int nbins, int k_rem, int tid, int lane, int warp) {
+  const int bpt = nbins / kSelThreads;   // 2 or 1
+  const int b0 = nbins - 1 - tid * bpt;
+  const int c0 = (int)fs.hist[b0];
+  const int c1 = bpt == 2 ? (int)fs.hist[b0 - 1] : 0;
+  int incl = c0 + c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) fs.red[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += fs.red[w];
+  incl += before;
+  const int excl = incl - c0 - c1;
+  if (excl < k_rem && k_rem <= incl) {
+    if (excl + c0 >= k_rem) {
+      fs.digit = b0;
+      fs.above = excl;
+      fs.in_bin = c0;
+    } else {
+      fs.digit = b0 - 1;
+      fs.above = excl + c0;
+      fs.in_bin = c1;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, const int32_t* __restrict__ bound,
+                        int top_k, int sel_width, int32_t* __restrict__ out) {
+  extern __shared__ __align__(16) uint32_t fast_smem[];
+  __shared__ FastShared fs;
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long row = blockIdx.x;
+  const int r = (int)(row / H);
+  const float4* src4 = reinterpret_cast<const float4*>(scores + row * (long long)n_keys);
+  int32_t* dst = out + row * (long long)sel_width;
+  const int last = min(bound[r], n_keys - 1);
+  const int n = last + 1 > 0 ? last + 1 : 0;
+  uint32_t* keys = fast_smem;                                           // [n_keys]
+  uint32_t* buf_key = fast_smem + ((n_keys + 3) & ~3);                  // [kFastCand]
+  int* buf_idx = reinterpret_cast<int*>(buf_key + kFastCand);           // [kFastCand]
+  const int seg = (((n + kSelWarps - 1) / kSelWarps) + 127) & ~127;     // keys per warp
+  const int beg = min(warp * seg, n), end = min(beg + seg, n);
+
+  // 1. staging: this warp's segment as 16-byte vectors, 8 in flight per lane
+  int elig = 0;
+  if (beg < end) {   // (a warp past the row's end has an empty segment)
+    const int i_beg = beg >> 2, i_end = (end + 3) >> 2;
+    for (int i0 = i_beg; i0 < i_end; i0 += 8 * 32) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 32 + lane;
+        v[u] = i < i_end ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i >= i_end) continue;
+        const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t k[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          k[e] = 4 * i + e < end ? score_key(x[e]) : 0u;
+          elig += k[e] != 0u;
+        }
+        *reinterpret_cast<uint4*>(keys + 4 * i) = make_uint4(k[0], k[1], k[2], k[3]);
+      }
+    }
+  }
+  elig = __reduce_add_sync(0xffffffffu, elig);
+  if (lane == 0) {
+    fs.warp_el[warp] = elig;
+    fs.warp_gt[warp] = 0;
+    fs.warp_eq[warp] = 0;
+  }
+  if (tid == 0) fs.nbuf = 0;
+  __syncthreads();
+  int E = 0;
+  for (int w = 0; w < kSelWarps; ++w) E += fs.warp_el[w];
+
+  // one warp step: the 4 keys of this lane at step start j0 (index order)
+  auto lane_keys = [&](int j0, uint32_t (&k)[4]) {
+    const int j = j0 + 4 * lane;
+    const uint4 v = j < end ? *reinterpret_cast<const uint4*>(keys + j) : make_uint4(0u, 0u, 0u, 0u);
+    k[0] = v.x; k[1] = v.y; k[2] = v.z; k[3] = v.w;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (j + e >= end) k[e] = 0u;
+  };
+
+  uint32_t T = 0u;
+  int need_eq = 0;
+  if (E > top_k && top_k > 0) {
+    // 2a. histogram of the first digit (bits 31..21)
+    for (int i = tid; i < kSelBins; i += kSelThreads) fs.hist[i] = 0u;
+    __syncthreads();
+    for (int j0 = beg; j0 < end; j0 += 128) {
+      uint32_t k[4];
+      lane_keys(j0, k);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (k[e] != 0u) atomicAdd(&fs.hist[k[e] >> 21], 1u);
+    }
+    __syncthreads();
+    find_digit(fs, kSelBins, top_k, tid, lane, warp);
+    const uint32_t d1 = (uint32_t)fs.digit;
+    int k_rem = top_k - fs.above;
+    const int in1 = fs.in_bin;
+    uint32_t prefix = d1 << 21, pmask = 2047u << 21;
+    bool exact = true;
+    if (in1 == k_rem) {   // the whole bin is kept
+      T = prefix - 1u;
+      exact = false;
+    }
+    const bool use_buf = exact && in1 <= kFastCand;
+    // 2b. candidate pass: per-warp count of keys above the bin; the bin's
+    // keys (key, index) into the buffer
+    int gt_above = 0;
+    for (int j0 = beg; j0 < end; j0 += 128) {
+      uint32_t k[4];
+      lane_keys(j0, k);
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        gt_above += (k[e] != 0u && (k[e] >> 21) > d1) ? 1 : 0;
+        c += (use_buf && k[e] != 0u && (k[e] >> 21) == d1) ? 1 : 0;
+      }
+      if (use_buf) {
+        int tot;
+        const int ex = warp_excl_scan(c, lane, tot);
+        int base = 0;
+        if (lane == 0 && tot > 0) base = atomicAdd(&fs.nbuf, tot);
+        base = __shfl_sync(0xffffffffu, base, 0);
+        int at = base + ex;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (k[e] != 0u && (k[e] >> 21) == d1) {
+            buf_key[at] = k[e];
+            buf_idx[at] = j0 + 4 * lane + e;
+            ++at;
+          }
+      }
+    }
+    gt_above = __reduce_add_sync(0xffffffffu, gt_above);
+    __syncthreads();
+    const int nb = use_buf ? fs.nbuf : 0;
+    // 2c. the remaining digits (bits 20..10, 9..0) on the buffer, or on the
+    // whole row when the bin did not fit
+    for (int pass = 1; pass < 3 && exact; ++pass) {
+      const int shift = pass == 1 ? 10 : 0;
+      const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+      const int nbins = (int)dmask + 1;
+      for (int i = tid; i < nbins; i += kSelThreads) fs.hist[i] = 0u;
+      __syncthreads();
+      if (use_buf) {
+        for (int i = tid; i < nb; i += kSelThreads) {
+          const uint32_t k = buf_key[i];
+          if ((k & pmask) == prefix) atomicAdd(&fs.hist[(k >> shift) & dmask], 1u);
+        }
+      } else {
+        for (int j0 = beg; j0 < end; j0 += 128) {
+          uint32_t k[4];
+          lane_keys(j0, k);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (k[e] != 0u && (k[e] & pmask) == prefix) atomicAdd(&fs.hist[(k[e] >> shift) & dmask], 1u);
+        }
+      }
+      __syncthreads();
+      find_digit(fs, nbins, k_rem, tid, lane, warp);
+      k_rem -= fs.above;
+      prefix |= (uint32_t)fs.digit << shift;
+      pmask |= dmask << shift;
+      if (fs.in_bin == k_rem) {
+        T = prefix - 1u;
+        exact = false;
+      }
+      __syncthreads();   // fs is rewritten by the next pass
+    }
+    if (exact) {
+      T = prefix;
+      need_eq = k_rem;
+    }
+    // 2d. per-warp counts of kept-above (> T) and equal (== T) keys
+    if (use_buf) {
+      if (lane == 0) fs.warp_gt[warp] = gt_above;
+      __syncthreads();
+      for (int i = tid; i < nb; i += kSelThreads) {
+        const uint32_t k = buf_key[i];
+        const int w = buf_idx[i] / seg;
+        if (k > T) atomicAdd(&fs.warp_gt[w], 1);
+        else if (need_eq > 0 && k == T) atomicAdd(&fs.warp_eq[w], 1);
+      }
+    } else {
+      int g = 0, q = 0;
+      for (int j0 = beg; j0 < end; j0 += 128) {
+        uint32_t k[4];
+        lane_keys(j0, k);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          g += k[e] > T ? 1 : 0;
+          q += (need_eq > 0 && k[e] == T) ? 1 : 0;
+        }
+      }
+      g = __reduce_add_sync(0xffffffffu, g);
+      q = __reduce_add_sync(0xffffffffu, q);
+      if (lane == 0) {
+        fs.warp_gt[warp] = g;
+        fs.warp_eq[warp] = q;
+      }
+    }
+    __syncthreads();
+  } else {
+    // every eligible key is kept (or none, top_k = 0): keys > 0
+    if (lane == 0) fs.warp_gt[warp] = top_k > 0 ? fs.warp_el[warp] : 0;
+    __syncthreads();
+  }
+  const int kept = E < top_k ? E : top_k;
+
+  // 3. write pass: kept indices in increasing order
+  if (kept > 0) {
+    int pos = 0, eq_seen = 0;
+    for (int w = 0; w < warp; ++w) {
+      pos += fs.warp_gt[w];
+      eq_seen += fs.warp_eq[w];
+    }
+    pos += min(eq_seen, need_eq);
+    for (int j0 = beg; j0 < end; j0 += 128) {
+      uint32_t k[4];
+      lane_keys(j0, k);
+      int nq = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) nq += (need_eq > 0 && k[e] == T) ? 1 : 0;
+      int q_tot;
+      const int q_ex = warp_excl_scan(nq, lane, q_tot);
+      bool take[4];
+      int nt = 0, qi = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool is_eq = need_eq > 0 && k[e] == T;
+        take[e] = k[e] > T || (is_eq && eq_seen + q_ex + qi < need_eq);
+        qi += is_eq ? 1 : 0;
+        nt += take[e] ? 1 : 0;
+      }
+      int t_tot;
+      const int t_ex = warp_excl_scan(nt, lane, t_tot);
+      int at = pos + t_ex;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (take[e]) dst[at++] = j0 + 4 * lane + e;
+      pos += t_tot;
+      eq_seen += q_tot;
+    }
+  }
+  // 4. padding up to the row's capacity
+  for (int i = kept + tid; i < sel_width; i += kSelThreads) dst[i] = -1;
+}
+
 }  // namespace spa
 
 using namespace spa;
@@ -251,6 +556,17 @@ extern "C" int spa_select_topk(const float* scores, int32_t R, int32_t H, int32_
   const int staged = n_keys <= kSelStageKeys ? 1 : 0;
   // whole-row 16-byte vectors: every row starts 16-byte aligned
   const int vec = (n_keys % 4 == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) ? 1 : 0;
+  if (vec && n_keys > 0 && n_keys <= kFastStageKeys) {
+    const size_t fsm = (size_t)n_keys * 4 + (size_t)kFastCand * 8;
+    if (fsm > 48 * 1024 &&
+        cudaFuncSetAttribute(select_topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kFastStageKeys * 4 + kFastCand * 8) != cudaSuccess)
+      return check_launch_public();
+    const int rc = launch_pdl(select_topk_fast_kernel, dim3((unsigned)(R * H)), dim3(kSelThreads), fsm,
+                              (cudaStream_t)stream, scores, H, n_keys, bound, top_k, sel_width, selected_idx);
+    if (rc != SPA_OK) return rc;
+    return check_launch_public();
+  }
   const size_t smem = staged ? (size_t)(n_keys > 0 ? ((n_keys + 3) & ~3) : 4) * sizeof(uint32_t) : 0;
   if (staged && smem > 48 * 1024) {
     if (cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
