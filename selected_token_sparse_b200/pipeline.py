@@ -92,6 +92,10 @@ class Step:
                                        out=self.out, lse=self.lse, num_splits=num_splits,
                                        status=self.status, **self.kw)
         self.workspace = spa.new_workspace(spa.workspace_size(self.args), dev)
+        self._bound = None
+        if mode == "step" and not self.pro:
+            self._bound = spa.BoundStep(self.args, d["past_seqlens"], d["k_new"], d["v_new"],
+                                        self.meta["slot_mapping"], self.workspace)
 
     def launches(self) -> int:
         """Kernel launches one call makes."""
@@ -108,8 +112,7 @@ class Step:
             spa.run_attention(self.args, self.workspace)
             return self.out
         if self.mode == "step":
-            spa.run_prepare_append_attention(self.args, d["past_seqlens"], d["k_new"], d["v_new"],
-                                             self.meta["slot_mapping"], self.workspace)
+            self._bound()   # spa_prepare_append_attention, arguments marshalled once
             return self.out
         if self.mode == "prepare_append":
             spa.prepare_append_kv(d["cu_seqlens_q"], d["past_seqlens"], d["block_table"],

@@ -355,6 +355,29 @@ def run_prepare_append_attention(args: AttentionArgs, past_seqlens: torch.Tensor
     _check(rc, "spa_prepare_append_attention")
 
 
+class BoundStep:
+    """spa_prepare_append_attention with every argument marshalled once: each
+    call passes the prepared pointers and the current stream, nothing else.
+    The tensors the arguments point at must stay alive and in place."""
+
+    def __init__(self, args: AttentionArgs, past_seqlens: torch.Tensor, k_new: torch.Tensor,
+                 v_new: torch.Tensor, slot_mapping: torch.Tensor, workspace: Optional[torch.Tensor]):
+        need = workspace_size(args)
+        if need and (workspace is None or workspace.numel() < need):
+            raise SpaError(SPA_ERR_WORKSPACE, "spa_prepare_append_attention")
+        self._fn = lib().spa_prepare_append_attention
+        self._args = ctypes.byref(args)
+        self._ptrs = (_ptr(past_seqlens), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping),
+                      _ptr(workspace) if need else None, need)
+        self._dev = k_new.device
+        self._keep = (args, past_seqlens, k_new, v_new, slot_mapping, workspace)
+
+    def __call__(self) -> None:
+        rc = self._fn(self._args, *self._ptrs, torch.cuda.current_stream(self._dev).cuda_stream)
+        if rc != SPA_OK:
+            raise SpaError(rc, "spa_prepare_append_attention")
+
+
 def prepare_append_attention_launches(args: AttentionArgs) -> int:
     """Kernel launches spa_prepare_append_attention makes for these arguments (1 or 2)."""
     rc = int(lib().spa_prepare_append_attention_launches(ctypes.byref(args)))
