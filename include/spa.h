@@ -258,8 +258,8 @@ typedef struct spa_attention_args {
 } spa_attention_args_t;
 
 /* Bytes of workspace spa_attention needs for these arguments (0 if none: one
-   split per unit, or splits that merge inside a thread-block cluster).
-   Returns 0 as well for invalid arguments; spa_attention then reports the error. */
+   split per unit).  Returns 0 as well for invalid arguments; spa_attention
+   then reports the error. */
 size_t spa_attention_workspace_size(const spa_attention_args_t* a);
 
 /*
@@ -275,14 +275,15 @@ size_t spa_attention_workspace_size(const spa_attention_args_t* a);
  * FP32 partial states are merged by log-sum-exp; the result does not depend
  * on num_splits beyond rounding.
  * workspace: device buffer of at least spa_attention_workspace_size() bytes,
- * 256-byte aligned; it may be NULL when the size is 0.  It must be zero-filled
- * before its first use: it holds per-unit split tickets that every call
- * leaves at zero again (the partial states around them need no
- * initialisation).  Calls that share a workspace must be ordered on one
- * stream.  The whole operation is one kernel launch: on the tensor-core
- * decode kernels the (at most 8) splits of a unit form one thread-block
- * cluster and merge through distributed shared memory; otherwise the last
- * CTA to finish a unit's splits merges them from the workspace.
+ * 256-byte aligned; it may be NULL when the size is 0.  It holds the splits'
+ * FP32 partial states (no initialisation needed) and, for plans that merge by
+ * ticket, per-unit split tickets: those must be zero before the first use and
+ * every call leaves them at zero again, so zero-fill a new workspace.  Calls
+ * that share a workspace must be ordered on one stream.  The whole operation
+ * is one kernel launch: on the tensor-core decode kernels the (at most 8)
+ * splits of a unit form one thread-block cluster, write their partial states
+ * to the workspace, pass a cluster barrier and merge a share of the rows
+ * each; otherwise the last CTA to finish a unit's splits merges them.
  */
 int spa_attention(const spa_attention_args_t* a, void* workspace, size_t workspace_bytes,
                   spa_stream_t stream);
@@ -421,8 +422,8 @@ int spa_prepare_qkv_append(const spa_qkv_args_t* a, spa_stream_t stream);
  * and no allocating routine.
  *   - A call whose plan needs more scratch than SPA_NOALLOC_SCRATCH_BYTES
  *     (spa_attention_workspace_size() of the same arguments) returns
- *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.  Plans whose splits merge
- *     inside a thread-block cluster need no scratch at all.
+ *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.  Plans with one split per
+ *     unit need no scratch at all.
  *   - The first call on each device resolves the array's device address (with
  *     that device current); make that first call before any stream capture.
  *     Every later call made outside a capture resolves it again; a call made

@@ -142,16 +142,16 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   pl->num_splits = (int)splits;
   pl->split_len = (int)std::min<long long>(per_tiles * KT, 0x7fffffffLL);
   pl->units = (int)units;
-  // the splits of a unit merge through distributed shared memory when they
-  // fit one cluster (tensor-core decode kernels) and need no workspace;
-  // otherwise through the workspace, where the CTA that finishes last merges
+  // split partial states go through the workspace; the splits of a unit
+  // merge after a cluster barrier when they fit one cluster (tensor-core
+  // decode kernels), otherwise the CTA that finishes last merges (tickets)
   pl->cluster_merge = (pl->kind == kPlanTc || pl->kind == kPlanMma) && pl->num_splits > 1 &&
                       pl->num_splits <= 8;
-  if (pl->num_splits > 1 && !pl->cluster_merge) {
+  if (pl->num_splits > 1) {
     const size_t rows = (size_t)a->T * a->H_q;
     pl->ws_acc_bytes = align256(rows * a->D * sizeof(float) * pl->num_splits);
     pl->ws_ml_bytes = align256(rows * 2 * sizeof(float) * pl->num_splits);
-    pl->ws_count_bytes = align256((size_t)units * sizeof(int));
+    if (!pl->cluster_merge) pl->ws_count_bytes = align256((size_t)units * sizeof(int));
   }
   if (pl->kind == kPlanScalar &&
       scalar_smem_bytes(a->D, pl->max_rows, pl->max_q) > 200 * 1024)
@@ -205,10 +205,11 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   p->split_len = pl.split_len;
   p->status = a->status;
   p->cluster_merge = pl.cluster_merge;
-  if (pl.num_splits > 1 && !pl.cluster_merge) {
+  if (pl.num_splits > 1) {
     p->ws_acc = static_cast<float*>(ws);
     p->ws_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.ws_acc_bytes);
-    p->ws_count = reinterpret_cast<int*>(static_cast<char*>(ws) + pl.ws_acc_bytes + pl.ws_ml_bytes);
+    if (!pl.cluster_merge)
+      p->ws_count = reinterpret_cast<int*>(static_cast<char*>(ws) + pl.ws_acc_bytes + pl.ws_ml_bytes);
   }
 }
 

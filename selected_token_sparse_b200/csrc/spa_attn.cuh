@@ -389,48 +389,49 @@ __device__ __forceinline__ void merge_rows(const AttnParams& p, int t0, int nq, 
   }
 }
 
-// Split merge through distributed shared memory.  The num_splits CTAs of a
-// unit form one cluster (rank = split); each has left its partial state at
-// the same shared-memory offsets: o [rows][D + 4] fp32 (row stride D + 4) and
-// (m, l, sink * log2(e), 0) [rows][4], log2 units.  After a cluster barrier, CTA k merges rows
-// k, k + S, k + 2S, ... with the sink as merge_rows does, in one pass: each
+// Split merge inside a thread-block cluster.  The num_splits CTAs of a unit
+// form one cluster (rank = split).  Each has written its partial state of the
+// unit's rows to the workspace, as the ticket merge's splits do (ws_acc
+// [split][T * H_q][D], ws_ml [split][T * H_q][2], log2 units), and passed a
+// cluster barrier (release / acquire) after that; then CTA k merges rows k,
+// k + S, k + 2S, ... with the sink as merge_rows does, in one pass: each
 // thread takes 4 output columns of a row, reads every split's (m, l) and
-// partial columns from the peers' shared memory at once, and forms the
-// weights itself.  The caller ends with another cluster barrier so that no
-// CTA leaves while its state is being read.
+// partial columns from L2 at once, and forms the weights itself.  No CTA
+// reads another's shared memory, so none waits for the others to leave.
+// (Pulling the partial states from the peers' shared memory instead costs a
+// second cluster barrier and moves them over the SM-to-SM network, which
+// measured slower than L2 for these sizes.)
 constexpr int kClusterMaxSplits = 8;
 
-// SMAX bounds the split count; IPT items of a thread have their peer loads in
-// flight together (a peer load is a round trip through the cluster network).
+// SMAX bounds the split count; IPT items of a thread have their loads in
+// flight together.
 template <typename ActT, int D, int SMAX, int IPT>
-__device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, int nq, int h_kv,
-                                                   const float* part_o, const float* part_ml) {
-  constexpr int C4 = D / 4, PS = D + 4;
+__device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, int nq, int h_kv) {
+  constexpr int C4 = D / 4;
   const int S = p.num_splits, k = (int)cluster_rank();
   const int R = nq * p.G;
+  const long long stride = (long long)p.T * p.H_q;
   const int mine = R > k ? (R - k + S - 1) / S : 0;   // rows k, k + S, ...
   const int n_items = mine * C4;
   for (int base = threadIdx.x; base < n_items; base += IPT * blockDim.x) {
     float2 ml[IPT][SMAX];
     float4 a[IPT][SMAX];
     float sink2[IPT];
+    long long rw[IPT];
 #pragma unroll
     for (int t = 0; t < IPT; ++t) {
       const int it = base + t * blockDim.x;
       const int r = k + (it / C4) * S, c = (it % C4) * 4;
-      sink2[t] = it < n_items ? part_ml[4 * r + 2] : -INFINITY;   // the same in every split
+      const int h = h_kv * p.G + r % p.G;
+      rw[t] = (long long)(t0 + r / p.G) * p.H_q + h;
+      sink2[t] = (p.sinks && it < n_items) ? __ldg(p.sinks + h) * kLog2e : -INFINITY;
 #pragma unroll
       for (int s = 0; s < SMAX; ++s) {
         ml[t][s] = make_float2(-INFINITY, 0.f);
         a[t][s] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (s < S && it < n_items) {
-          if (s == k) {   // this CTA's own state: a local read
-            ml[t][s] = *reinterpret_cast<const float2*>(part_ml + 4 * r);
-            a[t][s] = *reinterpret_cast<const float4*>(part_o + r * PS + c);
-          } else {
-            ml[t][s] = ld_peer2(peer_smem(part_ml + 4 * r, s));
-            a[t][s] = ld_peer4(peer_smem(part_o + r * PS + c, s));
-          }
+          ml[t][s] = __ldcg(reinterpret_cast<const float2*>(p.ws_ml + (s * stride + rw[t]) * 2));
+          a[t][s] = __ldcg(reinterpret_cast<const float4*>(p.ws_acc + (s * stride + rw[t]) * D + c));
         }
       }
     }
@@ -438,8 +439,7 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, 
     for (int t = 0; t < IPT; ++t) {
       const int it = base + t * blockDim.x;
       if (it >= n_items) continue;
-      const int r = k + (it / C4) * S, c = (it % C4) * 4;
-      const long long row = (long long)(t0 + r / p.G) * p.H_q + h_kv * p.G + r % p.G;
+      const int c = (it % C4) * 4;
       float M = sink2[t];
 #pragma unroll
       for (int s = 0; s < SMAX; ++s) M = fmaxf(M, ml[t][s].x);
@@ -459,8 +459,8 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnParams& p, int t0, 
         inv = 1.0f / Lsum;
         lse = (M + log2f(Lsum)) * kLn2;
       }
-      store_out4<ActT>(p, row * D + c, o.x * inv, o.y * inv, o.z * inv, o.w * inv);
-      if (c == 0 && p.lse) p.lse[row] = lse;
+      store_out4<ActT>(p, rw[t] * D + c, o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      if (c == 0 && p.lse) p.lse[rw[t]] = lse;
     }
   }
 }

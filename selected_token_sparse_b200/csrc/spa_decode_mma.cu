@@ -137,13 +137,8 @@ struct MmaCfg {
   // the cross-warp merge reuses the K/V ring once every tile is consumed
   static constexpr int OFF_RED = OFF_RAW;
   static constexpr int RED_BYTES = (KW > 1) ? NW * 32 * (D / 2 + 4) * 4 : 0;
-  // cluster split merge: the CTA's partial o [ROWS][D + 4] and (m, l, sink,
-  // 0) [ROWS][4], fp32, after the cross-warp buffer
-  static constexpr int OFF_PART = OFF_RED + RED_BYTES;
-  static constexpr int PART_ML = OFF_PART + ROWS * (D + 4) * 4;
-  static constexpr int END_PART = PART_ML + ROWS * 16;
-  static constexpr int SMEM = (END_PART > END) ? END_PART : END;
-  static_assert(END_PART <= OFF_KPOS, "merge buffers must not reach the scales / positions");
+  static constexpr int SMEM = END;
+  static_assert(OFF_RED + RED_BYTES <= OFF_KPOS, "the merge buffer must not reach the scales / positions");
 };
 
 // FUSED: one launch of the whole step (16-bit caches).  Every CTA rebuilds
@@ -168,6 +163,17 @@ decode_mma_kernel(const AttnParams p) {
   pdl_wait();
   pdl_trigger();
   SPA_PHASE(1);
+
+  // Issued first: the lengths every warp scans by itself (fused step, B + 1 <= 64:
+  // build_cs_warp, no block barrier that would wait for the loads in flight).
+  const bool warp_scan = FUSED && p.B + 1 <= 64;
+  int pc0 = 0, pc1 = 0, pp0 = 0, pp1 = 0;
+  if (warp_scan) {
+    pc0 = (lane >= 1 && lane <= p.B) ? ld_early(p.cu + lane) : 0;
+    pc1 = lane + 32 <= p.B ? ld_early(p.cu + lane + 32) : 0;
+    pp0 = lane < p.B ? ld_early(p.past + lane) : 0;
+    pp1 = lane + 32 < p.B ? ld_early(p.past + lane + 32) : 0;
+  }
 
   // Q rows of the unit in 16-byte chunks (row r = token r / G, head r % G).
   // A per-token unit knows its token from the block index, so its loads are
@@ -222,7 +228,8 @@ decode_mma_kernel(const AttnParams p) {
   if constexpr (FUSED) {
     cs_s = reinterpret_cast<int32_t*>(smem + C::SMEM);
     past_s = cs_s + p.B + 1;
-    build_cs<NT>(p.cu, p.B, p.T, cs_s, p.past, past_s);   // ends with a block barrier
+    if (warp_scan) build_cs_warp(p.B, p.T, cs_s, past_s, pc0, pc1, pp0, pp1);
+    else build_cs<NT>(p.cu, p.B, p.T, cs_s, p.past, past_s);   // ends with a block barrier
     has_rows = decode_unit_with(p, FusedMeta{p.cu, cs_s, past_s, p.B}, blockIdx.x, U);
     if (has_rows) {
       U.new_lo = max(past_s[U.b], 0);
@@ -417,6 +424,16 @@ decode_mma_kernel(const AttnParams p) {
         if (app_t >= 0 && app_thread) app_data = fused_load_row_vector<CacheT>(p, app_t, h_kv, tid, NV);
       }
       if (app_t >= 0) app_tl = token_meta_load(app_t, cs_s, p.B, past_s, p.block_table, p.MB, p.bs);
+      // steps 1-2 of the first token while this split's K/V copies are in
+      // flight: no CTA reads the cache rows it writes (keys at this step's
+      // positions are read from k_new / v_new)
+      if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits);
+      if (app_t >= 0) {
+        int tb = 0;
+        const TokenMeta m = token_meta_finish(app_tl, p.MB, p.bs, p.NB, tb);
+        fused_token_outputs(p, app_t, h_kv, m, tb, bits);
+        if (app_thread && m.slot >= 0) fused_store_row_vector<CacheT>(p, m.slot, h_kv, tid, NV, app_data);
+      }
     }
   }
   __syncthreads();
@@ -433,7 +450,7 @@ decode_mma_kernel(const AttnParams p) {
   const int r1 = r0 + 8;
   // the epilogue's sink logits, in flight from here
   float sink_raw[2] = {-INFINITY, -INFINITY};
-  if (p.sinks && (p.num_splits == 1 || p.cluster_merge)) {
+  if (p.sinks && p.num_splits == 1) {
     if (r0 < R) sink_raw[0] = ld_early(p.sinks + h_kv * G + r0 % G);
     if (r1 < R) sink_raw[1] = ld_early(p.sinks + h_kv * G + r1 % G);
   }
@@ -709,16 +726,6 @@ decode_mma_kernel(const AttnParams p) {
           *reinterpret_cast<uint32_t*>(out + d) = pack2<ActT>(fo[nn][hrow * 2 + 0] * f, fo[nn][hrow * 2 + 1] * f);
       }
       if (wk == 0 && (lane & 3) == 0 && p.lse) p.lse[row] = lse;
-    } else if (p.cluster_merge) {
-      float* po = reinterpret_cast<float*>(smem + C::OFF_PART) + r * (D + 4);
-#pragma unroll
-      for (int nn = 0; nn < NPW; ++nn) {
-        const int d = (n_lo + nn) * 8 + (lane & 3) * 2;
-        *reinterpret_cast<float2*>(po + d) = make_float2(fo[nn][hrow * 2], fo[nn][hrow * 2 + 1]);
-      }
-      if (wk == 0 && (lane & 3) == 0)
-        *reinterpret_cast<float4*>(smem + C::PART_ML + r * 16) =
-            make_float4(mf[hrow], lf[hrow], p.sinks ? sink_raw[hrow] * kLog2e : -INFINITY, 0.f);
     } else {
       const long long wrow = (long long)split * p.T * p.H_q + row;
       float* acc = p.ws_acc + wrow * D;
@@ -735,34 +742,24 @@ decode_mma_kernel(const AttnParams p) {
   }
 
   SPA_PHASE(7);
-  // fused step: the rest of steps 1-2 (off the attention's critical path)
+  // fused step: a request-grouped unit's further tokens (steps 1-2)
   if constexpr (FUSED) {
-    if (split == 0) {
-      if (blockIdx.x == 0) fused_request_outputs(p, cs_s, past_s, bits);
-      if (app_t >= 0) {
-        int tb = 0;
-        const TokenMeta m = token_meta_finish(app_tl, p.MB, p.bs, p.NB, tb);
-        fused_token_outputs(p, app_t, h_kv, m, tb, bits);
-        if (app_thread && m.slot >= 0) fused_store_row_vector<CacheT>(p, m.slot, h_kv, tid, NV, app_data);
-        // a request-grouped unit's further tokens
-        if (p.group_by_request) {
-          const int b = blockIdx.x / p.H_kv;
-          fused_append_tokens<CacheT>(p, cs_s, past_s, app_t + 1, cs_s[b + 1], h_kv, bits);
-        }
-      }
+    if (split == 0 && app_t >= 0 && p.group_by_request) {
+      const int b = blockIdx.x / p.H_kv;
+      fused_append_tokens<CacheT>(p, cs_s, past_s, app_t + 1, cs_s[b + 1], h_kv, bits);
     }
   }
   flag(p.status, bits);
   SPA_PHASE(8);
   if (p.num_splits > 1) {
     if (p.cluster_merge) {
-      // the unit's splits are one cluster: merge through distributed shared memory
+      // the unit's splits are one cluster: once every split's partial state
+      // is in the workspace, each CTA merges a share of the rows
       cluster_sync();
-      const float* po = reinterpret_cast<const float*>(smem + C::OFF_PART);
-      const float* pml = reinterpret_cast<const float*>(smem + C::PART_ML);
-      if (p.num_splits <= 4) cluster_merge_rows<ActT, D, 4, 2>(p, t0, nq, h_kv, po, pml);
-      else cluster_merge_rows<ActT, D, kClusterMaxSplits, 1>(p, t0, nq, h_kv, po, pml);
-      cluster_sync();
+      SPA_PHASE(10);
+      if (p.num_splits <= 4) cluster_merge_rows<ActT, D, 4, 2>(p, t0, nq, h_kv);
+      else cluster_merge_rows<ActT, D, kClusterMaxSplits, 1>(p, t0, nq, h_kv);
+      SPA_PHASE(11);
     } else {
       finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
     }

@@ -97,12 +97,7 @@ struct TcCfg {
   static constexpr int OFF_CONV = 0;                                   // [stage][K, V]
   static constexpr int OFF_RAW = OFF_CONV + kTcStages * 2 * KTILE;     // INT8: [raw stage][K, V]
   static constexpr int END_RING = OFF_RAW + RAW_ST * 2 * RAW;
-  // cluster split merge: partial o [128][D + 4] and (m, l, sink, 0) [128][4],
-  // fp32, over the rings once every tile is consumed
-  static constexpr int OFF_PART = 0;
-  static constexpr int PART_ML = OFF_PART + 128 * (D + 4) * 4;
-  static constexpr int END_PART = PART_ML + 128 * 4 * 4;
-  static constexpr int OFF_KVIS = END_RING > END_PART ? END_RING : END_PART;  // [stage][64] row intervals
+  static constexpr int OFF_KVIS = END_RING;                          // [stage][64] row intervals
   static constexpr int OFF_TVIS = OFF_KVIS + kTcStages * kTcKT * 8;           // [stage] tile seen by every row
   static constexpr int OFF_CAND = OFF_TVIS + 16;                    // [2 chunks] offsets + positions
   static constexpr int OFF_SCALE = OFF_CAND + 2 * kTcCand * 12;     // INT8: ks, vs
@@ -329,7 +324,7 @@ decode_tc_kernel(const AttnParams p) {
       for (int k = 0; k < QV; ++k) qv[k] = src[k];
     }
     // the epilogue's (or the cluster merge's) sink logit of row `row`
-    if (p.sinks && (p.num_splits == 1 || p.cluster_merge) && row < R) sink_raw = ld_early(p.sinks + h_kv * G + row % G);
+    if (p.sinks && p.num_splits == 1 && row < R) sink_raw = ld_early(p.sinks + h_kv * G + row % G);
   }
 
   if (producer) {
@@ -529,6 +524,7 @@ decode_tc_kernel(const AttnParams p) {
         }
       }
     }
+    SPA_PHASE_T(13, kTcCons);
     bar_sync(kTcBarProd, kTcProd);
     if constexpr (C::kInt8) {
       if (ntiles > 0) issue(0);
@@ -543,8 +539,10 @@ decode_tc_kernel(const AttnParams p) {
           issue(j + 1);   // raw stage (j+1) & 1 held tile j - 1, converted already
         }
         cp_async_commit();
+        if (j == 0) SPA_PHASE_T(14, kTcCons);
         cp_async_wait<1>();
         bar_sync(kTcBarProd, kTcProd);   // tile j's raw rows landed (every producer's copies)
+        if (j == 0) SPA_PHASE_T(15, kTcCons);
         wait_empty(j);
         if (bar_red_or(!ok, kTcBarProd, kTcProd)) {
           ok = false;
@@ -878,10 +876,6 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) out[e / 8] = pack8<ActT>(ov + e);
         }
-      } else if (p.cluster_merge) {
-        float* po = reinterpret_cast<float*>(smem + C::OFF_PART) + row * (D + 4) + col;
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(po + e) = make_float4(ov[e], ov[e + 1], ov[e + 2], ov[e + 3]);
       } else {
         float* acc = p.ws_acc + ((long long)split * p.T * p.H_q + orow) * D + col;
 #pragma unroll
@@ -891,9 +885,6 @@ decode_tc_kernel(const AttnParams p) {
     if (mine) {
       if (p.num_splits == 1) {
         if (p.lse) p.lse[orow] = lse;
-      } else if (p.cluster_merge) {
-        *reinterpret_cast<float4*>(smem + C::PART_ML + row * 16) =
-            make_float4(m_used, l_sum, p.sinks ? sink_raw * kLog2e : -INFINITY, 0.f);
       } else {
         const long long wrow = (long long)split * p.T * p.H_q + orow;
         p.ws_ml[wrow * 2 + 0] = m_used;
@@ -911,12 +902,13 @@ decode_tc_kernel(const AttnParams p) {
   }
   if (p.num_splits > 1) {
     if (p.cluster_merge) {
+      // every split's partial state is in the workspace once the cluster
+      // barrier passes; each CTA merges a share of the rows
       cluster_sync();
-      const float* po = reinterpret_cast<const float*>(smem + C::OFF_PART);
-      const float* pml = reinterpret_cast<const float*>(smem + C::PART_ML);
-      if (p.num_splits <= 4) cluster_merge_rows<ActT, D, 4, 3>(p, t0, nq, h_kv, po, pml);
-      else cluster_merge_rows<ActT, D, kClusterMaxSplits, 1>(p, t0, nq, h_kv, po, pml);
-      cluster_sync();
+      SPA_PHASE_T(11, 0);
+      if (p.num_splits <= 4) cluster_merge_rows<ActT, D, 4, 3>(p, t0, nq, h_kv);
+      else cluster_merge_rows<ActT, D, kClusterMaxSplits, 1>(p, t0, nq, h_kv);
+      SPA_PHASE_T(12, 0);
     } else {
       finish_split<ActT, D>(p, blockIdx.x, t0, nq, h_kv, &last_flag);
     }

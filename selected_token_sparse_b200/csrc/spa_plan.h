@@ -17,7 +17,7 @@ struct Plan {
   int num_splits;
   int split_len;
   int units;
-  int cluster_merge;  // splits of a unit merge in a thread-block cluster (no workspace)
+  int cluster_merge;  // splits of a unit merge after a cluster barrier (no tickets)
   size_t ws_acc_bytes;
   size_t ws_ml_bytes;
   size_t ws_count_bytes;

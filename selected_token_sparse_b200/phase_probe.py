@@ -17,6 +17,7 @@ TC_PHASES below):
   4 first candidate chunk resolved       5 first K/V stages issued
   6 key loop done (all copies landed)    7 output / partial state written
   8 fused metadata + append tail done    9 split merge done (CTA end)
+  10 cluster barrier passed               11 merged rows written (cluster merge)
 """
 from __future__ import annotations
 
@@ -33,18 +34,24 @@ from . import build, pipeline, spa, workloads as W
 TC_PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumulative-length scan)"),
              (2, 3, "producers: to their first candidates"), (3, 4, "producers: candidates of chunk 0"),
              (4, 5, "producers: INT8 staging, tile 0 copied, converted, published"),
+             (4, 13, "producers: this step's rows quantised (INT8) and appended"),
+             (13, 14, "producers: copies of tiles 0-1 issued"), (14, 15, "producers: tile 0 landed"),
+             (15, 5, "producers: tile 0 converted and published"),
              (2, 6, "softmax warps: Q (x key scale, hi / lo) into tensor memory"),
              (6, 7, "softmax warps: wait for S(0)"), (7, 8, "key loop (S, softmax, PV per tile)"),
              (8, 9, "epilogue: normalise, write output / partial"), (9, 10, "split merge"),
+             (9, 11, "merge: cluster barrier"), (11, 12, "merge: rows from the workspace"),
              (1, 10, "CTA after the wait"), (0, 10, "CTA incl. the wait")]
 PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumulative-length scan)"),
           (2, 3, "Q rows to shared memory"), (3, 4, "candidates: block ids, row offsets"),
           (4, 5, "issue the first K/V stages"), (5, 6, "key loop (copies, QK, softmax, PV)"),
           (6, 7, "epilogue: normalise, write output"), (7, 8, "fused metadata / append tail"),
-          (8, 9, "split merge"), (1, 9, "CTA after the wait"), (0, 9, "CTA incl. the wait")]
+          (8, 9, "split merge"), (8, 10, "merge: cluster barrier"),
+          (10, 11, "merge: rows from the workspace"),
+          (1, 9, "CTA after the wait"), (0, 9, "CTA incl. the wait")]
 
 
-def run(workload: str, lib_path: str, steps: int = 64):
+def run(workload: str, lib_path: str, steps: int = 64, raw: str = None):
     lib = spa.load_library(lib_path)
     for k in ("mma", "tc"):
         getattr(lib, f"spa_probe_read_{k}").restype = ctypes.c_int
@@ -85,6 +92,8 @@ def run(workload: str, lib_path: str, steps: int = 64):
     buf = np.zeros(nct * 16, dtype=np.uint64)
     assert read(buf.ctypes.data, buf.nbytes) == 0
     P = buf.reshape(nct, 16).astype(np.int64)
+    if raw:   # every CTA's stamps, indexed blockIdx.y * gridDim.x + blockIdx.x (0: not stamped)
+        np.save(raw, P)
     P = P[P[:, 0] > 0]
     lines = [f"workload {workload} ({tag} kernel): {len(P)} CTAs of the graph's last step ({steps} steps, "
              f"{R} instances)",
@@ -111,9 +120,10 @@ def main():
     ap.add_argument("--workload", default="gptoss_paged_decode_f16")
     ap.add_argument("--lib", default=None, help="probe library (default: build it with build.py --probe)")
     ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--raw", default=None, help="also save the raw stamps (.npy)")
     a = ap.parse_args()
     lib = a.lib or (build.PROBE_LIB if os.path.exists(build.PROBE_LIB) else build.build_probe())
-    print(run(a.workload, lib, a.steps))
+    print(run(a.workload, lib, a.steps, a.raw))
 
 
 if __name__ == "__main__":

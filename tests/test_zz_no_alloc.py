@@ -26,13 +26,15 @@ def _entry(lib):
     return fn
 
 
-# Cases whose partial states travel through the scratch array: more than 8
-# splits on the tensor-core kernels (beyond one cluster, so the last CTA of a
-# unit merges from the scratch), and the CUDA-core kernel, which always merges
-# there.  The sequence mixes workloads so that a call finds the previous
-# call's partials (of another shape) in the array.
+# Every split plan's partial states travel through the scratch array: up to 8
+# splits on the tensor-core kernels (one cluster per unit, merged after a
+# cluster barrier), more than 8 there (the last CTA of a unit merges, with
+# tickets), and the CUDA-core kernel (tickets).  The sequence mixes workloads
+# so that a call finds the previous call's partials (of another shape) in the
+# array.
 CASES = [("gptoss_paged_decode_f16", 16), ("tiny_decode_f32", 3), ("local_plus_selected_int8", 12),
-         ("selected_decode_bf16", 32), ("tiny_decode_f32", 5), ("gptoss_paged_decode_f16", 16)]
+         ("selected_decode_bf16", 4), ("selected_decode_bf16", 32), ("local_plus_selected_int8", 3),
+         ("tiny_decode_f32", 5), ("gptoss_paged_decode_f16", 2), ("gptoss_paged_decode_f16", 16)]
 
 
 def _prepare(name, splits):
