@@ -48,11 +48,42 @@ namespace spa {
 
 using namespace sm100;
 
+#ifdef SPA_PHASE_PROBE
+// Phase probe, compiled only into the separate probe library (build.py
+// --probe): a few threads of every CTA stamp %globaltimer at the points
+// listed in phase_probe.PF_SLOTS; the host reads the stamps of the last launch.
+constexpr int kPfProbeCtas = 2048, kPfProbeSlots = 64;
+static __device__ unsigned long long g_phase_pf[kPfProbeCtas * kPfProbeSlots];
+__device__ __forceinline__ void pf_stamp(int i) {
+  if (blockIdx.x >= kPfProbeCtas || i < 0 || i >= kPfProbeSlots) return;
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  g_phase_pf[blockIdx.x * kPfProbeSlots + i] = t;
+}
+#define SPA_PF_STAMP(cond, i) \
+  do {                          \
+    if (cond) pf_stamp(i);      \
+  } while (0)
+#else
+#define SPA_PF_STAMP(cond, i) ((void)0)
+#endif
+
 constexpr int kPfBM = 128;   // q rows per tile (TMEM lanes)
 constexpr int kPfBN = 128;   // keys per step
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint32_t kPfWaitLimit = 1u << 20;   // polls before a wait is declared lost
-constexpr int kPfThreads = 10 * 32;           // 2 softmax groups, the MMA warp, the K/V TMA warp
+// 3 warpgroups: softmax A (warps 0-3), softmax B (4-7), and warps 8-11: the
+// MMA warp, the K/V TMA warp and two idle warps.  The kernel is compiled for
+// kPfLaunchRegs registers a thread (one CTA per SM); the third warpgroup hands
+// registers to the softmax warpgroups (setmaxnreg), which hold a whole row of
+// S: 4 x 128 x (kPfSoftmaxRegs - 168) = 128 x (168 - kPfIssueRegs) registers.
+constexpr int kPfThreads = 12 * 32;
+constexpr int kPfLaunchRegs = 168;
+constexpr int kPfSoftmaxRegs = 200;
+constexpr int kPfIssueRegs = 104;
+static_assert(2 * (kPfSoftmaxRegs - kPfLaunchRegs) == kPfLaunchRegs - kPfIssueRegs,
+              "the registers released by the issue warpgroup must cover the softmax warpgroups' increase");
+static_assert(kPfThreads * kPfLaunchRegs <= 65536, "one CTA per SM");
 
 template <int D>
 struct PfCfg {
@@ -75,6 +106,13 @@ struct PfCfg {
 };
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+
+// max(a, b, c) in one instruction (three-input max.f32 of sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -214,6 +252,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
   pdl_trigger();
+  SPA_PF_STAMP(tid == 0, 0);
 
   unsigned char* const sQA = smem + C::OFF_QA;
   unsigned char* const sQB = smem + C::OFF_QB;
@@ -264,7 +303,12 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     while (item < n_items && !(pf_geom(p, item, n_pairs, max_tiles, gg) && gg.ntiles > 0)) item += gridDim.x;
     return item < n_items;
   };
-  if (warp == 9) {
+  // registers: warpgroup 2 (issue: warps 8-11) releases, the softmax
+  // warpgroups take them, each at the head of its role's code
+  if (warp >= 10) {
+    setmaxnreg_dec<kPfIssueRegs>();
+  } else if (warp == 9) {
+    setmaxnreg_dec<kPfIssueRegs>();
     // =================== K/V producer: the 2-stage ring over the CTA's key tiles ===================
     // Tile c of the stream goes to stage c % 2 once the MMAs of tile c - 2 are
     // complete (bar_ke), so the loads run ahead of the MMA warp.
@@ -282,6 +326,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           if (!ok) break;
           pf_issue_kv(p, g, &tm_k, &tm_v, sK + st * C::TILE, sV + st * C::TILE, bar_kf + st, bar_vf + st,
                       g.k_lo + j * kPfBN, box_rows, C::NCH, bits, C::TX_TILE);
+          SPA_PF_STAMP(c < 4, 40 + c);   // K/V tile c of the CTA's stream issued
           kv_issued = ++c;
         }
         item += gridDim.x;
@@ -296,6 +341,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       }
     }
   } else if (warp == 8) {
+    setmaxnreg_dec<kPfIssueRegs>();
     // =================== MMA issuer and Q loads (one thread) ===================
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -318,6 +364,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         issue_q(g);
         ++q_iss;
       }
+      SPA_PF_STAMP(true, 44);   // first Q issued
       bool ok = true;
       // wait for the outstanding PV of tile t (at most one)
       auto pv_done = [&](int t) {
@@ -351,8 +398,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           const int st = c_use & 1;
           const uint32_t ph = (c_use >> 1) & 1;
           ok = mbar_wait(bar_kf + st, ph, kPfWaitLimit, abort_flag);
+          SPA_PF_STAMP(q_seen < 2, 45 + 2 * q_seen);   // item's first K tile landed
           if (ok) {
             ok = mbar_wait(bar_q, q_seen & 1, kPfWaitLimit, abort_flag);
+            SPA_PF_STAMP(q_seen < 2, 46 + 2 * q_seen);   // item's Q landed
             if (ok) ++q_seen;
           }
           for (int t = 0; t < ntq && ok; ++t) {
@@ -435,6 +484,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         if (ke_iss[st] > 0) mbar_wait(bar_ke + st, (ke_iss[st] - 1) & 1, kPfWaitLimit);
     }
   } else {
+    setmaxnreg_inc<kPfSoftmaxRegs>();
     // =================== softmax group t (warps 4t .. 4t+3) ===================
     const int t = warp >> 2;
     const int r = tid & 127;                      // row within the q tile (TMEM lane)
@@ -444,6 +494,12 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     const float sl2 = p.scale_log2;
     int s_seen = 0, o_seen = 0;   // bar_s / bar_o phases this group has consumed
     bool ok = true;
+    int n_it = 0;   // items this group has worked on (probe only)
+    // probe: softmax thread 0 of group A (base 1) and of group B (base 21), items 0 and 1
+    const bool pr = (tid == 0 || tid == 128);
+    const int pbase = tid == 0 ? 1 : 21;
+    (void)pr;
+    (void)pbase;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       PfGeom g;
       if (!pf_geom(p, item, n_pairs, max_tiles, g)) continue;
@@ -457,8 +513,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       float l_sum = 0.f;
       const int nbox0 = kPfBN >> box_shift;
       int blk_next = g.ntiles > 0 ? pf_block_id(p, g.b, g.k_lo, lane, nbox0, box_shift) : -1;
+      SPA_PF_STAMP(pr && n_it < 2, pbase + n_it * 10);   // item geometry known
       for (int j = 0; j < g.ntiles; ++j) {
         ok = mbar_wait(bar_s + t, s_seen & 1, kPfWaitLimit, abort_flag);
+        SPA_PF_STAMP(pr && n_it < 2 && j < 3, pbase + n_it * 10 + 1 + 2 * j);   // S(j) ready
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -494,28 +552,26 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           }
           return m;
         };
-        // pass 1: row max over 32-column chunks of S (keeps few registers live)
-        float mx = -INFINITY;
-        if (full) {
-#pragma unroll 1
-          for (int c4 = 0; c4 < kPfBN / 32; ++c4) {
-            uint32_t v[32];
-            tmem_ld32(tS + c4 * 32, v);
-            tmem_wait_ld();
+        // the whole row of S in registers: four loads, one wait
+        uint32_t v[kPfBN];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, u2f(v[e]));
-          }
-        } else {
-#pragma unroll 1
-          for (int c4 = 0; c4 < kPfBN / 32; ++c4) {
-            uint32_t v[32];
-            tmem_ld32(tS + c4 * 32, v);
-            const uint32_t m = chunk_bits(c4);
-            tmem_wait_ld();
+        for (int c4 = 0; c4 < kPfBN / 32; ++c4) tmem_ld32(tS + c4 * 32, v + c4 * 32);
+        uint32_t msk[kPfBN / 32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, ((m >> e) & 1u) ? u2f(v[e]) : -INFINITY);
-          }
+        for (int c4 = 0; c4 < kPfBN / 32; ++c4) msk[c4] = full ? 0xffffffffu : chunk_bits(c4);
+        tmem_wait_ld();
+        // hidden keys (masked tiles) count as -inf in the max and give p = 0
+        if (!full) {
+#pragma unroll
+          for (int e = 0; e < kPfBN; ++e)
+            if (!((msk[e / 32] >> (e % 32)) & 1u)) v[e] = __float_as_uint(-INFINITY);
         }
+        // row max in four independent three-input max chains
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < kPfBN; e += 2) mq[(e / 2) & 3] = fmax3(mq[(e / 2) & 3], u2f(v[e]), u2f(v[e + 1]));
+        float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        SPA_PF_STAMP(tid == 0 && n_it == 0 && j == 1, 51);   // probe: step 1's row max known
         mx *= sl2;   // scores in log2 units (scale > 0)
         // lazy rescale: raise the reference max only when it grows by > 8 (x256).
         // The TMEM loads / stores of O are warp-collective, so the whole warp
@@ -523,7 +579,37 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         const bool need = mx > m_used + 8.0f;
         const float m_new = need ? mx : m_used;
         const float alpha = need ? ((m_used == -INFINITY) ? 0.f : ex2(m_used - m_new)) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY)) {
+        const bool rescale = j > 0 && __any_sync(0xffffffffu, need && m_used != -INFINITY);
+        l_sum *= alpha;
+        m_used = m_new;
+        const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+        SPA_PF_STAMP(tid == 0 && n_it == 0 && j == 1, 52);   // probe: step 1's rescale decided
+        // P = 2^(s*scale - m) (ex2(-inf) = 0 for hidden keys), packed in pairs
+        // into the TMEM columns that held the scores: fp16 P of keys hh*64 ..
+        // hh*64+63 in columns hh*32 ..; bf16 P_hi and P_lo (residual_pair) in
+        // columns hh*64 .. and hh*64+32 ..
+        float lq[4] = {0.f, 0.f, 0.f, 0.f};   // four independent sum chains
+#pragma unroll
+        for (int hh = 0; hh < kPfBN / 64; ++hh) {
+          uint32_t pk[32], pl[kPfLo<T> ? 32 : 1];
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float pa = ex2(fmaf(u2f(v[hh * 64 + e]), sl2, nm));
+            const float pb = ex2(fmaf(u2f(v[hh * 64 + e + 1]), sl2, nm));
+            lq[(e / 2) & 3] += pa + pb;
+            pk[e / 2] = pack_pair<T>(pa, pb);
+            if constexpr (kPfLo<T>) pl[e / 2] = residual_pair<T>(pa, pb, pk[e / 2]);
+          }
+          if constexpr (kPfLo<T>) {
+            tmem_st32(tS + hh * 64, pk);
+            tmem_st32(tS + hh * 64 + 32, pl);
+          } else {
+            tmem_st32(tS + hh * 32, pk);
+          }
+        }
+        // O *= alpha before this step's PV accumulates into it (the PV waits
+        // for this group's P arrival below)
+        if (rescale) {
           uint32_t o[32];
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -534,47 +620,14 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
             tmem_st32(tO + c * 32, o);
           }
         }
-        l_sum *= alpha;
-        m_used = m_new;
-        const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
-        // pass 2: P = 2^(s*scale - m) for 64 keys at a time, packed in pairs into
-        // the TMEM columns that held those keys' scores (already read)
-        // hidden keys (masked tiles) give p = 0
-        // bf16: P_hi and P_lo (residual_pair) of keys hh*64 .. hh*64+63 go
-        // to the 64 columns that held those keys' scores
-        float ls = 0.f;
-#pragma unroll
-        for (int hh = 0; hh < kPfBN / 64; ++hh) {
-          uint32_t pk[32], pl[kPfLo<T> ? 32 : 1];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            const int c0 = hh * 64 + half * 32;
-            tmem_ld32(tS + c0, v);
-            const uint32_t m = full ? 0xffffffffu : chunk_bits(hh * 2 + half);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float pa = ((m >> e) & 1u) ? ex2(fmaf(u2f(v[e]), sl2, nm)) : 0.f;
-              const float pb = ((m >> (e + 1)) & 1u) ? ex2(fmaf(u2f(v[e + 1]), sl2, nm)) : 0.f;
-              ls += pa + pb;
-              pk[half * 16 + e / 2] = pack_pair<T>(pa, pb);
-              if constexpr (kPfLo<T>) pl[half * 16 + e / 2] = residual_pair<T>(pa, pb, pk[half * 16 + e / 2]);
-            }
-          }
-          if constexpr (kPfLo<T>) {
-            tmem_st32(tS + hh * 64, pk);
-            tmem_st32(tS + hh * 64 + 32, pl);
-          } else {
-            tmem_st32(tS + hh * 32, pk);
-          }
-        }
-        l_sum += ls;
+        l_sum += (lq[0] + lq[1]) + (lq[2] + lq[3]);
+        SPA_PF_STAMP(tid == 0 && n_it == 0 && j == 1, 53);   // probe: step 1's P stores issued
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         const bool drop = p.test_expire_wait && warp == 0 && j == 0 && item == (int)blockIdx.x;
         if (lane == 0 && !drop) mbar_arrive(bar_p + t);
+        SPA_PF_STAMP(pr && n_it < 2 && j < 3, pbase + n_it * 10 + 2 + 2 * j);   // P(j) handed over
       }
       if (!ok) break;
       // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
@@ -587,6 +640,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           break;
         }
       }
+      SPA_PF_STAMP(pr && n_it < 2, pbase + n_it * 10 + 7);   // last PV complete
         tc_fence_after();
         const bool mine = r < rows_t;
         const int tok = g.t_begin + q0_t + r;
@@ -630,6 +684,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_e + t);
       }
+      SPA_PF_STAMP(pr && n_it < 2, pbase + n_it * 10 + 8);   // epilogue stored
+      ++n_it;
     }
     if (!ok) *abort_flag = 1;
   }
@@ -652,6 +708,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     tc_fence_after();
     tmem_dealloc(tmem, kPfTmemCols);
   }
+  SPA_PF_STAMP(tid == 0, 50);   // CTA end
 }
 
 // ---------------------------------------------------------------------------
@@ -724,6 +781,13 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   if (items > 0x7fffffffLL) return SPA_ERR_UNSUPPORTED;
   const int max_tiles = (p.max_k + kPfBN - 1) / kPfBN + 1;
   auto kern = prefill_tcgen05_kernel<T, D>;
+  // the register hand-over (setmaxnreg) balances only at the launch register
+  // count it was written for: a build with another count is not launched
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != kPfLaunchRegs) {
+    cudaGetLastError();
+    return SPA_ERR_UNSUPPORTED;
+  }
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   // persistent: one CTA per SM (all of TMEM, over half the shared memory),
   // items = heads fastest, then requests, then q-tile pairs from the last
@@ -752,3 +816,16 @@ int launch_prefill(const AttnParams& p, int act, cudaStream_t stream) {
 }
 
 }  // namespace spa
+
+#ifdef SPA_PHASE_PROBE
+// Probe library only: copy / clear the phase stamps of prefill_tcgen05_kernel.
+extern "C" int spa_probe_read_pf(void* host, size_t bytes) {
+  if (bytes > sizeof(spa::g_phase_pf)) bytes = sizeof(spa::g_phase_pf);
+  return (int)cudaMemcpyFromSymbol(host, spa::g_phase_pf, bytes);
+}
+extern "C" int spa_probe_clear_pf() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, spa::g_phase_pf) != cudaSuccess) return -1;
+  return (int)cudaMemset(p, 0, sizeof(spa::g_phase_pf));
+}
+#endif

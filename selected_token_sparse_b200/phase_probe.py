@@ -51,9 +51,65 @@ PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumul
           (1, 9, "CTA after the wait"), (0, 9, "CTA incl. the wait")]
 
 
+# Stamps of prefill_tcgen05_kernel (slot: point).  Softmax thread 0 of group
+# A (q tile A) uses slots 1-9 for its first item and 11-19 for its second,
+# thread 0 of group B slots 21-29 / 31-39: +0 geometry known, +1 S(0) ready,
+# +2 P(0) handed over, +3 / +4 the same for key step 1, +5 / +6 step 2,
+# +7 last PV complete, +8 epilogue stored.  40-43: the producer issued K/V
+# tiles 0-3 of the CTA's stream; 44: first Q issued; 45 / 46: the first
+# item's first K tile / Q landed (MMA thread), 47 / 48 the second item's;
+# 0 / 50: CTA start / end (thread 0); 51-53: inside group A's softmax of its
+# first item's key step 1 (row max known, rescale done, P stores issued).
+PF_PHASES = [(0, 1, "A item 0: geometry (metadata loads)"), (44, 46, "item 0: Q copy"),
+             (40, 45, "item 0: first K tile copy (from issue)"),
+             (1, 2, "A item 0: wait for S(0)"), (2, 3, "A item 0: softmax of key step 0"),
+             (3, 4, "A item 0: P(0) -> S(1) (PV + S on the tensor core)"), (4, 5, "A item 0: softmax of step 1"),
+             (4, 51, "A step 1: max pass (4 TMEM loads)"), (51, 52, "A step 1: rescale check"),
+             (52, 53, "A step 1: exp pass, P stores issued"), (53, 5, "A step 1: P stores complete, arrive"),
+             (5, 6, "A item 0: P(1) -> S(2)"), (6, 7, "A item 0: softmax of step 2"),
+             (8, 9, "A item 0: epilogue (O out of TMEM, stores)"), (9, 11, "A: next item's geometry"),
+             (11, 12, "A item 1: wait for S(0)"), (12, 13, "A item 1: softmax of step 0"),
+             (13, 14, "A item 1: P(0) -> S(1)"), (22, 23, "B item 0: softmax of step 0"),
+             (23, 24, "B item 0: P(0) -> S(1)"), (29, 31, "B: next item's geometry"),
+             (31, 32, "B item 1: wait for S(0)"), (0, 50, "CTA")]
+
+
+def run_pf(lib, insts, steps, R, raw=None):
+    clear, read = lib.spa_probe_clear_pf, lib.spa_probe_read_pf
+    stream = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            insts[i % R]()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert clear() == 0
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    nct, slots = 2048, 64
+    buf = np.zeros(nct * slots, dtype=np.uint64)
+    assert read(buf.ctypes.data, buf.nbytes) == 0
+    P = buf.reshape(nct, slots).astype(np.int64)
+    if raw:
+        np.save(raw, P)
+    P = P[P[:, 0] > 0]
+    lines = [f"prefill kernel: {len(P)} CTAs of the graph's last step ({steps} steps, {R} instances); "
+             f"span {(P[:, 50].max() - P[:, 0].min()) / 1e3:.2f} us", "",
+             "| interval | CTAs | median us | p90 us | max us |", "|---|---|---|---|---|"]
+    for a, b, name in PF_PHASES:
+        ok = (P[:, a] > 0) & (P[:, b] > 0)
+        if ok.any():
+            x = (P[ok, b] - P[ok, a]) / 1e3
+            lines.append(f"| {a}->{b} {name} | {int(ok.sum())} | {np.median(x):.2f} | {np.percentile(x, 90):.2f} | "
+                         f"{x.max():.2f} |")
+    return "\n".join(lines)
+
+
 def run(workload: str, lib_path: str, steps: int = 64, raw: str = None):
     lib = spa.load_library(lib_path)
-    for k in ("mma", "tc"):
+    for k in ("mma", "tc", "pf"):
         getattr(lib, f"spa_probe_read_{k}").restype = ctypes.c_int
         getattr(lib, f"spa_probe_read_{k}").argtypes = [ctypes.c_void_p, ctypes.c_size_t]
         getattr(lib, f"spa_probe_clear_{k}").restype = ctypes.c_int
@@ -69,6 +125,12 @@ def run(workload: str, lib_path: str, steps: int = 64, raw: str = None):
                                    "past_seqlens", "selected_idx") else v) for k, v in base.items()}
         insts.append(pipeline.Step(wl, d))
     kind = spa.attention_plan(insts[0].args)["kind"]
+    if kind == 2:
+        with torch.cuda.stream(torch.cuda.Stream()):
+            for st in insts:
+                st()
+        torch.cuda.synchronize()
+        return run_pf(lib, insts, steps, R, raw)
     assert kind in (1, 3), "the workload runs neither the warp-MMA nor the tcgen05 decode kernel"
     tag, phases, last, nct = ("mma", PHASES, 9, 8192) if kind == 1 else ("tc", TC_PHASES, 10, 4096)
     clear = getattr(lib, f"spa_probe_clear_{tag}")
