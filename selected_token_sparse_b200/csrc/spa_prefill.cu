@@ -142,6 +142,9 @@ struct PfGeom {
   int k_first;   // first key any row of the item attends (k_lo is it rounded down to a tile)
   int rlo;       // first key of this shard's range (0: all)
   int q0[2], rows[2];   // per q tile: first row within the request, rows present (0 = absent)
+  // per q tile: the key steps [j_lo, j_hi) holding a key some row of the tile
+  // may see (causal / window / shard limits); the item's key tiles are their union
+  int j_lo[2], j_hi[2];
 };
 
 // Block id of box `lane` of the key tile starting at kb (-1 when the lane has
@@ -228,6 +231,16 @@ __device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_pai
   g.k_hi = min(min(p_last + 1, g.L), rhi);
   g.ntiles = g.k_hi > g.k_lo ? (g.k_hi - g.k_lo + kPfBN - 1) / kPfBN : 0;
   g.ntiles = min(g.ntiles, max_tiles);
+  for (int t = 0; t < 2; ++t) {
+    g.j_lo[t] = g.j_hi[t] = 0;
+    if (g.rows[t] <= 0) continue;
+    const int lo_row = g.past + g.q0[t], hi_row = lo_row + g.rows[t] - 1;
+    const int first = max(p.window > 0 ? max(0, lo_row - p.window + 1) : 0, g.rlo);
+    const int hi = min(hi_row + 1, g.k_hi);
+    if (hi <= first) continue;
+    g.j_lo[t] = min((first - g.k_lo) / kPfBN, g.ntiles);
+    g.j_hi[t] = max(min((hi - g.k_lo + kPfBN - 1) / kPfBN, g.ntiles), g.j_lo[t]);
+  }
   return true;
 }
 
@@ -394,7 +407,9 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       // the other's MMAs.
       while (have && ok) {
         const int ntq = g.rows[1] > 0 ? 2 : 1;
-        {   // step 0: S of every q tile (after the tile's previous PV)
+        auto need = [&](int t, int j) { return t ? (j >= g.j_lo[1] && j < g.j_hi[1]) : (j >= g.j_lo[0] && j < g.j_hi[0]); };
+        bool pv_any[2] = {false, false};   // a PV of tile t issued in this item
+        {   // step 0: S of every q tile that sees key tile 0 (after the tile's previous PV)
           const int st = c_use & 1;
           const uint32_t ph = (c_use >> 1) & 1;
           ok = mbar_wait(bar_kf + st, ph, kPfWaitLimit, abort_flag);
@@ -405,6 +420,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
             if (ok) ++q_seen;
           }
           for (int t = 0; t < ntq && ok; ++t) {
+            if (!need(t, 0)) continue;
             pv_done(t);   // S_t overwrites P_t of the tile's previous step
             if (ok) issue_s(t, st);
           }
@@ -418,35 +434,39 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           bool k_next = false;
           ok = mbar_wait(bar_vf + st, ph, kPfWaitLimit, abort_flag);
           for (int t = 0; t < ntq && ok; ++t) {
-            ok = mbar_wait(bar_p + t, p_seen[t] & 1, p_wait_limit, abort_flag);
-            if (ok) ++p_seen[t];
-            // the first PV of an item overwrites O_t: the previous epilogue must have read it
-            while (ok && j == 0 && e_seen[t] < e_due[t]) {
-              ok = mbar_wait(bar_e + t, e_seen[t] & 1, kPfWaitLimit, abort_flag);
-              if (ok) ++e_seen[t];
-            }
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t tP = tmem + t * 128;
-            const uint32_t tO = tmem + 256 + t * 128;
-#pragma unroll
-            for (int kk = 0; kk < kPfBN / 16; ++kk) {
-              const uint64_t bd = smem_desc_sw128(smem_u32(sV + st * C::TILE + kk * 2048), C::CHUNK, 1024);
-              if constexpr (kPfLo<T>) {   // P_hi and P_lo of 64-key halves (see the softmax)
-                const uint32_t col = (kk / 4) * 64 + (kk % 4) * 8;
-                mma_ts(tO, tP + col, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-                mma_ts(tO, tP + col + 32, bd, IDESC_O, 1u);
-              } else {
-                mma_ts(tO, tP + kk * 8, bd, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+            if (need(t, j)) {
+              ok = mbar_wait(bar_p + t, p_seen[t] & 1, p_wait_limit, abort_flag);
+              if (ok) ++p_seen[t];
+              // the first PV of an item overwrites O_t: the previous epilogue must have read it
+              while (ok && !pv_any[t] && e_seen[t] < e_due[t]) {
+                ok = mbar_wait(bar_e + t, e_seen[t] & 1, kPfWaitLimit, abort_flag);
+                if (ok) ++e_seen[t];
               }
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t tP = tmem + t * 128;
+              const uint32_t tO = tmem + 256 + t * 128;
+              const uint32_t acc0 = pv_any[t] ? 1u : 0u;
+#pragma unroll
+              for (int kk = 0; kk < kPfBN / 16; ++kk) {
+                const uint64_t bd = smem_desc_sw128(smem_u32(sV + st * C::TILE + kk * 2048), C::CHUNK, 1024);
+                if constexpr (kPfLo<T>) {   // P_hi and P_lo of 64-key halves (see the softmax)
+                  const uint32_t col = (kk / 4) * 64 + (kk % 4) * 8;
+                  mma_ts(tO, tP + col, bd, IDESC_O, kk > 0 ? 1u : acc0);
+                  mma_ts(tO, tP + col + 32, bd, IDESC_O, 1u);
+                } else {
+                  mma_ts(tO, tP + kk * 8, bd, IDESC_O, kk > 0 ? 1u : acc0);
+                }
+              }
+              tc_commit(bar_o + t);
+              ++o_iss[t];
+              pv_any[t] = true;
             }
-            tc_commit(bar_o + t);
-            ++o_iss[t];
             if (t == ntq - 1) {   // every MMA reading this stage is issued: it empties on completion
               tc_commit(bar_ke + st);
               ++ke_iss[st];
             }
-            if (more) {
+            if (more && need(t, j + 1)) {
               if (!k_next) {
                 ok = mbar_wait(bar_kf + st1, ph1, kPfWaitLimit, abort_flag);
                 k_next = true;
@@ -459,7 +479,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           ++c_use;
         }
         if (!ok) break;
-        for (int t = 0; t < ntq; ++t) ++e_due[t];
+        for (int t = 0; t < ntq; ++t)
+          if (pv_any[t]) ++e_due[t];
         // every P of this item was observed, so its S MMAs are complete: Q may be replaced
         ci += gridDim.x;
         have = next_work(ci, g);
@@ -512,9 +533,11 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       float m_used = -INFINITY;   // log2 units
       float l_sum = 0.f;
       const int nbox0 = kPfBN >> box_shift;
-      int blk_next = g.ntiles > 0 ? pf_block_id(p, g.b, g.k_lo, lane, nbox0, box_shift) : -1;
+      // the key steps this tile sees; the MMA thread issues S and PV for these only
+      const int j_lo = t ? g.j_lo[1] : g.j_lo[0], j_hi = t ? g.j_hi[1] : g.j_hi[0];
+      int blk_next = j_hi > j_lo ? pf_block_id(p, g.b, g.k_lo + j_lo * kPfBN, lane, nbox0, box_shift) : -1;
       SPA_PF_STAMP(pr && n_it < 2, pbase + n_it * 10);   // item geometry known
-      for (int j = 0; j < g.ntiles; ++j) {
+      for (int j = j_lo; j < j_hi; ++j) {
         ok = mbar_wait(bar_s + t, s_seen & 1, kPfWaitLimit, abort_flag);
         SPA_PF_STAMP(pr && n_it < 2 && j < 3, pbase + n_it * 10 + 1 + 2 * j);   // S(j) ready
         if (!__all_sync(0xffffffffu, ok)) {
@@ -529,7 +552,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         // any row of this q tile?
         const int nbox = kPfBN >> box_shift;   // <= 8 (block_size >= 16)
         const uint32_t boxmask = __ballot_sync(0xffffffffu, lane < nbox && blk_next >= 0 && blk_next < p.NB);
-        if (j + 1 < g.ntiles) blk_next = pf_block_id(p, g.b, kb + kPfBN, lane, nbox, box_shift);
+        if (j + 1 < j_hi) blk_next = pf_block_id(p, g.b, kb + kPfBN, lane, nbox, box_shift);
         const bool all_mapped = boxmask == (1u << nbox) - 1u;
         const bool full = all_mapped && kb + kPfBN - 1 <= p_lo && kb + kPfBN <= g.k_hi &&
                           (p.window <= 0 || kb > p_hi - p.window) && kb >= g.rlo;
@@ -631,10 +654,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       }
       if (!ok) break;
       // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
-      bool have_o = g.ntiles > 0;
+      bool have_o = j_hi > j_lo;
       if (have_o) {
-        have_o = mbar_wait(bar_o + t, (o_seen + g.ntiles - 1) & 1, kPfWaitLimit, abort_flag);
-        o_seen += g.ntiles;
+        have_o = mbar_wait(bar_o + t, (o_seen + (j_hi - j_lo) - 1) & 1, kPfWaitLimit, abort_flag);
+        o_seen += j_hi - j_lo;
         if (!__all_sync(0xffffffffu, have_o)) {
           ok = false;
           break;
@@ -679,7 +702,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           }
         }
         if (mine && p.lse) p.lse[orow] = lse;
-      if (g.ntiles > 0) {   // O_t may now be overwritten by the next item
+      if (j_hi > j_lo) {   // O_t may now be overwritten by the next item
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_e + t);
