@@ -327,7 +327,10 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
   const int seg = (((n + kSelWarps - 1) / kSelWarps) + 127) & ~127;     // keys per warp
   const int beg = min(warp * seg, n), end = min(beg + seg, n);
 
-  // 1. staging: this warp's segment as 16-byte vectors, 8 in flight per lane
+  // 1. staging: this warp's segment as 16-byte vectors, 8 in flight per lane;
+  // the histogram of the first digit (bits 31..21) is counted on the way
+  for (int i = tid; i < kSelBins; i += kSelThreads) fs.hist[i] = 0u;
+  __syncthreads();
   int elig = 0;
   if (beg < end) {   // (a warp past the row's end has an empty segment)
     const int i_beg = beg >> 2, i_end = (end + 3) >> 2;
@@ -348,6 +351,7 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
         for (int e = 0; e < 4; ++e) {
           k[e] = 4 * i + e < end ? score_key(x[e]) : 0u;
           elig += k[e] != 0u;
+          if (k[e] != 0u) atomicAdd(&fs.hist[k[e] >> 21], 1u);
         }
         *reinterpret_cast<uint4*>(keys + 4 * i) = make_uint4(k[0], k[1], k[2], k[3]);
       }
@@ -374,20 +378,17 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
       if (j + e >= end) k[e] = 0u;
   };
 
+  // e-major view of a warp step: key j0 + 32 e + lane (index order is e, then lane)
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  auto key_e = [&](int j0, int e) -> uint32_t {
+    const int j = j0 + 32 * e + lane;
+    return j < end ? keys[j] : 0u;
+  };
+
   uint32_t T = 0u;
   int need_eq = 0;
   if (E > top_k && top_k > 0) {
-    // 2a. histogram of the first digit (bits 31..21)
-    for (int i = tid; i < kSelBins; i += kSelThreads) fs.hist[i] = 0u;
-    __syncthreads();
-    for (int j0 = beg; j0 < end; j0 += 128) {
-      uint32_t k[4];
-      lane_keys(j0, k);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (k[e] != 0u) atomicAdd(&fs.hist[k[e] >> 21], 1u);
-    }
-    __syncthreads();
+    // 2a. the first digit (its histogram was counted while staging)
     find_digit(fs, kSelBins, top_k, tid, lane, warp);
     const uint32_t d1 = (uint32_t)fs.digit;
     int k_rem = top_k - fs.above;
@@ -403,28 +404,29 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
     // keys (key, index) into the buffer
     int gt_above = 0;
     for (int j0 = beg; j0 < end; j0 += 128) {
-      uint32_t k[4];
-      lane_keys(j0, k);
-      int c = 0;
+      uint32_t k[4], bb[4];
+      int tot = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        gt_above += (k[e] != 0u && (k[e] >> 21) > d1) ? 1 : 0;
-        c += (use_buf && k[e] != 0u && (k[e] >> 21) == d1) ? 1 : 0;
+        k[e] = key_e(j0, e);
+        const uint32_t dg = k[e] >> 21;
+        gt_above += (k[e] != 0u && dg > d1) ? 1 : 0;
+        bb[e] = __ballot_sync(0xffffffffu, use_buf && k[e] != 0u && dg == d1);
+        tot += __popc(bb[e]);
       }
-      if (use_buf) {
-        int tot;
-        const int ex = warp_excl_scan(c, lane, tot);
+      if (tot > 0) {   // warp-uniform
         int base = 0;
-        if (lane == 0 && tot > 0) base = atomicAdd(&fs.nbuf, tot);
+        if (lane == 0) base = atomicAdd(&fs.nbuf, tot);
         base = __shfl_sync(0xffffffffu, base, 0);
-        int at = base + ex;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (k[e] != 0u && (k[e] >> 21) == d1) {
+        for (int e = 0; e < 4; ++e) {
+          if ((bb[e] >> lane) & 1u) {
+            const int at = base + __popc(bb[e] & lt_mask);
             buf_key[at] = k[e];
-            buf_idx[at] = j0 + 4 * lane + e;
-            ++at;
+            buf_idx[at] = j0 + 32 * e + lane;
           }
+          base += __popc(bb[e]);
+        }
       }
     }
     gt_above = __reduce_add_sync(0xffffffffu, gt_above);
@@ -512,30 +514,23 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
     }
     pos += min(eq_seen, need_eq);
     for (int j0 = beg; j0 < end; j0 += 128) {
-      uint32_t k[4];
-      lane_keys(j0, k);
-      int nq = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) nq += (need_eq > 0 && k[e] == T) ? 1 : 0;
-      int q_tot;
-      const int q_ex = warp_excl_scan(nq, lane, q_tot);
-      bool take[4];
-      int nt = 0, qi = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const bool is_eq = need_eq > 0 && k[e] == T;
-        take[e] = k[e] > T || (is_eq && eq_seen + q_ex + qi < need_eq);
-        qi += is_eq ? 1 : 0;
-        nt += take[e] ? 1 : 0;
+        const uint32_t k = key_e(j0, e);
+        bool take = k > T;
+        uint32_t bt = __ballot_sync(0xffffffffu, take);
+        if (need_eq > 0) {   // keys equal to T: the first need_eq of them by index
+          const bool eq = k == T;
+          const uint32_t be = __ballot_sync(0xffffffffu, eq);
+          if (be != 0u) {
+            take = take || (eq && eq_seen + __popc(be & lt_mask) < need_eq);
+            bt = __ballot_sync(0xffffffffu, take);
+            eq_seen += __popc(be);
+          }
+        }
+        if (take) dst[pos + __popc(bt & lt_mask)] = j0 + 32 * e + lane;
+        pos += __popc(bt);
       }
-      int t_tot;
-      const int t_ex = warp_excl_scan(nt, lane, t_tot);
-      int at = pos + t_ex;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (take[e]) dst[at++] = j0 + 4 * lane + e;
-      pos += t_tot;
-      eq_seen += q_tot;
     }
   }
   // 4. padding up to the row's capacity
