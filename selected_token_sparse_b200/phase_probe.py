@@ -44,7 +44,7 @@ TC_PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cu
              (1, 10, "CTA after the wait"), (0, 10, "CTA incl. the wait")]
 PHASES = [(0, 1, "wait for the predecessor (PDL)"), (1, 2, "unit metadata (cumulative-length scan)"),
           (2, 3, "Q rows to shared memory"), (3, 4, "candidates: block ids, row offsets"),
-          (4, 5, "issue the first K/V stages"), (5, 6, "key loop (copies, QK, softmax, PV)"),
+          (4, 5, "issue the first K/V stages; first token's append"), (5, 6, "key loop (copies, QK, softmax, PV)"),
           (6, 7, "epilogue: normalise, write output"), (7, 8, "fused metadata / append tail"),
           (8, 9, "split merge"), (8, 10, "merge: cluster barrier"),
           (10, 11, "merge: rows from the workspace"),
