@@ -23,9 +23,10 @@
 //     the main cache, always visible for auxiliary entries), a lazily raised
 //     max in log2 units, P into one of two TMEM buffers of its own; at the
 //     end O is scaled by the value scale (INT8), normalised with the sink and
-//     written (one split) or merged with the unit's other splits (a
-//     thread-block cluster through distributed shared memory, else the
-//     workspace);
+//     written (one split) or left in the workspace as a partial state and
+//     merged with the unit's other splits (up to 8 splits form a
+//     thread-block cluster and merge after a cluster barrier, more merge by
+//     ticket);
 //   * an MMA warp (one thread): S = Q K^T into one of two TMEM buffers, the
 //     next tile's S ahead of this tile's PV so that it is computed while the
 //     softmax runs, and O += P V (A from TMEM) once the four softmax warps
