@@ -20,7 +20,8 @@
 // its own online-softmax state (log2 units) and merges through shared memory
 // at the end.  With one split the learned sink is folded in and the output
 // written; otherwise FP32 partial states go to the workspace for the
-// log-sum-exp combine ("[WebGPU] Add SparsePagedAttention", File summaries;
+// log-sum-exp combine, after a cluster barrier (up to 8 splits) or by ticket
+// ("[WebGPU] Add SparsePagedAttention", File summaries;
 // "[WebGPU] Add DynamicSparseAttention", Attention: joint FP32 stable softmax
 // with optional sink; onnxruntime PR #33472: INT8 per-channel K/V scales).
 #include <type_traits>
@@ -194,7 +195,7 @@ decode_mma_kernel(const AttnParams p) {
   if (!p.group_by_request) load_q(blockIdx.x / p.H_kv, p.G);
   // fused step, split 0: this thread's vector of the unit's first token's
   // new K/V row is loaded early (a per-token unit knows its token now) and
-  // stored into the cache at the end
+  // stored into the cache while the split's K/V copies are in flight
   constexpr int NV = D * 2 / 16;
   const bool app_thread = FUSED && blockIdx.y == 0 && tid < 2 * NV;
   uint4 app_data = make_uint4(0, 0, 0, 0);

@@ -6,25 +6,30 @@
 // kernel is organised so that the tensor core and the softmax overlap:
 //
 //   CTA    = one q head x one request x a PAIR of 128-row q tiles (A, B);
-//            launched longest pairs first (q tiles in reverse order).
+//            launched longest pairs first (q tiles in reverse order); each q
+//            tile runs only the key tiles its own rows can see.
 //   TMEM   = S_A | S_B | O_A | O_B (4 x 128 columns); P of a tile overwrites
 //            its S as packed 16-bit pairs and feeds the PV MMA from TMEM.
-//   warp 8 = TMA producer and MMA issuer (one elected thread): Q_A, Q_B once;
-//            K and V tiles through a 2-stage ring from the paged cache (4-D
-//            tensor map over [num_blocks, block_size, H_kv, D]; the block id is
-//            a coordinate taken from the block table; an unmapped block is read
-//            from an out-of-range coordinate, i.e. zeros, and masked; 128-byte
-//            swizzle; no multicast).  Per 128-key step j it issues
-//              S_A = Q_A K_j^T, S_B = Q_B K_j^T, then O_A += P_A V_j and
-//              O_B += P_B V_j as each softmax group hands over its P,
-//            so S_B and PV_A run on the tensor core while the other group's
-//            softmax runs on the CUDA cores.
-//   warps 0-3 / 4-7 = softmax of tile A / B: thread i owns row i (TMEM lane i);
-//            masks only the tiles that cross the causal diagonal, the window
-//            edge, the end of the keys or an unmapped block; keeps a running
-//            max in log2 units that is raised (O rescaled in TMEM) only when a
-//            tile's max exceeds it by more than 8, so P <= 2^8; the scale is
-//            folded into one FFMA ahead of ex2.approx.
+//   warp 9 = K/V producer (one thread): K and V tiles through a 2-stage ring
+//            from the paged cache (4-D tensor map over [num_blocks,
+//            block_size, H_kv, D]; the block id is a coordinate taken from the
+//            block table; an unmapped block is read from an out-of-range
+//            coordinate, i.e. zeros, and masked; 128-byte swizzle; no
+//            multicast).
+//   warp 8 = MMA issuer (one thread) and the Q loads.  Per 128-key step j and
+//            q tile t it issues PV_t(j) (O_t += P_t V_j) as soon as the
+//            softmax group hands over P_t, then S_t(j + 1), so one group's
+//            MMAs run on the tensor core while the other group's softmax runs
+//            on the CUDA cores.
+//   warps 0-3 / 4-7 = softmax of tile A / B: thread i owns row i (TMEM lane i)
+//            and reads its row of S from TMEM once per step; masks only the
+//            tiles that cross the causal diagonal, the window edge, the end
+//            of the keys or an unmapped block; keeps a running max in log2
+//            units that is raised (O rescaled in TMEM) only when a tile's max
+//            exceeds it by more than 8, so P <= 2^8; the scale is folded into
+//            one FFMA ahead of ex2.approx.
+//   registers: warps 8-11 (warps 10-11 idle) hand registers to the softmax
+//            warpgroups (setmaxnreg), which need a row of S in registers.
 //   sink   = folded into the final normalisation (denominator only).
 //
 // The key loop starts at the earliest window tile, rounded down to the tile

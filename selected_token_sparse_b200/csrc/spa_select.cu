@@ -246,8 +246,8 @@ select_topk_kernel(const float* __restrict__ scores, int H, int n_keys, const in
 // two remaining digits are resolved on that buffer alone.  The per-warp
 // counts the final write needs are gathered on the way (keys above the bin in
 // the candidate pass, the buffer's keys once the threshold is exact), so the
-// row is read from shared memory three more times after staging: the first
-// histogram, the candidate pass and the write pass.  When the threshold bin
+// row is read from shared memory twice after staging (the first digit's
+// histogram is counted while staging): the candidate pass and the write pass.  When the threshold bin
 // is larger than the buffer (e.g. all scores equal), the remaining digits and
 // the counts run over the whole row instead.
 constexpr int kFastStageKeys = 40 * 1024;   // keys staged (160 KB)

@@ -1,4 +1,5 @@
-"""Warm, in-graph phase breakdown of the decode kernels (warp-MMA and tcgen05).
+"""Warm, in-graph phase breakdown of the decode kernels (warp-MMA and tcgen05)
+and of the tcgen05 prefill.
 
     python -m selected_token_sparse_b200.phase_probe [--workload NAME] [--lib PATH]
 
