@@ -255,6 +255,9 @@ constexpr int kFastCand = 4096;             // candidate buffer entries (32 KB)
 
 struct FastShared {
   uint32_t hist[kSelBins];
+  uint32_t hist1[kSelBins];   // CTA pair: digit 2's histogram (digit 3 reuses hist)
+  uint32_t histc[kSelBins];   // CTA pair: both halves' histogram of the current digit
+  int e_loc, peer_gt, peer_eq;
   int warp_el[kSelWarps];
   int warp_gt[kSelWarps];
   int warp_eq[kSelWarps];
@@ -276,11 +279,12 @@ __device__ __forceinline__ int warp_excl_scan(int x, int lane, int& total) {
 
 // Block-wide search of the histogram bin where the count of larger keys
 // reaches k_rem (bins ordered from the largest digit); results in fs.
-__device__ __forceinline__ void find_digit(FastShared& fs, int nbins, int k_rem, int tid, int lane, int warp) {
+__device__ __forceinline__ void find_digit(FastShared& fs, const uint32_t* hist, int nbins, int k_rem, int tid,
+                                           int lane, int warp) {
   const int bpt = nbins / kSelThreads;   // 2 or 1
   const int b0 = nbins - 1 - tid * bpt;
-  const int c0 = (int)fs.hist[b0];
-  const int c1 = bpt == 2 ? (int)fs.hist[b0 - 1] : 0;
+  const int c0 = (int)hist[b0];
+  const int c1 = bpt == 2 ? (int)hist[b0 - 1] : 0;
   int incl = c0 + c1;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -307,6 +311,30 @@ __device__ __forceinline__ void find_digit(FastShared& fs, int nbins, int k_rem,
   __syncthreads();
 }
 
+// The same word of shared memory in the other CTA of a pair (cluster of 2).
+__device__ __forceinline__ uint32_t pair_addr(const void* p, uint32_t peer) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n"
+               : "=r"(r)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(peer));
+  return r;
+}
+__device__ __forceinline__ uint32_t pair_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void pair_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
+
+// PAIR: a row's candidates are split over a CTA pair (a cluster of two along
+// y; rank = blockIdx.y): each stages and scans its half, the pair exchanges
+// every digit's histogram (and the eligible count) through distributed
+// shared memory after a cluster barrier, so both take the same digits; at
+// the end rank 0 hands its kept counts to rank 1, which writes after them.
+// Rows with few (row, kv head) pairs use twice the SMs this way.
+template <bool PAIR>
 __global__ void __launch_bounds__(kSelThreads, 1)
 select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, const int32_t* __restrict__ bound,
                         int top_k, int sel_width, int32_t* __restrict__ out) {
@@ -316,16 +344,29 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long row = blockIdx.x;
+  const int rank = PAIR ? (int)blockIdx.y : 0;
+  const uint32_t peer = (uint32_t)(rank ^ 1);
   const int r = (int)(row / H);
-  const float4* src4 = reinterpret_cast<const float4*>(scores + row * (long long)n_keys);
   int32_t* dst = out + row * (long long)sel_width;
   const int last = min(bound[r], n_keys - 1);
-  const int n = last + 1 > 0 ? last + 1 : 0;
-  uint32_t* keys = fast_smem;                                           // [n_keys]
-  uint32_t* buf_key = fast_smem + ((n_keys + 3) & ~3);                  // [kFastCand]
+  const int n_row = last + 1 > 0 ? last + 1 : 0;
+  // this CTA's candidates: [lo_c, lo_c + n) of the row (lo_c a multiple of 128)
+  const int half = PAIR ? ((((n_row + 1) / 2) + 127) & ~127) : n_row;
+  const int lo_c = PAIR ? min(rank * half, n_row) : 0;
+  const int n = PAIR ? min(half, n_row - lo_c) : n_row;
+  const float4* src4 = reinterpret_cast<const float4*>(scores + row * (long long)n_keys + lo_c);
+  uint32_t* keys = fast_smem;                                           // [n_keys or half]
+  uint32_t* buf_key = fast_smem + ((PAIR ? half : ((n_keys + 3) & ~3)));   // [kFastCand]
   int* buf_idx = reinterpret_cast<int*>(buf_key + kFastCand);           // [kFastCand]
   const int seg = (((n + kSelWarps - 1) / kSelWarps) + 127) & ~127;     // keys per warp
   const int beg = min(warp * seg, n), end = min(beg + seg, n);
+  // both halves' histogram of the digit counted in `h` (PAIR), after a
+  // cluster barrier that publishes this CTA's own
+  auto combine = [&](const uint32_t* h, int nbins) {
+    cluster_sync();
+    for (int i = tid; i < nbins; i += kSelThreads) fs.histc[i] = h[i] + pair_ld(pair_addr(h + i, peer));
+    __syncthreads();
+  };
 
   // 1. staging: this warp's segment as 16-byte vectors, 8 in flight per lane;
   // the histogram of the first digit (bits 31..21) is counted on the way
@@ -367,6 +408,12 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
   __syncthreads();
   int E = 0;
   for (int w = 0; w < kSelWarps; ++w) E += fs.warp_el[w];
+  const int E_loc = E;
+  if constexpr (PAIR) {
+    if (tid == 0) fs.e_loc = E;
+    combine(fs.hist, kSelBins);   // its barrier also publishes e_loc
+    E += (int)pair_ld(pair_addr(&fs.e_loc, peer));
+  }
 
   // one warp step: the 4 keys of this lane at step start j0 (index order)
   auto lane_keys = [&](int j0, uint32_t (&k)[4]) {
@@ -389,7 +436,7 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
   int need_eq = 0;
   if (E > top_k && top_k > 0) {
     // 2a. the first digit (its histogram was counted while staging)
-    find_digit(fs, kSelBins, top_k, tid, lane, warp);
+    find_digit(fs, PAIR ? fs.histc : fs.hist, kSelBins, top_k, tid, lane, warp);
     const uint32_t d1 = (uint32_t)fs.digit;
     int k_rem = top_k - fs.above;
     const int in1 = fs.in_bin;
@@ -438,12 +485,15 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
       const int shift = pass == 1 ? 10 : 0;
       const uint32_t dmask = pass == 2 ? 1023u : 2047u;
       const int nbins = (int)dmask + 1;
-      for (int i = tid; i < nbins; i += kSelThreads) fs.hist[i] = 0u;
+      // PAIR: digit 2 counts into hist1 (the peer may still read digit 1's
+      // hist until the barrier in combine), digit 3 into hist again
+      uint32_t* h = (PAIR && pass == 1) ? fs.hist1 : fs.hist;
+      for (int i = tid; i < nbins; i += kSelThreads) h[i] = 0u;
       __syncthreads();
       if (use_buf) {
         for (int i = tid; i < nb; i += kSelThreads) {
           const uint32_t k = buf_key[i];
-          if ((k & pmask) == prefix) atomicAdd(&fs.hist[(k >> shift) & dmask], 1u);
+          if ((k & pmask) == prefix) atomicAdd(&h[(k >> shift) & dmask], 1u);
         }
       } else {
         for (int j0 = beg; j0 < end; j0 += 128) {
@@ -451,11 +501,12 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
           lane_keys(j0, k);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (k[e] != 0u && (k[e] & pmask) == prefix) atomicAdd(&fs.hist[(k[e] >> shift) & dmask], 1u);
+            if (k[e] != 0u && (k[e] & pmask) == prefix) atomicAdd(&h[(k[e] >> shift) & dmask], 1u);
         }
       }
       __syncthreads();
-      find_digit(fs, nbins, k_rem, tid, lane, warp);
+      if constexpr (PAIR) combine(h, nbins);
+      find_digit(fs, PAIR ? fs.histc : h, nbins, k_rem, tid, lane, warp);
       k_rem -= fs.above;
       prefix |= (uint32_t)fs.digit << shift;
       pmask |= dmask << shift;
@@ -504,10 +555,29 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
     __syncthreads();
   }
   const int kept = E < top_k ? E : top_k;
+  // PAIR: rank 0's kept-above and equal counts, for rank 1's positions
+  int base_gt = 0, base_eq = 0;
+  if constexpr (PAIR) {
+    if (rank == 0 && tid == 0) {
+      int g = 0, q = 0;
+      for (int w = 0; w < kSelWarps; ++w) {
+        g += fs.warp_gt[w];
+        q += fs.warp_eq[w];
+      }
+      pair_st(pair_addr(&fs.peer_gt, peer), (uint32_t)g);
+      pair_st(pair_addr(&fs.peer_eq, peer), (uint32_t)q);
+    }
+    cluster_sync();   // the last access to the peer's shared memory precedes it
+    if (rank == 1) {
+      base_gt = fs.peer_gt;
+      base_eq = fs.peer_eq;
+    }
+  }
+  (void)E_loc;
 
   // 3. write pass: kept indices in increasing order
   if (kept > 0) {
-    int pos = 0, eq_seen = 0;
+    int pos = base_gt, eq_seen = base_eq;
     for (int w = 0; w < warp; ++w) {
       pos += fs.warp_gt[w];
       eq_seen += fs.warp_eq[w];
@@ -528,13 +598,14 @@ select_topk_fast_kernel(const float* __restrict__ scores, int H, int n_keys, con
             eq_seen += __popc(be);
           }
         }
-        if (take) dst[pos + __popc(bt & lt_mask)] = j0 + 32 * e + lane;
+        if (take) dst[pos + __popc(bt & lt_mask)] = lo_c + j0 + 32 * e + lane;
         pos += __popc(bt);
       }
     }
   }
-  // 4. padding up to the row's capacity
-  for (int i = kept + tid; i < sel_width; i += kSelThreads) dst[i] = -1;
+  // 4. padding up to the row's capacity (shared by the pair)
+  for (int i = kept + (PAIR ? rank * kSelThreads : 0) + tid; i < sel_width; i += (PAIR ? 2 : 1) * kSelThreads)
+    dst[i] = -1;
 }
 
 }  // namespace spa
@@ -552,13 +623,19 @@ extern "C" int spa_select_topk(const float* scores, int32_t R, int32_t H, int32_
   // whole-row 16-byte vectors: every row starts 16-byte aligned
   const int vec = (n_keys % 4 == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) ? 1 : 0;
   if (vec && n_keys > 0 && n_keys <= kFastStageKeys) {
-    const size_t fsm = (size_t)n_keys * 4 + (size_t)kFastCand * 8;
-    if (fsm > 48 * 1024 &&
-        cudaFuncSetAttribute(select_topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kFastStageKeys * 4 + kFastCand * 8) != cudaSuccess)
+    // few rows: each row over a CTA pair (twice the SMs, one wave at most)
+    const bool pair = 2LL * R * H <= 148 && n_keys >= 2 * 128;
+    const size_t keys_smem = pair ? (size_t)((((n_keys + 1) / 2) + 127) & ~127) * 4 : (size_t)((n_keys + 3) & ~3) * 4;
+    const size_t fsm = keys_smem + (size_t)kFastCand * 8;
+    auto kern = pair ? select_topk_fast_kernel<true> : select_topk_fast_kernel<false>;
+    // (the static shared memory counts toward the default 48 KB as well: always opt in)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm) != cudaSuccess)
       return check_launch_public();
-    const int rc = launch_pdl(select_topk_fast_kernel, dim3((unsigned)(R * H)), dim3(kSelThreads), fsm,
-                              (cudaStream_t)stream, scores, H, n_keys, bound, top_k, sel_width, selected_idx);
+    const int rc = pair ? launch_pdl_cluster_y(kern, dim3((unsigned)(R * H), 2), dim3(kSelThreads), fsm,
+                                               (cudaStream_t)stream, 2, scores, H, n_keys, bound, top_k, sel_width,
+                                               selected_idx)
+                        : launch_pdl(kern, dim3((unsigned)(R * H)), dim3(kSelThreads), fsm, (cudaStream_t)stream,
+                                     scores, H, n_keys, bound, top_k, sel_width, selected_idx);
     if (rc != SPA_OK) return rc;
     return check_launch_public();
   }
