@@ -36,7 +36,7 @@ __device__ __forceinline__ T from_f32_rn(float x) {
 }
 
 template <typename ActT, typename CacheT, int E>
-__global__ void __launch_bounds__(kProThreads)
+__global__ void __launch_bounds__(kProThreads, 1)
 prepare_qkv_append_kernel(const QkvParams P) {
   extern __shared__ int32_t pro_smem[];   // cs [B + 1], past [B], then per-warp rows [8][D]
   int32_t* cs = pro_smem;
@@ -57,34 +57,55 @@ prepare_qkv_append_kernel(const QkvParams P) {
     const void* base = kind == 0 ? P.q : (kind == 1 ? P.k : P.v);
     return static_cast<const ActT*>(base) + ((long long)t * (kind == 0 ? P.H_q : P.H_kv) + h) * D;
   };
-  // the warp's first row is loaded before the metadata is known
+  // Issued first: the lengths every warp scans by itself (B + 1 <= 64:
+  // build_cs_warp, no block barrier that would wait for the loads in flight)
+  const bool warp_scan = P.B + 1 <= 64;
+  int pc0 = 0, pc1 = 0, pp0 = 0, pp1 = 0;
+  if (warp_scan) {
+    pc0 = (lane >= 1 && lane <= P.B) ? ld_early(P.cu + lane) : 0;
+    pc1 = lane + 32 <= P.B ? ld_early(P.cu + lane + 32) : 0;
+    pp0 = lane < P.B ? ld_early(P.past + lane) : 0;
+    pp1 = lane + 32 < P.B ? ld_early(P.past + lane + 32) : 0;
+  }
+  // the warp's first row, its norm weights and (with explicit position ids)
+  // its rotary rows are loaded before the metadata is known
   const long long r0 = (long long)blockIdx.x * (kProThreads / 32) + warp;
+  const bool rope = P.cos_cache != nullptr && P.rotary_dim > 0;
+  const int rd = P.rotary_dim, half = rd / 2;
   ActT x0[E];
+  float w0[E], c0[E], s0[E];
+  int pos0 = -1;
   if (r0 < rows_total) {
-    const ActT* src = row_src((int)(r0 / NH), (int)(r0 % NH));
+    const int t0 = (int)(r0 / NH), hh0 = (int)(r0 % NH);
+    const ActT* src = row_src(t0, hh0);
 #pragma unroll
     for (int e = 0; e < E; ++e) x0[e] = src[lane * E + e];
+    const int kind0 = hh0 < P.H_q ? 0 : (hh0 < P.H_q + P.H_kv ? 1 : 2);
+    const float* w = kind0 == 0 ? P.q_norm : (kind0 == 1 ? P.k_norm : nullptr);
+#pragma unroll
+    for (int e = 0; e < E; ++e) w0[e] = w != nullptr ? ld_early(w + lane * E + e) : 0.f;
+    if (rope && kind0 != 2 && P.position_ids != nullptr) {
+      pos0 = ld_early(P.position_ids + t0);
+      if (pos0 >= 0 && pos0 < P.max_pos) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int d = lane * E + e;
+          const int i = d >= rd ? 0 : (P.interleaved ? d >> 1 : (d < half ? d : d - half));
+          c0[e] = ld_early(P.cos_cache + (long long)pos0 * half + i);
+          s0[e] = ld_early(P.sin_cache + (long long)pos0 * half + i);
+        }
+      }
+    }
   }
-  build_cs<kProThreads>(P.cu, P.B, P.T, cs, P.past, past_s);
+  if (warp_scan) build_cs_warp(P.B, P.T, cs, past_s, pc0, pc1, pp0, pp1);
+  else build_cs<kProThreads>(P.cu, P.B, P.T, cs, P.past, past_s);   // ends with a block barrier
   int bits = 0;
   if (blockIdx.x == 0)
     bits |= per_request(P.cu, past_s, cs, P.B, P.T, P.max_q, P.max_k, P.seqlens_q, P.seqlen_k);
-  const bool rope = P.cos_cache != nullptr && P.rotary_dim > 0;
-  const int rd = P.rotary_dim, half = rd / 2;
   for (long long r = r0; r < rows_total; r += (long long)gridDim.x * (kProThreads / 32)) {
     const int t = (int)(r / NH), hh = (int)(r % NH);
-    int tb = 0;
-    const TokenMeta m = token_meta(t, cs, P.B, past_s, P.block_table, P.MB, P.bs, P.NB, tb);
-    if (hh == 0 && lane == 0) {
-      bits |= tb;
-      P.token_batch[t] = m.b;
-      P.token_pos[t] = m.pos;
-      P.slot_mapping[t] = m.slot;
-    }
-    const int kind = hh < P.H_q ? 0 : (hh < P.H_q + P.H_kv ? 1 : 2);   // q, k, v
-    const int h = kind == 0 ? hh : (kind == 1 ? hh - P.H_q : hh - P.H_q - P.H_kv);
-    if (kind != 0 && m.slot < 0) continue;   // nothing to append
-    float x[E];
+    const TokenLoad l = token_meta_load(t, cs, P.B, past_s, P.block_table, P.MB, P.bs);
+    float x[E];   // the row, read before this iteration's metadata stores
     if (r == r0) {
 #pragma unroll
       for (int e = 0; e < E; ++e) x[e] = to_f32(x0[e]);
@@ -93,8 +114,38 @@ prepare_qkv_append_kernel(const QkvParams P) {
 #pragma unroll
       for (int e = 0; e < E; ++e) x[e] = to_f32(src[lane * E + e]);
     }
+    const int kind = hh < P.H_q ? 0 : (hh < P.H_q + P.H_kv ? 1 : 2);   // q, k, v
+    const int h = kind == 0 ? hh : (kind == 1 ? hh - P.H_q : hh - P.H_q - P.H_kv);
+    // the rotary position and its cos / sin entries, loaded while the
+    // block-table entry is in flight (l.pos is -1 for a token no request owns)
+    const bool pre = r == r0 && P.position_ids != nullptr;   // loaded up front
+    const int pos = !rope || kind == 2 ? -1
+                    : (pre ? pos0 : (P.position_ids ? P.position_ids[t] : l.pos + P.rotary_offset));
+    const bool rot = rope && kind != 2 && pos >= 0 && pos < P.max_pos;
+    const float* w = kind == 0 ? P.q_norm : (kind == 1 ? P.k_norm : nullptr);
+    float wv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) wv[e] = r == r0 ? w0[e] : (w != nullptr ? ld_early(w + lane * E + e) : 0.f);
+    float cv[E], sv[E];
+    if (rot) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int d = lane * E + e;
+        const int i = d >= rd ? 0 : (P.interleaved ? d >> 1 : (d < half ? d : d - half));
+        cv[e] = pre ? c0[e] : ld_early(P.cos_cache + (long long)pos * half + i);
+        sv[e] = pre ? s0[e] : ld_early(P.sin_cache + (long long)pos * half + i);
+      }
+    }
+    int tb = 0;
+    const TokenMeta m = token_meta_finish(l, P.MB, P.bs, P.NB, tb);
+    if (hh == 0 && lane == 0) {
+      bits |= tb;
+      P.token_batch[t] = m.b;
+      P.token_pos[t] = m.pos;
+      P.slot_mapping[t] = m.slot;
+    }
+    if (kind != 0 && m.slot < 0) continue;   // nothing to append
     if (kind != 2) {
-      const float* w = kind == 0 ? P.q_norm : P.k_norm;
       if (w != nullptr) {
         float ss = 0.f;
 #pragma unroll
@@ -103,33 +154,28 @@ prepare_qkv_append_kernel(const QkvParams P) {
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         const float inv = 1.0f / sqrtf(ss / (float)D + P.eps);
 #pragma unroll
-        for (int e = 0; e < E; ++e) x[e] = x[e] * inv * w[lane * E + e];
+        for (int e = 0; e < E; ++e) x[e] = x[e] * inv * wv[e];
       }
       if (rope) {
-        const int pos = P.position_ids ? P.position_ids[t] : m.pos + P.rotary_offset;
-        if (pos >= 0 && pos < P.max_pos) {
+        if (rot) {
 #pragma unroll
           for (int e = 0; e < E; ++e) xrow[lane * E + e] = x[e];
           __syncwarp();
-          const float* cr = P.cos_cache + (long long)pos * half;
-          const float* sr = P.sin_cache + (long long)pos * half;
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const int d = lane * E + e;
             if (d >= rd) continue;
-            int i, partner;
+            int partner;
             bool first;
             if (P.interleaved) {
-              i = d >> 1;
               first = (d & 1) == 0;
               partner = d ^ 1;
             } else {
               first = d < half;
-              i = first ? d : d - half;
               partner = first ? d + half : d - half;
             }
-            const float c = cr[i], s = sr[i], y = xrow[partner];
-            x[e] = first ? (x[e] * c - y * s) : (x[e] * c + y * s);
+            const float y = xrow[partner];
+            x[e] = first ? (x[e] * cv[e] - y * sv[e]) : (x[e] * cv[e] + y * sv[e]);
           }
           __syncwarp();
         } else {
