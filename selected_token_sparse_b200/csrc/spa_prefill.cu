@@ -95,12 +95,17 @@ struct PfCfg {
   static constexpr int NCH = D / 64;                  // 128-byte chunks along D
   static constexpr int CHUNK = 128 * 128;             // one chunk of a 128-row tile (bytes)
   static constexpr int TILE = NCH * CHUNK;            // one Q, K or V tile
-  static constexpr int OFF_QA = 0;
-  static constexpr int OFF_QB = OFF_QA + TILE;
-  static constexpr int OFF_K = OFF_QB + TILE;         // 2 stages
-  static constexpr int OFF_V = OFF_K + 2 * TILE;      // 2 stages
-  static constexpr int OFF_BAR = OFF_V + 2 * TILE;    // mbarriers
-  static constexpr int NBAR = 15;
+  // Q buffers (tiles A and B each): two where they fit next to the K/V ring,
+  // so that the next item's Q lands while this item runs
+  static constexpr int NQB = D == 64 ? 2 : 1;
+  static constexpr int OFF_Q = 0;                     // [NQB][2] tiles
+  // K/V ring stages: three where they fit, so that the next item's first two
+  // key tiles are in flight while this item's last ones are in use
+  static constexpr int NST = D == 64 ? 3 : 2;
+  static constexpr int OFF_K = OFF_Q + NQB * 2 * TILE;   // NST stages
+  static constexpr int OFF_V = OFF_K + NST * TILE;     // NST stages
+  static constexpr int OFF_BAR = OFF_V + NST * TILE;   // mbarriers
+  static constexpr int NBAR = 1 + 3 * NST + 8;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_FLAG = OFF_TMEM + 8;
   static constexpr int BYTES = OFF_FLAG + 8;
@@ -143,7 +148,8 @@ template <typename T>
 constexpr bool kPfLo = std::is_same<T, __nv_bfloat16>::value;
 
 struct PfGeom {
-  int b, h, h_kv, t_begin, q_len, past, L, k_lo, k_hi, ntiles;
+  int b, h_kv, t_begin, q_len, past, L, k_lo, k_hi, ntiles;
+  int hq[2];     // per q tile: its q head
   int k_first;   // first key any row of the item attends (k_lo is it rounded down to a tile)
   int rlo;       // first key of this shard's range (0: all)
   int q0[2], rows[2];   // per q tile: first row within the request, rows present (0 = absent)
@@ -162,23 +168,36 @@ __device__ __forceinline__ int pf_block_id(const AttnParams& p, int b, int kb, i
   return lb < p.MB ? ld_early(p.block_table + (long long)b * p.MB + lb) : -1;
 }
 
-// TMA loads of one key tile (keys [kb, kb + 128)) of K and of V, in boxes of
-// box_rows rows (one cache block, or 128 rows of one block).  The block ids of
-// all boxes are read first, as independent loads, and serve both tensors.
-__device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g, const CUtensorMap* map_k,
-                                            const CUtensorMap* map_v, unsigned char* dst_k,
-                                            unsigned char* dst_v, uint64_t* bar_k, uint64_t* bar_v, int kb,
-                                            int box_rows, int nch, int& bits, uint32_t tx) {
-  const int nbox = kPfBN / box_rows;   // <= 8 (block_size >= 16)
+// Block ids of the boxes of one key tile (keys [kb, kb + 128)) in boxes of
+// box_rows rows (one cache block, or 128 rows of one block): independent
+// loads, issued ahead of the wait for a free ring stage; they serve both K
+// and V.
+struct PfIds {
   int raw[8];
+};
+
+__device__ __forceinline__ PfIds pf_kv_ids(const AttnParams& p, const PfGeom& g, int kb, int box_rows) {
+  const int nbox = kPfBN / box_rows;   // <= 8 (block_size >= 16)
+  PfIds ids;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    raw[i] = -1;
+    ids.raw[i] = -1;
     if (i < nbox) {
       const int lb = (kb + i * box_rows) / p.bs;
-      if (lb < p.MB) raw[i] = ld_early(p.block_table + (long long)g.b * p.MB + lb);
+      if (lb < p.MB) ids.raw[i] = ld_early(p.block_table + (long long)g.b * p.MB + lb);
     }
   }
+  return ids;
+}
+
+// TMA loads of that key tile of K and of V, box by box.
+__device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g, const PfIds& ids,
+                                            const CUtensorMap* map_k, const CUtensorMap* map_v,
+                                            unsigned char* dst_k, unsigned char* dst_v, uint64_t* bar_k,
+                                            uint64_t* bar_v, int kb, int box_rows, int nch, int& bits,
+                                            uint32_t tx) {
+  const int nbox = kPfBN / box_rows;
+  const int* raw = ids.raw;
   mbar_arrive_expect_tx(bar_k, tx);
   mbar_arrive_expect_tx(bar_v, tx);
 #pragma unroll
@@ -204,33 +223,80 @@ __device__ __forceinline__ void pf_issue_kv(const AttnParams& p, const PfGeom& g
   }
 }
 
-// Geometry of work item `item` (q head, request, pair of 128-row q tiles;
-// items enumerate the longest pairs first).  Returns false for an empty item.
-__device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_pairs, int max_tiles, PfGeom& g) {
-  const int per_pair = p.H_q * p.B;
-  const int pz = item / per_pair, rem = item - pz * per_pair;
-  g.b = rem / p.H_q;
-  g.h = rem - g.b * p.H_q;
-  const int pair = n_pairs - 1 - pz;
-  g.t_begin = clampi(sanitised_start(p, g.b), 0, p.T);
-  g.q_len = clampi(p.seqlens_q[g.b], 0, p.T - g.t_begin);
-  g.q0[0] = pair * 2 * kPfBM;
-  g.q0[1] = g.q0[0] + kPfBM;
+// Work items.  An item is two 128-row q tiles (A, B) of one request that
+// read the same kv head: with an even group size G, the same q rows of two
+// q heads of one kv head ("head pair": both tiles see exactly the same key
+// tiles, so the two softmax groups run in step); otherwise two consecutive q
+// tiles of one q head ("tile pair"); `mode` bit 0 selects head pairs.
+// Items enumerate heads fastest, then requests, then the q-row slots from the
+// last (longest) down, for one CTA per item scheduled by the hardware (the
+// longest start first); or, for the persistent schedule (`mode` bit 1),
+// heads fastest, then slots from the first, then requests, which spreads
+// each request's items, and the empty slots past its end, evenly over the
+// CTAs' fixed strides.
+//
+// The per-request values an item's geometry is computed from are loaded in
+// one batch of independent loads (issued where pf_geom_load is called, so
+// that their latency can overlap other work before pf_geom_finish).
+struct PfRaw {
+  int b, h, slot, c0, c1, q, lk, r0, r1;
+};
+
+__device__ __forceinline__ PfRaw pf_geom_load(const AttnParams& p, int item, int n_slots, int mode) {
+  PfRaw r;
+  const int hn = (mode & 1) ? p.H_q / 2 : p.H_q;   // head slots per request
+  if (mode & 2) {
+    const int rest = item / hn;
+    r.h = item - rest * hn;
+    r.b = rest / n_slots;
+    r.slot = rest - r.b * n_slots;
+  } else {
+    const int per_slot = hn * p.B;
+    const int pz = item / per_slot, rem = item - pz * per_slot;
+    r.b = rem / hn;
+    r.h = rem - r.b * hn;
+    r.slot = n_slots - 1 - pz;
+  }
+  r.c0 = ld_early(p.cu + r.b);
+  r.c1 = ld_early(p.cu + r.b + 1);
+  r.q = ld_early(p.seqlens_q + r.b);
+  r.lk = ld_early(p.seqlen_k + r.b);
+  r.r0 = p.kv_range ? ld_early(p.kv_range + 2 * r.b) : 0;
+  r.r1 = p.kv_range ? ld_early(p.kv_range + 2 * r.b + 1) : INT_MAX;
+  return r;
+}
+
+// Geometry of a work item.  Returns false for an empty item.
+__device__ __forceinline__ bool pf_geom_finish(const AttnParams& p, const PfRaw& r, int max_tiles, int mode,
+                                               PfGeom& g) {
+  g.b = r.b;
+  int start = r.c0;   // the request's first token, as sanitised_start forms it
+  if (!(r.q > 0 && (long long)r.c1 - r.c0 == r.q)) {
+    start = 0;
+    for (int i = 0; i < g.b; ++i) start += max(p.seqlens_q[i], 0);
+  }
+  g.t_begin = clampi(start, 0, p.T);
+  g.q_len = clampi(r.q, 0, p.T - g.t_begin);
+  if (mode & 1) {   // head pair: q heads 2h, 2h + 1 (one kv head, G even), the same rows
+    g.hq[0] = 2 * r.h;
+    g.hq[1] = 2 * r.h + 1;
+    g.q0[0] = g.q0[1] = r.slot * kPfBM;
+  } else {    // tile pair: q head h, rows of two consecutive tiles
+    g.hq[0] = g.hq[1] = r.h;
+    g.q0[0] = r.slot * 2 * kPfBM;
+    g.q0[1] = g.q0[0] + kPfBM;
+  }
   if (g.q0[0] >= g.q_len) return false;
   g.rows[0] = min(kPfBM, g.q_len - g.q0[0]);
   g.rows[1] = max(0, min(kPfBM, g.q_len - g.q0[1]));
-  g.L = max(p.seqlen_k[g.b] + 1, 0);
+  g.L = max(r.lk + 1, 0);
   g.past = max(g.L - g.q_len, 0);
-  g.h_kv = g.h / p.G;
+  g.h_kv = g.hq[0] / p.G;
   const int last_row = g.rows[1] > 0 ? g.q0[1] + g.rows[1] - 1 : g.q0[0] + g.rows[0] - 1;
   const int p_first = g.past + g.q0[0];
   const int p_last = g.past + last_row;
-  g.rlo = 0;
-  int rhi = INT_MAX;
-  if (p.kv_range) {
-    g.rlo = max(p.kv_range[2 * g.b], 0);
-    rhi = p.kv_range[2 * g.b + 1];
-  }
+  g.rlo = max(r.r0, 0);
+  const int rhi = r.r1;
   g.k_first = max(p.window > 0 ? max(0, p_first - p.window + 1) : 0, g.rlo);
   g.k_lo = (g.k_first / kPfBN) * kPfBN;
   g.k_hi = min(min(p_last + 1, g.L), rhi);
@@ -249,6 +315,11 @@ __device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_pai
   return true;
 }
 
+__device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_slots, int max_tiles, int mode,
+                                        PfGeom& g) {
+  return pf_geom_finish(p, pf_geom_load(p, item, n_slots, mode), max_tiles, mode, g);
+}
+
 // Persistent: each CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
 // The K/V ring and every barrier's phases run on across items (phases come
 // from counters, not step indices); the next item's Q is loaded as soon as
@@ -259,7 +330,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                       int n_pairs, int box_rows, int box_shift, int max_tiles, int n_items) {
+                       int n_slots, int mode, int box_rows, int box_shift, int max_tiles, int n_items) {
   using C = PfCfg<D>;
   constexpr uint32_t FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = idesc_f16(FMT, kPfBM, kPfBN, 0);
@@ -272,32 +343,34 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   pdl_trigger();
   SPA_PF_STAMP(tid == 0, 0);
 
-  unsigned char* const sQA = smem + C::OFF_QA;
-  unsigned char* const sQB = smem + C::OFF_QB;
+  unsigned char* const sQ = smem + C::OFF_Q;   // Q tile t of buffer qb at sQ + (2 qb + t) TILE
   unsigned char* sK = smem + C::OFF_K;
   unsigned char* sV = smem + C::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  constexpr int NS = C::NST;
   uint64_t* bar_q = bars + 0;
-  uint64_t* bar_kf = bars + 1;    // [2] K stage full
-  uint64_t* bar_vf = bars + 3;    // [2] V stage full
-  uint64_t* bar_s = bars + 5;     // [2] S of tile A / B written
-  uint64_t* bar_o = bars + 7;     // [2] PV of tile A / B done
-  uint64_t* bar_p = bars + 9;     // [2] P of tile A / B in TMEM (4 warps arrive)
-  uint64_t* bar_e = bars + 11;    // [2] O of tile A / B read out by its epilogue (4 warps arrive)
-  uint64_t* bar_ke = bars + 13;   // [2] K/V stage empty (every MMA reading it is complete)
+  uint64_t* bar_kf = bars + 1;               // [NS] K stage full
+  uint64_t* bar_vf = bar_kf + NS;            // [NS] V stage full
+  uint64_t* bar_ke = bar_vf + NS;            // [NS] K/V stage empty (every MMA reading it is complete)
+  uint64_t* bar_s = bar_ke + NS;             // [2] S of tile A / B written
+  uint64_t* bar_o = bar_s + 2;               // [2] PV of tile A / B done
+  uint64_t* bar_p = bar_o + 2;               // [2] P of tile A / B in TMEM (4 warps arrive)
+  uint64_t* bar_e = bar_p + 2;               // [2] O of tile A / B read out by its epilogue (4 warps arrive)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(bar_kf + i, 1);
       mbar_init(bar_vf + i, 1);
+      mbar_init(bar_ke + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar_s + i, 1);
       mbar_init(bar_o + i, 1);
       mbar_init(bar_p + i, 4);
       mbar_init(bar_e + i, 4);
-      mbar_init(bar_ke + i, 1);
     }
     fence_mbar_init();
     *abort_flag = 0;
@@ -318,7 +391,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 
   // the next item, from `item` on, with key tiles (others need no tensor work)
   auto next_work = [&](int& item, PfGeom& gg) {
-    while (item < n_items && !(pf_geom(p, item, n_pairs, max_tiles, gg) && gg.ntiles > 0)) item += gridDim.x;
+    while (item < n_items && !(pf_geom(p, item, n_slots, max_tiles, mode, gg) && gg.ntiles > 0)) item += gridDim.x;
     return item < n_items;
   };
   // registers: warpgroup 2 (issue: warps 8-11) releases, the softmax
@@ -327,9 +400,9 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     setmaxnreg_dec<kPfIssueRegs>();
   } else if (warp == 9) {
     setmaxnreg_dec<kPfIssueRegs>();
-    // =================== K/V producer: the 2-stage ring over the CTA's key tiles ===================
-    // Tile c of the stream goes to stage c % 2 once the MMAs of tile c - 2 are
-    // complete (bar_ke), so the loads run ahead of the MMA warp.
+    // =================== K/V producer: the NS-stage ring over the CTA's key tiles ===================
+    // Tile c of the stream goes to stage c % NS once the MMAs of tile c - NS
+    // are complete (bar_ke), so the loads run ahead of the MMA warp.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -339,10 +412,11 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       PfGeom g;
       while (ok && next_work(item, g)) {
         for (int j = 0; j < g.ntiles && ok; ++j) {
-          const int st = c & 1;
-          if (c >= 2) ok = mbar_wait(bar_ke + st, ((c >> 1) - 1) & 1, kPfWaitLimit, abort_flag);
+          const int st = c % NS;
+          const PfIds ids = pf_kv_ids(p, g, g.k_lo + j * kPfBN, box_rows);
+          if (c >= NS) ok = mbar_wait(bar_ke + st, ((c / NS) - 1) & 1, kPfWaitLimit, abort_flag);
           if (!ok) break;
-          pf_issue_kv(p, g, &tm_k, &tm_v, sK + st * C::TILE, sV + st * C::TILE, bar_kf + st, bar_vf + st,
+          pf_issue_kv(p, g, ids, &tm_k, &tm_v, sK + st * C::TILE, sV + st * C::TILE, bar_kf + st, bar_vf + st,
                       g.k_lo + j * kPfBN, box_rows, C::NCH, bits, C::TX_TILE);
           SPA_PF_STAMP(c < 4, 40 + c);   // K/V tile c of the CTA's stream issued
           kv_issued = ++c;
@@ -352,9 +426,9 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       if (!ok) {   // the copies still in flight land before the CTA leaves (bounded)
         *abort_flag = 1;
         bits |= SPA_ST_TIMEOUT;
-        for (int k = c >= 2 ? c - 2 : 0; k < c; ++k) {
-          mbar_wait(bar_kf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
-          mbar_wait(bar_vf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
+        for (int k = c >= NS ? c - NS : 0; k < c; ++k) {
+          mbar_wait(bar_kf + k % NS, (k / NS) & 1, kPfWaitLimit);
+          mbar_wait(bar_vf + k % NS, (k / NS) & 1, kPfWaitLimit);
         }
       }
     }
@@ -363,25 +437,32 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     // =================== MMA issuer and Q loads (one thread) ===================
     if (lane == 0) {
       prefetch_tmap(&tm_q);
-      auto issue_q = [&](const PfGeom& gg) {
+      // Q of an item into buffer qb (completes one phase of bar_q; at most
+      // one such phase is outstanding at a time)
+      auto issue_q = [&](const PfGeom& gg, int qb) {
         const bool two = gg.rows[1] > 0;
+        unsigned char* const dq = sQ + 2 * qb * C::TILE;
         mbar_arrive_expect_tx(bar_q, (two ? 2 : 1) * C::TX_TILE);
         for (int c = 0; c < C::NCH; ++c) {
-          tma_load_3d(sQA + c * C::CHUNK, &tm_q, bar_q, c * 64, gg.h, gg.t_begin + gg.q0[0]);
-          if (two) tma_load_3d(sQB + c * C::CHUNK, &tm_q, bar_q, c * 64, gg.h, gg.t_begin + gg.q0[1]);
+          tma_load_3d(dq + c * C::CHUNK, &tm_q, bar_q, c * 64, gg.hq[0], gg.t_begin + gg.q0[0]);
+          if (two)
+            tma_load_3d(dq + C::TILE + c * C::CHUNK, &tm_q, bar_q, c * 64, gg.hq[1], gg.t_begin + gg.q0[1]);
         }
       };
       int c_use = 0;                              // key tiles consumed (stream index)
       int q_iss = 0, q_seen = 0;
       int s_iss[2] = {0, 0}, o_iss[2] = {0, 0}, o_seen[2] = {0, 0}, p_seen[2] = {0, 0};
-      int e_due[2] = {0, 0}, e_seen[2] = {0, 0}, ke_iss[2] = {0, 0};
+      int e_due[2] = {0, 0}, e_seen[2] = {0, 0}, ke_iss[NS] = {};
       int ci = blockIdx.x;
       PfGeom g;
       bool have = next_work(ci, g);
       if (have) {
-        issue_q(g);
+        issue_q(g, 0);
         ++q_iss;
       }
+      int cn = ci;     // with two Q buffers: the next item, taken up while this one runs
+      PfGeom gn;
+      bool have_n = false;
       SPA_PF_STAMP(true, 44);   // first Q issued
       bool ok = true;
       // wait for the outstanding PV of tile t (at most one)
@@ -391,11 +472,11 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           if (ok) ++o_seen[t];
         }
       };
-      // S_t = Q_t K^T for the key tile in `stage`
-      auto issue_s = [&](int t, int stage) {
+      // S_t = Q_t K^T for the key tile in `stage` (Q from buffer qb)
+      auto issue_s = [&](int t, int stage, int qb) {
         tc_fence_after();
         const uint32_t tS = tmem + t * 128;
-        unsigned char* const sq = t ? sQB : sQA;
+        unsigned char* const sq = sQ + (2 * qb + t) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk / 4, koff = (kk % 4) * 32;
@@ -414,9 +495,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         const int ntq = g.rows[1] > 0 ? 2 : 1;
         auto need = [&](int t, int j) { return t ? (j >= g.j_lo[1] && j < g.j_hi[1]) : (j >= g.j_lo[0] && j < g.j_hi[0]); };
         bool pv_any[2] = {false, false};   // a PV of tile t issued in this item
+        const int qb = q_seen % C::NQB;    // this item's Q buffer
         {   // step 0: S of every q tile that sees key tile 0 (after the tile's previous PV)
-          const int st = c_use & 1;
-          const uint32_t ph = (c_use >> 1) & 1;
+          const int st = c_use % NS;
+          const uint32_t ph = (c_use / NS) & 1;
           ok = mbar_wait(bar_kf + st, ph, kPfWaitLimit, abort_flag);
           SPA_PF_STAMP(q_seen < 2, 45 + 2 * q_seen);   // item's first K tile landed
           if (ok) {
@@ -427,15 +509,28 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           for (int t = 0; t < ntq && ok; ++t) {
             if (!need(t, 0)) continue;
             pv_done(t);   // S_t overwrites P_t of the tile's previous step
-            if (ok) issue_s(t, st);
+            if (ok) issue_s(t, st, qb);
+          }
+        }
+        if constexpr (C::NQB == 2) {
+          // the other buffer held the previous item's Q, whose S MMAs are all
+          // complete (every P of that item was observed): the next item's Q
+          // goes there now and lands while this item runs
+          if (ok) {
+            cn = ci + gridDim.x;
+            have_n = next_work(cn, gn);
+            if (have_n) {
+              issue_q(gn, qb ^ 1);
+              ++q_iss;
+            }
           }
         }
         for (int j = 0; j < g.ntiles && ok; ++j) {
-          const int st = c_use & 1;
-          const uint32_t ph = (c_use >> 1) & 1;
+          const int st = c_use % NS;
+          const uint32_t ph = (c_use / NS) & 1;
           const bool more = j + 1 < g.ntiles;
-          const int st1 = (c_use + 1) & 1;
-          const uint32_t ph1 = ((c_use + 1) >> 1) & 1;
+          const int st1 = (c_use + 1) % NS;
+          const uint32_t ph1 = ((c_use + 1) / NS) & 1;
           bool k_next = false;
           ok = mbar_wait(bar_vf + st, ph, kPfWaitLimit, abort_flag);
           for (int t = 0; t < ntq && ok; ++t) {
@@ -477,7 +572,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
                 k_next = true;
               }
               pv_done(t);   // P_t(j) consumed: S_t(j+1) may overwrite it
-              if (ok) issue_s(t, st1);
+              if (ok) issue_s(t, st1, qb);
             }
           }
           if (!ok) break;
@@ -487,11 +582,17 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         for (int t = 0; t < ntq; ++t)
           if (pv_any[t]) ++e_due[t];
         // every P of this item was observed, so its S MMAs are complete: Q may be replaced
-        ci += gridDim.x;
-        have = next_work(ci, g);
-        if (have) {
-          issue_q(g);
-          ++q_iss;
+        if constexpr (C::NQB == 2) {
+          ci = cn;
+          g = gn;
+          have = have_n;
+        } else {
+          ci += gridDim.x;
+          have = next_work(ci, g);
+          if (have) {
+            issue_q(g, 0);
+            ++q_iss;
+          }
         }
       }
       if (!ok) {
@@ -506,7 +607,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         for (int q = q_seen; q < q_iss; ++q) mbar_wait(bar_q, q & 1, kPfWaitLimit);
       }
       // the last stage-empty arrivals land before the CTA leaves (bounded)
-      for (int st = 0; st < 2; ++st)
+      for (int st = 0; st < NS; ++st)
         if (ke_iss[st] > 0) mbar_wait(bar_ke + st, (ke_iss[st] - 1) & 1, kPfWaitLimit);
     }
   } else {
@@ -526,12 +627,20 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     const int pbase = tid == 0 ? 1 : 21;
     (void)pr;
     (void)pbase;
+    // the raw per-request values of the group's next item are loaded ahead
+    // (before the current item's epilogue), so that its geometry is ready
+    PfRaw raw;
+    if ((int)blockIdx.x < n_items) raw = pf_geom_load(p, blockIdx.x, n_slots, mode);
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       PfGeom g;
-      if (!pf_geom(p, item, n_pairs, max_tiles, g)) continue;
+      const bool valid = pf_geom_finish(p, raw, max_tiles, mode, g);
+      const int item_next = item + gridDim.x;
       const int q0_t = t ? g.q0[1] : g.q0[0];
       const int rows_t = t ? g.rows[1] : g.rows[0];
-      if (rows_t <= 0) continue;
+      if (!valid || rows_t <= 0) {
+        if (item_next < n_items) raw = pf_geom_load(p, item_next, n_slots, mode);
+        continue;
+      }
       const int prow = g.past + q0_t + r;
       const int p_lo = g.past + q0_t;                         // first row of this tile
       const int p_hi = g.past + q0_t + rows_t - 1;
@@ -658,6 +767,9 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         SPA_PF_STAMP(pr && n_it < 2 && j < 3, pbase + n_it * 10 + 2 + 2 * j);   // P(j) handed over
       }
       if (!ok) break;
+      if (item_next < n_items) raw = pf_geom_load(p, item_next, n_slots, mode);
+      const int hq = g.hq[t];
+      const float sink_v = p.sinks ? ld_early(p.sinks + hq) : 0.f;
       // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
       bool have_o = j_hi > j_lo;
       if (have_o) {
@@ -672,8 +784,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         tc_fence_after();
         const bool mine = r < rows_t;
         const int tok = g.t_begin + q0_t + r;
-        const long long orow = (long long)tok * p.H_q + g.h;
-        const float sink2 = p.sinks ? p.sinks[g.h] * kLog2e : -INFINITY;
+        const long long orow = (long long)tok * p.H_q + hq;
+        const float sink2 = p.sinks ? sink_v * kLog2e : -INFINITY;
         float a, inv_l, lse;
         finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
         const float f = a * inv_l;
@@ -720,13 +832,13 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   __syncthreads();
   if (*abort_flag) {
     bits |= SPA_ST_TIMEOUT;
-    // another role gave up: the producer's last two K/V tiles may still be in
+    // another role gave up: the producer's last NS K/V tiles may still be in
     // flight although it finished issuing normally; they land before the CTA
     // leaves (bounded; the latest phase of each stage is unambiguous)
     if (warp == 9 && lane == 0)
-      for (int k = kv_issued >= 2 ? kv_issued - 2 : 0; k < kv_issued; ++k) {
-        mbar_wait(bar_kf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
-        mbar_wait(bar_vf + (k & 1), (k >> 1) & 1, kPfWaitLimit);
+      for (int k = kv_issued >= NS ? kv_issued - NS : 0; k < kv_issued; ++k) {
+        mbar_wait(bar_kf + k % NS, (k / NS) & 1, kPfWaitLimit);
+        mbar_wait(bar_vf + k % NS, (k / NS) & 1, kPfWaitLimit);
       }
   }
   flag(p.status, bits);
@@ -804,8 +916,10 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   if ((rc = encode(&tq, dt, 3, p.q, qd, qs, qb)) != SPA_OK) return rc;
   if ((rc = encode(&tk, dt, 4, p.k_cache, kd, ks, kbx)) != SPA_OK) return rc;
   if ((rc = encode(&tv, dt, 4, p.v_cache, kd, ks, kbx)) != SPA_OK) return rc;
-  const int n_pairs = (p.max_q + 2 * kPfBM - 1) / (2 * kPfBM);
-  const long long items = (long long)p.H_q * p.B * n_pairs;
+  // head pairs when the group size is even, tile pairs otherwise (see pf_geom_load)
+  const int hp = (p.G % 2 == 0) ? 1 : 0;
+  const int n_slots = hp ? (p.max_q + kPfBM - 1) / kPfBM : (p.max_q + 2 * kPfBM - 1) / (2 * kPfBM);
+  const long long items = (long long)(hp ? p.H_q / 2 : p.H_q) * p.B * n_slots;
   if (items > 0x7fffffffLL) return SPA_ERR_UNSUPPORTED;
   const int max_tiles = (p.max_k + kPfBN - 1) / kPfBN + 1;
   auto kern = prefill_tcgen05_kernel<T, D>;
@@ -817,9 +931,8 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
     return SPA_ERR_UNSUPPORTED;
   }
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  // persistent: one CTA per SM (all of TMEM, over half the shared memory),
-  // items = heads fastest, then requests, then q-tile pairs from the last
-  // (longest) down
+  // persistent: one CTA per SM (all of TMEM, over half the shared memory);
+  // the item order of each schedule is described at pf_geom_load
   // Short items (a window of at most two key tiles) run persistently, one CTA
   // per SM looping over them, so the per-CTA set-up and pipeline fill are paid
   // once per SM; long causal items keep one CTA each, which the hardware
@@ -829,7 +942,8 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const bool persistent = p.window > 0 && p.window <= 2 * kPfBN;
   const int grid = persistent ? (int)std::min<long long>(items, std::max(sms, 1)) : (int)items;
-  return launch_pdl(kern, dim3(grid), dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_pairs, box_rows,
+  const int mode = hp | (persistent ? 2 : 0);
+  return launch_pdl(kern, dim3(grid), dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_slots, mode, box_rows,
                     box_shift, max_tiles, (int)items);
 }
 
