@@ -257,9 +257,10 @@ typedef struct spa_attention_args {
   int32_t test_expire_wait;
 } spa_attention_args_t;
 
-/* Bytes of workspace spa_attention needs for these arguments (0 if none: one
-   split per unit).  Returns 0 as well for invalid arguments; spa_attention
-   then reports the error. */
+/* Bytes of workspace spa_attention needs for these arguments (0 if none:
+   decode with one split per unit, prefill without a local window of at most
+   256 keys).  Returns 0 as well for invalid arguments; spa_attention then
+   reports the error. */
 size_t spa_attention_workspace_size(const spa_attention_args_t* a);
 
 /*
@@ -276,10 +277,13 @@ size_t spa_attention_workspace_size(const spa_attention_args_t* a);
  * on num_splits beyond rounding.
  * workspace: device buffer of at least spa_attention_workspace_size() bytes,
  * 256-byte aligned; it may be NULL when the size is 0.  It holds the splits'
- * FP32 partial states (no initialisation needed) and, for plans that merge by
- * ticket, per-unit split tickets: those must be zero before the first use and
- * every call leaves them at zero again, so zero-fill a new workspace.  Calls
- * that share a workspace must be ordered on one stream.  The whole operation
+ * FP32 partial states (no initialisation needed), for plans that merge by
+ * ticket per-unit split tickets, and for prefill with a local window of at
+ * most 256 keys (one CTA per SM looping over work items) the work counter
+ * the CTAs claim items from: tickets and counter must be zero before the
+ * first use and every call leaves them at zero again (also when a bounded
+ * wait expired), so zero-fill a new workspace.  Calls that share a workspace
+ * must be ordered on one stream.  The whole operation
  * is one kernel launch: on the tensor-core decode kernels the (at most 8)
  * splits of a unit form one thread-block cluster, write their partial states
  * to the workspace, pass a cluster barrier and merge a share of the rows
@@ -422,8 +426,8 @@ int spa_prepare_qkv_append(const spa_qkv_args_t* a, spa_stream_t stream);
  * and no allocating routine.
  *   - A call whose plan needs more scratch than SPA_NOALLOC_SCRATCH_BYTES
  *     (spa_attention_workspace_size() of the same arguments) returns
- *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.  Plans with one split per
- *     unit need no scratch at all.
+ *     SPA_ERR_SCRATCH_LIMIT and enqueues nothing.  Plans whose
+ *     spa_attention_workspace_size() is 0 need no scratch at all.
  *   - The first call on each device resolves the array's device address (with
  *     that device current); make that first call before any stream capture.
  *     Every later call made outside a capture resolves it again; a call made

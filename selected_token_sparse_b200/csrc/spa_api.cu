@@ -36,6 +36,7 @@ int launch_prepare_qkv_append(const QkvParams& P, int act, int cache, cudaStream
 int mma_step_fits(int D, int max_rows, int B);
 int launch_prefill(const AttnParams& p, int act, cudaStream_t stream);
 int prefill_supported(const spa_attention_args_t* a);
+size_t prefill_ticket_bytes(const spa_attention_args_t* a);
 
 static thread_local char g_cuda_msg[256] = "no CUDA error recorded";
 
@@ -101,6 +102,7 @@ int make_plan(const spa_attention_args_t* a, Plan* pl) {
   if (prefill_supported(a)) {
     pl->kind = kPlanPrefill;
     pl->num_splits = 1;
+    pl->ws_count_bytes = prefill_ticket_bytes(a);   // the persistent schedule's work counter
     return SPA_OK;
   }
   // group all tokens of a request when their rows fit one CTA and the
@@ -205,6 +207,7 @@ void fill_params(const spa_attention_args_t* a, const Plan& pl, void* ws, AttnPa
   p->split_len = pl.split_len;
   p->status = a->status;
   p->cluster_merge = pl.cluster_merge;
+  if (pl.kind == kPlanPrefill && pl.ws_count_bytes > 0) p->ws_count = static_cast<int*>(ws);
   if (pl.num_splits > 1) {
     p->ws_acc = static_cast<float*>(ws);
     p->ws_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.ws_acc_bytes);

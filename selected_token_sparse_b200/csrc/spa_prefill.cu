@@ -77,6 +77,7 @@ constexpr int kPfBM = 128;   // q rows per tile (TMEM lanes)
 constexpr int kPfBN = 128;   // keys per step
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint32_t kPfWaitLimit = 1u << 20;   // polls before a wait is declared lost
+constexpr int kPfRing = 4;                     // item slots of the dynamic schedule
 // 3 warpgroups: softmax A (warps 0-3), softmax B (4-7), and warps 8-11: the
 // MMA warp, the K/V TMA warp and two idle warps.  The kernel is compiled for
 // kPfLaunchRegs registers a thread (one CTA per SM); the third warpgroup hands
@@ -105,10 +106,11 @@ struct PfCfg {
   static constexpr int OFF_K = OFF_Q + NQB * 2 * TILE;   // NST stages
   static constexpr int OFF_V = OFF_K + NST * TILE;     // NST stages
   static constexpr int OFF_BAR = OFF_V + NST * TILE;   // mbarriers
-  static constexpr int NBAR = 1 + 3 * NST + 8;
+  static constexpr int NBAR = 1 + 3 * NST + 8 + 2 * kPfRing;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_FLAG = OFF_TMEM + 8;
-  static constexpr int BYTES = OFF_FLAG + 8;
+  static constexpr int OFF_RING = OFF_FLAG + 8;       // [kPfRing] item indices
+  static constexpr int BYTES = OFF_RING + 4 * kPfRing;
   // + alignment slack; above half of the SM's shared memory so that exactly
   // one CTA (holding all 512 TMEM columns) is resident per SM
   static constexpr int SMEM = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
@@ -320,13 +322,21 @@ __device__ __forceinline__ bool pf_geom(const AttnParams& p, int item, int n_slo
   return pf_geom_finish(p, pf_geom_load(p, item, n_slots, mode), max_tiles, mode, g);
 }
 
-// Persistent: each CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...
+// Items: one CTA per item (grid = items), or persistent with a static
+// stride (items blockIdx.x, blockIdx.x + gridDim.x, ...), or persistent with
+// a dynamic schedule (`mode` bit 2, a work counter in the workspace): every
+// CTA starts with item blockIdx.x, then its producer thread claims items
+// gridDim.x + atomicAdd(counter, 1) as it needs them and publishes them, two
+// ahead, through a ring of kPfRing slots in shared memory (bar_if: slot
+// written, bar_ie: slot read by the MMA thread and the 8 softmax warps);
+// every role reads the same sequence, ended by -1.  The last CTA to finish
+// puts the counter back to zero.
 // The K/V ring and every barrier's phases run on across items (phases come
 // from counters, not step indices); the next item's Q is loaded as soon as
 // the current item's last P has been observed (its S MMAs are complete), and
 // a tile's first PV of an item waits until the softmax group has read the
 // previous item's O out of TMEM (bar_e).
-template <typename T, int D>
+template <typename T, int D, bool DYN>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -356,6 +366,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   uint64_t* bar_o = bar_s + 2;               // [2] PV of tile A / B done
   uint64_t* bar_p = bar_o + 2;               // [2] P of tile A / B in TMEM (4 warps arrive)
   uint64_t* bar_e = bar_p + 2;               // [2] O of tile A / B read out by its epilogue (4 warps arrive)
+  uint64_t* bar_if = bar_e + 2;              // [kPfRing] item slot written (producer)
+  uint64_t* bar_ie = bar_if + kPfRing;       // [kPfRing] item slot read (MMA thread + 8 softmax warps)
+  volatile int* ring = reinterpret_cast<volatile int*>(smem + C::OFF_RING);
+  constexpr bool dyn = DYN;   // `mode` bit 2 (the instance without it carries none of its code)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
 
@@ -371,6 +385,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       mbar_init(bar_o + i, 1);
       mbar_init(bar_p + i, 4);
       mbar_init(bar_e + i, 4);
+    }
+    for (int i = 0; i < kPfRing; ++i) {
+      mbar_init(bar_if + i, 1);
+      mbar_init(bar_ie + i, 9);
     }
     fence_mbar_init();
     *abort_flag = 0;
@@ -410,7 +428,42 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       bool ok = true;
       int item = blockIdx.x;
       PfGeom g;
-      while (ok && next_work(item, g)) {
+      // dynamic schedule: claim items (from `it` on; -1: from the counter)
+      // until one has key tiles, or -1 when none is left
+      const int hn = (mode & 1) ? p.H_q / 2 : p.H_q;
+      auto claim = [&](int it) -> int {
+        PfGeom gg;
+        for (;;) {
+          if (it < 0) it = (int)gridDim.x + atomicAdd(p.ws_count, 1);
+          if (it >= n_items) return -1;
+          const PfRaw r = pf_geom_load(p, it, n_slots, mode);
+          if (pf_geom_finish(p, r, max_tiles, mode, gg)) {
+            if (gg.ntiles > 0) return it;
+          } else {   // past the request's last q rows: so are its later items (request-major order)
+            atomicMax(p.ws_count, (r.b + 1) * n_slots * hn - (int)gridDim.x);
+          }
+          it = -1;
+        }
+      };
+      int k_pub = 0;   // items published
+      auto publish = [&](int it) {
+        const int sl = k_pub % kPfRing;
+        if (k_pub >= kPfRing) ok = ok && mbar_wait(bar_ie + sl, ((k_pub / kPfRing) - 1) & 1, kPfWaitLimit, abort_flag);
+        if (!ok) return;
+        ring[sl] = it;
+        mbar_arrive(bar_if + sl);
+        ++k_pub;
+      };
+      int nxt = -1, nnx = -1;
+      if (dyn) {
+        item = claim((int)blockIdx.x < n_items ? (int)blockIdx.x : n_items);
+        publish(item);
+        if (item >= 0) {
+          nxt = claim(-1);
+          publish(nxt);
+        }
+      }
+      while (ok && (dyn ? (item >= 0 && pf_geom(p, item, n_slots, max_tiles, mode, g)) : next_work(item, g))) {
         for (int j = 0; j < g.ntiles && ok; ++j) {
           const int st = c % NS;
           const PfIds ids = pf_kv_ids(p, g, g.k_lo + j * kPfBN, box_rows);
@@ -420,8 +473,18 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
                       g.k_lo + j * kPfBN, box_rows, C::NCH, bits, C::TX_TILE);
           SPA_PF_STAMP(c < 4, 40 + c);   // K/V tile c of the CTA's stream issued
           kv_issued = ++c;
+          if (dyn && j == 0 && nxt >= 0) {   // keep two items published ahead
+            nnx = claim(-1);
+            publish(nnx);
+          }
         }
-        item += gridDim.x;
+        if (dyn) {
+          item = nxt;
+          nxt = nnx;
+          nnx = -1;
+        } else {
+          item += gridDim.x;
+        }
       }
       if (!ok) {   // the copies still in flight land before the CTA leaves (bounded)
         *abort_flag = 1;
@@ -453,9 +516,25 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       int q_iss = 0, q_seen = 0;
       int s_iss[2] = {0, 0}, o_iss[2] = {0, 0}, o_seen[2] = {0, 0}, p_seen[2] = {0, 0};
       int e_due[2] = {0, 0}, e_seen[2] = {0, 0}, ke_iss[NS] = {};
+      bool ok = true;
+      int k_get = 0;   // item slots read (dynamic schedule)
+      // the CTA's next item after `it` (first: its first item); false when none is left
+      auto take = [&](int& it, PfGeom& gg, bool first) -> bool {
+        if (!dyn) {
+          if (!first) it += gridDim.x;
+          return next_work(it, gg);
+        }
+        const int sl = k_get % kPfRing;
+        ok = ok && mbar_wait(bar_if + sl, (k_get / kPfRing) & 1, kPfWaitLimit, abort_flag);
+        if (!ok) return false;
+        it = ring[sl];
+        mbar_arrive(bar_ie + sl);
+        ++k_get;
+        return it >= 0 && pf_geom(p, it, n_slots, max_tiles, mode, gg);
+      };
       int ci = blockIdx.x;
       PfGeom g;
-      bool have = next_work(ci, g);
+      bool have = take(ci, g, true);
       if (have) {
         issue_q(g, 0);
         ++q_iss;
@@ -464,7 +543,6 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       PfGeom gn;
       bool have_n = false;
       SPA_PF_STAMP(true, 44);   // first Q issued
-      bool ok = true;
       // wait for the outstanding PV of tile t (at most one)
       auto pv_done = [&](int t) {
         while (ok && o_seen[t] < o_iss[t]) {
@@ -517,8 +595,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           // complete (every P of that item was observed): the next item's Q
           // goes there now and lands while this item runs
           if (ok) {
-            cn = ci + gridDim.x;
-            have_n = next_work(cn, gn);
+            cn = ci;
+            have_n = take(cn, gn, false);
             if (have_n) {
               issue_q(gn, qb ^ 1);
               ++q_iss;
@@ -587,8 +665,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           g = gn;
           have = have_n;
         } else {
-          ci += gridDim.x;
-          have = next_work(ci, g);
+          have = take(ci, g, false);
           if (have) {
             issue_q(g, 0);
             ++q_iss;
@@ -629,16 +706,39 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     (void)pbase;
     // the raw per-request values of the group's next item are loaded ahead
     // (before the current item's epilogue), so that its geometry is ready
+    int k_get = 0;   // item slots this warp has read (dynamic schedule)
+    // the warp's next item after `prev` (-1: its first), or -1 when none is left
+    auto take = [&](int prev) -> int {
+      if (!dyn) {
+        const int it = prev < 0 ? (int)blockIdx.x : prev + (int)gridDim.x;
+        return it < n_items ? it : -1;
+      }
+      const int sl = k_get % kPfRing;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar_if + sl, (k_get / kPfRing) & 1, kPfWaitLimit,
+                                                         abort_flag));
+      if (!got) {
+        ok = false;
+        return -1;
+      }
+      const int it = ring[sl];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_ie + sl);
+      ++k_get;
+      return it;
+    };
+    int item = take(-1);
     PfRaw raw;
-    if ((int)blockIdx.x < n_items) raw = pf_geom_load(p, blockIdx.x, n_slots, mode);
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    if (item >= 0) raw = pf_geom_load(p, item, n_slots, mode);
+    for (; item >= 0 && ok;) {
       PfGeom g;
       const bool valid = pf_geom_finish(p, raw, max_tiles, mode, g);
-      const int item_next = item + gridDim.x;
+      const int item_next = take(item);
+      if (!ok) break;
       const int q0_t = t ? g.q0[1] : g.q0[0];
       const int rows_t = t ? g.rows[1] : g.rows[0];
       if (!valid || rows_t <= 0) {
-        if (item_next < n_items) raw = pf_geom_load(p, item_next, n_slots, mode);
+        if (item_next >= 0) raw = pf_geom_load(p, item_next, n_slots, mode);
+        item = item_next;
         continue;
       }
       const int prow = g.past + q0_t + r;
@@ -767,7 +867,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         SPA_PF_STAMP(pr && n_it < 2 && j < 3, pbase + n_it * 10 + 2 + 2 * j);   // P(j) handed over
       }
       if (!ok) break;
-      if (item_next < n_items) raw = pf_geom_load(p, item_next, n_slots, mode);
+      if (item_next >= 0) raw = pf_geom_load(p, item_next, n_slots, mode);
       const int hq = g.hq[t];
       const float sink_v = p.sinks ? ld_early(p.sinks + hq) : 0.f;
       // ---- epilogue: wait for the last PV of this tile, normalise with the sink, store
@@ -826,6 +926,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       }
       SPA_PF_STAMP(pr && n_it < 2, pbase + n_it * 10 + 8);   // epilogue stored
       ++n_it;
+      item = item_next;
     }
     if (!ok) *abort_flag = 1;
   }
@@ -847,6 +948,15 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kPfTmemCols);
+  }
+  // dynamic schedule: every role of this CTA is done claiming; the last CTA
+  // to get here puts the work counter (and this ticket) back to zero
+  if (dyn && tid == 0) {
+    __threadfence();
+    if (atomicAdd(p.ws_count + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(p.ws_count, 0);
+      atomicExch(p.ws_count + 1, 0);
+    }
   }
   SPA_PF_STAMP(tid == 0, 50);   // CTA end
 }
@@ -872,6 +982,14 @@ static EncodeTiledFn encode_fn() {
   });
   return fn;
 }
+
+// Short items (a window of at most two key tiles) run persistently, one CTA
+// per SM looping over them (see launch_pf).
+static bool pf_persistent(int window) { return window > 0 && window <= 2 * kPfBN; }
+
+// Workspace of a prefill plan: the persistent schedule's work counter and
+// its end-of-launch ticket (zero between calls).
+size_t prefill_ticket_bytes(const spa_attention_args_t* a) { return pf_persistent(a->window) ? 256 : 0; }
 
 int prefill_supported(const spa_attention_args_t* a) {
   if (a->act != SPA_F16 && a->act != SPA_BF16) return 0;
@@ -922,7 +1040,12 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   const long long items = (long long)(hp ? p.H_q / 2 : p.H_q) * p.B * n_slots;
   if (items > 0x7fffffffLL) return SPA_ERR_UNSUPPORTED;
   const int max_tiles = (p.max_k + kPfBN - 1) / kPfBN + 1;
-  auto kern = prefill_tcgen05_kernel<T, D>;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool persistent = pf_persistent(p.window);
+  // persistent items are claimed from a counter in the workspace when there is one
+  const bool dyn = persistent && p.ws_count != nullptr;
+  auto kern = dyn ? prefill_tcgen05_kernel<T, D, true> : prefill_tcgen05_kernel<T, D, false>;
   // the register hand-over (setmaxnreg) balances only at the launch register
   // count it was written for: a build with another count is not launched
   cudaFuncAttributes fa;
@@ -938,11 +1061,8 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   // once per SM; long causal items keep one CTA each, which the hardware
   // schedules dynamically (a static assignment of the unequal causal items
   // measured slower).
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const bool persistent = p.window > 0 && p.window <= 2 * kPfBN;
   const int grid = persistent ? (int)std::min<long long>(items, std::max(sms, 1)) : (int)items;
-  const int mode = hp | (persistent ? 2 : 0);
+  const int mode = hp | (persistent ? 2 : 0) | (dyn ? 4 : 0);
   return launch_pdl(kern, dim3(grid), dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_slots, mode, box_rows,
                     box_shift, max_tiles, (int)items);
 }

@@ -313,7 +313,7 @@ def attention_args(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
-    """A zero-filled workspace (its split tickets must start at zero)."""
+    """A zero-filled workspace (its tickets and work counter must start at zero)."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 

@@ -23,15 +23,27 @@ def _result(wl, st, d):
     return got
 
 
-def test_expired_wait_sets_timeout_and_the_next_call_is_correct():
-    wl = W.by_name("ragged_prefill_f16", small=True)
+def _counter_words(st):
+    """The persistent schedule's work counter and ticket (zero between calls)."""
+    if spa.workspace_size(st.args) == 0:
+        return [0, 0]
+    return st.workspace[:8].view(torch.int32).tolist()
+
+
+# one CTA per item (causal) and the persistent schedule with its work counter (window)
+@pytest.mark.parametrize("name", ["ragged_prefill_f16", "windowed_chunked_prefill_f16"])
+def test_expired_wait_sets_timeout_and_the_next_call_is_correct(name):
+    wl = W.by_name(name, small=True)
     d = pipeline.to_device(wl)
     st = pipeline.Step(wl, d, want_lse=True)
     assert spa.attention_plan(st.args)["kind"] == 2          # the tcgen05 prefill kernel
+    if name.startswith("windowed"):
+        assert spa.workspace_size(st.args) > 0              # the counter lives in the workspace
     ref = oracle_step(wl)
     st()                                                     # metadata, append, attention
     torch.cuda.synchronize()
     compare(wl, _result(wl, st, d), ref, strict=True)
+    assert _counter_words(st) == [0, 0]
 
     # the same attention call with the hook: a wait expires in every CTA
     st.status.zero_()
@@ -39,6 +51,7 @@ def test_expired_wait_sets_timeout_and_the_next_call_is_correct():
     spa.run_attention(st.args, st.workspace)                 # returns: nothing hangs
     torch.cuda.synchronize()
     assert int(st.status.item()) & SPA_ST_TIMEOUT
+    assert _counter_words(st) == [0, 0]                      # put back although the CTAs gave up
 
     # the context is intact: the next normal calls on the stream are correct
     st.args.test_expire_wait = 0
@@ -48,3 +61,4 @@ def test_expired_wait_sets_timeout_and_the_next_call_is_correct():
         spa.run_attention(st.args, st.workspace)
         torch.cuda.synchronize()
         compare(wl, _result(wl, st, d), ref, strict=True)
+        assert _counter_words(st) == [0, 0]

@@ -29,12 +29,14 @@ def _entry(lib):
 # Every split plan's partial states travel through the scratch array: up to 8
 # splits on the tensor-core kernels (one cluster per unit, merged after a
 # cluster barrier), more than 8 there (the last CTA of a unit merges, with
-# tickets), and the CUDA-core kernel (tickets).  The sequence mixes workloads
-# so that a call finds the previous call's partials (of another shape) in the
-# array.
+# tickets), and the CUDA-core kernel (tickets); the windowed prefill's
+# persistent schedule keeps its work counter there.  The sequence mixes
+# workloads so that a call finds the previous call's partials (of another
+# shape) in the array -- the prefill's counter words among them.
 CASES = [("gptoss_paged_decode_f16", 16), ("tiny_decode_f32", 3), ("local_plus_selected_int8", 12),
-         ("selected_decode_bf16", 4), ("selected_decode_bf16", 32), ("local_plus_selected_int8", 3),
-         ("tiny_decode_f32", 5), ("gptoss_paged_decode_f16", 2), ("gptoss_paged_decode_f16", 16)]
+         ("windowed_chunked_prefill_f16", 1), ("selected_decode_bf16", 4), ("selected_decode_bf16", 32),
+         ("local_plus_selected_int8", 3), ("windowed_chunked_prefill_f16", 1), ("tiny_decode_f32", 5),
+         ("gptoss_paged_decode_f16", 2), ("gptoss_paged_decode_f16", 16)]
 
 
 def _prepare(name, splits):
@@ -51,7 +53,7 @@ def _prepare(name, splits):
                               max_seqlen_q=wl.max_seqlen_q, max_seqlen_k=wl.max_seqlen_k,
                               out=out, lse=lse, num_splits=splits, status=st.status, **st.kw)
     need = spa.workspace_size(args)
-    assert 0 < need <= SCRATCH_LIMIT        # the partials go through the scratch, and they fit
+    assert 0 < need <= SCRATCH_LIMIT        # partials or counters go through the scratch, and they fit
     return wl, st, args, out, lse
 
 
