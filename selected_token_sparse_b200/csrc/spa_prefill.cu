@@ -429,7 +429,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       int item = blockIdx.x;
       PfGeom g;
       // dynamic schedule: claim items (from `it` on; -1: from the counter)
-      // until one has key tiles, or -1 when none is left
+      // until one has q rows, or -1 when none is left.  Items without key
+      // tiles are published too: the softmax warps write their rows.
       const int hn = (mode & 1) ? p.H_q / 2 : p.H_q;
       auto claim = [&](int it) -> int {
         PfGeom gg;
@@ -438,9 +439,12 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           if (it >= n_items) return -1;
           const PfRaw r = pf_geom_load(p, it, n_slots, mode);
           if (pf_geom_finish(p, r, max_tiles, mode, gg)) {
-            if (gg.ntiles > 0) return it;
-          } else {   // past the request's last q rows: so are its later items (request-major order)
-            atomicMax(p.ws_count, (r.b + 1) * n_slots * hn - (int)gridDim.x);
+            return it;
+          } else {
+            // past the request's last q rows: so are the request's other heads
+            // at this slot and, in request-major order, its later slots
+            const int skip = (mode & 2) ? (r.b + 1) * n_slots * hn : (it / hn + 1) * hn;
+            atomicMax(p.ws_count, skip - (int)gridDim.x);
           }
           it = -1;
         }
@@ -464,6 +468,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         }
       }
       while (ok && (dyn ? (item >= 0 && pf_geom(p, item, n_slots, max_tiles, mode, g)) : next_work(item, g))) {
+        if (dyn && g.ntiles == 0 && nxt >= 0) {   // no tiles to issue: keep two items published ahead now
+          nnx = claim(-1);
+          publish(nnx);
+        }
         for (int j = 0; j < g.ntiles && ok; ++j) {
           const int st = c % NS;
           const PfIds ids = pf_kv_ids(p, g, g.k_lo + j * kPfBN, box_rows);
@@ -524,13 +532,16 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           if (!first) it += gridDim.x;
           return next_work(it, gg);
         }
-        const int sl = k_get % kPfRing;
-        ok = ok && mbar_wait(bar_if + sl, (k_get / kPfRing) & 1, kPfWaitLimit, abort_flag);
-        if (!ok) return false;
-        it = ring[sl];
-        mbar_arrive(bar_ie + sl);
-        ++k_get;
-        return it >= 0 && pf_geom(p, it, n_slots, max_tiles, mode, gg);
+        for (;;) {   // items without key tiles need no tensor work
+          const int sl = k_get % kPfRing;
+          ok = ok && mbar_wait(bar_if + sl, (k_get / kPfRing) & 1, kPfWaitLimit, abort_flag);
+          if (!ok) return false;
+          it = ring[sl];
+          mbar_arrive(bar_ie + sl);
+          ++k_get;
+          if (it < 0) return false;
+          if (pf_geom(p, it, n_slots, max_tiles, mode, gg) && gg.ntiles > 0) return true;
+        }
       };
       int ci = blockIdx.x;
       PfGeom g;

@@ -76,7 +76,8 @@ def run_sharded(wl, R, num_splits=0):
     ("gptoss_paged_decode_f16", 2, 0), ("gptoss_paged_decode_f16", 3, 16),
     ("selected_decode_bf16", 4, 0), ("selected_decode_bf16", 3, 3),
     ("local_plus_selected_int8", 2, 0), ("local_plus_selected_int8", 3, 12),
-    ("tiny_decode_f32", 2, 0), ("ragged_prefill_f16", 3, 0), ("windowed_chunked_prefill_f16", 2, 0)])
+    ("tiny_decode_f32", 2, 0), ("ragged_prefill_f16", 3, 0), ("windowed_chunked_prefill_f16", 2, 0),
+    ("windowed_chunked_prefill_f16", 3, 0), ("windowed_chunked_prefill_f16", 4, 0)])
 def test_sharded_partials_merge_to_the_oracle(name, R, splits):
     wl = W.by_name(name, small=True)
     out, lse = run_sharded(wl, R, splits)
