@@ -115,6 +115,17 @@ EDGE = {
     "tc_empty_selection": dict(act="bf16", cache="i8", B=2, H_q=48, H_kv=4, D=128, block_size=64,
                                q_lens=[8, 3], past=[60, 10], sel_mode="main", sel_per_request=1,
                                sel_width=16, sel_valid=0),
+    # tcgen05 prefill work items: an odd group size pairs consecutive q tiles
+    # of one head (the last pair of a request may hold one tile), an even one
+    # pairs two heads; more items than SMs make the persistent (windowed)
+    # schedule claim further items and reuse its Q buffers and K/V stages
+    "prefill_tile_pairs_window_claimed": dict(act="f16", B=4, H_q=15, H_kv=5, D=64, block_size=16,
+                                              q_lens=[600, 260, 100, 513], past=[50, 0, 900, 7],
+                                              window=64),
+    "prefill_tile_pairs_causal_d128": dict(act="f16", B=2, H_q=3, H_kv=1, D=128, block_size=64,
+                                           q_lens=[300, 140], past=[0, 20]),
+    "prefill_head_pairs_window_d128_claimed": dict(act="bf16", B=2, H_q=32, H_kv=8, D=128, block_size=64,
+                                                   q_lens=[700, 500], past=[30, 0], window=200),
 }
 
 
