@@ -105,7 +105,11 @@ struct PfCfg {
   static constexpr int NST = D == 64 ? 3 : 2;
   static constexpr int OFF_K = OFF_Q + NQB * 2 * TILE;   // NST stages
   static constexpr int OFF_V = OFF_K + NST * TILE;     // NST stages
-  static constexpr int OFF_BAR = OFF_V + NST * TILE;   // mbarriers
+  // output staging (tiles A and B) for tiled stores of full 16-bit O tiles,
+  // where it fits
+  static constexpr int NOST = D == 64 ? 2 : 0;
+  static constexpr int OFF_OST = OFF_V + NST * TILE;
+  static constexpr int OFF_BAR = OFF_OST + NOST * TILE;   // mbarriers
   static constexpr int NBAR = 1 + 3 * NST + 8 + 2 * kPfRing;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int OFF_FLAG = OFF_TMEM + 8;
@@ -340,7 +344,8 @@ template <typename T, int D, bool DYN>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                       int n_slots, int mode, int box_rows, int box_shift, int max_tiles, int n_items) {
+                       const __grid_constant__ CUtensorMap tm_o, int n_slots, int mode, int box_rows,
+                       int box_shift, int max_tiles, int n_items) {
   using C = PfCfg<D>;
   constexpr uint32_t FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = idesc_f16(FMT, kPfBM, kPfBN, 0);
@@ -901,6 +906,18 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         finalize_row(m_used, l_sum, sink2, a, inv_l, lse);
         const float f = a * inv_l;
         T* out = static_cast<T*>(p.out) + orow * D;
+        // 16-bit output (`mode` bit 3): each warp whose 32 rows are all
+        // present writes them to its 128-byte-swizzled 4 KB of the group's
+        // staging tile (lane l's 16-byte chunk c at l * 128 + (c ^ (l & 7)) *
+        // 16) and its lane 0 stores them with one tiled store, instead of 32
+        // rows of scattered stores; no other warp takes part
+        const int w4 = warp & 3;
+        const bool tma_o = C::NOST > 0 && (mode & 8) && 32 * (w4 + 1) <= rows_t;   // warp-uniform
+        unsigned char* const stg = smem + C::OFF_OST + t * C::TILE + w4 * 4096;
+        if (tma_o) {
+          if (lane == 0) bulk_wait_read0();   // the warp's previous store has read its staging rows
+          __syncwarp();
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -911,7 +928,18 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-            if (mine && p.out_f32) {
+          if (tma_o) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = pack_pair<T>(u2f(o[e + 0]) * f, u2f(o[e + 1]) * f);
+              v.y = pack_pair<T>(u2f(o[e + 2]) * f, u2f(o[e + 3]) * f);
+              v.z = pack_pair<T>(u2f(o[e + 4]) * f, u2f(o[e + 5]) * f);
+              v.w = pack_pair<T>(u2f(o[e + 6]) * f, u2f(o[e + 7]) * f);
+              const int ch = c * 4 + e / 8;
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((ch ^ (lane & 7)) << 4)) = v;
+            }
+          } else if (mine && p.out_f32) {
             float* o32 = static_cast<float*>(p.out) + orow * D + c * 32;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
@@ -929,6 +957,14 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
             }
           }
         }
+        if (tma_o) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tm_o, stg, 0, hq, g.t_begin + q0_t + 32 * w4);
+            bulk_commit();
+          }
+        }
         if (mine && p.lse) p.lse[orow] = lse;
       if (j_hi > j_lo) {   // O_t may now be overwritten by the next item
         tc_fence_before();
@@ -940,6 +976,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       item = item_next;
     }
     if (!ok) *abort_flag = 1;
+    if (C::NOST > 0 && lane == 0) bulk_wait0();   // this warp's tiled stores are done
   }
   __syncthreads();
   if (*abort_flag) {
@@ -1033,7 +1070,7 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   const int box_rows = p.bs < kPfBN ? p.bs : kPfBN;
   int box_shift = 0;
   while ((1 << box_shift) < box_rows) ++box_shift;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const cuuint64_t qd[3] = {(cuuint64_t)D, (cuuint64_t)p.H_q, (cuuint64_t)p.T};
   const cuuint64_t qs[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.H_q * D * 2};
   const cuuint32_t qb[3] = {64, 1, (cuuint32_t)kPfBM};
@@ -1045,6 +1082,12 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   if ((rc = encode(&tq, dt, 3, p.q, qd, qs, qb)) != SPA_OK) return rc;
   if ((rc = encode(&tk, dt, 4, p.k_cache, kd, ks, kbx)) != SPA_OK) return rc;
   if ((rc = encode(&tv, dt, 4, p.v_cache, kd, ks, kbx)) != SPA_OK) return rc;
+  // tiled stores of the output, 32 rows of one head per box: 16-bit output
+  // (not a shard's fp32 partial) with room for the staging tiles
+  const bool tma_out = C::NOST > 0 && !p.out_f32 && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;
+  const cuuint32_t ob[3] = {64, 1, 32};
+  to = tq;
+  if (tma_out && (rc = encode(&to, dt, 3, p.out, qd, qs, ob)) != SPA_OK) return rc;
   // head pairs when the group size is even, tile pairs otherwise (see pf_geom_load)
   const int hp = (p.G % 2 == 0) ? 1 : 0;
   const int n_slots = hp ? (p.max_q + kPfBM - 1) / kPfBM : (p.max_q + 2 * kPfBM - 1) / (2 * kPfBM);
@@ -1073,8 +1116,8 @@ static int launch_pf(const AttnParams& p, CUtensorMapDataType dt, cudaStream_t s
   // schedules dynamically (a static assignment of the unequal causal items
   // measured slower).
   const int grid = persistent ? (int)std::min<long long>(items, std::max(sms, 1)) : (int)items;
-  const int mode = hp | (persistent ? 2 : 0) | (dyn ? 4 : 0);
-  return launch_pdl(kern, dim3(grid), dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, n_slots, mode, box_rows,
+  const int mode = hp | (persistent ? 2 : 0) | (dyn ? 4 : 0) | (tma_out ? 8 : 0);
+  return launch_pdl(kern, dim3(grid), dim3(kPfThreads), C::SMEM, stream, p, tq, tk, tv, to, n_slots, mode, box_rows,
                     box_shift, max_tiles, (int)items);
 }
 
