@@ -57,7 +57,7 @@ struct AttnParams {
   int32_t* slot_out;
   int max_seqlen_q;      // host bounds for the step-1 status bits
   int max_seqlen_k;
-  int cluster_merge;     // 1: the splits of a unit are one cluster, merged in shared memory
+  int cluster_merge;     // 1: the splits of a unit are one cluster, merged after a cluster barrier
   // one shard of a sequence split across devices: main-cache keys lo <= j < hi
   // of request b ([B, 2], or nullptr for all); out_f32: `out` is fp32 (the
   // shard's partial output; the host passes no sink then)

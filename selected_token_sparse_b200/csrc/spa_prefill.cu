@@ -5,29 +5,37 @@
 // real contractions, so they run as 128x128xD tcgen05.mma tiles, and the
 // kernel is organised so that the tensor core and the softmax overlap:
 //
-//   CTA    = one q head x one request x a PAIR of 128-row q tiles (A, B);
-//            launched longest pairs first (q tiles in reverse order); each q
-//            tile runs only the key tiles its own rows can see.
+//   item   = two 128-row q tiles (A, B) of one request that read one kv
+//            head: the same rows of two q heads when the group size is even
+//            (both tiles see the same key tiles), else two consecutive tiles
+//            of one q head; each q tile runs only the key tiles its own rows
+//            can see.  Causal items run one CTA each, longest first;
+//            window-bounded items run persistently, one CTA per SM claiming
+//            items from a work counter in the workspace (pf_geom_load and
+//            the kernel's comment give the orders and the claim protocol).
 //   TMEM   = S_A | S_B | O_A | O_B (4 x 128 columns); P of a tile overwrites
 //            its S as packed 16-bit pairs and feeds the PV MMA from TMEM.
-//   warp 9 = K/V producer (one thread): K and V tiles through a 2-stage ring
-//            from the paged cache (4-D tensor map over [num_blocks,
-//            block_size, H_kv, D]; the block id is a coordinate taken from the
-//            block table; an unmapped block is read from an out-of-range
+//   warp 9 = K/V producer (one thread): K and V tiles through a ring of 3
+//            stages (D = 64) or 2 (D = 128) from the paged cache (4-D tensor
+//            map over [num_blocks, block_size, H_kv, D]; the block id is a
+//            coordinate taken from the block table, read before the wait for
+//            a free stage; an unmapped block is read from an out-of-range
 //            coordinate, i.e. zeros, and masked; 128-byte swizzle; no
-//            multicast).
-//   warp 8 = MMA issuer (one thread) and the Q loads.  Per 128-key step j and
-//            q tile t it issues PV_t(j) (O_t += P_t V_j) as soon as the
-//            softmax group hands over P_t, then S_t(j + 1), so one group's
-//            MMAs run on the tensor core while the other group's softmax runs
-//            on the CUDA cores.
+//            multicast); on the persistent schedule it also claims the items.
+//   warp 8 = MMA issuer (one thread) and the Q loads (two Q buffers at
+//            D = 64: the next item's Q lands during this item).  Per 128-key
+//            step j and q tile t it issues PV_t(j) (O_t += P_t V_j) as soon as
+//            the softmax group hands over P_t, then S_t(j + 1), so one
+//            group's MMAs run on the tensor core while the other group's
+//            softmax runs on the CUDA cores.
 //   warps 0-3 / 4-7 = softmax of tile A / B: thread i owns row i (TMEM lane i)
 //            and reads its row of S from TMEM once per step; masks only the
 //            tiles that cross the causal diagonal, the window edge, the end
 //            of the keys or an unmapped block; keeps a running max in log2
 //            units that is raised (O rescaled in TMEM) only when a tile's max
 //            exceeds it by more than 8, so P <= 2^8; the scale is folded into
-//            one FFMA ahead of ex2.approx.
+//            one FFMA ahead of ex2.approx.  16-bit output leaves through
+//            per-warp tiled stores at D = 64.
 //   registers: warps 8-11 (warps 10-11 idle) hand registers to the softmax
 //            warpgroups (setmaxnreg), which need a row of S in registers.
 //   sink   = folded into the final normalisation (denominator only).
