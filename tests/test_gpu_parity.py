@@ -25,7 +25,10 @@ def test_workload_small(name):
 
 @pytest.mark.parametrize("name", W.WORKLOADS)
 def test_workload_full_size(name):
-    """The workloads at full size; prefill outputs are sampled rows."""
+    """The workloads at full size; prefill outputs are sampled rows: each
+    request's first and last two rows, six random rows, and one random row of
+    every 128-row q tile (every head of a sampled row is compared, so every
+    prefill work item is checked)."""
     wl = W.by_name(name, small=False)
     tokens = None
     if name in ("ragged_prefill_f16", "windowed_chunked_prefill_f16"):
@@ -35,6 +38,8 @@ def test_workload_full_size(name):
         for b in range(wl.B):
             picks |= {int(cu[b]), int(cu[b]) + 1, int(cu[b + 1]) - 1, int(cu[b + 1]) - 2}
             picks |= set(int(x) for x in rng.integers(cu[b], cu[b + 1], size=6))
+            for q0 in range(int(cu[b]), int(cu[b + 1]), 128):
+                picks.add(int(rng.integers(q0, min(q0 + 128, int(cu[b + 1])))))
         tokens = sorted(picks)
     got = run(wl)
     ref = oracle_step(wl, tokens=tokens)
