@@ -127,6 +127,9 @@ struct PfCfg {
   // one CTA (holding all 512 TMEM columns) is resident per SM
   static constexpr int SMEM = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
   static constexpr uint32_t TX_TILE = (uint32_t)TILE;
+  static_assert(SMEM <= 227 * 1024, "one CTA's shared memory");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_OST % 1024 == 0 && OFF_BAR % 8 == 0,
+                "128-byte-swizzled tiles start on 1024-byte boundaries");
 };
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
